@@ -1,0 +1,204 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library.
+ *
+ * KDA is the gated delta rule with a per-channel gate.  For every sequence and
+ * head the library carries a state S (d_k x d_v, fp32) and, for each token t
+ * with query q_t, key k_t (d_k), value v_t (d_v), per-channel log decay
+ * log_alpha_t (d_k) and write rate beta_t (scalar), computes
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * i.e. decay the old state channel by channel, read the old answer with the
+ * key, form the error against v_t, write beta_t times the error back along the
+ * key, then read the output with the query.
+ *
+ * Where the operation is defined (web pages, cited by title / address):
+ *   - delta rule S <- S + k^T (v - S k) and the scalar gate alpha in [0, 1]
+ *     (alpha = 1: pure delta rule, alpha = 0: memory cleared):
+ *     "From GPT-2 to Kimi K3" essay, pwwt.cn/news/3716252, delta-rule and
+ *     Gated DeltaNet paragraphs;
+ *   - one alpha per channel instead of one per head: same essay, Kimi Linear
+ *     paragraph; "我终于看懂了 KDA" explainer, pwwt.cn/news/3787313, section 9;
+ *   - order decay -> read -> error -> write and the learning rate beta:
+ *     the explainer, sections 6 and 8;
+ *   - chunkwise prefill (chunk C = 64 or 128, masked attention inside a chunk,
+ *     state-first recurrence across chunks) with WY / DPLR restructuring:
+ *     the essay's chunkwise paragraph; the explainer, sections 16 and 17;
+ *   - token-by-token decode (read state, emit output, update state):
+ *     the explainer, section 15.
+ *
+ * Conventions shared by all calls
+ *   - Device pointers are caller-owned CUDA device memory; the library keeps no
+ *     reference after a call returns and never allocates device memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  Input validation happens on the host before
+ *     anything is launched: a call that returns an error other than
+ *     KDA_ERR_CUDA has launched nothing and written nothing.
+ *   - Token-major layouts, last dimension contiguous:
+ *       q, k, log_alpha : [B, T, H, dk]      v, o : [B, T, H, dv]
+ *       beta            : [B, T, H]
+ *       states          : [N, H, dk, dv] fp32 (dv contiguous)
+ *     For packed variable-length batches B = 1, T = total tokens, and
+ *     cu_seqlens gives the N + 1 sequence offsets.
+ *   - q, k, v, log_alpha, beta and o share one dtype (KDA_BF16 or KDA_F32);
+ *     states are always fp32; accumulation is fp32.
+ *   - log_alpha <= 0 (alpha in [0, 1]); -inf means alpha = 0.  Kernels clamp
+ *     log_alpha at -100 (exp(-100) is below every fp32 normal number).
+ *   - No scaling of q is applied: o_t = S_t^T q_t exactly.
+ *   - Supported sizes: dk, dv in {64, 128}; every pointer 16-byte aligned.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_NULL = -1,       /* a required pointer is NULL                     */
+    KDA_ERR_SHAPE = -2,      /* unsupported or inconsistent sizes              */
+    KDA_ERR_DTYPE = -3,      /* unknown dtype                                  */
+    KDA_ERR_ALIGN = -4,      /* a pointer is not 16-byte aligned               */
+    KDA_ERR_CHUNK = -5,      /* chunk size is not 64 or 128                    */
+    KDA_ERR_SEQLENS = -6,    /* cu_seqlens not 0-based, non-decreasing, = T    */
+    KDA_ERR_WORKSPACE = -7,  /* workspace NULL or smaller than required        */
+    KDA_ERR_CUDA = -8,       /* a CUDA runtime call or launch failed           */
+    KDA_ERR_TIMEOUT = -9,    /* a bounded device-side wait gave up             */
+    KDA_ERR_DEVICE = -10     /* the current device is not sm_100 (B200)       */
+} kda_status;
+
+typedef enum {
+    KDA_BF16 = 0,
+    KDA_F32 = 1
+} kda_dtype;
+
+/* Prefill algorithm.  AUTO picks the tensor-core path for bf16 with
+ * dk = dv = 128 and the CUDA-core path otherwise.  SIMT is the four-kernel
+ * CUDA-core split (cumulative decay, WY/UT, state carry, output) that keeps
+ * its intermediates in the workspace; TC is the tcgen05 tensor-core path. */
+typedef enum {
+    KDA_ALGO_AUTO = 0,
+    KDA_ALGO_SIMT = 1,
+    KDA_ALGO_TC = 2
+} kda_algo;
+
+/* Human-readable name of a status code (static string, never NULL). */
+KDA_API const char* kda_status_string(int status);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+KDA_API int kda_version(void);
+
+/*
+ * Workspace bytes kda_chunk_fwd needs for this problem (0 on invalid sizes).
+ *   cu_seqlens_host : NULL for B sequences of length T each; else a HOST array of
+ *                     n_seqs + 1 int32 offsets (requires B == 1).
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                    kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                    int n_seqs);
+
+/* As above for a chosen algorithm (AUTO resolves as kda_chunk_fwd does). */
+KDA_API size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int C,
+                                       kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                       int n_seqs, kda_algo algo);
+
+/*
+ * Chunkwise prefill.  Processes every sequence from its initial state and
+ * writes o for every token and (optionally) the final state of every sequence.
+ *
+ *   q, k, v, log_alpha, beta : device inputs (layouts above), dtype `dtype`
+ *   init_state      : device [N, H, dk, dv] fp32, or NULL for zero states
+ *   cu_seqlens_host : NULL (B sequences of T tokens) or a HOST array of
+ *                     n_seqs + 1 int32 offsets, cu[0] = 0, non-decreasing,
+ *                     cu[n_seqs] = T, with B = 1; empty sequences are allowed
+ *   n_seqs          : number of sequences when cu_seqlens_host != NULL
+ *   C               : chunk size, 64 or 128; chunks restart at each sequence
+ *                     start and the last chunk of a sequence may be partial
+ *   o               : device output [B, T, H, dv], dtype `dtype`
+ *   final_state     : device [N, H, dk, dv] fp32, or NULL; may alias init_state
+ *   workspace       : device scratch of at least kda_chunk_fwd_workspace_size()
+ *                     bytes, 256-byte aligned; contents on entry are ignored
+ *   stream          : cudaStream_t (as void*)
+ * T == 0 (or all sequences empty) is valid: final_state = init_state (or 0).
+ */
+KDA_API kda_status kda_chunk_fwd(const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta, kda_dtype dtype,
+                         const float* init_state, const int32_t* cu_seqlens_host,
+                         int n_seqs, int B, int T, int H, int dk, int dv, int C,
+                         void* o, float* final_state, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* kda_chunk_fwd with an explicit algorithm choice (same arguments otherwise). */
+KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                            const void* log_alpha, const void* beta, kda_dtype dtype,
+                            const float* init_state, const int32_t* cu_seqlens_host,
+                            int n_seqs, int B, int T, int H, int dk, int dv, int C,
+                            void* o, float* final_state, void* workspace,
+                            size_t workspace_bytes, void* stream, kda_algo algo);
+
+/*
+ * Byte offsets, inside the workspace of the SIMT algorithm, of the
+ * intermediates that its four kernels exchange (for inspection by tests):
+ *   offsets[0] g       fp32 [T_total, H, dk]  chunk-local inclusive cumulative log decay
+ *   offsets[1] U       fp32 [T_total, H, dv]  (I + A)^-1 Diag(beta) V
+ *   offsets[2] Wk      fp32 [T_total, H, dk]  (I + A)^-1 Diag(beta) (K . exp(g))
+ *   offsets[3] W       fp32 [T_total, H, dv]  per-token corrections U - Wk S_n
+ *   offsets[4] S_chunk fp32 [n_chunks, H, dk, dv] start state of every chunk
+ * (T_total = B * T; chunks are numbered sequence by sequence.)  Same size
+ * arguments as kda_chunk_fwd_workspace_size.
+ */
+KDA_API kda_status kda_chunk_simt_offsets(int B, int T, int H, int dk, int dv, int C,
+                                  const int32_t* cu_seqlens_host, int n_seqs,
+                                  size_t offsets[5]);
+
+/*
+ * Optional per-kernel timing hook for the calling host thread.  When n_events
+ * > 0, the next kda_chunk_fwd / kda_chunk_fwd_ex call made from this thread
+ * records events[0] on its stream before its first kernel and events[i] after
+ * its i-th kernel (i = 1 .. number of kernels), then clears the hook.  Calls
+ * that launch more kernels than n_events - 1 record only the first ones.
+ *   events   : array of cudaEvent_t (as void*), created by the caller
+ *   n_events : number of entries (0 clears the hook)
+ * The events only observe the launches; kda_chunk_fwd_kernels tells how many
+ * kernels a call launches and their names.
+ */
+KDA_API kda_status kda_set_timing_events(void* const* events, int n_events);
+
+/*
+ * Number of kernels kda_chunk_fwd_ex launches for this problem and algorithm
+ * (after AUTO resolution), and their names through names[i] (static strings;
+ * names may be NULL, at most max_names entries are written).  Returns the
+ * count, or a negative kda_status on invalid sizes.
+ */
+KDA_API int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype dtype,
+                                  const int32_t* cu_seqlens_host, int n_seqs, kda_algo algo,
+                                  const char** names, int max_names);
+
+/*
+ * One decode step for N independent sequences, one token each; the state is
+ * updated in place (read once, written once).
+ *   q, k, log_alpha : device [N, H, dk]; v : device [N, H, dv]; beta : [N, H]
+ *   state           : device [N, H, dk, dv] fp32, read and overwritten
+ *   o               : device [N, H, dv], dtype `dtype`
+ */
+KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, kda_dtype dtype,
+                           float* state, int N, int H, int dk, int dv, void* o,
+                           void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

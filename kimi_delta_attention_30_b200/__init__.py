@@ -1,0 +1,220 @@
+"""Python binding of the KDA C ABI (``include/kda.h``, ``libkda.so``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory and streams.  There
+is no CPU path: tensors must live on a CUDA device, and a missing or unloadable
+``libkda.so`` raises :class:`KdaError`.
+
+Calls:
+
+* :func:`chunk_fwd` -- chunkwise prefill (``kda_chunk_fwd``).
+* :func:`decode_step` -- one recurrent step, state updated in place
+  (``kda_decode_step``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_BF16, KDA_F32 = 0, 1
+ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+_DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = _lib_or_none().kda_status_string(status).decode() if _lib_or_none() else f"status {status}"
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def _declare(lib):
+    c_int, c_size, vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    lib.kda_status_string.argtypes = [c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    lib.kda_version.restype = c_int
+    lib.kda_chunk_fwd_workspace_size.argtypes = [c_int] * 6 + [c_int, i32p, c_int]
+    lib.kda_chunk_fwd_workspace_size.restype = c_size
+    lib.kda_chunk_fwd_workspace_size_ex.argtypes = [c_int] * 6 + [c_int, i32p, c_int, c_int]
+    lib.kda_chunk_fwd_workspace_size_ex.restype = c_size
+    lib.kda_chunk_fwd.argtypes = [vp] * 5 + [c_int, vp, i32p, c_int] + [c_int] * 6 + [vp, vp, vp, c_size, vp]
+    lib.kda_chunk_fwd.restype = c_int
+    lib.kda_chunk_fwd_ex.argtypes = lib.kda_chunk_fwd.argtypes + [c_int]
+    lib.kda_chunk_fwd_ex.restype = c_int
+    lib.kda_chunk_simt_offsets.argtypes = [c_int] * 6 + [i32p, c_int, ctypes.POINTER(c_size)]
+    lib.kda_chunk_simt_offsets.restype = c_int
+    lib.kda_decode_step.argtypes = [vp] * 5 + [c_int, vp] + [c_int] * 4 + [vp, vp]
+    lib.kda_decode_step.restype = c_int
+    lib.kda_set_timing_events.argtypes = [ctypes.POINTER(vp), c_int]
+    lib.kda_set_timing_events.restype = c_int
+    lib.kda_chunk_fwd_kernels.argtypes = [c_int] * 7 + [i32p, c_int, c_int, ctypes.POINTER(ctypes.c_char_p), c_int]
+    lib.kda_chunk_fwd_kernels.restype = c_int
+    return lib
+
+
+def _lib_or_none():
+    return _lib
+
+
+def lib():
+    """Load ``libkda.so`` (building it first when it is missing or stale and
+    nvcc is present).  Raises :class:`KdaError` when it cannot be loaded."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            try:
+                from . import build as _build
+                if _build._stale():
+                    _build.build()
+            except Exception as exc:  # noqa: BLE001 - report any build problem
+                if not os.path.exists(LIB_PATH):
+                    raise KdaError(-8, f"libkda.so missing and could not be built ({exc})") from exc
+            try:
+                _lib = _declare(ctypes.CDLL(LIB_PATH))
+            except OSError as exc:
+                raise RuntimeError(f"cannot load {LIB_PATH}: {exc}") from exc
+    return _lib
+
+
+def exported_symbols():
+    return ["kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
+            "kda_chunk_fwd_workspace_size_ex", "kda_chunk_fwd", "kda_chunk_fwd_ex",
+            "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels"]
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cu_arg(cu_seqlens):
+    if cu_seqlens is None:
+        return None, 0, None
+    arr = np.ascontiguousarray(np.asarray(cu_seqlens), dtype=np.int32)
+    return arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(arr) - 1, arr
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_cuda(name, t, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def workspace_size(B, T, H, dk, dv, C, dtype, cu_seqlens=None, algo="auto") -> int:
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    d = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return int(lib().kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, C, d, cu, n, ALGOS[algo]))
+
+
+def simt_offsets(B, T, H, dk, dv, C, cu_seqlens=None):
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    out = (ctypes.c_size_t * 5)()
+    st = lib().kda_chunk_simt_offsets(B, T, H, dk, dv, C, cu, n, out)
+    if st != 0:
+        raise KdaError(st, "kda_chunk_simt_offsets")
+    return [int(x) for x in out]
+
+
+def chunk_kernels(B, T, H, dk, dv, C, dtype, cu_seqlens=None, algo="auto"):
+    """Names of the kernels one chunk_fwd call launches, in launch order."""
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    d = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    names = (ctypes.c_char_p * 32)()
+    cnt = lib().kda_chunk_fwd_kernels(B, T, H, dk, dv, C, d, cu, n, ALGOS[algo], names, 32)
+    if cnt < 0:
+        raise KdaError(cnt, "kda_chunk_fwd_kernels")
+    return [names[i].decode() for i in range(cnt)]
+
+
+def set_timing_events(events):
+    """Per-kernel timing hook for the next chunk_fwd on this thread: a list of
+    torch.cuda.Event (recorded before the first kernel and after each kernel)."""
+    arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    st = lib().kda_set_timing_events(arr, len(events))
+    if st != 0:
+        raise KdaError(st, "kda_set_timing_events")
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int = 64,
+              output_final_state: bool = True, o=None, final_state=None, workspace=None,
+              algo: str = "auto", stream=None):
+    """Chunkwise KDA prefill.
+
+    q, k, log_alpha ``[B, T, H, dk]``; v ``[B, T, H, dv]``; beta ``[B, T, H]``;
+    all one dtype (bf16 or fp32), contiguous, on one CUDA device.  ``cu_seqlens``
+    (host sequence, N + 1 offsets) selects packed varlen mode with B = 1.
+    ``init_state`` ``[N, H, dk, dv]`` fp32 or None.  Returns ``(o, final_state)``
+    (final_state is None when ``output_final_state`` is False).
+    """
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        _check_cuda(name, t, dt)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu, n_seqs, _keep = _cu_arg(cu_seqlens)
+    N = n_seqs if cu_seqlens is not None else B
+    _check_cuda("init_state", init_state, torch.float32)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_cuda("o", o, dt)
+    _check_cuda("final_state", final_state, torch.float32)
+    need = lib().kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, C, _DTYPES[dt], cu, n_seqs, ALGOS[algo])
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
+    _check_cuda("workspace", workspace)
+    st = lib().kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o), _ptr(final_state),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream_handle(stream), ALGOS[algo])
+    if st != 0:
+        raise KdaError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+def decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
+    """One KDA decode step for N sequences; ``state`` ``[N, H, dk, dv]`` fp32 is
+    updated in place.  q, k, log_alpha ``[N, H, dk]``, v ``[N, H, dv]``, beta
+    ``[N, H]``.  Returns o ``[N, H, dv]``."""
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        _check_cuda(name, t, dt)
+    _check_cuda("state", state, torch.float32)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dt, device=q.device)
+    _check_cuda("o", o, dt)
+    st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], _ptr(state),
+                               N, H, dk, dv, _ptr(o), _stream_handle(stream))
+    if st != 0:
+        raise KdaError(st, "kda_decode_step")
+    return o

@@ -1,0 +1,281 @@
+// Host side of the C ABI declared in include/kda.h: argument validation,
+// workspace planning, the sequence table and kernel dispatch.  Nothing here
+// allocates device memory; all scratch lives in the caller's workspace.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+
+cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              const float* init_state, void* o, float* final_state, const ChunkMap& cmap,
+                              const SeqMap& smap, int n_chunks, int n_seqs, int H, int C, void* tc_ws,
+                              cudaStream_t stream);
+size_t tc_workspace_bytes(int n_chunks, int H, int C);
+bool tc_available();
+
+TimingHook& timing_hook() {
+    static thread_local TimingHook hook{{nullptr}, 0};
+    return hook;
+}
+
+extern const char* const kTcKernelNames[];
+extern const int kTcKernelCount;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+const char* const kSimtKernelNames[] = {"k1_cumsum", "k2_wy", "k3_state", "k4_output"};
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Problem geometry shared by the workspace query and the launch.
+struct Plan {
+    int n_seqs = 0;
+    int n_chunks = 0;
+    long long total_tokens = 0;
+    bool varlen = false;
+    std::vector<SeqInfo> natural;   // chunk0 non-decreasing (varlen only)
+    std::vector<SeqInfo> by_len;    // longest first (varlen only)
+};
+
+kda_status make_plan(int B, int T, int H, int dk, int dv, int C, const int32_t* cu, int n_seqs, Plan& p) {
+    if (H <= 0 || B < 0 || T < 0) return KDA_ERR_SHAPE;
+    if (!((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_SHAPE;
+    if (C != 64 && C != 128) return KDA_ERR_CHUNK;
+    if (cu == nullptr) {
+        p.n_seqs = B;
+        long long ncps = (T + C - 1) / C;
+        if ((long long)B * ncps > 0x7fffffffLL || (long long)B * T > 0x7fffffffLL) return KDA_ERR_SHAPE;
+        p.n_chunks = (int)(B * ncps);
+        p.total_tokens = (long long)B * T;
+        return KDA_OK;
+    }
+    if (B != 1 || n_seqs < 1) return KDA_ERR_SEQLENS;
+    if (cu[0] != 0 || cu[n_seqs] != T) return KDA_ERR_SEQLENS;
+    p.varlen = true;
+    p.n_seqs = n_seqs;
+    p.total_tokens = T;
+    p.natural.resize(n_seqs);
+    long long chunks = 0;
+    for (int s = 0; s < n_seqs; ++s) {
+        if (cu[s + 1] < cu[s]) return KDA_ERR_SEQLENS;
+        int len = cu[s + 1] - cu[s];
+        p.natural[s] = SeqInfo{cu[s], len, (int)chunks, s};
+        chunks += (len + C - 1) / C;
+    }
+    if (chunks > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    p.n_chunks = (int)chunks;
+    p.by_len = p.natural;
+    std::stable_sort(p.by_len.begin(), p.by_len.end(),
+                     [](const SeqInfo& a, const SeqInfo& b) { return a.len > b.len; });
+    return KDA_OK;
+}
+
+// Workspace layout: [sequence tables][algorithm scratch]
+size_t table_bytes(const Plan& p) { return p.varlen ? align_up(2 * sizeof(SeqInfo) * (size_t)p.n_seqs) : 0; }
+
+struct SimtLayout {
+    size_t off[5];
+    size_t total;
+};
+
+SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
+    SimtLayout L;
+    size_t o = table_bytes(p);
+    const size_t tok = (size_t)p.total_tokens * H;
+    L.off[0] = o; o = align_up(o + tok * dk * sizeof(float));               // g
+    L.off[1] = o; o = align_up(o + tok * dv * sizeof(float));               // U
+    L.off[2] = o; o = align_up(o + tok * dk * sizeof(float));               // Wk
+    L.off[3] = o; o = align_up(o + tok * dv * sizeof(float));               // W
+    L.off[4] = o; o = align_up(o + (size_t)p.n_chunks * H * dk * dv * sizeof(float));  // S_chunk
+    L.total = o;
+    return L;
+}
+
+kda_algo resolve(kda_algo algo, kda_dtype dtype, int dk, int dv) {
+    if (algo != KDA_ALGO_AUTO) return algo;
+    return (tc_available() && dtype == KDA_BF16 && dk == 128 && dv == 128) ? KDA_ALGO_TC : KDA_ALGO_SIMT;
+}
+
+size_t workspace_for(const Plan& p, int H, int dk, int dv, int C, kda_algo algo) {
+    if (algo == KDA_ALGO_TC) return align_up(table_bytes(p) + tc_workspace_bytes(p.n_chunks, H, C));
+    return simt_layout(p, H, dk, dv).total;
+}
+
+// Device capability check, cached per device ordinal.
+kda_status check_device() {
+    static std::mutex mu;
+    static int cached[64];
+    static bool init = false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!init) { std::fill(cached, cached + 64, -1); init = true; }
+    if (dev < 0 || dev >= 64) return KDA_ERR_DEVICE;
+    if (cached[dev] < 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 0;
+    }
+    return cached[dev] ? KDA_OK : KDA_ERR_DEVICE;
+}
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_NULL: return "KDA_ERR_NULL: a required pointer is NULL";
+        case KDA_ERR_SHAPE: return "KDA_ERR_SHAPE: unsupported or inconsistent sizes";
+        case KDA_ERR_DTYPE: return "KDA_ERR_DTYPE: unknown dtype";
+        case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: pointer not 16-byte aligned";
+        case KDA_ERR_CHUNK: return "KDA_ERR_CHUNK: chunk size must be 64 or 128";
+        case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: invalid cu_seqlens";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait expired";
+        case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: current device is not sm_100 (B200)";
+        default: return "KDA: unknown status";
+    }
+}
+
+int kda_version(void) { return 100; }
+
+size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int C, kda_dtype dtype,
+                                       const int32_t* cu_seqlens_host, int n_seqs, kda_algo algo) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return 0;
+    Plan p;
+    if (make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
+    algo = resolve(algo, dtype, dk, dv);
+    if (algo == KDA_ALGO_TC && !(dtype == KDA_BF16 && dk == 128 && dv == 128)) return 0;
+    return std::max<size_t>(workspace_for(p, H, dk, dv, C, algo), kAlign);
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int C, kda_dtype dtype,
+                                    const int32_t* cu_seqlens_host, int n_seqs) {
+    return kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, C, dtype, cu_seqlens_host, n_seqs, KDA_ALGO_AUTO);
+}
+
+kda_status kda_chunk_simt_offsets(int B, int T, int H, int dk, int dv, int C, const int32_t* cu_seqlens_host,
+                                  int n_seqs, size_t offsets[5]) {
+    if (!offsets) return KDA_ERR_NULL;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    SimtLayout L = simt_layout(p, H, dk, dv);
+    for (int i = 0; i < 5; ++i) offsets[i] = L.off[i];
+    return KDA_OK;
+}
+
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                            kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs,
+                            int B, int T, int H, int dk, int dv, int C, void* o, float* final_state,
+                            void* workspace, size_t workspace_bytes, void* stream, kda_algo algo) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_SHAPE;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    algo = resolve(algo, dtype, dk, dv);
+    if (algo == KDA_ALGO_TC && !(dtype == KDA_BF16 && dk == 128 && dv == 128)) return KDA_ERR_SHAPE;
+    const bool has_tokens = p.total_tokens > 0;
+    if (has_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, o, final_state};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return KDA_ERR_ALIGN;
+    if (workspace_bytes < workspace_for(p, H, dk, dv, C, algo)) return KDA_ERR_WORKSPACE;
+    if ((st = check_device()) != KDA_OK) return st;
+    if (p.n_seqs == 0) return KDA_OK;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    const int ncps = (int)((T + C - 1) / C);
+    ChunkMap cmap{nullptr, p.n_seqs, T, C, ncps};
+    SeqMap smap{nullptr, T, C, ncps};
+    if (p.varlen) {
+        std::vector<SeqInfo> both(p.natural);
+        both.insert(both.end(), p.by_len.begin(), p.by_len.end());
+        if (cudaMemcpyAsync(ws, both.data(), both.size() * sizeof(SeqInfo), cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        cmap.seqs = (const SeqInfo*)ws;
+        smap.order = (const SeqInfo*)ws + p.n_seqs;
+    }
+    timing_mark(s, 0);
+    cudaError_t err;
+    if (algo == KDA_ALGO_SIMT) {
+        SimtLayout L = simt_layout(p, H, dk, dv);
+        SimtWorkspace w{(float*)(ws + L.off[0]), (float*)(ws + L.off[1]), (float*)(ws + L.off[2]),
+                        (float*)(ws + L.off[3]), (float*)(ws + L.off[4])};
+        err = launch_simt_prefill(dtype, q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap,
+                                  p.n_chunks, p.n_seqs, H, dk, dv, C, w, s);
+    } else {
+        err = launch_tc_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap, p.n_chunks,
+                                p.n_seqs, H, C, ws + table_bytes(p), s);
+    }
+    timing_hook().n = 0;
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                         kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs,
+                         int B, int T, int H, int dk, int dv, int C, void* o, float* final_state, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, dtype, init_state, cu_seqlens_host, n_seqs, B, T, H, dk, dv,
+                            C, o, final_state, workspace, workspace_bytes, stream, KDA_ALGO_AUTO);
+}
+
+kda_status kda_set_timing_events(void* const* events, int n_events) {
+    TimingHook& h = timing_hook();
+    if (n_events < 0 || n_events > 32) return KDA_ERR_SHAPE;
+    if (n_events > 0 && !events) return KDA_ERR_NULL;
+    for (int i = 0; i < 32; ++i) h.ev[i] = (i < n_events) ? events[i] : nullptr;
+    h.n = n_events;
+    return KDA_OK;
+}
+
+int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype dtype,
+                          const int32_t* cu_seqlens_host, int n_seqs, kda_algo algo, const char** names,
+                          int max_names) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    algo = resolve(algo, dtype, dk, dv);
+    const char* const* list = (algo == KDA_ALGO_TC) ? kTcKernelNames : kSimtKernelNames;
+    const int n = (algo == KDA_ALGO_TC) ? kTcKernelCount : 4;
+    for (int i = 0; names && i < n && i < max_names; ++i) names[i] = list[i];
+    return n;
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                           kda_dtype dtype, float* state, int N, int H, int dk, int dv, void* o, void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (N < 0 || H <= 0 || !((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_SHAPE;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_NULL;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, state, o};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
+    kda_status st = check_device();
+    if (st != KDA_OK) return st;
+    cudaError_t err = launch_decode(dtype, q, k, v, log_alpha, beta, state, N, H, dk, dv, o, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,271 @@
+// CUDA-core (SIMT, fp32 arithmetic) chunkwise KDA prefill: four kernels that
+// exchange their intermediates through the workspace.
+//
+//   K1 cumulative log decay  g_r = sum_{j<=r} log alpha_j   (restarting per chunk)
+//   K2 WY/UT transform       A_{r,i} = beta_r sum_c k_rc k_ic exp(g_rc - g_ic), i < r
+//                            (I + A) U  = Diag(beta) V
+//                            (I + A) Wk = Diag(beta) (K . exp(g))
+//   K3 state carry           for each chunk in order: S_n -> workspace,
+//                            W = U - Wk S_n,
+//                            S_{n+1} = Diag(exp(g_C)) S_n + (K . exp(g_C - g))^T W
+//   K4 output                O = (Q . exp(g)) S_n + (M_incl . [(Q x K) exp(g_r - g_i)]) W
+//
+// Chunkwise form: "From GPT-2 to Kimi K3" essay (pwwt.cn/news/3716252),
+// chunkwise and Gated DeltaNet paragraphs (masked attention inside a chunk,
+// state-first recurrence across chunks, cumulative decay factors across
+// chunks); WY / DPLR restructuring: "我终于看懂了 KDA" explainer
+// (pwwt.cn/news/3787313), sections 16-17.  This path evaluates every decay
+// as exp of a non-positive difference g_r - g_i (r >= i), so it is exact for
+// any decay range; it serves the fp32 inputs and is the CUDA-core reference
+// for the tensor-core path.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBV = 32;   // d_v columns per state-carry block
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// K1: one block per (chunk, head), one thread per key channel.
+template <typename Tin>
+__global__ void __launch_bounds__(128) k1_cumsum(const Tin* __restrict__ la, float* __restrict__ g,
+                                                 ChunkMap cmap, int H, int dk) {
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, c = threadIdx.x;
+    float acc = 0.f;
+    for (int r = 0; r < len; ++r) {
+        size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
+        acc += fmaxf(to_f32(la[off]), kLogAlphaFloor);
+        g[off] = acc;
+    }
+}
+
+// K2: one block per (chunk, head).  Dynamic shared memory:
+//   A [C][C] | phase 1: Ks [C][dk], Gs [C][dk]  / phase 2: X [C][dk + dv]
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, const Tin* __restrict__ v,
+                                                  const Tin* __restrict__ beta, const float* __restrict__ g,
+                                                  float* __restrict__ U, float* __restrict__ Wk, ChunkMap cmap,
+                                                  int H, int dk, int dv, int C) {
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* A = smem;
+    float* Ks = A + C * C;
+    float* Gs = Ks + C * dk;
+
+    for (int e = tid; e < len * dk; e += kThreads) {
+        int r = e / dk, c = e - r * dk;
+        size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
+        Ks[r * dk + c] = to_f32(k[off]);
+        Gs[r * dk + c] = g[off];
+    }
+    __syncthreads();
+    // A, one warp per (r, i) pair, lanes over channels
+    for (int p = warp; p < len * len; p += kThreads / 32) {
+        int r = p / len, i = p - r * len;
+        float s = 0.f;
+        if (i < r) {
+            for (int c = lane; c < dk; c += 32)
+                s += Ks[r * dk + c] * Ks[i * dk + c] * expf(Gs[r * dk + c] - Gs[i * dk + c]);
+            s = warp_sum(s) * to_f32(beta[(size_t)(tok0 + r) * H + h]);
+        }
+        if (lane == 0) A[r * C + i] = s;
+    }
+    __syncthreads();
+    // forward substitution, one column per thread; X reuses the Ks/Gs region
+    float* X = Ks;
+    const int ncol = dk + dv;
+    for (int j = tid; j < ncol; j += kThreads) {
+        for (int r = 0; r < len; ++r) {
+            const size_t tok = (size_t)(tok0 + r) * H + h;
+            const float br = to_f32(beta[tok]);
+            float s;
+            if (j < dv) {
+                s = br * to_f32(v[tok * dv + j]);
+            } else {
+                const int c = j - dv;
+                s = br * to_f32(k[tok * dk + c]) * expf(g[tok * dk + c]);
+            }
+            for (int i = 0; i < r; ++i) s -= A[r * C + i] * X[i * ncol + j];
+            X[r * ncol + j] = s;
+            if (j < dv) U[tok * dv + j] = s;
+            else Wk[tok * dk + (j - dv)] = s;
+        }
+    }
+}
+
+// K3: one block per (sequence, head, d_v tile of kBV columns), sequential over
+// the sequence's chunks.  Shared: S [dk][kBV], M [C][dk] (Wk, then K . decay),
+// Ws [C][kBV], gC [dk].
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
+                                                     const float* __restrict__ U, const float* __restrict__ Wkg,
+                                                     float* __restrict__ Wg, float* __restrict__ S_chunk,
+                                                     const float* __restrict__ init_state,
+                                                     float* __restrict__ final_state, SeqMap smap, int H, int dk,
+                                                     int dv, int C) {
+    extern __shared__ float smem[];
+    const SeqInfo sq = smap.get(blockIdx.x);
+    const int h = blockIdx.y, j0 = blockIdx.z * kBV, tid = threadIdx.x;
+    float* S = smem;
+    float* M = S + dk * kBV;
+    float* Ws = M + C * dk;
+    float* gC = Ws + C * kBV;
+
+    const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
+    for (int e = tid; e < dk * kBV; e += kThreads) {
+        int c = e / kBV, j = e - c * kBV;
+        S[e] = init_state ? init_state[st_base + (size_t)c * dv + j0 + j] : 0.f;
+    }
+    __syncthreads();
+    const int nch = (sq.len + C - 1) / C;
+    for (int n = 0; n < nch; ++n) {
+        const int t0 = sq.tok0 + n * C;
+        const int L = min(C, sq.len - n * C);
+        const size_t sc_base = ((size_t)(sq.chunk0 + n) * H + h) * dk * dv;
+        for (int e = tid; e < dk * kBV; e += kThreads) {
+            int c = e / kBV, j = e - c * kBV;
+            S_chunk[sc_base + (size_t)c * dv + j0 + j] = S[e];
+        }
+        for (int e = tid; e < L * dk; e += kThreads) {
+            int r = e / dk, c = e - r * dk;
+            M[e] = Wkg[((size_t)(t0 + r) * H + h) * dk + c];
+        }
+        __syncthreads();
+        // W = U - Wk S
+        for (int e = tid; e < L * kBV; e += kThreads) {
+            int r = e / kBV, j = e - r * kBV;
+            float s = U[((size_t)(t0 + r) * H + h) * dv + j0 + j];
+            for (int c = 0; c < dk; ++c) s -= M[r * dk + c] * S[c * kBV + j];
+            Ws[e] = s;
+            Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = s;
+        }
+        __syncthreads();
+        for (int c = tid; c < dk; c += kThreads) gC[c] = g[((size_t)(t0 + L - 1) * H + h) * dk + c];
+        __syncthreads();
+        for (int e = tid; e < L * dk; e += kThreads) {
+            int r = e / dk, c = e - r * dk;
+            size_t off = ((size_t)(t0 + r) * H + h) * dk + c;
+            M[e] = to_f32(k[off]) * expf(gC[c] - g[off]);
+        }
+        __syncthreads();
+        // S <- Diag(exp(g_C)) S + (K . exp(g_C - g))^T W
+        for (int e = tid; e < dk * kBV; e += kThreads) {
+            int c = e / kBV, j = e - c * kBV;
+            float s = expf(gC[c]) * S[e];
+            for (int r = 0; r < L; ++r) s += M[r * dk + c] * Ws[r * kBV + j];
+            S[e] = s;
+        }
+        __syncthreads();
+    }
+    if (final_state) {
+        for (int e = tid; e < dk * kBV; e += kThreads) {
+            int c = e / kBV, j = e - c * kBV;
+            final_state[st_base + (size_t)c * dv + j0 + j] = S[e];
+        }
+    }
+}
+
+// K4: one block per (chunk, head).  Shared: Ks [C][dk] (then Q . exp(g)),
+// Gs [C][dk], P [C][C].
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                      const float* __restrict__ g, const float* __restrict__ Wg,
+                                                      const float* __restrict__ S_chunk, Tin* __restrict__ o,
+                                                      ChunkMap cmap, int H, int dk, int dv, int C) {
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* Ks = smem;
+    float* Gs = Ks + C * dk;
+    float* P = Gs + C * dk;
+    for (int e = tid; e < len * dk; e += kThreads) {
+        int r = e / dk, c = e - r * dk;
+        size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
+        Ks[e] = to_f32(k[off]);
+        Gs[e] = g[off];
+    }
+    __syncthreads();
+    // P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic), i <= r (inclusive mask)
+    for (int p = warp; p < len * len; p += kThreads / 32) {
+        int r = p / len, i = p - r * len;
+        float s = 0.f;
+        if (i <= r) {
+            const size_t qoff = ((size_t)(tok0 + r) * H + h) * dk;
+            for (int c = lane; c < dk; c += 32)
+                s += to_f32(q[qoff + c]) * Ks[i * dk + c] * expf(Gs[r * dk + c] - Gs[i * dk + c]);
+            s = warp_sum(s);
+        }
+        if (lane == 0) P[r * C + i] = s;
+    }
+    __syncthreads();
+    for (int e = tid; e < len * dk; e += kThreads) {
+        int r = e / dk, c = e - r * dk;
+        size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
+        Ks[e] = to_f32(q[off]) * expf(Gs[e]);
+    }
+    __syncthreads();
+    const size_t sc_base = ((size_t)blockIdx.x * H + h) * dk * dv;
+    for (int e = tid; e < len * dv; e += kThreads) {
+        int r = e / dv, j = e - r * dv;
+        float s = 0.f;
+        for (int c = 0; c < dk; ++c) s += Ks[r * dk + c] * S_chunk[sc_base + (size_t)c * dv + j];
+        for (int i = 0; i <= r; ++i) s += P[r * C + i] * Wg[((size_t)(tok0 + i) * H + h) * dv + j];
+        o[((size_t)(tok0 + r) * H + h) * dv + j] = from_f32<Tin>(s);
+    }
+}
+
+template <typename Tin>
+cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const Tin* beta, const float* init_state,
+                Tin* o, float* final_state, const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs,
+                int H, int dk, int dv, int C, const SimtWorkspace& ws, cudaStream_t stream) {
+    const size_t smem2 = sizeof(float) * ((size_t)C * C + (size_t)C * (size_t)((2 * dk > dk + dv) ? 2 * dk : dk + dv));
+    const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + dk);
+    const size_t smem4 = sizeof(float) * (2 * (size_t)C * dk + (size_t)C * C);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
+    if ((e = cudaFuncSetAttribute(k3_state<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
+    if ((e = cudaFuncSetAttribute(k4_output<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4))) return e;
+    if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, cmap, H, dk);
+    timing_mark(stream, 1);
+    if (n_chunks > 0)
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.U, ws.Wk, cmap, H, dk, dv, C);
+    timing_mark(stream, 2);
+    if (n_seqs > 0)
+        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.U, ws.Wk, ws.W, ws.S_chunk,
+                                                                            init_state, final_state, smap, H, dk,
+                                                                            dv, C);
+    timing_mark(stream, 3);
+    if (n_chunks > 0)
+        k4_output<Tin><<<dim3(n_chunks, H), kThreads, smem4, stream>>>(q, k, ws.g, ws.W, ws.S_chunk, o, cmap, H, dk,
+                                                                     dv, C);
+    timing_mark(stream, 4);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_simt_prefill(kda_dtype dtype, const void* q, const void* k, const void* v, const void* log_alpha,
+                                const void* beta, const float* init_state, void* o, float* final_state,
+                                const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs, int H, int dk,
+                                int dv, int C, const SimtWorkspace& ws, cudaStream_t stream) {
+    if (dtype == KDA_F32)
+        return run<float>((const float*)q, (const float*)k, (const float*)v, (const float*)log_alpha,
+                          (const float*)beta, init_state, (float*)o, final_state, cmap, smap, n_chunks, n_seqs, H,
+                          dk, dv, C, ws, stream);
+    return run<__nv_bfloat16>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                              (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, init_state,
+                              (__nv_bfloat16*)o, final_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws, stream);
+}
+
+}  // namespace kda

@@ -1,0 +1,64 @@
+"""Helpers shared by the tests: parity metric and oracle calls on sampled slices.
+
+The oracle (``oracle/``) is imported here only; the CUDA binding never is.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from kda_inputs import to_f64
+
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+
+
+def rel_err(got, ref) -> float:
+    """max |got - ref| / rms(ref) over the compared elements."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref ** 2))
+    if rms == 0.0:
+        return float(np.max(np.abs(got - ref))) if got.size else 0.0
+    return float(np.max(np.abs(got - ref)) / rms)
+
+
+def oracle_prefill(inp, heads=None, seqs=None, n_threads=0):
+    """Oracle o / final_state for the given heads and sequences of a PrefillInputs.
+
+    Returns (o_ref [n_tok_sel, n_heads, dv], fs_ref [n_seq_sel, n_heads, dk, dv],
+    token index array, seq list, head list)."""
+    H = inp.q.shape[2]
+    heads = list(range(H)) if heads is None else list(heads)
+    ss = inp.seq_start
+    seqs = list(range(len(ss) - 1)) if seqs is None else list(seqs)
+    flat = lambda t: t.reshape(-1, *t.shape[2:])
+    tok_idx = np.concatenate([np.arange(ss[s], ss[s + 1]) for s in seqs]) if seqs else np.zeros(0, np.int64)
+    lens = [int(ss[s + 1] - ss[s]) for s in seqs]
+    sub_start = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    ti = torch.as_tensor(tok_idx, device=inp.q.device, dtype=torch.long)
+    hi = torch.as_tensor(heads, device=inp.q.device, dtype=torch.long)
+
+    def pick(t):
+        return to_f64(flat(t).index_select(0, ti).index_select(1, hi))
+
+    s0 = None
+    if inp.init_state is not None:
+        si = torch.as_tensor(seqs, device=inp.q.device, dtype=torch.long)
+        s0 = to_f64(inp.init_state.index_select(0, si).index_select(1, hi))
+    o, fs = oracle.forward(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.log_alpha), pick(inp.beta),
+                           sub_start, init_state=s0, n_threads=n_threads)
+    return o, fs, tok_idx, seqs, heads
+
+
+def gpu_slices(o_gpu, fs_gpu, tok_idx, seqs, heads):
+    """The same slices of the GPU outputs as host fp64 arrays."""
+    dev = o_gpu.device
+    ti = torch.as_tensor(tok_idx, device=dev, dtype=torch.long)
+    hi = torch.as_tensor(heads, device=dev, dtype=torch.long)
+    o = to_f64(o_gpu.reshape(-1, *o_gpu.shape[2:]).index_select(0, ti).index_select(1, hi))
+    fs = None
+    if fs_gpu is not None:
+        si = torch.as_tensor(seqs, device=dev, dtype=torch.long)
+        fs = to_f64(fs_gpu.index_select(0, si).index_select(1, hi))
+    return o, fs

@@ -1,0 +1,124 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects invalid arguments on the host before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kimi_delta_attention_30_b200 as kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+OK, E_NULL, E_SHAPE, E_DTYPE, E_ALIGN, E_CHUNK, E_SEQ, E_WS = 0, -1, -2, -3, -4, -5, -6, -7
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]*?\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    names = header_functions()
+    assert "kda_chunk_fwd" in names and "kda_decode_step" in names
+    assert set(names) == set(kda.exported_symbols())
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(kda.lib()._name)
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    lib = kda.lib()
+    for code in range(-10, 1):
+        s = lib.kda_status_string(code).decode()
+        assert s.startswith("KDA")
+    assert "unknown" in lib.kda_status_string(-99).decode()
+    assert lib.kda_version() >= 100
+
+
+def _ws(B=1, T=256, H=2, dk=64, dv=64, C=64, dtype=1, cu=None, algo="auto"):
+    return kda.workspace_size(B, T, H, dk, dv, C, dtype, cu_seqlens=cu, algo=algo)
+
+
+def test_workspace_size_queries():
+    assert _ws() > 0
+    assert _ws(C=32) == 0
+    assert _ws(dk=96) == 0
+    assert _ws(dtype=7) == 0
+    assert _ws(B=1, T=10, cu=[0, 4, 10]) > 0
+    assert _ws(B=2, T=10, cu=[0, 4, 10]) == 0          # varlen needs B = 1
+    assert _ws(B=1, T=10, cu=[0, 6, 4, 10]) == 0       # decreasing
+    assert _ws(B=1, T=10, cu=[1, 4, 10]) == 0          # does not start at 0
+    assert _ws(B=1, T=10, cu=[0, 4, 9]) == 0           # does not end at T
+    assert _ws(T=0) > 0                                # empty problem is valid
+    # SIMT workspace holds g, U, Wk, W and the chunk start states
+    B, T, H, d, C = 2, 200, 3, 64, 64
+    n_chunks = B * ((T + C - 1) // C)
+    need = B * T * H * d * 4 * 4 + n_chunks * H * d * d * 4
+    assert _ws(B=B, T=T, H=H, dk=d, dv=d, C=C, dtype=1, algo="simt") >= need
+
+
+def test_simt_offsets_are_disjoint_and_ordered():
+    off = kda.simt_offsets(2, 200, 3, 64, 64, 64)
+    assert off == sorted(off) and len(set(off)) == 5
+    assert all(o % 256 == 0 for o in off)
+
+
+def _call(**kw):
+    """kda_chunk_fwd_ex with fake (never dereferenced) device pointers."""
+    lib = kda.lib()
+    a = dict(q=0x10000, k=0x20000, v=0x30000, la=0x40000, beta=0x50000, dtype=1, s0=None, cu=None, n=0,
+             B=1, T=256, H=2, dk=64, dv=64, C=64, o=0x60000, fs=None, ws=0x100000, wsb=1 << 40, algo=0)
+    a.update(kw)
+    cu = None
+    keep = None
+    if a["cu"] is not None:
+        keep = (ctypes.c_int32 * len(a["cu"]))(*a["cu"])
+        cu = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int32))
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.kda_chunk_fwd_ex(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["la"]), vp(a["beta"]), a["dtype"],
+                                vp(a["s0"]), cu, a["n"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["C"],
+                                vp(a["o"]), vp(a["fs"]), vp(a["ws"]), a["wsb"], None, a["algo"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=5), E_DTYPE),
+    (dict(C=32), E_CHUNK),
+    (dict(dk=96), E_SHAPE),
+    (dict(H=0), E_SHAPE),
+    (dict(q=None), E_NULL),
+    (dict(o=None), E_NULL),
+    (dict(ws=None), E_WS),
+    (dict(wsb=16), E_WS),
+    (dict(k=0x20004), E_ALIGN),
+    (dict(ws=0x100010), E_ALIGN),
+    (dict(cu=[0, 100, 50, 256], n=3), E_SEQ),
+    (dict(cu=[0, 100, 200], n=2), E_SEQ),
+    (dict(cu=[0, 256], n=1, B=2), E_SEQ),
+    (dict(algo=2, dtype=1), E_SHAPE),          # tensor-core path is bf16 only
+    (dict(algo=9), E_SHAPE),
+])
+def test_chunk_fwd_rejects_before_launch(kw, code):
+    assert _call(**kw) == code
+
+
+def test_decode_rejects_before_launch():
+    lib = kda.lib()
+    vp = ctypes.c_void_p
+    args = [vp(0x10000)] * 5
+    assert lib.kda_decode_step(*args, 3, vp(0x70000), 4, 2, 64, 64, vp(0x80000), None) == E_DTYPE
+    assert lib.kda_decode_step(*args, 0, vp(0x70000), 4, 2, 96, 64, vp(0x80000), None) == E_SHAPE
+    assert lib.kda_decode_step(*args, 0, None, 4, 2, 64, 64, vp(0x80000), None) == E_NULL
+    assert lib.kda_decode_step(*args, 0, vp(0x70004), 4, 2, 64, 64, vp(0x80000), None) == E_ALIGN
+    assert lib.kda_decode_step(*args, 0, vp(0x70000), 0, 2, 64, 64, vp(0x80000), None) == OK   # N = 0: no work
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
