@@ -273,6 +273,9 @@ def main():
         prefill_step()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(a.steps)]
+    for row in ev:            # torch creates the CUDA event on its first record
+        for e in row:
+            e.record(stream)
     barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()

@@ -151,7 +151,10 @@ def chunk_kernels(B, T, H, dk, dv, C, dtype, cu_seqlens=None, algo="auto"):
 
 def set_timing_events(events):
     """Per-kernel timing hook for the next chunk_fwd on this thread: a list of
-    torch.cuda.Event (recorded before the first kernel and after each kernel)."""
+    torch.cuda.Event (recorded before the first kernel and after each kernel).
+    Each event must already exist (torch creates it on its first record)."""
+    if any(e.cuda_event == 0 for e in events):
+        raise ValueError("record every event once before handing it to the timing hook")
     arr = (ctypes.c_void_p * max(1, len(events)))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     st = lib().kda_set_timing_events(arr, len(events))
     if st != 0:

@@ -13,14 +13,33 @@ from kda_inputs import to_f64
 TOL = {"bf16": 2e-2, "f32": 1e-4}
 
 
-def rel_err(got, ref) -> float:
-    """max |got - ref| / rms(ref) over the compared elements."""
+def bf16_half_ulp(x):
+    """Half the bf16 spacing at each (bf16-representable) value of x: the most
+    that round-to-nearest-even moves a value when it is stored as bf16."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.where(ax > 0, 2.0 ** (e - 8), 2.0 ** -134)
+
+
+def rel_err(got, ref, stored_as=None) -> float:
+    """max |got - ref| / rms(ref) over the compared elements.
+
+    With ``stored_as="bf16"`` the GPU values were rounded once to bf16 when
+    they were written (the output dtype follows the inputs); that rounding is
+    not an error of the computation, so each |got - ref| is first reduced by
+    the half-ulp the storage may add (and floored at 0)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
+    if got.size == 0:
+        return 0.0
+    d = np.abs(got - ref)
+    if stored_as == "bf16":
+        d = np.maximum(d - bf16_half_ulp(got), 0.0)
     rms = np.sqrt(np.mean(ref ** 2))
     if rms == 0.0:
-        return float(np.max(np.abs(got - ref))) if got.size else 0.0
-    return float(np.max(np.abs(got - ref)) / rms)
+        return float(np.max(d))
+    return float(np.max(d) / rms)
 
 
 def oracle_prefill(inp, heads=None, seqs=None, n_threads=0):
