@@ -46,6 +46,10 @@ def _args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample length")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+                    help="profiling aid: run only one part (the JSON line then lacks the other)")
+    ap.add_argument("--decode-n", type=int, default=DECODE["N"], help="profiling aid: decode sequences")
+    ap.add_argument("--prefill-b", type=int, default=PREFILL["B"], help="profiling aid: prefill batch")
     a = ap.parse_args()
     a.warmup = max(3, a.warmup)
     return a
@@ -249,69 +253,75 @@ def main():
         gpu_id = None
     pk = peaks()
     p = PREFILL
-    B, T, H, dk, dv, C = p["B"], p["T"], p["H"], p["dk"], p["dv"], p["C"]
+    B, T, H, dk, dv, C = a.prefill_b, p["T"], p["H"], p["dk"], p["dv"], p["C"]
+    DECODE["N"] = a.decode_n
 
-    inp = make_prefill("prefill", device=dev, seed=rank)
-    kernels = kda.chunk_kernels(B, T, H, dk, dv, C, torch.bfloat16, algo=a.algo)
-    nk = len(kernels)
-    ws = torch.empty(kda.workspace_size(B, T, H, dk, dv, C, torch.bfloat16, algo=a.algo), dtype=torch.uint8,
-                     device=dev)
-    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
-    fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+    run_prefill = a.only in ("all", "prefill")
+    run_decode = a.only in ("all", "decode") and not a.no_decode
     stream = torch.cuda.current_stream()
-
-    def prefill_step(evs=None):
-        if evs is not None:
-            kda.set_timing_events(evs)
-        kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, init_state=inp.init_state, C=C, o=o,
-                      final_state=fs, workspace=ws, algo=a.algo)
-
     clocks = ClockSampler(gpu_id if rank == 0 else None)
-    for _ in range(a.warmup):
-        flush.zero_()
-        prefill_step()
-    torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(a.steps)]
-    for row in ev:            # torch creates the CUDA event on its first record
-        for e in row:
-            e.record(stream)
-    barrier()
-    torch.cuda.synchronize()
-    t_wall = time.perf_counter()
-    for i in range(a.steps):
-        flush.zero_()
-        prefill_step(ev[i])
-    torch.cuda.synchronize()
-    barrier()
-    t_wall = time.perf_counter() - t_wall
-    step_ms = [ev[i][0].elapsed_time(ev[i][nk]) for i in range(a.steps)]
-    k_ms = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(a.steps)] for j in range(nk)]
-    total_ms = max_over_ranks(sum(step_ms))
-    ms_per_step = total_ms / a.steps
-    tokens = B * T
-    value = world * tokens * a.steps / (total_ms / 1e3)
-    k_avg = [statistics.mean(x) for x in k_ms]
-    dom = max(range(nk), key=lambda j: k_avg[j])
-    dom_bytes = kernel_bytes(kernels[dom], B, T, H, dk, dv, C)
-    kernel_table = {kernels[j]: {"avg_us": k_avg[j] * 1e3, "share": k_avg[j] / max(sum(k_avg), 1e-12)}
-                    for j in range(nk)}
-    roofline = None
-    if dom_bytes is not None:
-        ach = dom_bytes / (k_avg[dom] / 1e3) / 1e9
-        roofline = {"kernel": kernels[dom], "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                    "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_bytes": dom_bytes,
-                    "peak_source": pk["source"]}
-    min_b = minimal_bytes(B, T, H, dk, dv)
-    path_roofline = {"minimal_bytes": min_b, "time_min_us": min_b / (pk["hbm_gbs"] * 1e9) * 1e6,
-                     "frac_of_hbm_bound": (min_b / (pk["hbm_gbs"] * 1e9)) / (ms_per_step / 1e3)}
+    value = ms_per_step = roofline = path_roofline = kernel_table = t_wall = None
+    kernels, nk = [], 0
+    if run_prefill:
+        inp = make_prefill("prefill", device=dev, seed=rank, B=B)
+        kernels = kda.chunk_kernels(B, T, H, dk, dv, C, torch.bfloat16, algo=a.algo)
+        nk = len(kernels)
+        ws = torch.empty(kda.workspace_size(B, T, H, dk, dv, C, torch.bfloat16, algo=a.algo), dtype=torch.uint8,
+                         device=dev)
+        o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+        fs = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+        flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+
+        def prefill_step(evs=None):
+            if evs is not None:
+                kda.set_timing_events(evs)
+            kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, init_state=inp.init_state, C=C, o=o,
+                          final_state=fs, workspace=ws, algo=a.algo)
+
+        for _ in range(a.warmup):
+            flush.zero_()
+            prefill_step()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(a.steps)]
+        for row in ev:            # torch creates the CUDA event on its first record
+            for e in row:
+                e.record(stream)
+        barrier()
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter()
+        for i in range(a.steps):
+            flush.zero_()
+            prefill_step(ev[i])
+        torch.cuda.synchronize()
+        barrier()
+        t_wall = time.perf_counter() - t_wall
+        step_ms = [ev[i][0].elapsed_time(ev[i][nk]) for i in range(a.steps)]
+        k_ms = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(a.steps)] for j in range(nk)]
+        total_ms = max_over_ranks(sum(step_ms))
+        ms_per_step = total_ms / a.steps
+        tokens = B * T
+        value = world * tokens * a.steps / (total_ms / 1e3)
+        k_avg = [statistics.mean(x) for x in k_ms]
+        dom = max(range(nk), key=lambda j: k_avg[j])
+        dom_bytes = kernel_bytes(kernels[dom], B, T, H, dk, dv, C)
+        kernel_table = {kernels[j]: {"avg_us": k_avg[j] * 1e3, "share": k_avg[j] / max(sum(k_avg), 1e-12)}
+                        for j in range(nk)}
+        roofline = None
+        if dom_bytes is not None:
+            ach = dom_bytes / (k_avg[dom] / 1e3) / 1e9
+            roofline = {"kernel": kernels[dom], "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_bytes": dom_bytes,
+                        "peak_source": pk["source"]}
+        min_b = minimal_bytes(B, T, H, dk, dv)
+        path_roofline = {"minimal_bytes": min_b, "time_min_us": min_b / (pk["hbm_gbs"] * 1e9) * 1e6,
+                         "frac_of_hbm_bound": (min_b / (pk["hbm_gbs"] * 1e9)) / (ms_per_step / 1e3)}
 
     # ---------------------------------------------------------------- decode
     decode = None
-    if not a.no_decode:
+    if run_decode:
         d = DECODE
-        state = make_decode_state("decode", device=dev, seed=rank)
-        toks = [make_decode_token("decode", step=s, device=dev, seed=rank) for s in range(d["steps"])]
+        state = make_decode_state("decode", device=dev, seed=rank, N=d["N"])
+        toks = [make_decode_token("decode", step=s, device=dev, seed=rank, N=d["N"]) for s in range(d["steps"])]
         od = torch.empty((d["N"], d["H"], d["dv"]), dtype=torch.bfloat16, device=dev)
 
         def decode_round(evs=None):
@@ -355,7 +365,7 @@ def main():
 
     # ---------------------------------------------------------------- end to end
     e2e = None
-    if not a.no_e2e:
+    if run_prefill and not a.no_e2e:
         host = {n: getattr(inp, n).to("cpu").pin_memory() for n in ("q", "k", "v", "log_alpha", "beta")}
         host["init_state"] = inp.init_state.to("cpu").pin_memory()
         o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -389,7 +399,7 @@ def main():
 
     # ---------------------------------------------------------------- CPU baseline
     cpu = None
-    if rank == 0 and world == 1 and not a.no_cpu:
+    if rank == 0 and world == 1 and run_prefill and not a.no_cpu:
         smp = OracleSample(a.cpu_seconds)
         dt = smp.time()
         cpu = {"value": smp.tokens() / dt, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
@@ -404,7 +414,7 @@ def main():
                            "kernels": kernels, "l2": "flushed before every timed step (256 MiB write)",
                            "parallelism": f"replicas x{world} (independent sequences per GPU)"},
                 "roofline": roofline, "path_roofline": path_roofline, "kernel_times": kernel_table,
-                "gpu_launches": nk * a.steps, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clk, "wall_s_timed": t_wall, "gpu": props.name}
         print(json.dumps(line), flush=True)
     if world > 1:
