@@ -75,7 +75,8 @@ typedef enum {
     KDA_ERR_WORKSPACE = -7,  /* workspace NULL or smaller than required        */
     KDA_ERR_CUDA = -8,       /* a CUDA runtime call or launch failed           */
     KDA_ERR_TIMEOUT = -9,    /* a bounded device-side wait gave up             */
-    KDA_ERR_DEVICE = -10     /* the current device is not sm_100 (B200)       */
+    KDA_ERR_DEVICE = -10,    /* the current device is not sm_100 (B200)       */
+    KDA_ERR_SCRATCH = -11    /* problem too large for the built-in scratch     */
 } kda_status;
 
 typedef enum {
@@ -184,6 +185,41 @@ KDA_API kda_status kda_set_timing_events(void* const* events, int n_events);
 KDA_API int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype dtype,
                                   const int32_t* cu_seqlens_host, int n_seqs, kda_algo algo,
                                   const char** names, int max_names);
+
+/*
+ * Prefill that allocates nothing (no counterpart on the pages: this is a
+ * deployment aid, not part of the method).
+ *
+ * For callers that cannot allocate device memory -- a plugin host that passes
+ * the operator only its input and output buffers and no allocator, or a
+ * serving runtime whose memory pool already owns the whole device, where a
+ * cudaMalloc from inside the operator fails or forces a device-wide
+ * synchronisation.  Same arguments and results as kda_chunk_fwd, without the
+ * workspace: the scratch is a fixed array of KDA_NOALLOC_SCRATCH_BYTES in
+ * device memory that the library itself declares.  Every device that loads the
+ * library holds that array until the process exits.
+ *
+ *   - Problems whose kda_chunk_fwd_workspace_size() exceeds
+ *     KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_SCRATCH before
+ *     anything is launched (about 16 K token-heads at dk = dv = 128 on the
+ *     CUDA-core path, e.g. B = 1, T = 1024, H = 16).
+ *   - The call never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - The first call on a device looks up the array's device address with that
+ *     device current (cudaGetSymbolAddress) and caches it; make that first call
+ *     before any stream capture on the device.
+ *   - All calls share the one array, and it keeps the last call's contents
+ *     (the prefill writes every scratch byte before reading it, so nothing needs
+ *     clearing).  Calls whose execution overlaps on the GPU -- on different
+ *     streams, or from different host threads -- race on the array and give
+ *     wrong results: serialise them.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+KDA_API kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                         const void* log_alpha, const void* beta, kda_dtype dtype,
+                                         const float* init_state, const int32_t* cu_seqlens_host,
+                                         int n_seqs, int B, int T, int H, int dk, int dv, int C,
+                                         void* o, float* final_state, void* stream);
 
 /*
  * One decode step for N independent sequences, one token each; the state is

@@ -62,6 +62,8 @@ def _declare(lib):
     lib.kda_set_timing_events.restype = c_int
     lib.kda_chunk_fwd_kernels.argtypes = [c_int] * 7 + [i32p, c_int, c_int, ctypes.POINTER(ctypes.c_char_p), c_int]
     lib.kda_chunk_fwd_kernels.restype = c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 5 + [c_int, vp, i32p, c_int] + [c_int] * 6 + [vp, vp, vp]
+    lib.kda_chunk_fwd_noalloc.restype = c_int
     return lib
 
 
@@ -92,7 +94,8 @@ def lib():
 def exported_symbols():
     return ["kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
             "kda_chunk_fwd_workspace_size_ex", "kda_chunk_fwd", "kda_chunk_fwd_ex",
-            "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels"]
+            "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
+            "kda_chunk_fwd_noalloc"]
 
 
 def _ptr(t):
@@ -198,6 +201,40 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
                                 _stream_handle(stream), ALGOS[algo])
     if st != 0:
         raise KdaError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20   # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int = 64,
+                      o=None, final_state=None, stream=None):
+    """Prefill through ``kda_chunk_fwd_noalloc``: no workspace argument, the
+    library's own fixed device scratch is used (for callers that cannot
+    allocate).  Problems needing more than NOALLOC_SCRATCH_BYTES of scratch
+    raise KdaError (KDA_ERR_SCRATCH).  Calls that overlap on the GPU share the
+    scratch and must be serialised."""
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        _check_cuda(name, t, dt)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu, n_seqs, _keep = _cu_arg(cu_seqlens)
+    N = n_seqs if cu_seqlens is not None else B
+    _check_cuda("init_state", init_state, torch.float32)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check_cuda("o", o, dt)
+    _check_cuda("final_state", final_state, torch.float32)
+    st = lib().kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                     _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o), _ptr(final_state),
+                                     _stream_handle(stream))
+    if st != 0:
+        raise KdaError(st, "kda_chunk_fwd_noalloc")
     return o, final_state
 
 

@@ -148,6 +148,8 @@ const char* kda_status_string(int status) {
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime error";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait expired";
         case KDA_ERR_DEVICE: return "KDA_ERR_DEVICE: current device is not sm_100 (B200)";
+        case KDA_ERR_SCRATCH:
+            return "KDA_ERR_SCRATCH: problem needs more scratch than the built-in KDA_NOALLOC_SCRATCH_BYTES";
         default: return "KDA: unknown status";
     }
 }

@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     lib = kda.lib()
-    for code in range(-10, 1):
+    for code in range(-11, 1):
         s = lib.kda_status_string(code).decode()
         assert s.startswith("KDA")
     assert "unknown" in lib.kda_status_string(-99).decode()
