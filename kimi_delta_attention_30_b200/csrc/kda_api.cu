@@ -16,6 +16,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
                               cudaStream_t stream);
 size_t tc_workspace_bytes(int n_chunks, int H, int C);
 bool tc_available();
+bool tc_supports(int C);
 
 TimingHook& timing_hook() {
     static thread_local TimingHook hook{{nullptr}, 0};
@@ -98,9 +99,13 @@ SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
     return L;
 }
 
-kda_algo resolve(kda_algo algo, kda_dtype dtype, int dk, int dv) {
+bool tc_shape(kda_dtype dtype, int dk, int dv, int C) {
+    return dtype == KDA_BF16 && dk == 128 && dv == 128 && tc_supports(C);
+}
+
+kda_algo resolve(kda_algo algo, kda_dtype dtype, int dk, int dv, int C) {
     if (algo != KDA_ALGO_AUTO) return algo;
-    return (tc_available() && dtype == KDA_BF16 && dk == 128 && dv == 128) ? KDA_ALGO_TC : KDA_ALGO_SIMT;
+    return (tc_available() && tc_shape(dtype, dk, dv, C)) ? KDA_ALGO_TC : KDA_ALGO_SIMT;
 }
 
 size_t workspace_for(const Plan& p, int H, int dk, int dv, int C, kda_algo algo) {
@@ -161,8 +166,8 @@ size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int 
     if (dtype != KDA_BF16 && dtype != KDA_F32) return 0;
     Plan p;
     if (make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
-    algo = resolve(algo, dtype, dk, dv);
-    if (algo == KDA_ALGO_TC && !(dtype == KDA_BF16 && dk == 128 && dv == 128)) return 0;
+    algo = resolve(algo, dtype, dk, dv, C);
+    if (algo == KDA_ALGO_TC && !tc_shape(dtype, dk, dv, C)) return 0;
     return std::max<size_t>(workspace_for(p, H, dk, dv, C, algo), kAlign);
 }
 
@@ -191,8 +196,8 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
     Plan p;
     kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
     if (st != KDA_OK) return st;
-    algo = resolve(algo, dtype, dk, dv);
-    if (algo == KDA_ALGO_TC && !(dtype == KDA_BF16 && dk == 128 && dv == 128)) return KDA_ERR_SHAPE;
+    algo = resolve(algo, dtype, dk, dv, C);
+    if (algo == KDA_ALGO_TC && !tc_shape(dtype, dk, dv, C)) return KDA_ERR_SHAPE;
     const bool has_tokens = p.total_tokens > 0;
     if (has_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
     if (!workspace) return KDA_ERR_WORKSPACE;
@@ -257,7 +262,7 @@ int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype 
     Plan p;
     kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
     if (st != KDA_OK) return st;
-    algo = resolve(algo, dtype, dk, dv);
+    algo = resolve(algo, dtype, dk, dv, C);
     const char* const* list = (algo == KDA_ALGO_TC) ? kTcKernelNames : kSimtKernelNames;
     const int n = (algo == KDA_ALGO_TC) ? kTcKernelCount : 4;
     for (int i = 0; names && i < n && i < max_names; ++i) names[i] = list[i];

@@ -108,11 +108,11 @@ def test_prefill_tiny_f32(cuda_ok):
     _check_all(inp, o, fs, TOL["f32"])
 
 
-@pytest.mark.parametrize("algo", ["auto", "simt"])
-@pytest.mark.parametrize("C", [64, 128])
-@pytest.mark.parametrize("T", [1, 63, 200, 300])
+@pytest.mark.parametrize("algo,C", [("auto", 64), ("auto", 128), ("simt", 64), ("simt", 128), ("tc", 64)])
+@pytest.mark.parametrize("T", [1, 63, 64, 200, 300])
 def test_prefill_bf16_ragged(cuda_ok, algo, C, T):
-    """bf16, d=128, several chunks and a ragged tail, random initial state."""
+    """bf16, d=128, several chunks and a ragged tail, random initial state;
+    the tensor-core path (chunk 64) and the CUDA-core split."""
     inp = _to(make_prefill("prefill", B=2, T=T, H=3, seed=T), DEV)
     o, fs = _run(inp, algo=algo, C=C)
     _check_all(inp, o, fs, TOL["bf16"])
@@ -128,33 +128,36 @@ def test_prefill_small_heads(cuda_ok, dk, dv):
         _check_all(inp, o, fs, TOL[dt])
 
 
-def test_prefill_varlen_with_empty_and_tiny_sequences(cuda_ok):
+@pytest.mark.parametrize("algo,C", [("auto", 64), ("auto", 128), ("simt", 64)])
+def test_prefill_varlen_with_empty_and_tiny_sequences(cuda_ok, algo, C):
     lengths = [5, 0, 64, 129, 1, 300, 0, 77]
-    for C in (64, 128):
-        inp = _to(make_prefill("varlen", H=4, lengths=lengths, seed=11, C=C), DEV)
-        o, fs = _run(inp, C=C)
-        _check_all(inp, o, fs, TOL["bf16"])
+    inp = _to(make_prefill("varlen", H=4, lengths=lengths, seed=11, C=C), DEV)
+    o, fs = _run(inp, algo=algo, C=C)
+    _check_all(inp, o, fs, TOL["bf16"])
 
 
-def test_prefill_gate_regimes_and_special_heads(cuda_ok):
-    """Near-0 gates (log alpha down to -16 per token), near-1 gates, mixed; and
-    the alpha = 1 / scalar-alpha heads."""
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+def test_prefill_gate_regimes_and_special_heads(cuda_ok, algo):
+    """Near-0 gates (log alpha down to -16 per token: the tensor-core path's
+    pairwise fallback for diagonal blocks), near-1 gates, mixed; and the
+    alpha = 1 / scalar-alpha heads."""
     inp = _to(make_prefill("varlen", H=6, lengths=[700, 333], seed=12), DEV)
-    o, fs = _run(inp)
+    o, fs = _run(inp, algo=algo)
     _check_all(inp, o, fs, TOL["bf16"])
     inp = _to(make_prefill("long", T=500, H=4, seed=13), DEV)
-    o, fs = _run(inp)
+    o, fs = _run(inp, algo=algo)
     _check_all(inp, o, fs, TOL["bf16"])
 
 
-def test_prefill_alpha_zero_beta_edges(cuda_ok):
+@pytest.mark.parametrize("algo", ["auto", "simt"])
+def test_prefill_alpha_zero_beta_edges(cuda_ok, algo):
     inp = make_prefill("prefill", B=1, T=200, H=2, seed=14)
     inp.log_alpha[0, 50:60, 0] = float("-inf")
     inp.log_alpha[0, 100, 1, :7] = float("-inf")
     inp.beta[0, 10:20, 0] = 0.0
     inp.beta[0, 30:40, 1] = 1.0
     inp = _to(inp, DEV)
-    o, fs = _run(inp)
+    o, fs = _run(inp, algo=algo)
     _check_all(inp, o, fs, TOL["bf16"])
 
 
