@@ -118,7 +118,10 @@ def kernel_bytes(name, B, T, H, dk, dv, C, in_bytes=2):
     n_chunks = B * ((T + C - 1) // C)
     st = B * H * dk * dv * 4
     schunk = n_chunks * H * dk * dv * 4
+    ws_tok = 5 * 4 * 128      # workspace per token-head of the tensor-core path: Wk, Q', Kd (hi+lo bf16), U, U' (fp32)
     table = {
+        "tc_intra": tok * ((3 * dk + dv) * in_bytes + in_bytes) + tok * ws_tok + n_chunks * H * dk * 4,
+        "tc_recur": tok * ws_tok + n_chunks * H * dk * 4 + tok * dv * in_bytes + 2 * st,
         "k1_cumsum": tok * dk * (in_bytes + 4),
         "k2_wy": tok * (2 * dk * in_bytes + dv * in_bytes + in_bytes + 4 * dk) + tok * 4 * (dv + dk),
         "k3_state": tok * (4 * dk + 4 * dv + in_bytes * dk + 4 * dk) + tok * 4 * dv + schunk + 2 * st,

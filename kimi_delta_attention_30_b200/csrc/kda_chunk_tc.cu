@@ -3,16 +3,15 @@
 //
 // Two kernels:
 //
-//   tc_intra  (one CTA per (chunk, head), all chunks in parallel)
-//     cumulative log decay g (row a1), then on the tensor cores the
-//     decay-weighted strictly-lower A = Diag(beta) (K K^T . exp(g_r - g_i)) and
-//     the inclusive score matrix P = (Q K^T . exp(g_r - g_i)); T = (I + A)^{-1}
-//     by blocked forward substitution on CUDA cores; then (tensor cores)
-//       U  = T Diag(beta) V,        Wk = T Diag(beta) (K . exp(g))       (row a2)
-//       U' = P U,                   Q' = Q . exp(g) - P Wk
-//       Kd = K . exp(g_C - g),      Gamma_C = exp(g_C)
-//     written to the workspace in the exact shared-memory layout the second
-//     kernel's MMAs consume (so its loads are plain 1-D bulk copies).
+//   tc_intra  (one CTA per (chunk, head), all chunks in parallel, 2 CTAs/SM)
+//     cumulative log decay g (row a1); on the tensor cores the decay-weighted
+//     strictly-lower A = Diag(beta) (K K^T . exp(g_r - g_i)) and the inclusive
+//     score matrix P = (Q K^T . exp(g_r - g_i)); T = (I + A)^{-1} by blocked
+//     substitution on CUDA cores; then on the tensor cores P T and
+//       [T ; P T] [beta V | beta K exp(g)] = [U | Wk ; U' | P Wk]          (row a2)
+//     i.e. U = T Diag(beta) V, Wk = T Diag(beta)(K . exp(g)), U' = P U and
+//     Q' = Q . exp(g) - P Wk, plus Kd = K . exp(g_C - g) and Gamma_C = exp(g_C).
+//     Results go to the workspace in the layout the second kernel consumes.
 //
 //   tc_recur  (one CTA per (sequence, head, d_v tile), sequential over chunks)
 //     with the fp32 state tile S (d_k x BV) in TMEM:
@@ -20,7 +19,7 @@
 //       W   = U - D[0:64]                         per-token corrections
 //       O   = D[64:128] + U'                      outputs (row a4)
 //       S  <- Diag(Gamma_C) S + Kd^T W            M = 128 MMA accumulating in TMEM (row a3)
-//     The next chunk's operands stream in by bulk copies (TMA engine, no
+//     The next chunk's operands stream in by 1-D bulk copies (TMA engine, no
 //     multicast) while the current chunk is processed.
 //
 // Derivation (ours; the oracle's chunk form checks it against the token
@@ -35,9 +34,9 @@
 // Precision.  Every tensor-core product is formed in three bf16 terms,
 // a_hi b_hi + a_hi b_lo + a_lo b_hi (hi = RN_bf16(x), lo = RN_bf16(x - hi)),
 // with fp32 accumulation: about 16 significant bits per operand.  Heavy decay
-// makes single tokens dominate many of the sums, so a single bf16 rounding of
-// an operand would show up at ~2^-9 times the (heavy) tail of o; three terms
-// keep the whole path within the fp32 regime.  U and U' are kept in fp32.
+// lets single tokens dominate many of the sums, so one bf16 rounding of an
+// operand would show up at ~2^-9 times the heavy tail of o; three terms keep
+// the path in the fp32 regime.  U and U' are stored in fp32.
 //
 // Decay factors.  Rows form 16-row blocks; gb[b] is g at the row before block
 // b (gb[0] = 0), gb[4] = g_C.  Every factor handed to the tensor cores is exp of
@@ -61,75 +60,64 @@ constexpr int kD = 128;
 constexpr float kDiagRange = 80.0f;
 
 // ---- workspace image of one (chunk, head) --------------------------------------
-constexpr uint32_t kOffWkQh = 0;         // [128 rows][128 k] bf16 SW128: rows 0-63 Wk, 64-127 Q' (hi)
+constexpr uint32_t kOffWkQh = 0;         // [128 rows][128 k] bf16 SW128 K-major: rows 0-63 Wk, 64-127 Q' (hi)
 constexpr uint32_t kOffWkQl = 32768;     // lo parts
-constexpr uint32_t kOffKdTh = 65536;     // [128 rows (channel)][64 k (token)] bf16 SW128 (hi)
+constexpr uint32_t kOffKdTh = 65536;     // [128 rows (channel)][64 k (token)] bf16 SW128 K-major (hi)
 constexpr uint32_t kOffKdTl = 81920;     // lo parts
-constexpr uint32_t kOffU = 98304;        // U : [4 column blocks][64 rows][32] fp32
+constexpr uint32_t kOffU = 98304;        // U : fp32, see u_index()
 constexpr uint32_t kOffU2 = 131072;      // U': same layout
 constexpr uint32_t kOffGam = 163840;     // Gamma_C fp32 [128]
 constexpr uint32_t kChunkBytes = 164352;
 constexpr uint32_t kErrHeader = 256;     // first bytes of the TC scratch: error word
 
+// U / U' tiles: [4 column blocks of 32][64 rows][8 chunks of 4 floats], chunk
+// permuted by row % 8 so that row-per-thread float4 reads hit distinct banks.
+__host__ __device__ __forceinline__ int u_index(int r, int j) {   // j % 4 == 0
+    return (j >> 5) * 2048 + r * 32 + (((((j & 31) >> 2)) ^ (r & 7)) << 2);
+}
+
 // ---- tc_intra shared memory (byte offsets from a 1024-aligned base) -----------
 constexpr int kIntraThreads = 256;
-// phase 1: MMA-1 operands
-constexpr uint32_t kAKQh = 0;            // [K.E ; Q.E]  128 x 128
-constexpr uint32_t kAKQl = 32768;
-constexpr uint32_t kKFh = 65536;         // decayed key versions 160 x 128
-constexpr uint32_t kKFl = 106496;
-constexpr uint32_t kXVh = 147456;        // (beta V)^T 128 x 64
-constexpr uint32_t kXVl = 163840;
-// phase 2 (after MMA 1, inside [0, 147456))
-constexpr uint32_t kXKh = 0;             // (beta K exp(g))^T 128 x 64
-constexpr uint32_t kXKl = 16384;
-constexpr uint32_t kAs = 32768;          // A fp32 [64][64]
-constexpr uint32_t kPh = 49152;          // P 64 x 64
-constexpr uint32_t kPl = 57344;
-constexpr uint32_t kTs = 65536;          // T fp32 [64][64]
-constexpr uint32_t kScr = 81920;         // 8 KB scratch
-constexpr uint32_t kTh = 90112;          // T 64 x 64
-constexpr uint32_t kTl = 98304;
-// phase 3 (after MMA 2): U^T and Wk^T operands in the dead X regions
-constexpr uint32_t kUTh = 0, kUTl = 16384, kWTh = kXVh, kWTl = kXVl;
-constexpr uint32_t kTab = 180224;        // tables
+// first MMA, one half of the channels at a time
+constexpr uint32_t kAKQh = 0;            // [K.E ; Q.E]  128 rows x 64 k
+constexpr uint32_t kAKQl = 16384;
+constexpr uint32_t kKFh = 32768;         // decayed key versions 160 rows x 64 k
+constexpr uint32_t kKFl = 53248;
+// after the first MMA
+constexpr uint32_t kAs = 0;              // A fp32 [64][65]
+constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
+constexpr uint32_t kPl = 25600;
+constexpr uint32_t kScr = 33792;         // 8 KB scratch
+constexpr uint32_t kTs = 41984;          // T fp32 [64][65]
+// [T ; P T] (128 rows x 64 k, K-major; rows 0-63 also serve as the MN-major T)
+constexpr uint32_t kTPh = 65536;
+constexpr uint32_t kTPl = 81920;
+// [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns)
+constexpr uint32_t kXh = 0;
+constexpr uint32_t kXl = 32768;
+constexpr uint32_t kTab = 98304;         // tables
 constexpr int kNumTab = 18;              // tau[4], sigma[6], exp(gb)[4], exp(g_C - gb[b+1])[4]
 constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 64 * 4 + 64;
 constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
+constexpr int kAS = 65;                  // row stride of As / Ts (floats)
 
 // rows of the decayed-key versions: version R covers keys [0, 16 R + 16)
-__device__ __forceinline__ int kf_off(int R) { return (R * (R + 1)) * 8; }   // 0, 16, 48, 96
+__host__ __device__ __forceinline__ int kf_off(int R) { return (R * (R + 1)) * 8; }   // 0, 16, 48, 96
 
 __device__ __forceinline__ int tab_tau(int R) { return R; }                                  // exp(gb[R] - gb[R+1])
 __device__ __forceinline__ int tab_sigma(int R, int I) { return 4 + (R * (R - 1)) / 2 + I; } // exp(gb[R] - gb[I+1]), I < R
 __device__ __forceinline__ int tab_e0(int I) { return 10 + I; }                              // exp(gb[I])
 __device__ __forceinline__ int tab_ec(int I) { return 14 + I; }                              // exp(g_C - gb[I+1])
 
-__device__ __forceinline__ void unpack4(uint2 v, float (&f)[4]) {
-    f[0] = bf16_lo(v.x);
-    f[1] = bf16_hi(v.x);
-    f[2] = bf16_lo(v.y);
-    f[3] = bf16_hi(v.y);
+// two values of one row -> 4-byte stores into the hi and lo tiles
+__device__ __forceinline__ void store2_split(uint8_t* hi_tile, uint8_t* lo_tile, uint32_t off, float a, float b) {
+    uint32_t hv, lv;
+    split2(a, b, hv, lv);
+    *reinterpret_cast<uint32_t*>(hi_tile + off) = hv;
+    *reinterpret_cast<uint32_t*>(lo_tile + off) = lv;
 }
 
-// four consecutive k values of one row, split into the hi and lo tiles
-__device__ __forceinline__ void store4_split(uint8_t* hi_tile, uint8_t* lo_tile, uint32_t off, float a, float b,
-                                             float c, float d) {
-    uint2 hv, lv;
-    split2(a, b, hv.x, lv.x);
-    split2(c, d, hv.y, lv.y);
-    *reinterpret_cast<uint2*>(hi_tile + off) = hv;
-    *reinterpret_cast<uint2*>(lo_tile + off) = lv;
-}
-
-__device__ __forceinline__ void store1_split(uint8_t* hi_tile, uint8_t* lo_tile, uint32_t off, float x) {
-    __nv_bfloat16 hv, lv;
-    split1(x, hv, lv);
-    *reinterpret_cast<__nv_bfloat16*>(hi_tile + off) = hv;
-    *reinterpret_cast<__nv_bfloat16*>(lo_tile + off) = lv;
-}
-
-// eight consecutive k values (one 16-byte chunk) split into hi and lo tiles
+// eight consecutive values (one 16-byte chunk) split into hi and lo tiles
 __device__ __forceinline__ void store8_split(uint8_t* hi_tile, uint8_t* lo_tile, uint32_t off, const float* x) {
     uint4 hv, lv;
     split2(x[0], x[1], hv.x, lv.x);
@@ -140,25 +128,34 @@ __device__ __forceinline__ void store8_split(uint8_t* hi_tile, uint8_t* lo_tile,
     *reinterpret_cast<uint4*>(lo_tile + off) = lv;
 }
 
+__device__ __forceinline__ void unpack8(uint4 v, float* f) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
 __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
-// D (+)= A B^T in three bf16 terms over `ksteps` K-slices of 16.
+// D (+)= A B^T over `ksteps` K-slices of 16, in three bf16 terms; A K-major,
+// B K-major (b_mn = false) or MN-major (b_mn = true, `brows` = K rows).
 __device__ __forceinline__ void mma3(uint32_t d, uint32_t ah, uint32_t al, int arows, uint32_t bh, uint32_t bl,
-                                     int brows, int ksteps, uint32_t idesc, bool accumulate) {
+                                     int brows, bool b_mn, int ksteps, uint32_t idesc, bool accumulate) {
     for (int s = 0; s < ksteps; ++s) {
         const uint32_t acc0 = (accumulate || s > 0) ? 1u : 0u;
-        mma_bf16(d, sw128_desc_k(ah, arows, s), sw128_desc_k(bh, brows, s), idesc, acc0);
-        mma_bf16(d, sw128_desc_k(ah, arows, s), sw128_desc_k(bl, brows, s), idesc, 1u);
-        mma_bf16(d, sw128_desc_k(al, arows, s), sw128_desc_k(bh, brows, s), idesc, 1u);
+        const uint64_t dah = sw128_desc_k(ah, arows, s), dal = sw128_desc_k(al, arows, s);
+        const uint64_t dbh = b_mn ? mn_desc_k(bh, brows, s) : sw128_desc_k(bh, brows, s);
+        const uint64_t dbl = b_mn ? mn_desc_k(bl, brows, s) : sw128_desc_k(bl, brows, s);
+        mma_bf16(d, dah, dbh, idesc, acc0);
+        mma_bf16(d, dah, dbl, idesc, 1u);
+        mma_bf16(d, dal, dbh, idesc, 1u);
     }
 }
 
 // ============================================================================
 // tc_intra
 // ============================================================================
-__global__ void __launch_bounds__(kIntraThreads, 1)
+__global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
@@ -172,8 +169,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __shared__ uint64_t mbar;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c0 = 4 * lane, r0 = 8 * warp;    // this thread: channels [c0, c0+4), rows [r0, r0+8)
-    const int I = warp >> 1;                   // 16-row block of this thread's rows
+    // this thread: rows [8 w, 8 w + 8) of 16-row block I = w / 2, and channels
+    // 2 lane, 2 lane + 1 of each 64-channel half (index x = 2 half + e)
+    const int I = warp >> 1;
+    const int kc = 2 * lane;                  // channel inside a half
+    const int r0 = 8 * warp;
     int seq, tok0, len, cidx;
     cmap.locate(blockIdx.x, seq, tok0, len, cidx);
     const int h = blockIdx.y;
@@ -191,52 +191,51 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     }
     if (tid < 64) sbeta[tid] = (tid < len) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
 
-    // ---- this thread's 8 rows x 4 channels of k, q, v, log alpha ----------
-    uint2 kr[8], qr[8], vr[8];
+    // ---- log alpha of 8 rows x 4 channels; k, q, v prefetched into L2 ---------
+    // (k and q are read in the round that uses them, v at the end; holding them
+    // in registers through the chunk would push the kernel past 128 registers)
     float g[8][4];
+    if (lane < 16) {
+        const int r = r0 + (lane & 7);
+        if (r < len) {
+            const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * (lane >> 3);
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(k + off));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(q + off));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(v + off));
+        }
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int r = r0 + j;
-        if (r < len) {
-            const size_t off = ((size_t)(tok0 + r) * H + h) * kD + c0;
-            kr[j] = *reinterpret_cast<const uint2*>(k + off);
-            qr[j] = *reinterpret_cast<const uint2*>(q + off);
-            vr[j] = *reinterpret_cast<const uint2*>(v + off);
-            float a[4];
-            unpack4(*reinterpret_cast<const uint2*>(la + off), a);
 #pragma unroll
-            for (int x = 0; x < 4; ++x) g[j][x] = fmaxf(a[x], kLogAlphaFloor);
-        } else {
-            kr[j] = make_uint2(0, 0);
-            qr[j] = kr[j];
-            vr[j] = kr[j];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) g[j][x] = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t a = 0u;
+            if (r < len) a = *reinterpret_cast<const uint32_t*>(la + ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc);
+            g[j][2 * hh] = (r < len) ? fmaxf(bf16_lo(a), kLogAlphaFloor) : 0.f;
+            g[j][2 * hh + 1] = (r < len) ? fmaxf(bf16_hi(a), kLogAlphaFloor) : 0.f;
         }
     }
-    // ---- cumulative log decay (row a1): local prefix, then carries --------
+    // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
     for (int j = 1; j < 8; ++j)
 #pragma unroll
         for (int x = 0; x < 4; ++x) g[j][x] += g[j - 1][x];
-    float* tot = tab;   // [8][128] partial totals (the table space is free until the tables are built)
+    float* tot = tab;   // [8][128] per-warp totals; the tables are built after their last use
 #pragma unroll
-    for (int x = 0; x < 4; ++x) tot[warp * 128 + c0 + x] = g[7][x];
+    for (int x = 0; x < 4; ++x) tot[warp * 128 + 64 * (x >> 1) + kc + (x & 1)] = g[7][x];
     __syncthreads();
-    {
-        float carry[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int p = 0; p < warp; ++p)
+    float carry[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int p = 0; p < warp; ++p)
 #pragma unroll
-            for (int x = 0; x < 4; ++x) carry[x] += tot[p * 128 + c0 + x];
+        for (int x = 0; x < 4; ++x) carry[x] += tot[p * 128 + 64 * (x >> 1) + kc + (x & 1)];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int x = 0; x < 4; ++x) g[j][x] += carry[x];
-    }
+        for (int x = 0; x < 4; ++x) g[j][x] += carry[x];
     if (tid < 128) gb[tid] = 0.f;
     if (warp & 1) {
 #pragma unroll
-        for (int x = 0; x < 4; ++x) gb[(I + 1) * 128 + c0 + x] = g[7][x];
+        for (int x = 0; x < 4; ++x) gb[(I + 1) * 128 + 64 * (x >> 1) + kc + (x & 1)] = g[7][x];
     }
     __syncthreads();
 
@@ -268,86 +267,82 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             if (fbmask & (1u << R)) tab[tab_tau(R) * 128 + tid] = 0.f;
     }
     __syncthreads();
+    if (tid < 128) reinterpret_cast<float*>(out + kOffGam)[tid] = __expf(gb[4 * 128 + tid]);
 
-    // ---- MMA-1 operands, Q exp(g) and Kd into the workspace, (beta V)^T ------
-    {
-        float e0[4], ec[4], gref[4], glast[4];
+    const uint32_t tbase = sflags[2];
+    uint32_t phase = 0;
+    bool abort = false;
+
+    // ---- first MMA in two channel halves --------------------------------------------
+    // Round hr: every thread reads k and q of its 8 rows for its two channels in
+    // half hr, builds that half's MMA operands and writes its Q exp(g) and Kd
+    // values to the workspace.
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            e0[x] = tab[tab_e0(I) * 128 + c0 + x];
-            ec[x] = tab[tab_ec(I) * 128 + c0 + x];
-            gref[x] = gb[I * 128 + c0 + x];
-            glast[x] = gb[(I + 1) * 128 + c0 + x];
-        }
-        float kd[4][8], bv[4][8];
+    for (int hr = 0; hr < 2; ++hr) {
+        const int ch = 64 * hr + kc;
+        const float gref0 = gb[I * 128 + ch], gref1 = gb[I * 128 + ch + 1];
+        const float glast0 = gb[(I + 1) * 128 + ch], glast1 = gb[(I + 1) * 128 + ch + 1];
+        const float x0 = tab[tab_e0(I) * 128 + ch], x1 = tab[tab_e0(I) * 128 + ch + 1];
+        const float y0 = tab[tab_ec(I) * 128 + ch], y1 = tab[tab_ec(I) * 128 + ch + 1];
+        uint32_t kv[8], qv[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = r0 + j;
-            float kk[4], qq[4], vv[4], E[4], F[4];
-            unpack4(kr[j], kk);
-            unpack4(qr[j], qq);
-            unpack4(vr[j], vv);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                E[x] = __expf(g[j][x] - gref[x]);
-                F[x] = __expf(glast[x] - g[j][x]);
-            }
-            store4_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, c0, 128), kk[0] * E[0], kk[1] * E[1],
-                         kk[2] * E[2], kk[3] * E[3]);
-            store4_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, c0, 128), qq[0] * E[0], qq[1] * E[1],
-                         qq[2] * E[2], qq[3] * E[3]);
-            // Q exp(g) into the Q' rows of the workspace image (completed at the end)
-            store4_split(out + kOffWkQh, out + kOffWkQl, sw128_offset(64 + r, c0, 128), qq[0] * E[0] * e0[0],
-                         qq[1] * E[1] * e0[1], qq[2] * E[2] * e0[2], qq[3] * E[3] * e0[3]);
-#pragma unroll
-            for (int R = 0; R < 4; ++R) {
-                if (R < I) continue;
-                float f[4];
-#pragma unroll
-                for (int x = 0; x < 4; ++x)
-                    f[x] = kk[x] * F[x] * tab[((R == I) ? tab_tau(R) : tab_sigma(R, I)) * 128 + c0 + x];
-                store4_split(sm + kKFh, sm + kKFl, sw128_offset(kf_off(R) + r, c0, 160), f[0], f[1], f[2], f[3]);
-            }
-            const float b = sbeta[r];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                kd[x][j] = kk[x] * F[x] * ec[x];
-                bv[x][j] = b * vv[x];
+            kv[j] = qv[j] = 0u;
+            if (r < len) {
+                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + ch;
+                kv[j] = *reinterpret_cast<const uint32_t*>(k + off);
+                qv[j] = *reinterpret_cast<const uint32_t*>(q + off);
             }
         }
+        float kd0[8], kd1[8];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(c0 + x, r0, 128), kd[x]);
-            store8_split(sm + kXVh, sm + kXVl, sw128_chunk(c0 + x, r0, 128), bv[x]);
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
+            const float e0 = __expf(g[j][2 * hr] - gref0), e1 = __expf(g[j][2 * hr + 1] - gref1);
+            const float f0 = __expf(glast0 - g[j][2 * hr]), f1 = __expf(glast1 - g[j][2 * hr + 1]);
+            const float k0 = bf16_lo(kv[j]), k1 = bf16_hi(kv[j]);
+            const float q0 = bf16_lo(qv[j]), q1 = bf16_hi(qv[j]);
+            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, kc, 128), k0 * e0, k1 * e1);
+            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, kc, 128), q0 * e0, q1 * e1);
+#pragma unroll 1
+            for (int R = I; R < 4; ++R) {
+                const float* sg = tab + ((R == I) ? tab_tau(R) : tab_sigma(R, I)) * 128 + ch;
+                store2_split(sm + kKFh, sm + kKFl, sw128_offset(kf_off(R) + r, kc, 160), k0 * f0 * sg[0],
+                             k1 * f1 * sg[1]);
+            }
+            store2_split(out + kOffWkQh, out + kOffWkQl, sw128_offset(64 + r, ch, 128), q0 * e0 * x0, q1 * e1 * x1);
+            kd0[j] = k0 * f0 * y0;
+            kd1[j] = k1 * f1 * y1;
         }
-        if (tid < 128) reinterpret_cast<float*>(out + kOffGam)[tid] = __expf(gb[4 * 128 + tid]);
+        store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch, r0, 128), kd0);
+        store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch + 1, r0, 128), kd1);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+            mma3(tbase, smem_u32(sm + kAKQh), smem_u32(sm + kAKQl), 128, smem_u32(sm + kKFh), smem_u32(sm + kKFl),
+                 160, false, 4, idesc_bf16_f32(128, 160), hr > 0);
+            mma_commit(&mbar);
+        }
+        if (!mbar_wait(&mbar, phase)) {
+            record_error(err, KDA_ERR_TIMEOUT);
+            atomicExch(&sflags[1], 1u);
+        }
+        phase ^= 1;
+        tc_fence_after();
+        __syncthreads();
+        if (sflags[1]) {
+            abort = true;
+            break;
+        }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tbase = sflags[2];
-
-    // ---- MMA 1: [K.E ; Q.E] (128 x 128) x versions^T (160 x 128), three terms --
-    if (tid == 0) {
-        mma3(tbase, smem_u32(sm + kAKQh), smem_u32(sm + kAKQl), 128, smem_u32(sm + kKFh), smem_u32(sm + kKFl), 160,
-             kD / 16, idesc_bf16_f32(128, 160), false);
-        mma_commit(&mbar);
-    }
-    uint32_t phase = 0;
-    if (!mbar_wait(&mbar, phase)) {
-        record_error(err, KDA_ERR_TIMEOUT);
-        atomicExch(&sflags[1], 1u);
-    }
-    phase ^= 1;
-    tc_fence_after();
-    __syncthreads();
-    const bool abort1 = sflags[1] != 0;
 
     float* As = reinterpret_cast<float*>(sm + kAs);
     float* Ts = reinterpret_cast<float*>(sm + kTs);
     float* scr = reinterpret_cast<float*>(sm + kScr);
-    if (!abort1) {
+    if (!abort) {
         // ---- A and P out of TMEM ---------------------------------------------------
         // lane L < 64: row L of the key products; L >= 64: row L-64 of the query
         // products.  Warps w and w+4 share sub-partition w % 4 and split its columns.
@@ -362,42 +357,37 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         const float br = sbeta[r];
         for (int gi = gbeg; gi < gend; ++gi) {
             float vals[16];
-            tmem_ld16(tmem_addr(tbase, 32 * sp, cbeg + 16 * gi), vals);
+            const int col0 = cbeg + 16 * gi;
+            tmem_ld16(tmem_addr(tbase, 32 * sp, col0), vals);
             tmem_ld_wait();
+            const int i0 = col0 - kf_off(R);              // multiple of 16
+            if (i0 < 0 || i0 >= 16 * R + 16) continue;    // another block's version
+            if (!is_p) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const int col = cbeg + 16 * gi + e;
-                const int i = col - kf_off(R);
-                if (i < 0 || i >= 16 * R + 16) continue;   // another block's version
-                if (!is_p) As[r * 64 + i] = (i < r) ? br * vals[e] : 0.f;
-                else store1_split(sm + kPh, sm + kPl, sw128_offset(r, i, 64), (i <= r) ? vals[e] : 0.f);
+                for (int e = 0; e < 16; ++e) As[r * kAS + i0 + e] = (i0 + e < r) ? br * vals[e] : 0.f;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vals[e] = (i0 + e <= r) ? vals[e] : 0.f;
+                store8_split(sm + kPh, sm + kPl, sw128_chunk(r, i0, 64), vals);
+                store8_split(sm + kPh, sm + kPl, sw128_chunk(r, i0 + 8, 64), vals + 8);
             }
         }
         if (warp < 4) {
-            for (int i = 16 * R + 16; i < 64; ++i) {
-                if (!is_p) As[r * 64 + i] = 0.f;
-                else store1_split(sm + kPh, sm + kPl, sw128_offset(r, i, 64), 0.f);
+            const float zero[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int i = 16 * R + 16; i < 64; i += 8) {
+                if (!is_p) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) As[r * kAS + i + e] = 0.f;
+                } else {
+                    store8_split(sm + kPh, sm + kPl, sw128_chunk(r, i, 64), zero);
+                }
             }
         }
-        // (beta K exp(g))^T, three-term operand (MMA 1 no longer reads this region)
-        float bk[4][8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float kk[4];
-            unpack4(kr[j], kk);
-            const float b = sbeta[r0 + j];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) bk[x][j] = b * kk[x] * __expf(g[j][x]);
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x) store8_split(sm + kXKh, sm + kXKl, sw128_chunk(c0 + x, r0, 128), bk[x]);
     }
-    tc_fence_before();
     __syncthreads();
-    tc_fence_after();
 
     // ---- diagonal blocks with a large decay range: pairwise on CUDA cores ----------
-    if (!abort1 && fbmask) {
+    if (!abort && fbmask) {
         for (int R = 0; R < 4; ++R) {
             if (!(fbmask & (1u << R))) continue;
             float* sh = scr;   // [16][128] block-local cumulative log decay
@@ -431,8 +421,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                     spq += __shfl_xor_sync(0xffffffffu, spq, o);
                 }
                 if (lane == 0) {
-                    As[row * 64 + col] = (ii < rr) ? sbeta[row] * sa : 0.f;
-                    store1_split(sm + kPh, sm + kPl, sw128_offset(row, col, 64), spq);
+                    As[row * kAS + col] = (ii < rr) ? sbeta[row] * sa : 0.f;
+                    __nv_bfloat16 ph, pl;
+                    split1(spq, ph, pl);
+                    *reinterpret_cast<__nv_bfloat16*>(sm + kPh + sw128_offset(row, col, 64)) = ph;
+                    *reinterpret_cast<__nv_bfloat16*>(sm + kPl + sw128_offset(row, col, 64)) = pl;
                 }
             }
             __syncthreads();
@@ -440,22 +433,28 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     }
 
     // ---- T = (I + A)^{-1}: diagonal 16 x 16 blocks, then by block distance -----------
-    if (!abort1) {
+    if (!abort) {
         if (warp < 4 && lane < 16) {
+            // column j of the inverse of the unit lower-triangular diagonal block,
+            // built top-down in registers: t[rr] = -sum_{i<rr} A[rr][i] t[i]
             const int base = 16 * warp, j = lane;
-            for (int rr = 0; rr < 16; ++rr) Ts[(base + rr) * 64 + base + j] = (rr == j) ? 1.f : 0.f;
-            for (int rr = j + 1; rr < 16; ++rr) {
+            float t[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
                 float s = 0.f;
-                for (int i = j; i < rr; ++i) s += As[(base + rr) * 64 + base + i] * Ts[(base + i) * 64 + base + j];
-                Ts[(base + rr) * 64 + base + j] = -s;
+#pragma unroll
+                for (int i = 0; i < rr; ++i) s += As[(base + rr) * kAS + base + i] * t[i];
+                t[rr] = (rr == j) ? 1.f : ((rr < j) ? 0.f : -s);
             }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) Ts[(base + rr) * kAS + base + j] = t[rr];
         }
         for (int e = tid; e < 64 * 64; e += kIntraThreads) {
             const int rr = e >> 6, cc = e & 63;
-            if ((cc >> 4) > (rr >> 4)) Ts[e] = 0.f;
+            if ((cc >> 4) > (rr >> 4)) Ts[rr * kAS + cc] = 0.f;
         }
         __syncthreads();
-        float* Y = scr;   // [3][16][16]
+        float* Y = scr;   // [3][16][17]
         for (int d = 1; d < 4; ++d) {
             const int nb = 4 - d;
             for (int e = tid; e < nb * 256; e += kIntraThreads) {
@@ -463,23 +462,29 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 const int R = bi + d, I2 = bi;
                 float s = 0.f;
                 for (int J = I2; J < R; ++J)
+#pragma unroll
                     for (int m = 0; m < 16; ++m)
-                        s += As[(16 * R + rr) * 64 + 16 * J + m] * Ts[(16 * J + m) * 64 + 16 * I2 + ii];
-                Y[e] = s;
+                        s += As[(16 * R + rr) * kAS + 16 * J + m] * Ts[(16 * J + m) * kAS + 16 * I2 + ii];
+                Y[bi * 272 + rr * 17 + ii] = s;
             }
             __syncthreads();
             for (int e = tid; e < nb * 256; e += kIntraThreads) {
                 const int bi = e >> 8, rr = (e >> 4) & 15, ii = e & 15;
                 const int R = bi + d, I2 = bi;
                 float s = 0.f;
-                for (int m = 0; m < 16; ++m) s += Ts[(16 * R + rr) * 64 + 16 * R + m] * Y[bi * 256 + m * 16 + ii];
-                Ts[(16 * R + rr) * 64 + 16 * I2 + ii] = -s;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) s += Ts[(16 * R + rr) * kAS + 16 * R + m] * Y[bi * 272 + m * 17 + ii];
+                Ts[(16 * R + rr) * kAS + 16 * I2 + ii] = -s;
             }
             __syncthreads();
         }
+        // T (hi/lo) into rows 0-63 of [T ; P T]
         for (int e = tid; e < 64 * 8; e += kIntraThreads) {
             const int rr = e >> 3, k8 = (e & 7) * 8;
-            store8_split(sm + kTh, sm + kTl, sw128_chunk(rr, k8, 64), Ts + rr * 64 + k8);
+            float t8[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) t8[x] = Ts[rr * kAS + k8 + x];
+            store8_split(sm + kTPh, sm + kTPl, sw128_chunk(rr, k8, 128), t8);
         }
     }
     fence_async_smem();
@@ -487,51 +492,72 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
 
-    // ---- MMA 2: [U | Wk] = T [beta V | beta K exp(g)] ------------------------------------
-    if (tid == 0 && !abort1) {
-        const uint32_t th = smem_u32(sm + kTh), tl = smem_u32(sm + kTl);
-        mma3(tmem_addr(tbase, 0, 0), th, tl, 64, smem_u32(sm + kXVh), smem_u32(sm + kXVl), 128, kC / 16,
-             idesc_bf16_f32(64, 128), false);
-        mma3(tmem_addr(tbase, 0, 128), th, tl, 64, smem_u32(sm + kXKh), smem_u32(sm + kXKl), 128, kC / 16,
-             idesc_bf16_f32(64, 128), false);
+    // ---- P T  (M = 64; B = T read as an MN-major 64 x 64 tile) -----------------------
+    if (tid == 0 && !abort) {
+        mma3(tmem_addr(tbase, 0, 0), smem_u32(sm + kPh), smem_u32(sm + kPl), 64, smem_u32(sm + kTPh),
+             smem_u32(sm + kTPl), 64, true, kC / 16, idesc_bf16_f32_bmn(64, 64), false);
         mma_commit(&mbar);
     }
-    if (!abort1 && !mbar_wait(&mbar, phase)) {
+    if (!abort && !mbar_wait(&mbar, phase)) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
     }
     phase ^= 1;
     tc_fence_after();
     __syncthreads();
-    const bool abort2 = sflags[1] != 0;
+    abort = abort || sflags[1] != 0;
 
-    // ---- epilogue 2: U (fp32) and Wk (hi/lo image) to the workspace; U^T, Wk^T operands --
-    // M = 64 layout: sub-partition sp, lanes 0-15 hold rows 16 sp + lane.
-    if (!abort2) {
-        const int sp = warp & 3;
-        const int r = 16 * sp + (lane & 15);
-        const bool second = warp >= 4;     // warps 4-7: the Wk half
-        const bool active = lane < 16;
-        for (int gi = 0; gi < 8; ++gi) {
-            float vals[16];
-            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi), vals);
-            tmem_ld_wait();
-            if (!active) continue;
-            if (!second) {
-                const int cb = (16 * gi) >> 5, cc = (16 * gi) & 31;
-                float4* dst = reinterpret_cast<float4*>(out + kOffU + cb * 8192 + r * 128 + cc * 4);
+    if (!abort) {
+        // ---- P T (hi/lo) into rows 64-127 of [T ; P T] --------------------------------
+        {
+            const int sp = warp & 3;
+            const int r = 16 * sp + (lane & 15);
+            const int cb = (warp < 4) ? 0 : 32;
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    dst[e] = make_float4(vals[4 * e], vals[4 * e + 1], vals[4 * e + 2], vals[4 * e + 3]);
+            for (int gi = 0; gi < 2; ++gi) {
+                float vals[16];
+                tmem_ld16(tmem_addr(tbase, 32 * sp, cb + 16 * gi), vals);
+                tmem_ld_wait();
+                if (lane < 16) {
+                    store8_split(sm + kTPh, sm + kTPl, sw128_chunk(64 + r, cb + 16 * gi, 128), vals);
+                    store8_split(sm + kTPh, sm + kTPl, sw128_chunk(64 + r, cb + 16 * gi + 8, 128), vals + 8);
+                }
+            }
+        }
+        // ---- [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns) ----------
+        // k, v and log alpha are read again (from L2) and g is rebuilt from the
+        // carries, so that no per-row state stays in registers through the middle.
+        uint32_t vv[8][2], kv[8][2], lv[8][2];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    store1_split(sm + kUTh, sm + kUTl, sw128_offset(16 * gi + e, r, 128), vals[e]);
-            } else {
-                store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, 16 * gi, 128), vals);
-                store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, 16 * gi + 8, 128), vals + 8);
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    store1_split(sm + kWTh, sm + kWTl, sw128_offset(16 * gi + e, r, 128), vals[e]);
+            for (int hh = 0; hh < 2; ++hh) {
+                vv[j][hh] = kv[j][hh] = lv[j][hh] = 0u;
+                if (r < len) {
+                    const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
+                    vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
+                    kv[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
+                    lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
+                }
+            }
+        }
+        float a[4] = {carry[0], carry[1], carry[2], carry[3]};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
+            const float b = sbeta[r];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int ch = 64 * hh + kc;
+                if (r < len) {
+                    a[2 * hh] += fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor);
+                    a[2 * hh + 1] += fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor);
+                }
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, ch, 64), b * bf16_lo(vv[j][hh]),
+                             b * bf16_hi(vv[j][hh]));
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), b * bf16_lo(kv[j][hh]) * __expf(a[2 * hh]),
+                             b * bf16_hi(kv[j][hh]) * __expf(a[2 * hh + 1]));
             }
         }
     }
@@ -540,54 +566,67 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
 
-    // ---- MMA 3: [U' | P Wk] = P [U | Wk] -------------------------------------------------
-    if (tid == 0 && !abort2) {
-        const uint32_t ph = smem_u32(sm + kPh), pl = smem_u32(sm + kPl);
-        mma3(tmem_addr(tbase, 0, 0), ph, pl, 64, smem_u32(sm + kUTh), smem_u32(sm + kUTl), 128, kC / 16,
-             idesc_bf16_f32(64, 128), false);
-        mma3(tmem_addr(tbase, 0, 128), ph, pl, 64, smem_u32(sm + kWTh), smem_u32(sm + kWTl), 128, kC / 16,
-             idesc_bf16_f32(64, 128), false);
+    // ---- [U | Wk ; U' | P Wk] = [T ; P T] [beta V | beta K exp(g)] --------------------
+    if (tid == 0 && !abort) {
+        const uint32_t ah = smem_u32(sm + kTPh), al = smem_u32(sm + kTPl);
+        const uint32_t bh = smem_u32(sm + kXh), bl = smem_u32(sm + kXl);
+        mma3(tmem_addr(tbase, 0, 0), ah, al, 128, bh, bl, 64, true, kC / 16, idesc_bf16_f32_bmn(128, 128), false);
+        mma3(tmem_addr(tbase, 0, 128), ah, al, 128, bh + 16384, bl + 16384, 64, true, kC / 16,
+             idesc_bf16_f32_bmn(128, 128), false);
         mma_commit(&mbar);
     }
-    if (!abort2 && !mbar_wait(&mbar, phase)) {
+    if (!abort && !mbar_wait(&mbar, phase)) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
     }
     tc_fence_after();
     __syncthreads();
-    const bool abort3 = sflags[1] != 0;
+    abort = abort || sflags[1] != 0;
 
-    // ---- epilogue 3: U' (fp32); Q' = Q exp(g) - P Wk (hi/lo image) -------------------------
-    if (!abort3) {
-        const int sp = warp & 3;
-        const int r = 16 * sp + (lane & 15);
-        const bool second = warp >= 4;
-        const bool active = lane < 16;
-        for (int gi = 0; gi < 8; ++gi) {
-            float vals[16];
-            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi), vals);
+    // ---- epilogue: U, U' (fp32); Wk and Q' = Q exp(g) - P Wk (hi/lo images) ----------
+    if (!abort) {
+        const int sp = warp & 3, L = 32 * sp + lane;
+        const bool second = warp >= 4;      // columns [128, 256): Wk / P Wk
+        const int r = L & 63;
+        float* uo = reinterpret_cast<float*>(out + ((L < 64) ? kOffU : kOffU2));
+        const bool qrow = second && L >= 64;   // warp-uniform (sub-partitions 2, 3)
+        for (int gi = 0; gi < 8; gi += 2) {
+            uint4 qh[4], ql[4];
+            if (qrow) {
+                // Q exp(g) of the two column groups, read before the TMEM loads so
+                // the four 16-byte reads overlap
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const uint32_t off = sw128_chunk(64 + r, 16 * gi + 8 * x, 128);
+                    qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
+                    ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
+                }
+            }
+            float vals[2][16];
+            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi), vals[0]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi + 16), vals[1]);
             tmem_ld_wait();
-            if (!active) continue;
-            if (!second) {
-                const int cb = (16 * gi) >> 5, cc = (16 * gi) & 31;
-                float4* dst = reinterpret_cast<float4*>(out + kOffU2 + cb * 8192 + r * 128 + cc * 4);
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    dst[e] = make_float4(vals[4 * e], vals[4 * e + 1], vals[4 * e + 2], vals[4 * e + 3]);
-            } else {
+            for (int x = 0; x < 2; ++x) {
+                const int j0 = 16 * (gi + x);
+                if (!second) {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t off = sw128_chunk(64 + r, 16 * gi + 8 * hh, 128);
-                    const uint4 qh = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
-                    const uint4 ql = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
-                    const float* pv = vals + 8 * hh;
-                    float qv[8] = {bf16_lo(qh.x) + bf16_lo(ql.x), bf16_hi(qh.x) + bf16_hi(ql.x),
-                                   bf16_lo(qh.y) + bf16_lo(ql.y), bf16_hi(qh.y) + bf16_hi(ql.y),
-                                   bf16_lo(qh.z) + bf16_lo(ql.z), bf16_hi(qh.z) + bf16_hi(ql.z),
-                                   bf16_lo(qh.w) + bf16_lo(ql.w), bf16_hi(qh.w) + bf16_hi(ql.w)};
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<float4*>(uo + u_index(r, j0 + 4 * e)) =
+                            make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
+                } else if (!qrow) {
+                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0, 128), vals[x]);
+                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 8, 128), vals[x] + 8);
+                } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) qv[e] -= pv[e];
-                    store8_split(out + kOffWkQh, out + kOffWkQl, off, qv);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float a[8], b[8];
+                        unpack8(qh[2 * x + hh], a);
+                        unpack8(ql[2 * x + hh], b);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) a[e] = a[e] + b[e] - vals[x][8 * hh + e];
+                        store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(64 + r, j0 + 8 * hh, 128), a);
+                    }
                 }
             }
         }
@@ -610,9 +649,9 @@ struct RecurLayout {
     static constexpr uint32_t kUtile = (uint32_t)BV * 64 * 4;                  // U (or U') tile, fp32
     static constexpr uint32_t kUStage = 2 * kUtile + 512;                      // U, U', Gamma_C
     static constexpr uint32_t kUU = 98304;                                     // two U stages
-    static constexpr uint32_t kST = (kUU + 2 * kUStage + 1023) / 1024 * 1024;  // S^T hi/lo [BV][128 k]
-    static constexpr uint32_t kWT = kST + 2 * (uint32_t)BV * 256;              // W^T hi/lo [BV][64 k]
-    static constexpr uint32_t kBars = kWT + 2 * (uint32_t)BV * 128;
+    static constexpr uint32_t kS = (kUU + 2 * kUStage + 1023) / 1024 * 1024;  // S hi/lo: 128 rows x 128 B (MN-major)
+    static constexpr uint32_t kW = kS + 2 * 16384;                             // W hi/lo: 64 rows x 128 B (MN-major)
+    static constexpr uint32_t kBars = kW + 2 * 8192;
     static constexpr uint32_t kSmem = kBars + 128;
     static constexpr uint32_t kAlloc = kSmem + 1024;
     static constexpr uint32_t kTmemCols = (2 * BV < 32) ? 32 : 2 * BV;
@@ -632,10 +671,10 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     uint64_t* bar1 = bars + 4;
     uint64_t* bar2 = bars + 5;
     uint32_t* sflags = reinterpret_cast<uint32_t*>(bars + 6);        // [0] tmem base, [1] abort
-    uint8_t* sth = sm + Lay::kST;
-    uint8_t* stl = sth + BV * 256;
-    uint8_t* wth = sm + Lay::kWT;
-    uint8_t* wtl = wth + BV * 128;
+    uint8_t* s_h = sm + Lay::kS;
+    uint8_t* s_l = s_h + 16384;
+    uint8_t* w_h = sm + Lay::kW;
+    uint8_t* w_l = w_h + 8192;
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const SeqInfo sq = smap.get(blockIdx.x);
@@ -706,9 +745,9 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     for (int n = 0; n < nch; ++n) {
         const int stage = n & 1;
         const uint8_t* uu = sm + Lay::kUU + stage * Lay::kUStage;
-        // S_n as the B operand of MMA 1 (three-term): element (row j, k = c)
+        // S_n as the MN-major B operand of MMA 1 (K = channel row c, N = columns)
 #pragma unroll
-        for (int j = 0; j < BV; ++j) store1_split(sth, stl, sw128_offset(j, c, BV), s[j]);
+        for (int j = 0; j < BV; j += 8) store8_split(s_h, s_l, mn_chunk(c, j, 128), s + j);
         if (!mbar_wait(&uu_full[stage], (uint32_t)(n >> 1) & 1u)) {
             record_error(err, KDA_ERR_TIMEOUT);
             atomicExch(&sflags[1], 1u);
@@ -734,8 +773,8 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 atomicExch(&sflags[1], 1u);
             } else {
                 const uint32_t a = smem_u32(sm + Lay::kWkQ);
-                mma3(t_d, a, a + 32768, 128, smem_u32(sth), smem_u32(stl), BV, kD / 16, idesc_bf16_f32(128, BV),
-                     false);
+                mma3(t_d, a, a + 32768, 128, smem_u32(s_h), smem_u32(s_l), 128, true, kD / 16,
+                     idesc_bf16_f32_bmn(128, BV), false);
             }
             mma_commit(bar1);
         }
@@ -745,62 +784,72 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         }
         tc_fence_after();
         if (tid == 0 && n + 1 < nch) load_wkq(n + 1);   // MMA 1 is done with the buffer
-        // lanes 0-63: W = U - Wk S (rows are tokens); lanes 64-127: O = Q' S + U'
-        {
-            const int r = tid & 63;
-            const float* ut = reinterpret_cast<const float*>(uu + ((tid < 64) ? 0 : Lay::kUtile));
+        const int r = tid & 63;
+        const float* ut = reinterpret_cast<const float*>(uu + ((tid < 64) ? 0 : Lay::kUtile));
+        if (tid < 64) {
+            // W = U - Wk S (rows are tokens) -> MN-major B operand of MMA 2
+#pragma unroll
+            for (int jb = 0; jb < BV; jb += 16) {
+                float d[16];
+                tmem_ld16(tmem_addr(t_d, 32 * warp, jb), d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
+                    d[e] = u.x - d[e]; d[e + 1] = u.y - d[e + 1]; d[e + 2] = u.z - d[e + 2]; d[e + 3] = u.w - d[e + 3];
+                }
+                store8_split(w_h, w_l, mn_chunk(r, jb, 64), d);
+                store8_split(w_h, w_l, mn_chunk(r, jb + 8, 64), d + 8);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            asm volatile("bar.sync 1, 64;" ::: "memory");   // warps 0-1 only: W is ready
+            tc_fence_after();
+            if (tid == 0) {
+                if (!mbar_wait(kdt_full, (uint32_t)n & 1u)) {
+                    record_error(err, KDA_ERR_TIMEOUT);
+                    atomicExch(&sflags[1], 1u);
+                } else {
+                    const uint32_t a = smem_u32(sm + Lay::kKdT);
+                    mma3(t_s, a, a + 16384, 128, smem_u32(w_h), smem_u32(w_l), 64, true, kC / 16,
+                         idesc_bf16_f32_bmn(128, BV), true);
+                }
+                mma_commit(bar2);
+            }
+        } else {
+            // O = Q' S + U' (rows are tokens), overlapping MMA 2
             const int rows_here = min(kC, sq.len - n * kC);
 #pragma unroll
             for (int jb = 0; jb < BV; jb += 16) {
                 float d[16];
                 tmem_ld16(tmem_addr(t_d, 32 * warp, jb), d);
                 tmem_ld_wait();
-                float u[16];
+                if (r < rows_here) {
 #pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const int j = jb + e;
-                    const float4 w = *reinterpret_cast<const float4*>(ut + (j >> 5) * 2048 + r * 32 + (j & 31));
-                    u[e] = w.x; u[e + 1] = w.y; u[e + 2] = w.z; u[e + 3] = w.w;
-                }
-                if (tid < 64) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) store1_split(wth, wtl, sw128_offset(jb + e, r, BV), u[e] - d[e]);
-                } else if (r < rows_here) {
+                    for (int e = 0; e < 16; e += 4) {
+                        const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
+                        d[e] += u.x; d[e + 1] += u.y; d[e + 2] += u.z; d[e + 3] += u.w;
+                    }
                     __nv_bfloat16* dst = o + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + jb;
                     uint4 w0, w1;
-                    w0.x = pack_bf16(d[0] + u[0], d[1] + u[1]); w0.y = pack_bf16(d[2] + u[2], d[3] + u[3]);
-                    w0.z = pack_bf16(d[4] + u[4], d[5] + u[5]); w0.w = pack_bf16(d[6] + u[6], d[7] + u[7]);
-                    w1.x = pack_bf16(d[8] + u[8], d[9] + u[9]); w1.y = pack_bf16(d[10] + u[10], d[11] + u[11]);
-                    w1.z = pack_bf16(d[12] + u[12], d[13] + u[13]); w1.w = pack_bf16(d[14] + u[14], d[15] + u[15]);
+                    w0.x = pack_bf16(d[0], d[1]); w0.y = pack_bf16(d[2], d[3]);
+                    w0.z = pack_bf16(d[4], d[5]); w0.w = pack_bf16(d[6], d[7]);
+                    w1.x = pack_bf16(d[8], d[9]); w1.y = pack_bf16(d[10], d[11]);
+                    w1.z = pack_bf16(d[12], d[13]); w1.w = pack_bf16(d[14], d[15]);
                     reinterpret_cast<uint4*>(dst)[0] = w0;
                     reinterpret_cast<uint4*>(dst)[1] = w1;
                 }
             }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (sflags[1]) break;
-        tc_fence_after();
-        if (tid == 0) {
-            if (!mbar_wait(kdt_full, (uint32_t)n & 1u)) {
-                record_error(err, KDA_ERR_TIMEOUT);
-                atomicExch(&sflags[1], 1u);
-            } else {
-                const uint32_t a = smem_u32(sm + Lay::kKdT);
-                mma3(t_s, a, a + 16384, 128, smem_u32(wth), smem_u32(wtl), BV, kC / 16, idesc_bf16_f32(128, BV),
-                     true);
-            }
-            mma_commit(bar2);
         }
         if (!mbar_wait(bar2, (uint32_t)n & 1u)) {
             record_error(err, KDA_ERR_TIMEOUT);
             atomicExch(&sflags[1], 1u);
         }
         tc_fence_after();
+        __syncthreads();   // every thread is past its reads of this chunk's U / U' stage
         if (tid == 0) {
             if (n + 1 < nch) load_kdt(n + 1);          // MMA 2 is done with the buffer
-            if (n + 2 < nch) load_uu(n + 2, stage);    // every thread is past its reads of this stage
+            if (n + 2 < nch) load_uu(n + 2, stage);
         }
 #pragma unroll
         for (int jb = 0; jb < BV; jb += 16) {

@@ -54,6 +54,38 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Same with B MN-major (N contiguous).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+    return idesc_bf16_f32(M, N) | (1u << 16);
+}
+
+// ---------------------------------------------------------------------------
+// MN-major B tiles (K rows, N contiguous), 128-byte swizzle, bf16.
+// N is split into blocks of 64 elements; block b holds K rows of 128 bytes at
+// byte offset b * K * 128, with the same chunk ^ (row % 8) permutation as the
+// K-major tiles.  (A 64-wide MN-major tile and a 64-deep K-major tile of the
+// same row-major matrix therefore have the same bytes.)
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint32_t mn_chunk(int k, int n, int K) {   // n % 8 == 0
+    return (uint32_t)((n >> 6) * K * 128 + k * 128 + ((((n & 63) >> 3) ^ (k & 7)) << 4));
+}
+__host__ __device__ __forceinline__ uint32_t mn_offset(int k, int n, int K) {
+    return mn_chunk(k, n & ~7, K) + ((n & 7) << 1);
+}
+
+// Descriptor of the K-slice [16 s, 16 s + 16) of an MN-major tile with K rows:
+// LBO = K * 128 bytes between 64-wide N blocks, SBO = 1024 bytes between
+// 8-row groups.
+__device__ __forceinline__ uint64_t mn_desc_k(uint32_t tile_addr, int K, int s) {
+    const uint32_t addr = tile_addr + (uint32_t)s * 2048u;
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(((uint32_t)K * 128u >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
