@@ -305,8 +305,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             const float q0 = bf16_lo(qv[j]), q1 = bf16_hi(qv[j]);
             store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, kc, 128), k0 * e0, k1 * e1);
             store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, kc, 128), q0 * e0, q1 * e1);
-#pragma unroll 1
-            for (int R = I; R < 4; ++R) {
+#pragma unroll
+            for (int R = 0; R < 4; ++R) {
+                if (R < I) continue;
                 const float* sg = tab + ((R == I) ? tab_tau(R) : tab_sigma(R, I)) * 128 + ch;
                 store2_split(sm + kKFh, sm + kKFl, sw128_offset(kf_off(R) + r, kc, 160), k0 * f0 * sg[0],
                              k1 * f1 * sg[1]);
