@@ -88,7 +88,7 @@ constexpr uint32_t kAs = 0;              // A fp32 [64][65]
 constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
 constexpr uint32_t kPl = 25600;
 constexpr uint32_t kScr = 33792;         // 8 KB scratch
-constexpr uint32_t kTs = 41984;          // T fp32 [64][65]
+constexpr uint32_t kTs = 41984;          // T fp32 [64][68]
 // [T ; P T] (128 rows x 64 k, K-major; rows 0-63 also serve as the MN-major T)
 constexpr uint32_t kTPh = 65536;
 constexpr uint32_t kTPl = 81920;
@@ -99,7 +99,9 @@ constexpr uint32_t kTab = 98304;         // tables
 constexpr int kNumTab = 18;              // tau[4], sigma[6], exp(gb)[4], exp(g_C - gb[b+1])[4]
 constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 64 * 4 + 64;
 constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
-constexpr int kAS = 65;                  // row stride of As / Ts (floats)
+constexpr int kAS = 65;                  // row stride of As (floats)
+constexpr int kTS = 68;                  // row stride of Ts (floats; rows 16-byte aligned)
+constexpr int kYS = 20;                  // row stride of the 16 x 16 blocks Y (floats)
 
 // rows of the decayed-key versions: version R covers keys [0, 16 R + 16)
 __host__ __device__ __forceinline__ int kf_off(int R) { return (R * (R + 1)) * 8; }   // 0, 16, 48, 96
@@ -192,9 +194,23 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     if (tid < 64) sbeta[tid] = (tid < len) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
 
     // ---- log alpha of 8 rows x 4 channels; k, q, v prefetched into L2 ---------
-    // (k and q are read in the round that uses them, v at the end; holding them
-    // in registers through the chunk would push the kernel past 128 registers)
+    // (k and q of a channel half are read one phase before the round that uses
+    // them, v at the end; holding them in registers through the chunk would push
+    // the kernel past 128 registers)
     float g[8][4];
+    uint32_t kv[8], qv[8];
+    auto load_kq = [&](int hr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
+            kv[j] = qv[j] = 0u;
+            if (r < len) {
+                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hr + kc;
+                kv[j] = *reinterpret_cast<const uint32_t*>(k + off);
+                qv[j] = *reinterpret_cast<const uint32_t*>(q + off);
+            }
+        }
+    };
     if (lane < 16) {
         const int r = r0 + (lane & 7);
         if (r < len) {
@@ -215,6 +231,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             g[j][2 * hh + 1] = (r < len) ? fmaxf(bf16_hi(a), kLogAlphaFloor) : 0.f;
         }
     }
+    load_kq(0);
     // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
     for (int j = 1; j < 8; ++j)
@@ -284,17 +301,6 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         const float glast0 = gb[(I + 1) * 128 + ch], glast1 = gb[(I + 1) * 128 + ch + 1];
         const float x0 = tab[tab_e0(I) * 128 + ch], x1 = tab[tab_e0(I) * 128 + ch + 1];
         const float y0 = tab[tab_ec(I) * 128 + ch], y1 = tab[tab_ec(I) * 128 + ch + 1];
-        uint32_t kv[8], qv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = r0 + j;
-            kv[j] = qv[j] = 0u;
-            if (r < len) {
-                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + ch;
-                kv[j] = *reinterpret_cast<const uint32_t*>(k + off);
-                qv[j] = *reinterpret_cast<const uint32_t*>(q + off);
-            }
-        }
         float kd0[8], kd1[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -318,6 +324,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         }
         store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch, r0, 128), kd0);
         store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch + 1, r0, 128), kd1);
+        if (hr == 0) load_kq(1);   // in flight during this round's MMA
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -435,56 +442,71 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 
     // ---- T = (I + A)^{-1}: diagonal 16 x 16 blocks, then by block distance -----------
     if (!abort) {
-        if (warp < 4 && lane < 16) {
-            // column j of the inverse of the unit lower-triangular diagonal block,
-            // built top-down in registers: t[rr] = -sum_{i<rr} A[rr][i] t[i]
-            const int base = 16 * warp, j = lane;
-            float t[16];
+        if (warp < 4) {
+            // inverse of the unit lower-triangular diagonal block K = warp by
+            // right-looking elimination: lane = (row rr, column half hc); pivot row i
+            // is final after step i - 1 and reaches the rows below by shuffles
+            const int K = warp, rr = lane & 15, hc = lane >> 4;
+            float arow[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float s = 0.f;
+            for (int i = 0; i < 16; ++i) arow[i] = As[(16 * K + rr) * kAS + 16 * K + i];   // zero for i >= rr
+            float t[8];
 #pragma unroll
-                for (int i = 0; i < rr; ++i) s += As[(base + rr) * kAS + base + i] * t[i];
-                t[rr] = (rr == j) ? 1.f : ((rr < j) ? 0.f : -s);
-            }
+            for (int c = 0; c < 8; ++c) t[c] = (8 * hc + c == rr) ? 1.f : 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Ts[(base + rr) * kAS + base + j] = t[rr];
-        }
-        for (int e = tid; e < 64 * 64; e += kIntraThreads) {
-            const int rr = e >> 6, cc = e & 63;
-            if ((cc >> 4) > (rr >> 4)) Ts[rr * kAS + cc] = 0.f;
+            for (int i = 0; i < 15; ++i)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) t[c] = fmaf(-arow[i], __shfl_sync(0xffffffffu, t[c], i + 16 * hc), t[c]);
+            float* trow = Ts + (16 * K + rr) * kTS + 16 * K + 8 * hc;
+            reinterpret_cast<float4*>(trow)[0] = make_float4(t[0], t[1], t[2], t[3]);
+            reinterpret_cast<float4*>(trow)[1] = make_float4(t[4], t[5], t[6], t[7]);
         }
         __syncthreads();
-        float* Y = scr;   // [3][16][17]
+        // block (R, I) at distance d = R - I: Y = sum_{I <= J < R} A_RJ T_JI, then
+        // T_RI = -T_RR Y; each thread forms four adjacent columns of one row
+        float* Y = scr;   // [3][16][kYS]
         for (int d = 1; d < 4; ++d) {
             const int nb = 4 - d;
-            for (int e = tid; e < nb * 256; e += kIntraThreads) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, ii = e & 15;
-                const int R = bi + d, I2 = bi;
-                float s = 0.f;
+            const int e = tid;
+            const int bi = e >> 6, rr = (e >> 2) & 15, i4 = (e & 3) * 4;
+            const int R = bi + d, I2 = bi;
+            if (e < nb * 64) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int J = I2; J < R; ++J)
 #pragma unroll
-                    for (int m = 0; m < 16; ++m)
-                        s += As[(16 * R + rr) * kAS + 16 * J + m] * Ts[(16 * J + m) * kAS + 16 * I2 + ii];
-                Y[bi * 272 + rr * 17 + ii] = s;
+                    for (int m = 0; m < 16; ++m) {
+                        const float av = As[(16 * R + rr) * kAS + 16 * J + m];
+                        const float4 tv = *reinterpret_cast<const float4*>(Ts + (16 * J + m) * kTS + 16 * I2 + i4);
+                        acc.x = fmaf(av, tv.x, acc.x); acc.y = fmaf(av, tv.y, acc.y);
+                        acc.z = fmaf(av, tv.z, acc.z); acc.w = fmaf(av, tv.w, acc.w);
+                    }
+                *reinterpret_cast<float4*>(Y + (bi * 16 + rr) * kYS + i4) = acc;
             }
             __syncthreads();
-            for (int e = tid; e < nb * 256; e += kIntraThreads) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, ii = e & 15;
-                const int R = bi + d, I2 = bi;
-                float s = 0.f;
+            if (e < nb * 64) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) s += Ts[(16 * R + rr) * kAS + 16 * R + m] * Y[bi * 272 + m * 17 + ii];
-                Ts[(16 * R + rr) * kAS + 16 * I2 + ii] = -s;
+                for (int m = 0; m < 16; ++m) {
+                    const float dv = Ts[(16 * R + rr) * kTS + 16 * R + m];
+                    const float4 yv = *reinterpret_cast<const float4*>(Y + (bi * 16 + m) * kYS + i4);
+                    acc.x = fmaf(dv, yv.x, acc.x); acc.y = fmaf(dv, yv.y, acc.y);
+                    acc.z = fmaf(dv, yv.z, acc.z); acc.w = fmaf(dv, yv.w, acc.w);
+                }
+                *reinterpret_cast<float4*>(Ts + (16 * R + rr) * kTS + 16 * I2 + i4) =
+                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
-        // T (hi/lo) into rows 0-63 of [T ; P T]
+        // T (hi/lo) into rows 0-63 of [T ; P T]; blocks above the diagonal are zero
         for (int e = tid; e < 64 * 8; e += kIntraThreads) {
             const int rr = e >> 3, k8 = (e & 7) * 8;
-            float t8[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) t8[x] = Ts[rr * kAS + k8 + x];
+            float t8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if ((k8 >> 4) <= (rr >> 4)) {
+                const float4 x0 = *reinterpret_cast<const float4*>(Ts + rr * kTS + k8);
+                const float4 x1 = *reinterpret_cast<const float4*>(Ts + rr * kTS + k8 + 4);
+                t8[0] = x0.x; t8[1] = x0.y; t8[2] = x0.z; t8[3] = x0.w;
+                t8[4] = x1.x; t8[5] = x1.y; t8[6] = x1.z; t8[7] = x1.w;
+            }
             store8_split(sm + kTPh, sm + kTPl, sw128_chunk(rr, k8, 128), t8);
         }
     }
@@ -494,6 +516,24 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     tc_fence_after();
 
     // ---- P T  (M = 64; B = T read as an MN-major 64 x 64 tile) -----------------------
+    // v, k and log alpha for the [beta V | beta K exp(g)] operand are read again
+    // (from L2) while this product runs; g is rebuilt from the carries, so that no
+    // per-row state stays in registers through the middle of the kernel.
+    uint32_t vv[8][2], kx[8][2], lv[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int r = r0 + j;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            vv[j][hh] = kx[j][hh] = lv[j][hh] = 0u;
+            if (r < len && !abort) {
+                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
+                vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
+                kx[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
+                lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
+            }
+        }
+    }
     if (tid == 0 && !abort) {
         mma3(tmem_addr(tbase, 0, 0), smem_u32(sm + kPh), smem_u32(sm + kPl), 64, smem_u32(sm + kTPh),
              smem_u32(sm + kTPl), 64, true, kC / 16, idesc_bf16_f32_bmn(64, 64), false);
@@ -526,23 +566,6 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             }
         }
         // ---- [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns) ----------
-        // k, v and log alpha are read again (from L2) and g is rebuilt from the
-        // carries, so that no per-row state stays in registers through the middle.
-        uint32_t vv[8][2], kv[8][2], lv[8][2];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = r0 + j;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                vv[j][hh] = kv[j][hh] = lv[j][hh] = 0u;
-                if (r < len) {
-                    const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
-                    vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
-                    kv[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
-                    lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
-                }
-            }
-        }
         float a[4] = {carry[0], carry[1], carry[2], carry[3]};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -557,8 +580,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 }
                 store2_split(sm + kXh, sm + kXl, mn_offset(r, ch, 64), b * bf16_lo(vv[j][hh]),
                              b * bf16_hi(vv[j][hh]));
-                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), b * bf16_lo(kv[j][hh]) * __expf(a[2 * hh]),
-                             b * bf16_hi(kv[j][hh]) * __expf(a[2 * hh + 1]));
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), b * bf16_lo(kx[j][hh]) * __expf(a[2 * hh]),
+                             b * bf16_hi(kx[j][hh]) * __expf(a[2 * hh + 1]));
             }
         }
     }
@@ -585,50 +608,60 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     abort = abort || sflags[1] != 0;
 
     // ---- epilogue: U, U' (fp32); Wk and Q' = Q exp(g) - P Wk (hi/lo images) ----------
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. row L of [U | Wk ; U' | P Wk];
+    // the two warp groups take 64 of the 128 columns of each part.
     if (!abort) {
         const int sp = warp & 3, L = 32 * sp + lane;
-        const bool second = warp >= 4;      // columns [128, 256): Wk / P Wk
         const int r = L & 63;
-        float* uo = reinterpret_cast<float*>(out + ((L < 64) ? kOffU : kOffU2));
-        const bool qrow = second && L >= 64;   // warp-uniform (sub-partitions 2, 3)
-        for (int gi = 0; gi < 8; gi += 2) {
-            uint4 qh[4], ql[4];
-            if (qrow) {
-                // Q exp(g) of the two column groups, read before the TMEM loads so
-                // the four 16-byte reads overlap
+        const bool qrow = L >= 64;              // warp-uniform (sub-partitions 2, 3)
+        const int cg = (warp >> 2) * 64;
+        float* uo = reinterpret_cast<float*>(out + (qrow ? kOffU2 : kOffU));
+        uint4 qh[4], ql[4];
+        auto load_qg = [&](int j0) {            // Q exp(g) of columns [j0, j0 + 32)
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const uint32_t off = sw128_chunk(64 + r, 16 * gi + 8 * x, 128);
-                    qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
-                    ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
-                }
+            for (int x = 0; x < 4; ++x) {
+                const uint32_t off = sw128_chunk(64 + r, j0 + 8 * x, 128);
+                qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
+                ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
             }
+        };
+        if (qrow) load_qg(cg);
+#pragma unroll
+        for (int bt = 0; bt < 2; ++bt) {
+            const int j0 = cg + 32 * bt;
             float vals[2][16];
-            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi), vals[0]);
-            tmem_ld16(tmem_addr(tbase, 32 * sp, (second ? 128 : 0) + 16 * gi + 16), vals[1]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, j0), vals[0]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, j0 + 16), vals[1]);
             tmem_ld_wait();
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int j0 = 16 * (gi + x);
-                if (!second) {
+            for (int x = 0; x < 2; ++x)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        *reinterpret_cast<float4*>(uo + u_index(r, j0 + 4 * e)) =
-                            make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
-                } else if (!qrow) {
-                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0, 128), vals[x]);
-                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 8, 128), vals[x] + 8);
-                } else {
+                for (int e = 0; e < 4; ++e)
+                    *reinterpret_cast<float4*>(uo + u_index(r, j0 + 16 * x + 4 * e)) =
+                        make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0), vals[0]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0 + 16), vals[1]);
+            tmem_ld_wait();
+            if (!qrow) {
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 16 * x, 128), vals[x]);
+                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 16 * x + 8, 128), vals[x] + 8);
+                }
+            } else {
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        float a[8], b[8];
-                        unpack8(qh[2 * x + hh], a);
-                        unpack8(ql[2 * x + hh], b);
+                        float qa[8], qb[8];
+                        unpack8(qh[2 * x + hh], qa);
+                        unpack8(ql[2 * x + hh], qb);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) a[e] = a[e] + b[e] - vals[x][8 * hh + e];
-                        store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(64 + r, j0 + 8 * hh, 128), a);
+                        for (int e = 0; e < 8; ++e) qa[e] = qa[e] + qb[e] - vals[x][8 * hh + e];
+                        store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(64 + r, j0 + 16 * x + 8 * hh, 128),
+                                     qa);
                     }
-                }
+                if (bt == 0) load_qg(cg + 32);
             }
         }
     }
@@ -641,7 +674,10 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 // ============================================================================
 // tc_recur
 // ============================================================================
-constexpr int kRecurThreads = 128;
+// 256 threads: warp w reads TMEM lanes 32 (w % 4) .. + 31 and owns the state
+// columns [BV/2 (w / 4), BV/2 (w / 4 + 1)) of its rows, so both warp groups
+// share every per-chunk step of the chain.
+constexpr int kRecurThreads = 256;
 
 template <int BV>
 struct RecurLayout {
@@ -663,6 +699,8 @@ __global__ void __launch_bounds__(kRecurThreads, 1)
 tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, float* __restrict__ final_state,
          __nv_bfloat16* __restrict__ o, int* __restrict__ err, SeqMap smap, int H) {
     using Lay = RecurLayout<BV>;
+    constexpr int HB = BV / 2;          // state columns per thread
+    constexpr int NG = HB / 16;         // 16-column TMEM groups per thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBars);
@@ -677,7 +715,9 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     uint8_t* w_h = sm + Lay::kW;
     uint8_t* w_l = w_h + 8192;
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int sp = warp & 3;            // TMEM sub-partition: lanes 32 sp .. 32 sp + 31
+    const int cq = (warp >> 2) * HB;    // first state column of this thread (relative to j0)
     const SeqInfo sq = smap.get(blockIdx.x);
     const int h = blockIdx.y;
     const int j0 = blockIdx.z * BV;
@@ -730,13 +770,13 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         if (nch > 1) load_uu(1, 1);
     }
 
-    // this thread's state row c = tid, columns [j0, j0 + BV)
-    const int c = tid;
-    float s[BV];
+    // this thread's state row c, columns j0 + cq + [0, HB)
+    const int c = 32 * sp + lane;
+    float s[HB];
     {
-        const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0;
+        const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
-        for (int j = 0; j < BV; j += 4) {
+        for (int j = 0; j < HB; j += 4) {
             float4 x = init_state ? *reinterpret_cast<const float4*>(init_state + base + j)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
             s[j] = x.x; s[j + 1] = x.y; s[j + 2] = x.z; s[j + 3] = x.w;
@@ -748,7 +788,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         const uint8_t* uu = sm + Lay::kUU + stage * Lay::kUStage;
         // S_n as the MN-major B operand of MMA 1 (K = channel row c, N = columns)
 #pragma unroll
-        for (int j = 0; j < BV; j += 8) store8_split(s_h, s_l, mn_chunk(c, j, 128), s + j);
+        for (int j = 0; j < HB; j += 8) store8_split(s_h, s_l, mn_chunk(c, cq + j, 128), s + j);
         if (!mbar_wait(&uu_full[stage], (uint32_t)(n >> 1) & 1u)) {
             record_error(err, KDA_ERR_TIMEOUT);
             atomicExch(&sflags[1], 1u);
@@ -756,11 +796,11 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         // Diag(Gamma_C) S_n into TMEM; MMA 2 accumulates on top of it
         const float gam = reinterpret_cast<const float*>(uu + 2 * Lay::kUtile)[c];
 #pragma unroll
-        for (int jb = 0; jb < BV; jb += 16) {
+        for (int g = 0; g < NG; ++g) {
             float t[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) t[e] = gam * s[jb + e];
-            tmem_st16(tmem_addr(t_s, 32 * warp, jb), t);
+            for (int e = 0; e < 16; ++e) t[e] = gam * s[16 * g + e];
+            tmem_st16(tmem_addr(t_s, 32 * sp, cq + 16 * g), t);
         }
         tmem_st_wait();
         fence_async_smem();
@@ -785,26 +825,29 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         }
         tc_fence_after();
         if (tid == 0 && n + 1 < nch) load_wkq(n + 1);   // MMA 1 is done with the buffer
-        const int r = tid & 63;
-        const float* ut = reinterpret_cast<const float*>(uu + ((tid < 64) ? 0 : Lay::kUtile));
-        if (tid < 64) {
+        const int r = c & 63;
+        const float* ut = reinterpret_cast<const float*>(uu + ((sp < 2) ? 0 : Lay::kUtile));
+        float d[NG][16];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
+        tmem_ld_wait();
+        if (sp < 2) {
             // W = U - Wk S (rows are tokens) -> MN-major B operand of MMA 2
 #pragma unroll
-            for (int jb = 0; jb < BV; jb += 16) {
-                float d[16];
-                tmem_ld16(tmem_addr(t_d, 32 * warp, jb), d);
-                tmem_ld_wait();
+            for (int g = 0; g < NG; ++g) {
+                const int jb = cq + 16 * g;
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
                     const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
-                    d[e] = u.x - d[e]; d[e + 1] = u.y - d[e + 1]; d[e + 2] = u.z - d[e + 2]; d[e + 3] = u.w - d[e + 3];
+                    d[g][e] = u.x - d[g][e]; d[g][e + 1] = u.y - d[g][e + 1];
+                    d[g][e + 2] = u.z - d[g][e + 2]; d[g][e + 3] = u.w - d[g][e + 3];
                 }
-                store8_split(w_h, w_l, mn_chunk(r, jb, 64), d);
-                store8_split(w_h, w_l, mn_chunk(r, jb + 8, 64), d + 8);
+                store8_split(w_h, w_l, mn_chunk(r, jb, 64), d[g]);
+                store8_split(w_h, w_l, mn_chunk(r, jb + 8, 64), d[g] + 8);
             }
             fence_async_smem();
             tc_fence_before();
-            asm volatile("bar.sync 1, 64;" ::: "memory");   // warps 0-1 only: W is ready
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 0, 1, 4, 5: W is ready
             tc_fence_after();
             if (tid == 0) {
                 if (!mbar_wait(kdt_full, (uint32_t)n & 1u)) {
@@ -817,29 +860,24 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 }
                 mma_commit(bar2);
             }
-        } else {
+        } else if (r < min(kC, sq.len - n * kC)) {
             // O = Q' S + U' (rows are tokens), overlapping MMA 2
-            const int rows_here = min(kC, sq.len - n * kC);
+            __nv_bfloat16* dst = o + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + cq;
 #pragma unroll
-            for (int jb = 0; jb < BV; jb += 16) {
-                float d[16];
-                tmem_ld16(tmem_addr(t_d, 32 * warp, jb), d);
-                tmem_ld_wait();
-                if (r < rows_here) {
+            for (int g = 0; g < NG; ++g) {
+                const int jb = cq + 16 * g;
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4) {
-                        const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
-                        d[e] += u.x; d[e + 1] += u.y; d[e + 2] += u.z; d[e + 3] += u.w;
-                    }
-                    __nv_bfloat16* dst = o + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + jb;
-                    uint4 w0, w1;
-                    w0.x = pack_bf16(d[0], d[1]); w0.y = pack_bf16(d[2], d[3]);
-                    w0.z = pack_bf16(d[4], d[5]); w0.w = pack_bf16(d[6], d[7]);
-                    w1.x = pack_bf16(d[8], d[9]); w1.y = pack_bf16(d[10], d[11]);
-                    w1.z = pack_bf16(d[12], d[13]); w1.w = pack_bf16(d[14], d[15]);
-                    reinterpret_cast<uint4*>(dst)[0] = w0;
-                    reinterpret_cast<uint4*>(dst)[1] = w1;
+                for (int e = 0; e < 16; e += 4) {
+                    const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
+                    d[g][e] += u.x; d[g][e + 1] += u.y; d[g][e + 2] += u.z; d[g][e + 3] += u.w;
                 }
+                uint4 w0, w1;
+                w0.x = pack_bf16(d[g][0], d[g][1]); w0.y = pack_bf16(d[g][2], d[g][3]);
+                w0.z = pack_bf16(d[g][4], d[g][5]); w0.w = pack_bf16(d[g][6], d[g][7]);
+                w1.x = pack_bf16(d[g][8], d[g][9]); w1.y = pack_bf16(d[g][10], d[g][11]);
+                w1.z = pack_bf16(d[g][12], d[g][13]); w1.w = pack_bf16(d[g][14], d[g][15]);
+                reinterpret_cast<uint4*>(dst + 16 * g)[0] = w0;
+                reinterpret_cast<uint4*>(dst + 16 * g)[1] = w1;
             }
         }
         if (!mbar_wait(bar2, (uint32_t)n & 1u)) {
@@ -852,21 +890,23 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
             if (n + 1 < nch) load_kdt(n + 1);          // MMA 2 is done with the buffer
             if (n + 2 < nch) load_uu(n + 2, stage);
         }
+        {
+            float t[NG][16];
 #pragma unroll
-        for (int jb = 0; jb < BV; jb += 16) {
-            float t[16];
-            tmem_ld16(tmem_addr(t_s, 32 * warp, jb), t);
+            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_s, 32 * sp, cq + 16 * g), t[g]);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) s[jb + e] = t[e];
+            for (int g = 0; g < NG; ++g)
+#pragma unroll
+                for (int e = 0; e < 16; ++e) s[16 * g + e] = t[g][e];
         }
     }
     __syncthreads();
     const bool failed = sflags[1] != 0;
     if (!failed && final_state) {
-        const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0;
+        const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
-        for (int j = 0; j < BV; j += 4)
+        for (int j = 0; j < HB; j += 4)
             *reinterpret_cast<float4*>(final_state + base + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
     }
     if (failed && tid == 0) {
