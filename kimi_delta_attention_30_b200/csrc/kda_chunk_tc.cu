@@ -83,6 +83,7 @@ constexpr uint32_t kAKQh = 0;            // [K.E ; Q.E]  128 rows x 64 k
 constexpr uint32_t kAKQl = 16384;
 constexpr uint32_t kKFh = 32768;         // decayed key versions 160 rows x 64 k
 constexpr uint32_t kKFl = 53248;
+constexpr uint32_t kKdStage = 73728;     // Kd^T rows of one channel half, hi 8 KB + lo 8 KB (bulk-copied out)
 // after the first MMA
 constexpr uint32_t kAs = 0;              // A fp32 [64][65]
 constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
-         int H) {
+         int H, int ahead) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* tab = reinterpret_cast<float*>(sm + kTab);                 // [18][128]
@@ -191,7 +192,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         tmem_alloc(&sflags[2], 256);
         tmem_relinquish();
     }
-    if (tid < 64) sbeta[tid] = (tid < len) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+    const float beta_t = (tid < len && tid < 64) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
 
     // ---- log alpha of 8 rows x 4 channels; k, q, v prefetched into L2 ---------
     // (k and q of a channel half are read one phase before the round that uses
@@ -232,6 +233,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         }
     }
     load_kq(0);
+    if (tid < 64) sbeta[tid] = beta_t;
     // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
     for (int j = 1; j < 8; ++j)
@@ -322,8 +324,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             kd0[j] = k0 * f0 * y0;
             kd1[j] = k1 * f1 * y1;
         }
-        store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch, r0, 128), kd0);
-        store8_split(out + kOffKdTh, out + kOffKdTl, sw128_chunk(ch + 1, r0, 128), kd1);
+        // Kd^T rows ch, ch + 1 (this half's 64 rows are staged, then copied out whole)
+        store8_split(sm + kKdStage, sm + kKdStage + 8192, sw128_chunk(kc, r0, 64), kd0);
+        store8_split(sm + kKdStage, sm + kKdStage + 8192, sw128_chunk(kc + 1, r0, 64), kd1);
         if (hr == 0) load_kq(1);   // in flight during this round's MMA
         fence_async_smem();
         tc_fence_before();
@@ -333,11 +336,15 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             mma3(tbase, smem_u32(sm + kAKQh), smem_u32(sm + kAKQl), 128, smem_u32(sm + kKFh), smem_u32(sm + kKFl),
                  160, false, 4, idesc_bf16_f32(128, 160), hr > 0);
             mma_commit(&mbar);
+            bulk_s2g(out + kOffKdTh + 64 * hr * 128, sm + kKdStage, 8192);
+            bulk_s2g(out + kOffKdTl + 64 * hr * 128, sm + kKdStage + 8192, 8192);
+            bulk_commit();
         }
         if (!mbar_wait(&mbar, phase)) {
             record_error(err, KDA_ERR_TIMEOUT);
             atomicExch(&sflags[1], 1u);
         }
+        if (tid == 0) bulk_wait_read_all();   // the stage is rewritten next round (or by [T ; P T])
         phase ^= 1;
         tc_fence_after();
         __syncthreads();
@@ -607,25 +614,39 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     abort = abort || sflags[1] != 0;
 
+    // ---- inputs of the (chunk, head) that starts about one wave later into L2 ----------
+    // (`ahead` = co-resident CTAs; its loads then hit L2 instead of waiting on DRAM)
+    {
+        const int next = blockIdx.x + blockIdx.y * gridDim.x + ahead;
+        if (next < (int)(gridDim.x * gridDim.y)) {
+            const int nx = next % gridDim.x, ny = next / gridDim.x;
+            int nseq, ntok0, nlen, nidx;
+            cmap.locate(nx, nseq, ntok0, nlen, nidx);
+            const int row = tid & 63, which = tid >> 6;
+            if (row < nlen) {
+                const __nv_bfloat16* src = (which == 0) ? la : (which == 1) ? k : (which == 2) ? q : v;
+                const __nv_bfloat16* p = src + ((size_t)(ntok0 + row) * H + ny) * kD;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 64));
+            }
+        }
+    }
+
     // ---- epilogue: U, U' (fp32); Wk and Q' = Q exp(g) - P Wk (hi/lo images) ----------
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. row L of [U | Wk ; U' | P Wk];
-    // the two warp groups take 64 of the 128 columns of each part.
+    // the two warp groups take 64 of the 128 columns of each part.  Rows go to
+    // shared-memory copies of the workspace images (free after the last MMA) and
+    // leave in whole-line bulk copies: a row per thread written straight to
+    // global memory would put each warp store into 32 different lines.
     if (!abort) {
+        uint8_t* st_u = sm;                    // U | U' (64 KB, same bytes as the workspace)
+        uint8_t* st_h = sm + 65536;            // [Wk ; Q'] hi (32 KB)
+        uint8_t* st_l = sm;                    // [Wk ; Q'] lo (32 KB), after U | U' has left
         const int sp = warp & 3, L = 32 * sp + lane;
         const int r = L & 63;
         const bool qrow = L >= 64;              // warp-uniform (sub-partitions 2, 3)
         const int cg = (warp >> 2) * 64;
-        float* uo = reinterpret_cast<float*>(out + (qrow ? kOffU2 : kOffU));
-        uint4 qh[4], ql[4];
-        auto load_qg = [&](int j0) {            // Q exp(g) of columns [j0, j0 + 32)
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const uint32_t off = sw128_chunk(64 + r, j0 + 8 * x, 128);
-                qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
-                ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
-            }
-        };
-        if (qrow) load_qg(cg);
+        float* uo = reinterpret_cast<float*>(st_u + (qrow ? (kOffU2 - kOffU) : 0));
 #pragma unroll
         for (int bt = 0; bt < 2; ++bt) {
             const int j0 = cg + 32 * bt;
@@ -639,14 +660,37 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 for (int e = 0; e < 4; ++e)
                     *reinterpret_cast<float4*>(uo + u_index(r, j0 + 16 * x + 4 * e)) =
                         make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(out + kOffU, st_u, 65536);     // U and U' are adjacent in the workspace
+            bulk_commit();
+        }
+        uint4 qh[4], ql[4];
+        auto load_qg = [&](int j0) {            // Q exp(g) of columns [j0, j0 + 32), from the rounds
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const uint32_t off = sw128_chunk(64 + r, j0 + 8 * x, 128);
+                qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
+                ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
+            }
+        };
+        if (qrow) load_qg(cg);
+        if (tid == 0) bulk_wait_read_all();    // U | U' has left shared memory
+        __syncthreads();
+#pragma unroll
+        for (int bt = 0; bt < 2; ++bt) {
+            const int j0 = cg + 32 * bt;
+            float vals[2][16];
             tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0), vals[0]);
             tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0 + 16), vals[1]);
             tmem_ld_wait();
             if (!qrow) {
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 16 * x, 128), vals[x]);
-                    store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(r, j0 + 16 * x + 8, 128), vals[x] + 8);
+                    store8_split(st_h, st_l, sw128_chunk(r, j0 + 16 * x, 128), vals[x]);
+                    store8_split(st_h, st_l, sw128_chunk(r, j0 + 16 * x + 8, 128), vals[x] + 8);
                 }
             } else {
 #pragma unroll
@@ -658,11 +702,21 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                         unpack8(ql[2 * x + hh], qb);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) qa[e] = qa[e] + qb[e] - vals[x][8 * hh + e];
-                        store8_split(out + kOffWkQh, out + kOffWkQl, sw128_chunk(64 + r, j0 + 16 * x + 8 * hh, 128),
-                                     qa);
+                        store8_split(st_h, st_l, sw128_chunk(64 + r, j0 + 16 * x + 8 * hh, 128), qa);
                     }
                 if (bt == 0) load_qg(cg + 32);
             }
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            // the rows 64-127 being replaced were written (Q exp(g)) and read back
+            // through the generic proxy
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            bulk_s2g(out + kOffWkQh, st_h, 32768);
+            bulk_s2g(out + kOffWkQl, st_l, 32768);
+            bulk_commit();
+            bulk_wait_read_all();                // shared memory stays valid until read
         }
     }
     tc_fence_before();
@@ -932,6 +986,19 @@ cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* fina
     return cudaGetLastError();
 }
 
+// multiprocessors of the current device, looked up once per device
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 }  // namespace
 
 bool tc_available() { return true; }
@@ -957,14 +1024,14 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         tc_intra<<<dim3(n_chunks, H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 2 * sm_count());
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     timing_mark(stream, 1);
     if (n_seqs > 0) {
         const long units = (long)n_seqs * H;
-        if (units * 4 <= 148)
+        if (units * 4 <= sm_count())
             e = launch_recur<32>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream);
         else
             e = launch_recur<64>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream);
