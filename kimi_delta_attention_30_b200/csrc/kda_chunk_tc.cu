@@ -299,30 +299,37 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
         const int ch = 64 * hr + kc;
-        const float gref0 = gb[I * 128 + ch], gref1 = gb[I * 128 + ch + 1];
-        const float glast0 = gb[(I + 1) * 128 + ch], glast1 = gb[(I + 1) * 128 + ch + 1];
-        const float x0 = tab[tab_e0(I) * 128 + ch], x1 = tab[tab_e0(I) * 128 + ch + 1];
-        const float y0 = tab[tab_ec(I) * 128 + ch], y1 = tab[tab_ec(I) * 128 + ch + 1];
+        // e = exp(g - gb[I]), f = exp(gb[I+1] - g)
+        const float2 gref = make_float2(gb[I * 128 + ch], gb[I * 128 + ch + 1]);
+        const float2 glast = make_float2(gb[(I + 1) * 128 + ch], gb[(I + 1) * 128 + ch + 1]);
+        const float2 xq = make_float2(tab[tab_e0(I) * 128 + ch], tab[tab_e0(I) * 128 + ch + 1]);
+        const float2 yk = make_float2(tab[tab_ec(I) * 128 + ch], tab[tab_ec(I) * 128 + ch + 1]);
+        float2 sgv[4];
+#pragma unroll
+        for (int R = 0; R < 4; ++R) {
+            const float* sg = tab + ((R == I) ? tab_tau(R) : tab_sigma(R > I ? R : I + 1, I)) * 128 + ch;
+            sgv[R] = (R < I) ? make_float2(0.f, 0.f) : make_float2(sg[0], sg[1]);
+        }
         float kd0[8], kd1[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = r0 + j;
-            const float e0 = __expf(g[j][2 * hr] - gref0), e1 = __expf(g[j][2 * hr + 1] - gref1);
-            const float f0 = __expf(glast0 - g[j][2 * hr]), f1 = __expf(glast1 - g[j][2 * hr + 1]);
-            const float k0 = bf16_lo(kv[j]), k1 = bf16_hi(kv[j]);
-            const float q0 = bf16_lo(qv[j]), q1 = bf16_hi(qv[j]);
-            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, kc, 128), k0 * e0, k1 * e1);
-            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, kc, 128), q0 * e0, q1 * e1);
+            const float2 gj = make_float2(g[j][2 * hr], g[j][2 * hr + 1]);
+            const float2 e = exp_diff2(gj, gref), f = exp_diff2(glast, gj);
+            const float2 k2 = unpack_bf16x2(kv[j]), q2 = unpack_bf16x2(qv[j]);
+            const float2 ke = mul2(k2, e), qe = mul2(q2, e), kf = mul2(k2, f);
+            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, kc, 128), ke.x, ke.y);
+            store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, kc, 128), qe.x, qe.y);
 #pragma unroll
             for (int R = 0; R < 4; ++R) {
                 if (R < I) continue;
-                const float* sg = tab + ((R == I) ? tab_tau(R) : tab_sigma(R, I)) * 128 + ch;
-                store2_split(sm + kKFh, sm + kKFl, sw128_offset(kf_off(R) + r, kc, 160), k0 * f0 * sg[0],
-                             k1 * f1 * sg[1]);
+                const float2 kfs = mul2(kf, sgv[R]);
+                store2_split(sm + kKFh, sm + kKFl, sw128_offset(kf_off(R) + r, kc, 160), kfs.x, kfs.y);
             }
-            store2_split(out + kOffWkQh, out + kOffWkQl, sw128_offset(64 + r, ch, 128), q0 * e0 * x0, q1 * e1 * x1);
-            kd0[j] = k0 * f0 * y0;
-            kd1[j] = k1 * f1 * y1;
+            const float2 qg = mul2(qe, xq), kd = mul2(kf, yk);
+            store2_split(out + kOffWkQh, out + kOffWkQl, sw128_offset(64 + r, ch, 128), qg.x, qg.y);
+            kd0[j] = kd.x;
+            kd1[j] = kd.y;
         }
         // Kd^T rows ch, ch + 1 (this half's 64 rows are staged, then copied out whole)
         store8_split(sm + kKdStage, sm + kKdStage + 8192, sw128_chunk(kc, r0, 64), kd0);
@@ -478,29 +485,29 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             const int bi = e >> 6, rr = (e >> 2) & 15, i4 = (e & 3) * 4;
             const int R = bi + d, I2 = bi;
             if (e < nb * 64) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
                 for (int J = I2; J < R; ++J)
 #pragma unroll
                     for (int m = 0; m < 16; ++m) {
                         const float av = As[(16 * R + rr) * kAS + 16 * J + m];
                         const float4 tv = *reinterpret_cast<const float4*>(Ts + (16 * J + m) * kTS + 16 * I2 + i4);
-                        acc.x = fmaf(av, tv.x, acc.x); acc.y = fmaf(av, tv.y, acc.y);
-                        acc.z = fmaf(av, tv.z, acc.z); acc.w = fmaf(av, tv.w, acc.w);
+                        acc0 = fma2(make_float2(av, av), make_float2(tv.x, tv.y), acc0);
+                        acc1 = fma2(make_float2(av, av), make_float2(tv.z, tv.w), acc1);
                     }
-                *reinterpret_cast<float4*>(Y + (bi * 16 + rr) * kYS + i4) = acc;
+                *reinterpret_cast<float4*>(Y + (bi * 16 + rr) * kYS + i4) = make_float4(acc0.x, acc0.y, acc1.x, acc1.y);
             }
             __syncthreads();
             if (e < nb * 64) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int m = 0; m < 16; ++m) {
                     const float dv = Ts[(16 * R + rr) * kTS + 16 * R + m];
                     const float4 yv = *reinterpret_cast<const float4*>(Y + (bi * 16 + m) * kYS + i4);
-                    acc.x = fmaf(dv, yv.x, acc.x); acc.y = fmaf(dv, yv.y, acc.y);
-                    acc.z = fmaf(dv, yv.z, acc.z); acc.w = fmaf(dv, yv.w, acc.w);
+                    acc0 = fma2(make_float2(dv, dv), make_float2(yv.x, yv.y), acc0);
+                    acc1 = fma2(make_float2(dv, dv), make_float2(yv.z, yv.w), acc1);
                 }
                 *reinterpret_cast<float4*>(Ts + (16 * R + rr) * kTS + 16 * I2 + i4) =
-                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+                    make_float4(-acc0.x, -acc0.y, -acc1.x, -acc1.y);
             }
             __syncthreads();
         }
@@ -573,22 +580,22 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             }
         }
         // ---- [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns) ----------
-        float a[4] = {carry[0], carry[1], carry[2], carry[3]};
+        float2 a2[2] = {make_float2(carry[0], carry[1]), make_float2(carry[2], carry[3])};
+        const float2 zero2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = r0 + j;
-            const float b = sbeta[r];
+            const float2 b2 = make_float2(sbeta[r], sbeta[r]);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int ch = 64 * hh + kc;
-                if (r < len) {
-                    a[2 * hh] += fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor);
-                    a[2 * hh + 1] += fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor);
-                }
-                store2_split(sm + kXh, sm + kXl, mn_offset(r, ch, 64), b * bf16_lo(vv[j][hh]),
-                             b * bf16_hi(vv[j][hh]));
-                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), b * bf16_lo(kx[j][hh]) * __expf(a[2 * hh]),
-                             b * bf16_hi(kx[j][hh]) * __expf(a[2 * hh + 1]));
+                if (r < len)
+                    a2[hh] = __fadd2_rn(a2[hh], make_float2(fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor),
+                                                            fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor)));
+                const float2 vb = mul2(b2, unpack_bf16x2(vv[j][hh]));
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, ch, 64), vb.x, vb.y);
+                const float2 kb = mul2(mul2(b2, unpack_bf16x2(kx[j][hh])), exp_diff2(a2[hh], zero2));
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), kb.x, kb.y);
             }
         }
     }
@@ -701,7 +708,13 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                         unpack8(qh[2 * x + hh], qa);
                         unpack8(ql[2 * x + hh], qb);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) qa[e] = qa[e] + qb[e] - vals[x][8 * hh + e];
+                        for (int e = 0; e < 8; e += 2) {
+                            const float2 t = __fadd2_rn(make_float2(qa[e], qa[e + 1]), make_float2(qb[e], qb[e + 1]));
+                            const float2 d = fma2(make_float2(vals[x][8 * hh + e], vals[x][8 * hh + e + 1]),
+                                                  make_float2(-1.f, -1.f), t);
+                            qa[e] = d.x;
+                            qa[e + 1] = d.y;
+                        }
                         store8_split(st_h, st_l, sw128_chunk(64 + r, j0 + 16 * x + 8 * hh, 128), qa);
                     }
                 if (bt == 0) load_qg(cg + 32);

@@ -230,9 +230,32 @@ __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x 
 // hi + lo carries about 16 significant bits.  Products computed as
 // a_hi b_hi + a_hi b_lo + a_lo b_hi ("three-term bf16") keep a relative error
 // near 2^-16 while running on the bf16 tensor-core path.
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t x) { return make_float2(bf16_lo(x), bf16_hi(x)); }
+
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16(a, b);
-    lo = pack_bf16(a - bf16_lo(hi), b - bf16_hi(hi));
+    // x - hi is exact in fp32; one packed fma forms both differences
+    const float2 d = __ffma2_rn(unpack_bf16x2(hi), make_float2(-1.f, -1.f), make_float2(a, b));
+    lo = pack_bf16(d.x, d.y);
+}
+
+// Packed fp32 pair arithmetic (one instruction for both lanes of the pair).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// 2^x on the special-function unit (approximate, flushes subnormal results to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// exp(a - b) for a pair, as 2^((a - b) log2 e).  The difference is formed first
+// (exact when a and b are close, as cumulative decays within a block are), so
+// large |a|, |b| cost no accuracy.
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float2 exp_diff2(float2 a, float2 b) {
+    const float2 t = __fmul2_rn(__ffma2_rn(b, make_float2(-1.f, -1.f), a), make_float2(kLog2e, kLog2e));
+    return make_float2(ex2_approx(t.x), ex2_approx(t.y));
 }
 
 __device__ __forceinline__ void split1(float a, __nv_bfloat16& hi, __nv_bfloat16& lo) {
