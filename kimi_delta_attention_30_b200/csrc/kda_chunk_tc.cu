@@ -162,14 +162,15 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
-         int H, int ahead) {
+         int H) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* tab = reinterpret_cast<float*>(sm + kTab);                 // [18][128]
     float* gb = tab + kNumTab * 128;                                  // [5][128]
     float* sbeta = gb + 5 * 128;                                      // [64]
     uint32_t* sflags = reinterpret_cast<uint32_t*>(sbeta + 64);       // [0] fallback mask, [1] abort, [2] tmem base
-    __shared__ uint64_t mbar;
+    __shared__ uint64_t mbar;    // tensor-core products, in issue order
+    __shared__ uint64_t mbar_k;  // the second half of the last product
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this thread: rows [8 w, 8 w + 8) of 16-row block I = w / 2, and channels
@@ -186,6 +187,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         sflags[0] = 0;
         sflags[1] = 0;
         mbar_init(&mbar, 1);
+        mbar_init(&mbar_k, 1);
         mbar_init_fence();
     }
     if (warp == 0) {
@@ -580,22 +582,15 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             }
         }
         // ---- [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns) ----------
-        float2 a2[2] = {make_float2(carry[0], carry[1]), make_float2(carry[2], carry[3])};
-        const float2 zero2 = make_float2(0.f, 0.f);
+        // first beta V (columns 0-127), whose product starts while beta K exp(g) is built
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = r0 + j;
             const float2 b2 = make_float2(sbeta[r], sbeta[r]);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const int ch = 64 * hh + kc;
-                if (r < len)
-                    a2[hh] = __fadd2_rn(a2[hh], make_float2(fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor),
-                                                            fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor)));
                 const float2 vb = mul2(b2, unpack_bf16x2(vv[j][hh]));
-                store2_split(sm + kXh, sm + kXl, mn_offset(r, ch, 64), vb.x, vb.y);
-                const float2 kb = mul2(mul2(b2, unpack_bf16x2(kx[j][hh])), exp_diff2(a2[hh], zero2));
-                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + ch, 64), kb.x, kb.y);
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, 64 * hh + kc, 64), vb.x, vb.y);
             }
         }
     }
@@ -604,40 +599,48 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
 
-    // ---- [U | Wk ; U' | P Wk] = [T ; P T] [beta V | beta K exp(g)] --------------------
+    // ---- [U | Wk ; U' | P Wk] = [T ; P T] [beta V | beta K exp(g)], in two halves -----
+    const uint32_t tp_h = smem_u32(sm + kTPh), tp_l = smem_u32(sm + kTPl);
+    const uint32_t x_h = smem_u32(sm + kXh), x_l = smem_u32(sm + kXl);
     if (tid == 0 && !abort) {
-        const uint32_t ah = smem_u32(sm + kTPh), al = smem_u32(sm + kTPl);
-        const uint32_t bh = smem_u32(sm + kXh), bl = smem_u32(sm + kXl);
-        mma3(tmem_addr(tbase, 0, 0), ah, al, 128, bh, bl, 64, true, kC / 16, idesc_bf16_f32_bmn(128, 128), false);
-        mma3(tmem_addr(tbase, 0, 128), ah, al, 128, bh + 16384, bl + 16384, 64, true, kC / 16,
-             idesc_bf16_f32_bmn(128, 128), false);
+        mma3(tmem_addr(tbase, 0, 0), tp_h, tp_l, 128, x_h, x_l, 64, true, kC / 16, idesc_bf16_f32_bmn(128, 128),
+             false);
         mma_commit(&mbar);
     }
-    if (!abort && !mbar_wait(&mbar, phase)) {
+    if (!abort) {
+        float2 a2[2] = {make_float2(carry[0], carry[1]), make_float2(carry[2], carry[3])};
+        const float2 zero2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + j;
+            const float2 b2 = make_float2(sbeta[r], sbeta[r]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                if (r < len)
+                    a2[hh] = __fadd2_rn(a2[hh], make_float2(fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor),
+                                                            fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor)));
+                const float2 kb = mul2(mul2(b2, unpack_bf16x2(kx[j][hh])), exp_diff2(a2[hh], zero2));
+                store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + 64 * hh + kc, 64), kb.x, kb.y);
+            }
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0 && !abort) {
+        mma3(tmem_addr(tbase, 0, 128), tp_h, tp_l, 128, x_h + 16384, x_l + 16384, 64, true, kC / 16,
+             idesc_bf16_f32_bmn(128, 128), false);
+        mma_commit(&mbar_k);
+    }
+    // both halves: the epilogue reuses the operand space as its staging area
+    if (!abort && (!mbar_wait(&mbar, phase) || !mbar_wait(&mbar_k, 0))) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
     }
     tc_fence_after();
     __syncthreads();
     abort = abort || sflags[1] != 0;
-
-    // ---- inputs of the (chunk, head) that starts about one wave later into L2 ----------
-    // (`ahead` = co-resident CTAs; its loads then hit L2 instead of waiting on DRAM)
-    {
-        const int next = blockIdx.x + blockIdx.y * gridDim.x + ahead;
-        if (next < (int)(gridDim.x * gridDim.y)) {
-            const int nx = next % gridDim.x, ny = next / gridDim.x;
-            int nseq, ntok0, nlen, nidx;
-            cmap.locate(nx, nseq, ntok0, nlen, nidx);
-            const int row = tid & 63, which = tid >> 6;
-            if (row < nlen) {
-                const __nv_bfloat16* src = (which == 0) ? la : (which == 1) ? k : (which == 2) ? q : v;
-                const __nv_bfloat16* p = src + ((size_t)(ntok0 + row) * H + ny) * kD;
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 64));
-            }
-        }
-    }
 
     // ---- epilogue: U, U' (fp32); Wk and Q' = Q exp(g) - P Wk (hi/lo images) ----------
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. row L of [U | Wk ; U' | P Wk];
@@ -1037,7 +1040,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         tc_intra<<<dim3(n_chunks, H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 2 * sm_count());
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
