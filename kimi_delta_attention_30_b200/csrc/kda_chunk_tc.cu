@@ -651,7 +651,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     if (!abort) {
         uint8_t* st_u = sm;                    // U | U' (64 KB, same bytes as the workspace)
         uint8_t* st_h = sm + 65536;            // [Wk ; Q'] hi (32 KB)
-        uint8_t* st_l = sm;                    // [Wk ; Q'] lo (32 KB), after U | U' has left
+        uint8_t* st_l = sm;                    // [Wk ; Q'] lo (32 KB), once U has left
         const int sp = warp & 3, L = 32 * sp + lane;
         const int r = L & 63;
         const bool qrow = L >= 64;              // warp-uniform (sub-partitions 2, 3)
@@ -674,7 +674,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         fence_async_smem();
         __syncthreads();
         if (tid == 0) {
-            bulk_s2g(out + kOffU, st_u, 65536);     // U and U' are adjacent in the workspace
+            bulk_s2g(out + kOffU, st_u, 32768);     // U, then U', as separate groups
+            bulk_commit();
+            bulk_s2g(out + kOffU2, st_u + 32768, 32768);
             bulk_commit();
         }
         uint4 qh[4], ql[4];
@@ -687,7 +689,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             }
         };
         if (qrow) load_qg(cg);
-        if (tid == 0) bulk_wait_read_all();    // U | U' has left shared memory
+        if (tid == 0) bulk_wait_read_but1();   // U has left shared memory (U' may still be leaving)
         __syncthreads();
 #pragma unroll
         for (int bt = 0; bt < 2; ++bt) {
