@@ -19,6 +19,7 @@ Prints ONE JSON line on rank 0.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -137,6 +138,26 @@ def minimal_bytes(B, T, H, dk, dv, in_bytes=2, with_state=True):
     if with_state:
         b += 2 * B * H * dk * dv * 4
     return b
+
+
+def measured_traffic(kernel, B, T, H, C):
+    """DRAM bytes per launch of `kernel` on this workload from the committed ncu
+    table, or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(ROOT, "kimi_delta_attention_30_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("kda_chunk_tc.cu", "kda_tc.cuh", "kda_internal.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    want = f"prefill_b{B}_h{H}_t{T}_c{C}"
+    for line in open(path):
+        f = line.split()
+        if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] == want and f[4] == digest:
+            return int(f[2]) + int(f[3])
+    return None
 
 
 def peaks():
@@ -313,7 +334,8 @@ def main():
         if dom_bytes is not None:
             ach = dom_bytes / (k_avg[dom] / 1e3) / 1e9
             roofline = {"kernel": kernels[dom], "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": ach / pk["hbm_gbs"], "traffic": None, "algorithmic_bytes": dom_bytes,
+                        "frac": ach / pk["hbm_gbs"], "traffic": measured_traffic(kernels[dom], B, T, H, C),
+                        "algorithmic_bytes": dom_bytes,
                         "peak_source": pk["source"]}
         min_b = minimal_bytes(B, T, H, dk, dv)
         path_roofline = {"minimal_bytes": min_b, "time_min_us": min_b / (pk["hbm_gbs"] * 1e9) * 1e6,
