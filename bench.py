@@ -119,7 +119,9 @@ def kernel_bytes(name, B, T, H, dk, dv, C, in_bytes=2):
     n_chunks = B * ((T + C - 1) // C)
     st = B * H * dk * dv * 4
     schunk = n_chunks * H * dk * dv * 4
-    ws_tok = 5 * 4 * 128      # workspace per token-head of the tensor-core path: Wk, Q', Kd (hi+lo bf16), U, U' (fp32)
+    # workspace per token-head of the tensor-core path: Wk, Q exp(g), Kd (hi+lo bf16, 4 B per
+    # channel each), U (fp32), one row of P (hi+lo bf16, C entries)
+    ws_tok = 3 * 4 * dk + 4 * dv + 4 * C
     table = {
         "tc_intra": tok * ((3 * dk + dv) * in_bytes + in_bytes) + tok * ws_tok + n_chunks * H * dk * 4,
         "tc_recur": tok * ws_tok + n_chunks * H * dk * 4 + tok * dv * in_bytes + 2 * st,

@@ -7,26 +7,25 @@
 //     cumulative log decay g (row a1); on the tensor cores the decay-weighted
 //     strictly-lower A = Diag(beta) (K K^T . exp(g_r - g_i)) and the inclusive
 //     score matrix P = (Q K^T . exp(g_r - g_i)); T = (I + A)^{-1} by blocked
-//     substitution on CUDA cores; then on the tensor cores P T and
-//       [T ; P T] [beta V | beta K exp(g)] = [U | Wk ; U' | P Wk]          (row a2)
-//     i.e. U = T Diag(beta) V, Wk = T Diag(beta)(K . exp(g)), U' = P U and
-//     Q' = Q . exp(g) - P Wk, plus Kd = K . exp(g_C - g) and Gamma_C = exp(g_C).
-//     Results go to the workspace in the layout the second kernel consumes.
+//     substitution on CUDA cores; then on the tensor cores
+//       T [beta V | beta K exp(g)] = [U | Wk]                                  (row a2)
+//     i.e. U = T Diag(beta) V, Wk = T Diag(beta)(K . exp(g)), plus Q . exp(g),
+//     P, Kd = K . exp(g_C - g) and Gamma_C = exp(g_C).  Results go to the
+//     workspace in the layout the second kernel consumes.
 //
 //   tc_recur  (one CTA per (sequence, head, d_v tile), sequential over chunks)
 //     with the fp32 state tile S (d_k x BV) in TMEM:
-//       D   = [Wk ; Q'] S                         M = 128 MMA
+//       D   = [Wk ; Q . exp(g)] S                 M = 128 MMA
 //       W   = U - D[0:64]                         per-token corrections
-//       O   = D[64:128] + U'                      outputs (row a4)
 //       S  <- Diag(Gamma_C) S + Kd^T W            M = 128 MMA accumulating in TMEM (row a3)
+//       D  += [0 ; P] W,  O = D[64:128]           outputs (row a4), read during the next chunk
 //     The next chunk's operands stream in by 1-D bulk copies (TMA engine, no
 //     multicast) while the current chunk is processed.
 //
 // Derivation (ours; the oracle's chunk form checks it against the token
 // recurrence): with Gamma_r = exp(g_r) the per-token corrections W solve
 // (I + A) W = Diag(beta)(V - (K . Gamma) S_0), so W = U - Wk S_0; the outputs
-// are O = (Q . Gamma) S_0 + P W = Q' S_0 + U'; the next state is
-// Diag(Gamma_C) S_0 + Kd^T W.  Chunkwise form: "From GPT-2 to Kimi K3" essay
+// are O = (Q . Gamma) S_0 + P W; the next state is Diag(Gamma_C) S_0 + Kd^T W.  Chunkwise form: "From GPT-2 to Kimi K3" essay
 // (pwwt.cn/news/3716252), chunkwise and Gated DeltaNet paragraphs; WY / DPLR
 // restructuring: "我终于看懂了 KDA" explainer (pwwt.cn/news/3787313),
 // sections 16-17.
@@ -36,7 +35,7 @@
 // with fp32 accumulation: about 16 significant bits per operand.  Heavy decay
 // lets single tokens dominate many of the sums, so one bf16 rounding of an
 // operand would show up at ~2^-9 times the heavy tail of o; three terms keep
-// the path in the fp32 regime.  U and U' are stored in fp32.
+// the path in the fp32 regime.  U is stored in fp32.
 //
 // Decay factors.  Rows form 16-row blocks; gb[b] is g at the row before block
 // b (gb[0] = 0), gb[4] = g_C.  Every factor handed to the tensor cores is exp of
@@ -60,17 +59,18 @@ constexpr int kD = 128;
 constexpr float kDiagRange = 80.0f;
 
 // ---- workspace image of one (chunk, head) --------------------------------------
-constexpr uint32_t kOffWkQh = 0;         // [128 rows][128 k] bf16 SW128 K-major: rows 0-63 Wk, 64-127 Q' (hi)
+constexpr uint32_t kOffWkQh = 0;         // [128 rows][128 k] bf16 SW128 K-major: rows 0-63 Wk, 64-127 Q exp(g) (hi)
 constexpr uint32_t kOffWkQl = 32768;     // lo parts
 constexpr uint32_t kOffKdTh = 65536;     // [128 rows (channel)][64 k (token)] bf16 SW128 K-major (hi)
 constexpr uint32_t kOffKdTl = 81920;     // lo parts
 constexpr uint32_t kOffU = 98304;        // U : fp32, see u_index()
-constexpr uint32_t kOffU2 = 131072;      // U': same layout
-constexpr uint32_t kOffGam = 163840;     // Gamma_C fp32 [128]
-constexpr uint32_t kChunkBytes = 164352;
+constexpr uint32_t kOffPh = 131072;      // P [64 rows][64 k] bf16 SW128 K-major (hi)
+constexpr uint32_t kOffPl = 139264;      // lo parts
+constexpr uint32_t kOffGam = 147456;     // Gamma_C fp32 [128]
+constexpr uint32_t kChunkBytes = 147968;
 constexpr uint32_t kErrHeader = 256;     // first bytes of the TC scratch: error word
 
-// U / U' tiles: [4 column blocks of 32][64 rows][8 chunks of 4 floats], chunk
+// U tiles: [4 column blocks of 32][64 rows][8 chunks of 4 floats], chunk
 // permuted by row % 8 so that row-per-thread float4 reads hit distinct banks.
 __host__ __device__ __forceinline__ int u_index(int r, int j) {   // j % 4 == 0
     return (j >> 5) * 2048 + r * 32 + (((((j & 31) >> 2)) ^ (r & 7)) << 2);
@@ -90,7 +90,7 @@ constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
 constexpr uint32_t kPl = 25600;
 constexpr uint32_t kScr = 33792;         // 8 KB scratch
 constexpr uint32_t kTs = 41984;          // T fp32 [64][68]
-// [T ; P T] (128 rows x 64 k, K-major; rows 0-63 also serve as the MN-major T)
+// T (64 rows x 64 k, K-major), the A operand of the last product
 constexpr uint32_t kTPh = 65536;
 constexpr uint32_t kTPl = 81920;
 // [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns)
@@ -129,11 +129,6 @@ __device__ __forceinline__ void store8_split(uint8_t* hi_tile, uint8_t* lo_tile,
     split2(x[6], x[7], hv.w, lv.w);
     *reinterpret_cast<uint4*>(hi_tile + off) = hv;
     *reinterpret_cast<uint4*>(lo_tile + off) = lv;
-}
-
-__device__ __forceinline__ void unpack8(uint4 v, float* f) {
-    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
-    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
 }
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -456,6 +451,34 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         }
     }
 
+    // ---- P (hi/lo image, complete after the fallback) to the workspace ---------------
+    // The output's intra-chunk term P W is formed by the state carry, which knows W.
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0 && !abort) {
+        bulk_s2g(out + kOffPh, sm + kPh, 8192);
+        bulk_s2g(out + kOffPl, sm + kPl, 8192);
+        bulk_commit();
+    }
+    // v, k and log alpha for the [beta V | beta K exp(g)] operand are read again
+    // (from L2) while T is solved; g is rebuilt from the carries, so that no
+    // per-row state stays in registers through the middle of the kernel.
+    uint32_t vv[8][2], kx[8][2], lv[8][2];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int r = r0 + j;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            vv[j][hh] = kx[j][hh] = lv[j][hh] = 0u;
+            if (r < len && !abort) {
+                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
+                vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
+                kx[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
+                lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
+            }
+        }
+    }
+
     // ---- T = (I + A)^{-1}: diagonal 16 x 16 blocks, then by block distance -----------
     if (!abort) {
         if (warp < 4) {
@@ -513,7 +536,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             }
             __syncthreads();
         }
-        // T (hi/lo) into rows 0-63 of [T ; P T]; blocks above the diagonal are zero
+        // T (hi/lo) as a K-major tile; blocks above the diagonal are zero
         for (int e = tid; e < 64 * 8; e += kIntraThreads) {
             const int rr = e >> 3, k8 = (e & 7) * 8;
             float t8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -531,56 +554,10 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
 
-    // ---- P T  (M = 64; B = T read as an MN-major 64 x 64 tile) -----------------------
-    // v, k and log alpha for the [beta V | beta K exp(g)] operand are read again
-    // (from L2) while this product runs; g is rebuilt from the carries, so that no
-    // per-row state stays in registers through the middle of the kernel.
-    uint32_t vv[8][2], kx[8][2], lv[8][2];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const int r = r0 + j;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            vv[j][hh] = kx[j][hh] = lv[j][hh] = 0u;
-            if (r < len && !abort) {
-                const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
-                vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
-                kx[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
-                lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
-            }
-        }
-    }
-    if (tid == 0 && !abort) {
-        mma3(tmem_addr(tbase, 0, 0), smem_u32(sm + kPh), smem_u32(sm + kPl), 64, smem_u32(sm + kTPh),
-             smem_u32(sm + kTPl), 64, true, kC / 16, idesc_bf16_f32_bmn(64, 64), false);
-        mma_commit(&mbar);
-    }
-    if (!abort && !mbar_wait(&mbar, phase)) {
-        record_error(err, KDA_ERR_TIMEOUT);
-        atomicExch(&sflags[1], 1u);
-    }
-    phase ^= 1;
-    tc_fence_after();
+    if (tid == 0) bulk_wait_read_all();   // P has left shared memory (the operand below overwrites it)
     __syncthreads();
-    abort = abort || sflags[1] != 0;
 
     if (!abort) {
-        // ---- P T (hi/lo) into rows 64-127 of [T ; P T] --------------------------------
-        {
-            const int sp = warp & 3;
-            const int r = 16 * sp + (lane & 15);
-            const int cb = (warp < 4) ? 0 : 32;
-#pragma unroll
-            for (int gi = 0; gi < 2; ++gi) {
-                float vals[16];
-                tmem_ld16(tmem_addr(tbase, 32 * sp, cb + 16 * gi), vals);
-                tmem_ld_wait();
-                if (lane < 16) {
-                    store8_split(sm + kTPh, sm + kTPl, sw128_chunk(64 + r, cb + 16 * gi, 128), vals);
-                    store8_split(sm + kTPh, sm + kTPl, sw128_chunk(64 + r, cb + 16 * gi + 8, 128), vals + 8);
-                }
-            }
-        }
         // ---- [beta V | beta K exp(g)] (MN-major, 64 token rows x 256 columns) ----------
         // first beta V (columns 0-127), whose product starts while beta K exp(g) is built
 #pragma unroll
@@ -599,11 +576,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
 
-    // ---- [U | Wk ; U' | P Wk] = [T ; P T] [beta V | beta K exp(g)], in two halves -----
+    // ---- [U | Wk] = T [beta V | beta K exp(g)]  (M = 64), in two halves -----------------
     const uint32_t tp_h = smem_u32(sm + kTPh), tp_l = smem_u32(sm + kTPl);
     const uint32_t x_h = smem_u32(sm + kXh), x_l = smem_u32(sm + kXl);
     if (tid == 0 && !abort) {
-        mma3(tmem_addr(tbase, 0, 0), tp_h, tp_l, 128, x_h, x_l, 64, true, kC / 16, idesc_bf16_f32_bmn(128, 128),
+        mma3(tmem_addr(tbase, 0, 0), tp_h, tp_l, 64, x_h, x_l, 64, true, kC / 16, idesc_bf16_f32_bmn(64, 128),
              false);
         mma_commit(&mbar);
     }
@@ -629,8 +606,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     tc_fence_after();
     if (tid == 0 && !abort) {
-        mma3(tmem_addr(tbase, 0, 128), tp_h, tp_l, 128, x_h + 16384, x_l + 16384, 64, true, kC / 16,
-             idesc_bf16_f32_bmn(128, 128), false);
+        mma3(tmem_addr(tbase, 0, 128), tp_h, tp_l, 64, x_h + 16384, x_l + 16384, 64, true, kC / 16,
+             idesc_bf16_f32_bmn(64, 128), false);
         mma_commit(&mbar_k);
     }
     // both halves: the epilogue reuses the operand space as its staging area
@@ -642,21 +619,21 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     abort = abort || sflags[1] != 0;
 
-    // ---- epilogue: U, U' (fp32); Wk and Q' = Q exp(g) - P Wk (hi/lo images) ----------
-    // Warp w reads TMEM lanes 32 (w % 4) .. + 31, i.e. row L of [U | Wk ; U' | P Wk];
-    // the two warp groups take 64 of the 128 columns of each part.  Rows go to
+    // ---- epilogue: U (fp32) and Wk (hi/lo) ----------------------------------------------
+    // M = 64 results: row r sits in TMEM lane 32 (r / 16) + r % 16, so warp w
+    // (sub-partition w % 4) holds rows 16 (w % 4) .. + 15 in its lanes 0-15; the two
+    // warp groups take 64 of the 128 columns of each part.  Rows go to
     // shared-memory copies of the workspace images (free after the last MMA) and
-    // leave in whole-line bulk copies: a row per thread written straight to
-    // global memory would put each warp store into 32 different lines.
+    // leave in whole bulk copies: a row per thread written straight to global
+    // memory would put each warp store into 16 different lines.
     if (!abort) {
-        uint8_t* st_u = sm;                    // U | U' (64 KB, same bytes as the workspace)
-        uint8_t* st_h = sm + 65536;            // [Wk ; Q'] hi (32 KB)
-        uint8_t* st_l = sm;                    // [Wk ; Q'] lo (32 KB), once U has left
-        const int sp = warp & 3, L = 32 * sp + lane;
-        const int r = L & 63;
-        const bool qrow = L >= 64;              // warp-uniform (sub-partitions 2, 3)
+        uint8_t* st_u = sm;                    // U (32 KB, same bytes as the workspace)
+        uint8_t* st_w = sm + 32768;            // Wk hi, K blocks 0 and 1 (8 KB each), then lo
+        const int sp = warp & 3;
+        const int r = 16 * sp + (lane & 15);
+        const bool row_lane = lane < 16;
         const int cg = (warp >> 2) * 64;
-        float* uo = reinterpret_cast<float*>(st_u + (qrow ? (kOffU2 - kOffU) : 0));
+        float* uo = reinterpret_cast<float*>(st_u);
 #pragma unroll
         for (int bt = 0; bt < 2; ++bt) {
             const int j0 = cg + 32 * bt;
@@ -664,75 +641,36 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             tmem_ld16(tmem_addr(tbase, 32 * sp, j0), vals[0]);
             tmem_ld16(tmem_addr(tbase, 32 * sp, j0 + 16), vals[1]);
             tmem_ld_wait();
-#pragma unroll
-            for (int x = 0; x < 2; ++x)
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    *reinterpret_cast<float4*>(uo + u_index(r, j0 + 16 * x + 4 * e)) =
-                        make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
-        }
-        fence_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(out + kOffU, st_u, 32768);     // U, then U', as separate groups
-            bulk_commit();
-            bulk_s2g(out + kOffU2, st_u + 32768, 32768);
-            bulk_commit();
-        }
-        uint4 qh[4], ql[4];
-        auto load_qg = [&](int j0) {            // Q exp(g) of columns [j0, j0 + 32), from the rounds
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const uint32_t off = sw128_chunk(64 + r, j0 + 8 * x, 128);
-                qh[x] = *reinterpret_cast<const uint4*>(out + kOffWkQh + off);
-                ql[x] = *reinterpret_cast<const uint4*>(out + kOffWkQl + off);
-            }
-        };
-        if (qrow) load_qg(cg);
-        if (tid == 0) bulk_wait_read_but1();   // U has left shared memory (U' may still be leaving)
-        __syncthreads();
-#pragma unroll
-        for (int bt = 0; bt < 2; ++bt) {
-            const int j0 = cg + 32 * bt;
-            float vals[2][16];
-            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0), vals[0]);
-            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0 + 16), vals[1]);
-            tmem_ld_wait();
-            if (!qrow) {
-#pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    store8_split(st_h, st_l, sw128_chunk(r, j0 + 16 * x, 128), vals[x]);
-                    store8_split(st_h, st_l, sw128_chunk(r, j0 + 16 * x + 8, 128), vals[x] + 8);
-                }
-            } else {
+            if (row_lane) {
 #pragma unroll
                 for (int x = 0; x < 2; ++x)
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float qa[8], qb[8];
-                        unpack8(qh[2 * x + hh], qa);
-                        unpack8(ql[2 * x + hh], qb);
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<float4*>(uo + u_index(r, j0 + 16 * x + 4 * e)) =
+                            make_float4(vals[x][4 * e], vals[x][4 * e + 1], vals[x][4 * e + 2], vals[x][4 * e + 3]);
+            }
+            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0), vals[0]);
+            tmem_ld16(tmem_addr(tbase, 32 * sp, 128 + j0 + 16), vals[1]);
+            tmem_ld_wait();
+            if (row_lane) {
+                uint8_t* wh = st_w + (j0 >> 6) * 8192;
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2) {
-                            const float2 t = __fadd2_rn(make_float2(qa[e], qa[e + 1]), make_float2(qb[e], qb[e + 1]));
-                            const float2 d = fma2(make_float2(vals[x][8 * hh + e], vals[x][8 * hh + e + 1]),
-                                                  make_float2(-1.f, -1.f), t);
-                            qa[e] = d.x;
-                            qa[e + 1] = d.y;
-                        }
-                        store8_split(st_h, st_l, sw128_chunk(64 + r, j0 + 16 * x + 8 * hh, 128), qa);
-                    }
-                if (bt == 0) load_qg(cg + 32);
+                for (int x = 0; x < 2; ++x) {
+                    const int kk = (j0 & 63) + 16 * x;
+                    store8_split(wh, wh + 16384, sw128_chunk(r, kk, 64), vals[x]);
+                    store8_split(wh, wh + 16384, sw128_chunk(r, kk + 8, 64), vals[x] + 8);
+                }
             }
         }
         fence_async_smem();
         __syncthreads();
         if (tid == 0) {
-            // the rows 64-127 being replaced were written (Q exp(g)) and read back
-            // through the generic proxy
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            bulk_s2g(out + kOffWkQh, st_h, 32768);
-            bulk_s2g(out + kOffWkQl, st_l, 32768);
+            bulk_s2g(out + kOffU, st_u, 32768);
+            // rows 0-63 of each 64-wide K block of the [Wk ; Q exp(g)] hi and lo images
+            bulk_s2g(out + kOffWkQh, st_w, 8192);
+            bulk_s2g(out + kOffWkQh + 16384, st_w + 8192, 8192);
+            bulk_s2g(out + kOffWkQl, st_w + 16384, 8192);
+            bulk_s2g(out + kOffWkQl + 16384, st_w + 24576, 8192);
             bulk_commit();
             bulk_wait_read_all();                // shared memory stays valid until read
         }
@@ -747,23 +685,28 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 // tc_recur
 // ============================================================================
 // 256 threads: warp w reads TMEM lanes 32 (w % 4) .. + 31 and owns the state
-// columns [BV/2 (w / 4), BV/2 (w / 4 + 1)) of its rows, so both warp groups
-// share every per-chunk step of the chain.
+// columns [BV/2 (w / 4), BV/2 (w / 4 + 1)) of its rows.  Warps with w % 4 < 2
+// form W (rows 0-63 of D); the others finish the outputs.  The output product
+// [0 ; P] W of chunk n is issued (by thread 64, after thread 0 has issued chunk
+// n + 1's first product) into chunk n's D buffer, and runs on the tensor core
+// while the CUDA cores form chunk n + 1's W: D and W alternate between two
+// buffers, so nothing on the chain waits for it.
 constexpr int kRecurThreads = 256;
 
 template <int BV>
 struct RecurLayout {
     static constexpr uint32_t kWkQ = 0;                                        // hi 32 KB + lo 32 KB
     static constexpr uint32_t kKdT = 65536;                                    // hi 16 KB + lo 16 KB
-    static constexpr uint32_t kUtile = (uint32_t)BV * 64 * 4;                  // U (or U') tile, fp32
-    static constexpr uint32_t kUStage = 2 * kUtile + 512;                      // U, U', Gamma_C
+    static constexpr uint32_t kUtile = (uint32_t)BV * 64 * 4;                  // U tile, fp32
+    static constexpr uint32_t kUStage = kUtile + 512;                          // U, Gamma_C
     static constexpr uint32_t kUU = 98304;                                     // two U stages
-    static constexpr uint32_t kS = (kUU + 2 * kUStage + 1023) / 1024 * 1024;  // S hi/lo: 128 rows x 128 B (MN-major)
-    static constexpr uint32_t kW = kS + 2 * 16384;                             // W hi/lo: 64 rows x 128 B (MN-major)
-    static constexpr uint32_t kBars = kW + 2 * 8192;
+    static constexpr uint32_t kP = (kUU + 2 * kUStage + 1023) / 1024 * 1024;  // [0 ; P] hi 16 KB + lo 16 KB
+    static constexpr uint32_t kS = kP + 2 * 16384;                             // S hi/lo: 128 rows x 128 B (MN-major)
+    static constexpr uint32_t kW = kS + 2 * 16384;                             // W hi/lo: 64 rows x 128 B (MN-major), x2
+    static constexpr uint32_t kBars = kW + 2 * 2 * 8192;
     static constexpr uint32_t kSmem = kBars + 128;
     static constexpr uint32_t kAlloc = kSmem + 1024;
-    static constexpr uint32_t kTmemCols = (2 * BV < 32) ? 32 : 2 * BV;
+    static constexpr uint32_t kTmemCols = (3 * BV <= 32) ? 32 : (3 * BV <= 64) ? 64 : (3 * BV <= 128) ? 128 : 256;
 };
 
 template <int BV>
@@ -779,13 +722,15 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     uint64_t* wkq_full = bars + 0;
     uint64_t* kdt_full = bars + 1;
     uint64_t* uu_full = bars + 2;     // [2]
-    uint64_t* bar1 = bars + 4;
-    uint64_t* bar2 = bars + 5;
-    uint32_t* sflags = reinterpret_cast<uint32_t*>(bars + 6);        // [0] tmem base, [1] abort
+    uint64_t* bar_d = bars + 4;       // D = [Wk ; Q exp(g)] S done
+    uint64_t* bar_s = bars + 5;       // S update done
+    uint64_t* bar_o = bars + 6;       // D += [0 ; P] W done (outputs ready)
+    uint64_t* p_full = bars + 7;      // P landed
+    uint64_t* d_issued = bars + 8;    // the chunk's first product has been issued
+    uint32_t* sflags = reinterpret_cast<uint32_t*>(bars + 9);        // [0] tmem base, [1] abort
     uint8_t* s_h = sm + Lay::kS;
     uint8_t* s_l = s_h + 16384;
-    uint8_t* w_h = sm + Lay::kW;
-    uint8_t* w_l = w_h + 8192;
+    auto w_hi = [&](int n) { return sm + Lay::kW + (n & 1) * 16384; };   // lo parts 8 KB further
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3;            // TMEM sub-partition: lanes 32 sp .. 32 sp + 31
@@ -794,10 +739,10 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     const int h = blockIdx.y;
     const int j0 = blockIdx.z * BV;
     const int nch = (sq.len + kC - 1) / kC;
-    const int cb0 = j0 / 32;   // first 32-column block of U / U'
+    const int cb0 = j0 / 32;   // first 32-column block of U
 
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
         sflags[1] = 0;
         mbar_init_fence();
     }
@@ -805,12 +750,17 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         tmem_alloc(&sflags[0], Lay::kTmemCols);
         tmem_relinquish();
     }
+    // rows 0-63 of the [0 ; P] operand are zero (hi and lo)
+    for (int i = tid; i < 1024; i += kRecurThreads) {
+        const int img = i >> 9, off = (i & 511) * 16;
+        *reinterpret_cast<uint4*>(sm + Lay::kP + img * 16384 + off) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sflags[0];
-    const uint32_t t_d = tbase;              // D = [Wk ; Q'] S   (columns [0, BV))
-    const uint32_t t_s = tbase + BV;         // S                 (columns [BV, 2 BV))
+    const uint32_t t_s = tbase + 2 * BV;     // S (columns [2 BV, 3 BV)); D of chunk n: columns [BV (n % 2), + BV)
 
     auto chunk_src = [&](int n) {
         return ws + (size_t)((size_t)(sq.chunk0 + n) * H + h) * kChunkBytes;
@@ -832,13 +782,23 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         uint8_t* dst = sm + Lay::kUU + stage * Lay::kUStage;
         mbar_arrive_expect_tx(&uu_full[stage], Lay::kUStage);
         bulk_g2s(dst, src + kOffU + cb0 * 8192, Lay::kUtile, &uu_full[stage]);
-        bulk_g2s(dst + Lay::kUtile, src + kOffU2 + cb0 * 8192, Lay::kUtile, &uu_full[stage]);
-        bulk_g2s(dst + 2 * Lay::kUtile, src + kOffGam, 512, &uu_full[stage]);
+        bulk_g2s(dst + Lay::kUtile, src + kOffGam, 512, &uu_full[stage]);
+    };
+    auto load_p = [&](int n) {   // P into rows 64-127 of the [0 ; P] hi and lo tiles
+        const uint8_t* src = chunk_src(n);
+        mbar_arrive_expect_tx(p_full, 16384);
+        bulk_g2s(sm + Lay::kP + 8192, src + kOffPh, 8192, p_full);
+        bulk_g2s(sm + Lay::kP + 16384 + 8192, src + kOffPl, 8192, p_full);
+    };
+    auto fail = [&]() {
+        record_error(err, KDA_ERR_TIMEOUT);
+        atomicExch(&sflags[1], 1u);
     };
     if (tid == 0 && nch > 0) {
         load_wkq(0);
         load_kdt(0);
         load_uu(0, 0);
+        load_p(0);
         if (nch > 1) load_uu(1, 1);
     }
 
@@ -855,18 +815,53 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         }
     }
 
-    for (int n = 0; n < nch; ++n) {
+    // D(m) += [0 ; P] W(m): the output product of chunk m (thread 64)
+    auto issue_o = [&](int m) {
+        if (!mbar_wait(p_full, (uint32_t)m & 1u)) {
+            fail();
+        } else {
+            const uint32_t a = smem_u32(sm + Lay::kP);
+            const uint32_t wh = smem_u32(w_hi(m));
+            mma3(tbase + (uint32_t)(BV * (m & 1)), a, a + 16384, 128, wh, wh + 8192, 64, true, kC / 16,
+                 idesc_bf16_f32_bmn(128, BV), true);
+        }
+        mma_commit(bar_o);
+    };
+    // O rows of chunk m out of D (warps with sp >= 2: rows 64-127 = token rows 0-63)
+    auto emit_o = [&](int m) {
+        const uint32_t t_d = tbase + (uint32_t)(BV * (m & 1));
+        float d[NG][16];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
+        tmem_ld_wait();
+        const int r = c - 64;
+        if (r < min(kC, sq.len - m * kC)) {
+            __nv_bfloat16* dst = o + ((size_t)(sq.tok0 + m * kC + r) * H + h) * kD + j0 + cq;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                uint4 w0, w1;
+                w0.x = pack_bf16(d[g][0], d[g][1]); w0.y = pack_bf16(d[g][2], d[g][3]);
+                w0.z = pack_bf16(d[g][4], d[g][5]); w0.w = pack_bf16(d[g][6], d[g][7]);
+                w1.x = pack_bf16(d[g][8], d[g][9]); w1.y = pack_bf16(d[g][10], d[g][11]);
+                w1.z = pack_bf16(d[g][12], d[g][13]); w1.w = pack_bf16(d[g][14], d[g][15]);
+                reinterpret_cast<uint4*>(dst + 16 * g)[0] = w0;
+                reinterpret_cast<uint4*>(dst + 16 * g)[1] = w1;
+            }
+        }
+    };
+
+    int n = 0;
+    for (; n < nch; ++n) {
         const int stage = n & 1;
         const uint8_t* uu = sm + Lay::kUU + stage * Lay::kUStage;
-        // S_n as the MN-major B operand of MMA 1 (K = channel row c, N = columns)
+        const uint32_t par = (uint32_t)n & 1u;
+        const uint32_t t_d = tbase + (uint32_t)(BV * (n & 1));
+        // S_n as the MN-major B operand (K = channel row c, N = columns)
 #pragma unroll
         for (int j = 0; j < HB; j += 8) store8_split(s_h, s_l, mn_chunk(c, cq + j, 128), s + j);
-        if (!mbar_wait(&uu_full[stage], (uint32_t)(n >> 1) & 1u)) {
-            record_error(err, KDA_ERR_TIMEOUT);
-            atomicExch(&sflags[1], 1u);
-        }
-        // Diag(Gamma_C) S_n into TMEM; MMA 2 accumulates on top of it
-        const float gam = reinterpret_cast<const float*>(uu + 2 * Lay::kUtile)[c];
+        if (!mbar_wait(&uu_full[stage], (uint32_t)(n >> 1) & 1u)) fail();
+        // Diag(Gamma_C) S_n into TMEM; the S update accumulates on top of it
+        const float gam = reinterpret_cast<const float*>(uu + Lay::kUtile)[c];
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             float t[16];
@@ -881,30 +876,28 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         if (sflags[1]) break;
         tc_fence_after();
         if (tid == 0) {
-            if (!mbar_wait(wkq_full, (uint32_t)n & 1u)) {
-                record_error(err, KDA_ERR_TIMEOUT);
-                atomicExch(&sflags[1], 1u);
+            if (!mbar_wait(wkq_full, par)) {
+                fail();
             } else {
                 const uint32_t a = smem_u32(sm + Lay::kWkQ);
                 mma3(t_d, a, a + 32768, 128, smem_u32(s_h), smem_u32(s_l), 128, true, kD / 16,
                      idesc_bf16_f32_bmn(128, BV), false);
             }
-            mma_commit(bar1);
+            mma_commit(bar_d);
+            mbar_arrive(d_issued);   // the previous chunk's output product may follow it
         }
-        if (!mbar_wait(bar1, (uint32_t)n & 1u)) {
-            record_error(err, KDA_ERR_TIMEOUT);
-            atomicExch(&sflags[1], 1u);
-        }
+        if (!mbar_wait(bar_d, par)) fail();
         tc_fence_after();
-        if (tid == 0 && n + 1 < nch) load_wkq(n + 1);   // MMA 1 is done with the buffer
-        const int r = c & 63;
-        const float* ut = reinterpret_cast<const float*>(uu + ((sp < 2) ? 0 : Lay::kUtile));
-        float d[NG][16];
-#pragma unroll
-        for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
-        tmem_ld_wait();
+        if (tid == 0 && n + 1 < nch) load_wkq(n + 1);   // the product is done with the buffer
         if (sp < 2) {
-            // W = U - Wk S (rows are tokens) -> MN-major B operand of MMA 2
+            // W = U - Wk S (rows are tokens) -> MN-major B operand of the S update and of [0 ; P] W
+            const int r = c;
+            const float* ut = reinterpret_cast<const float*>(uu);
+            uint8_t* w_h = w_hi(n);
+            float d[NG][16];
+#pragma unroll
+            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
+            tmem_ld_wait();
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
                 const int jb = cq + 16 * g;
@@ -914,52 +907,43 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                     d[g][e] = u.x - d[g][e]; d[g][e + 1] = u.y - d[g][e + 1];
                     d[g][e + 2] = u.z - d[g][e + 2]; d[g][e + 3] = u.w - d[g][e + 3];
                 }
-                store8_split(w_h, w_l, mn_chunk(r, jb, 64), d[g]);
-                store8_split(w_h, w_l, mn_chunk(r, jb + 8, 64), d[g] + 8);
+                store8_split(w_h, w_h + 8192, mn_chunk(r, jb, 64), d[g]);
+                store8_split(w_h, w_h + 8192, mn_chunk(r, jb + 8, 64), d[g] + 8);
             }
             fence_async_smem();
             tc_fence_before();
             asm volatile("bar.sync 1, 128;" ::: "memory");   // warps 0, 1, 4, 5: W is ready
             tc_fence_after();
             if (tid == 0) {
-                if (!mbar_wait(kdt_full, (uint32_t)n & 1u)) {
-                    record_error(err, KDA_ERR_TIMEOUT);
-                    atomicExch(&sflags[1], 1u);
+                if (!mbar_wait(kdt_full, par)) {
+                    fail();
                 } else {
                     const uint32_t a = smem_u32(sm + Lay::kKdT);
-                    mma3(t_s, a, a + 16384, 128, smem_u32(w_h), smem_u32(w_l), 64, true, kC / 16,
+                    mma3(t_s, a, a + 16384, 128, smem_u32(w_h), smem_u32(w_h) + 8192, 64, true, kC / 16,
                          idesc_bf16_f32_bmn(128, BV), true);
                 }
-                mma_commit(bar2);
+                mma_commit(bar_s);
             }
-        } else if (r < min(kC, sq.len - n * kC)) {
-            // O = Q' S + U' (rows are tokens), overlapping MMA 2
-            __nv_bfloat16* dst = o + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + cq;
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-                const int jb = cq + 16 * g;
-#pragma unroll
-                for (int e = 0; e < 16; e += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
-                    d[g][e] += u.x; d[g][e + 1] += u.y; d[g][e + 2] += u.z; d[g][e + 3] += u.w;
-                }
-                uint4 w0, w1;
-                w0.x = pack_bf16(d[g][0], d[g][1]); w0.y = pack_bf16(d[g][2], d[g][3]);
-                w0.z = pack_bf16(d[g][4], d[g][5]); w0.w = pack_bf16(d[g][6], d[g][7]);
-                w1.x = pack_bf16(d[g][8], d[g][9]); w1.y = pack_bf16(d[g][10], d[g][11]);
-                w1.z = pack_bf16(d[g][12], d[g][13]); w1.w = pack_bf16(d[g][14], d[g][15]);
-                reinterpret_cast<uint4*>(dst + 16 * g)[0] = w0;
-                reinterpret_cast<uint4*>(dst + 16 * g)[1] = w1;
+        } else if (n > 0) {
+            // outputs of the previous chunk: its product goes in behind this chunk's
+            // first one and runs while W is formed; then its P tile may be replaced
+            if (tid == 64) {
+                if (!mbar_wait(d_issued, par)) fail();
+                issue_o(n - 1);
             }
+            if (!mbar_wait(bar_o, par ^ 1u)) {
+                fail();
+            } else if (tid == 64) {
+                load_p(n);
+            }
+            tc_fence_after();
+            emit_o(n - 1);
         }
-        if (!mbar_wait(bar2, (uint32_t)n & 1u)) {
-            record_error(err, KDA_ERR_TIMEOUT);
-            atomicExch(&sflags[1], 1u);
-        }
+        if (!mbar_wait(bar_s, par)) fail();
         tc_fence_after();
-        __syncthreads();   // every thread is past its reads of this chunk's U / U' stage
+        __syncthreads();   // every thread is past its reads of this chunk's U stage
         if (tid == 0) {
-            if (n + 1 < nch) load_kdt(n + 1);          // MMA 2 is done with the buffer
+            if (n + 1 < nch) load_kdt(n + 1);          // the S update is done with Kd^T
             if (n + 2 < nch) load_uu(n + 2, stage);
         }
         {
@@ -975,13 +959,21 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     }
     __syncthreads();
     const bool failed = sflags[1] != 0;
+    if (!failed && nch > 0 && sp >= 2) {
+        // outputs of the last chunk
+        if (tid == 64) issue_o(nch - 1);
+        if (!mbar_wait(bar_o, (uint32_t)(nch - 1) & 1u)) fail();
+        tc_fence_after();
+        emit_o(nch - 1);
+    }
     if (!failed && final_state) {
         const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
         for (int j = 0; j < HB; j += 4)
             *reinterpret_cast<float4*>(final_state + base + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
     }
-    if (failed && tid == 0) {
+    __syncthreads();
+    if (sflags[1] && tid == 0) {
         // a wait gave up: give in-flight copies and MMAs a bounded time to land before freeing TMEM
         const uint64_t t0 = globaltimer_ns();
         while (globaltimer_ns() - t0 < 100000000ull) {
