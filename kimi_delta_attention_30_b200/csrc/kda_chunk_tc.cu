@@ -84,6 +84,7 @@ constexpr uint32_t kAKQl = 16384;
 constexpr uint32_t kKFh = 32768;         // decayed key versions 160 rows x 64 k
 constexpr uint32_t kKFl = 53248;
 constexpr uint32_t kKdStage = 73728;     // Kd^T rows of one channel half, hi 8 KB + lo 8 KB (bulk-copied out)
+constexpr uint32_t kLaStage = 73728;     // at the start: the chunk's log alpha rows (64 x 256 B, bulk-copied in)
 // after the first MMA
 constexpr uint32_t kAs = 0;              // A fp32 [64][65]
 constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
@@ -166,6 +167,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     uint32_t* sflags = reinterpret_cast<uint32_t*>(sbeta + 64);       // [0] fallback mask, [1] abort, [2] tmem base
     __shared__ uint64_t mbar;    // tensor-core products, in issue order
     __shared__ uint64_t mbar_k;  // the second half of the last product
+    __shared__ uint64_t mbar_la; // log alpha rows landed
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this thread: rows [8 w, 8 w + 8) of 16-row block I = w / 2, and channels
@@ -174,20 +176,34 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     const int kc = 2 * lane;                  // channel inside a half
     const int r0 = 8 * warp;
     int seq, tok0, len, cidx;
-    cmap.locate(blockIdx.x, seq, tok0, len, cidx);
-    const int h = blockIdx.y;
-    uint8_t* out = ws + (size_t)((size_t)blockIdx.x * H + h) * kChunkBytes;
+    // heads vary fastest over the grid: CTAs that run together read neighbouring
+    // 256-byte pieces of the same token rows and write neighbouring workspace images
+    const int chunk = (int)(blockIdx.x / (unsigned)H);
+    const int h = (int)(blockIdx.x - (unsigned)chunk * (unsigned)H);
+    cmap.locate(chunk, seq, tok0, len, cidx);
+    uint8_t* out = ws + (size_t)((size_t)chunk * H + h) * kChunkBytes;
 
     if (tid == 0) {
         sflags[0] = 0;
         sflags[1] = 0;
         mbar_init(&mbar, 1);
         mbar_init(&mbar_k, 1);
+        mbar_init(&mbar_la, 64);
         mbar_init_fence();
     }
     if (warp == 0) {
         tmem_alloc(&sflags[2], 256);
         tmem_relinquish();
+    }
+    __syncthreads();   // barriers initialised
+    // log alpha rows by the bulk-copy engine (one 256-byte row per thread of the first two warps)
+    if (tid < 64) {
+        if (tid < len) {
+            mbar_arrive_expect_tx(&mbar_la, 256);
+            bulk_g2s(sm + kLaStage + tid * 256, la + ((size_t)(tok0 + tid) * H + h) * kD, 256, &mbar_la);
+        } else {
+            mbar_arrive(&mbar_la);
+        }
     }
     const float beta_t = (tid < len && tid < 64) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
 
@@ -218,18 +234,22 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             asm volatile("prefetch.global.L2 [%0];" ::"l"(v + off));
         }
     }
+    load_kq(0);
+    if (!mbar_wait(&mbar_la, 0)) {
+        record_error(err, KDA_ERR_TIMEOUT);
+        atomicExch(&sflags[1], 1u);
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int r = r0 + j;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             uint32_t a = 0u;
-            if (r < len) a = *reinterpret_cast<const uint32_t*>(la + ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc);
+            if (r < len) a = *reinterpret_cast<const uint32_t*>(sm + kLaStage + r * 256 + (64 * hh + kc) * 2);
             g[j][2 * hh] = (r < len) ? fmaxf(bf16_lo(a), kLogAlphaFloor) : 0.f;
             g[j][2 * hh + 1] = (r < len) ? fmaxf(bf16_hi(a), kLogAlphaFloor) : 0.f;
         }
     }
-    load_kq(0);
     if (tid < 64) sbeta[tid] = beta_t;
     // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
@@ -1032,7 +1052,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
     if (n_chunks > 0) {
         e = cudaFuncSetAttribute(tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIntraAlloc);
         if (e != cudaSuccess) return e;
-        tc_intra<<<dim3(n_chunks, H), kIntraThreads, kIntraAlloc, stream>>>(
+        tc_intra<<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
             (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H);
         e = cudaGetLastError();
