@@ -103,7 +103,6 @@ constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 64 * 4 
 constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
 constexpr int kAS = 65;                  // row stride of As (floats)
 constexpr int kTS = 68;                  // row stride of Ts (floats; rows 16-byte aligned)
-constexpr int kYS = 20;                  // row stride of the 16 x 16 blocks Y (floats)
 
 // rows of the decayed-key versions: version R covers keys [0, 16 R + 16)
 __host__ __device__ __forceinline__ int kf_off(int R) { return (R * (R + 1)) * 8; }   // 0, 16, 48, 96
@@ -148,6 +147,51 @@ __device__ __forceinline__ void mma3(uint32_t d, uint32_t ah, uint32_t al, int a
         mma_bf16(d, dah, dbh, idesc, acc0);
         mma_bf16(d, dah, dbl, idesc, 1u);
         mma_bf16(d, dal, dbh, idesc, 1u);
+    }
+}
+
+// Columns [c0, c0 + 2 NC) of the block column I of T = (I + A)^{-1}, below the
+// diagonal, given the diagonal inverses T_JJ in Ts: for R = I+1 .. 3,
+// Y = sum_{I <= J < R} A_RJ T_JI and T_RI = -T_RR Y.  One warp: lane = (row r of
+// the block, column group lane / 16 of NC columns).
+template <int NC>
+__device__ __forceinline__ void tsolve_cols(const float* As, float* Ts, float* Yw, int I, int c0, int lane) {
+    const int r = lane & 15;
+    const int cl = (lane >> 4) * NC;        // first column of this lane inside the slice
+    const int col = c0 + cl;
+    for (int R = I + 1; R < 4; ++R) {
+        float2 acc[NC / 2];
+#pragma unroll
+        for (int x = 0; x < NC / 2; ++x) acc[x] = make_float2(0.f, 0.f);
+        for (int J = I; J < R; ++J) {
+            const float* arow = As + (16 * R + r) * kAS + 16 * J;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float2 av = make_float2(arow[m], arow[m]);
+                const float* trow = Ts + (16 * J + m) * kTS + col;
+#pragma unroll
+                for (int x = 0; x < NC / 2; ++x)
+                    acc[x] = fma2(av, *reinterpret_cast<const float2*>(trow + 2 * x), acc[x]);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < NC / 2; ++x) *reinterpret_cast<float2*>(Yw + r * 8 + cl + 2 * x) = acc[x];
+        __syncwarp();
+        float2 t[NC / 2];
+#pragma unroll
+        for (int x = 0; x < NC / 2; ++x) t[x] = make_float2(0.f, 0.f);
+        const float* drow = Ts + (16 * R + r) * kTS + 16 * R;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const float2 dv = make_float2(drow[m], drow[m]);
+#pragma unroll
+            for (int x = 0; x < NC / 2; ++x)
+                t[x] = fma2(dv, *reinterpret_cast<const float2*>(Yw + m * 8 + cl + 2 * x), t[x]);
+        }
+#pragma unroll
+        for (int x = 0; x < NC / 2; ++x)
+            *reinterpret_cast<float2*>(Ts + (16 * R + r) * kTS + col + 2 * x) = make_float2(-t[x].x, -t[x].y);
+        __syncwarp();   // T_RI is read at the next level; Yw is reused
     }
 }
 
@@ -521,41 +565,19 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             reinterpret_cast<float4*>(trow)[1] = make_float4(t[4], t[5], t[6], t[7]);
         }
         __syncthreads();
-        // block (R, I) at distance d = R - I: Y = sum_{I <= J < R} A_RJ T_JI, then
-        // T_RI = -T_RR Y; each thread forms four adjacent columns of one row
-        float* Y = scr;   // [3][16][kYS]
-        for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            const int e = tid;
-            const int bi = e >> 6, rr = (e >> 2) & 15, i4 = (e & 3) * 4;
-            const int R = bi + d, I2 = bi;
-            if (e < nb * 64) {
-                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-                for (int J = I2; J < R; ++J)
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float av = As[(16 * R + rr) * kAS + 16 * J + m];
-                        const float4 tv = *reinterpret_cast<const float4*>(Ts + (16 * J + m) * kTS + 16 * I2 + i4);
-                        acc0 = fma2(make_float2(av, av), make_float2(tv.x, tv.y), acc0);
-                        acc1 = fma2(make_float2(av, av), make_float2(tv.z, tv.w), acc1);
-                    }
-                *reinterpret_cast<float4*>(Y + (bi * 16 + rr) * kYS + i4) = make_float4(acc0.x, acc0.y, acc1.x, acc1.y);
-            }
-            __syncthreads();
-            if (e < nb * 64) {
-                float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float dv = Ts[(16 * R + rr) * kTS + 16 * R + m];
-                    const float4 yv = *reinterpret_cast<const float4*>(Y + (bi * 16 + m) * kYS + i4);
-                    acc0 = fma2(make_float2(dv, dv), make_float2(yv.x, yv.y), acc0);
-                    acc1 = fma2(make_float2(dv, dv), make_float2(yv.z, yv.w), acc1);
-                }
-                *reinterpret_cast<float4*>(Ts + (16 * R + rr) * kTS + 16 * I2 + i4) =
-                    make_float4(-acc0.x, -acc0.y, -acc1.x, -acc1.y);
-            }
-            __syncthreads();
-        }
+        // off-diagonal blocks, column by column (columns of T are independent):
+        // T_RI = -T_RR sum_{I <= J < R} A_RJ T_JI for R = I+1 .. 3, one warp per
+        // slice of a block column, so the levels need only warp-level syncs.
+        // Warps 0-3: block column 0 (4 columns each), 4-5: block column 1 and
+        // 6-7: block column 2 (8 columns each).
+        float* Yw = scr + warp * 128;   // [16][8] per warp
+        if (warp < 4)
+            tsolve_cols<2>(As, Ts, Yw, 0, 4 * warp, lane);
+        else if (warp < 6)
+            tsolve_cols<4>(As, Ts, Yw, 1, 16 + 8 * (warp - 4), lane);
+        else
+            tsolve_cols<4>(As, Ts, Yw, 2, 32 + 8 * (warp - 6), lane);
+        __syncthreads();
         // T (hi/lo) as a K-major tile; blocks above the diagonal are zero
         for (int e = tid; e < 64 * 8; e += kIntraThreads) {
             const int rr = e >> 3, k8 = (e & 7) * 8;
