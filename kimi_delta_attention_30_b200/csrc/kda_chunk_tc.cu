@@ -361,15 +361,18 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     for (int hr = 0; hr < 2; ++hr) {
         const int ch = 64 * hr + kc;
         // e = exp(g - gb[I]), f = exp(gb[I+1] - g)
-        const float2 gref = make_float2(gb[I * 128 + ch], gb[I * 128 + ch + 1]);
-        const float2 glast = make_float2(gb[(I + 1) * 128 + ch], gb[(I + 1) * 128 + ch + 1]);
-        const float2 xq = make_float2(tab[tab_e0(I) * 128 + ch], tab[tab_e0(I) * 128 + ch + 1]);
-        const float2 yk = make_float2(tab[tab_ec(I) * 128 + ch], tab[tab_ec(I) * 128 + ch + 1]);
+        // (pairs of channels as one 8-byte load: the lanes of a warp read 256
+        // consecutive bytes without bank conflicts)
+        auto pair = [](const float* p) { return *reinterpret_cast<const float2*>(p); };
+        const float2 gref = pair(gb + I * 128 + ch);
+        const float2 glast = pair(gb + (I + 1) * 128 + ch);
+        const float2 xq = pair(tab + tab_e0(I) * 128 + ch);
+        const float2 yk = pair(tab + tab_ec(I) * 128 + ch);
         float2 sgv[4];
 #pragma unroll
         for (int R = 0; R < 4; ++R) {
             const float* sg = tab + ((R == I) ? tab_tau(R) : tab_sigma(R > I ? R : I + 1, I)) * 128 + ch;
-            sgv[R] = (R < I) ? make_float2(0.f, 0.f) : make_float2(sg[0], sg[1]);
+            sgv[R] = (R < I) ? make_float2(0.f, 0.f) : pair(sg);
         }
         float kd0[8], kd1[8];
 #pragma unroll
@@ -392,9 +395,23 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             kd0[j] = kd.x;
             kd1[j] = kd.y;
         }
-        // Kd^T rows ch, ch + 1 (this half's 64 rows are staged, then copied out whole)
-        store8_split(sm + kKdStage, sm + kKdStage + 8192, sw128_chunk(kc, r0, 64), kd0);
-        store8_split(sm + kKdStage, sm + kKdStage + 8192, sw128_chunk(kc + 1, r0, 64), kd1);
+        // Kd^T rows ch, ch + 1 (this half's 64 rows are staged, then copied out whole).
+        // Lanes 4m..4m+3 store the even row first when m is even and the odd row
+        // first when m is odd, so each store covers all eight 16-byte bank groups.
+        {
+            uint4 h0, l0, h1, l1;
+            split2(kd0[0], kd0[1], h0.x, l0.x); split2(kd0[2], kd0[3], h0.y, l0.y);
+            split2(kd0[4], kd0[5], h0.z, l0.z); split2(kd0[6], kd0[7], h0.w, l0.w);
+            split2(kd1[0], kd1[1], h1.x, l1.x); split2(kd1[2], kd1[3], h1.y, l1.y);
+            split2(kd1[4], kd1[5], h1.z, l1.z); split2(kd1[6], kd1[7], h1.w, l1.w);
+            const bool odd_first = (lane >> 2) & 1;
+            const uint32_t oa = sw128_chunk(kc + (odd_first ? 1 : 0), r0, 64);
+            const uint32_t ob = sw128_chunk(kc + (odd_first ? 0 : 1), r0, 64);
+            *reinterpret_cast<uint4*>(sm + kKdStage + oa) = odd_first ? h1 : h0;
+            *reinterpret_cast<uint4*>(sm + kKdStage + 8192 + oa) = odd_first ? l1 : l0;
+            *reinterpret_cast<uint4*>(sm + kKdStage + ob) = odd_first ? h0 : h1;
+            *reinterpret_cast<uint4*>(sm + kKdStage + 8192 + ob) = odd_first ? l0 : l1;
+        }
         if (hr == 0) load_kq(1);   // in flight during this round's MMA
         fence_async_smem();
         tc_fence_before();
