@@ -63,6 +63,33 @@ def _dist():
     return world, rank, local
 
 
+def rank_helpers(world, device=None):
+    """barrier() and max_over_ranks(x) for a step timed on every rank: with one
+    rank both are no-ops; otherwise they use the initialised process group
+    (NCCL on GPUs, gloo in the CPU tests)."""
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    return barrier, max_over_ranks
+
+
+def job_throughput(world, units_per_rank_step, steps, max_total_ms):
+    """Whole-job units/s: every rank processes its own batch (weak scaling), the
+    job takes as long as its slowest rank."""
+    return world * units_per_rank_step * steps / (max_total_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -260,16 +287,7 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier, max_over_ranks = rank_helpers(world, dev)
 
     props = torch.cuda.get_device_properties(dev)
     gpu_id = None
@@ -326,7 +344,7 @@ def main():
         total_ms = max_over_ranks(sum(step_ms))
         ms_per_step = total_ms / a.steps
         tokens = B * T
-        value = world * tokens * a.steps / (total_ms / 1e3)
+        value = job_throughput(world, tokens, a.steps, total_ms)
         k_avg = [statistics.mean(x) for x in k_ms]
         dom = max(range(nk), key=lambda j: k_avg[j])
         dom_bytes = kernel_bytes(kernels[dom], B, T, H, dk, dv, C)
@@ -378,7 +396,7 @@ def main():
         tok_bytes = d["N"] * d["H"] * ((3 * d["dk"] + 2 * d["dv"]) * 2 + 2)
         alg = 2 * st_bytes + tok_bytes
         gbs = alg / (us * 1e-6) / 1e9
-        decode = {"value": world * d["N"] * n_launch / (dtot / 1e3), "unit": "tokens/s",
+        decode = {"value": job_throughput(world, d["N"], n_launch, dtot), "unit": "tokens/s",
                   "us_per_step": us, "hbm_gbs": gbs,
                   "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"],
                                "unit": "GB/s", "frac": gbs / pk["hbm_gbs"], "traffic": None,
@@ -421,7 +439,7 @@ def main():
         torch.cuda.synchronize()
         barrier()
         et = max_over_ranks(e0.elapsed_time(e1))
-        e2e = {"value": world * tokens * a.steps / (et / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(world, tokens, a.steps, et), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": et / a.steps}
 
     # ---------------------------------------------------------------- CPU baseline
