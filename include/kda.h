@@ -125,7 +125,10 @@ KDA_API size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int 
  *                     cu[n_seqs] = T, with B = 1; empty sequences are allowed
  *   n_seqs          : number of sequences when cu_seqlens_host != NULL
  *   C               : chunk size, 64 or 128; chunks restart at each sequence
- *                     start and the last chunk of a sequence may be partial
+ *                     start and the last chunk of a sequence may be partial.
+ *                     The chunk form's result does not depend on C (up to
+ *                     rounding), so the tensor-core path serves both sizes with
+ *                     64-token chunks; the CUDA-core path uses C as given
  *   o               : device output [B, T, H, dv], dtype `dtype`
  *   final_state     : device [N, H, dk, dv] fp32, or NULL; may alias init_state
  *   workspace       : device scratch of at least kda_chunk_fwd_workspace_size()

@@ -17,6 +17,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
 size_t tc_workspace_bytes(int n_chunks, int H, int C);
 bool tc_available();
 bool tc_supports(int C);
+int tc_chunk();
 
 TimingHook& timing_hook() {
     static thread_local TimingHook hook{{nullptr}, 0};
@@ -168,6 +169,10 @@ size_t kda_chunk_fwd_workspace_size_ex(int B, int T, int H, int dk, int dv, int 
     if (make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
     algo = resolve(algo, dtype, dk, dv, C);
     if (algo == KDA_ALGO_TC && !tc_shape(dtype, dk, dv, C)) return 0;
+    if (algo == KDA_ALGO_TC && C != tc_chunk()) {
+        C = tc_chunk();
+        if (make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
+    }
     return std::max<size_t>(workspace_for(p, H, dk, dv, C, algo), kAlign);
 }
 
@@ -198,6 +203,12 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
     if (st != KDA_OK) return st;
     algo = resolve(algo, dtype, dk, dv, C);
     if (algo == KDA_ALGO_TC && !tc_shape(dtype, dk, dv, C)) return KDA_ERR_SHAPE;
+    if (algo == KDA_ALGO_TC && C != tc_chunk()) {
+        // the tensor-core kernels tile by 64 tokens; the chunk form gives the
+        // same result for either chunk length
+        C = tc_chunk();
+        if ((st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p)) != KDA_OK) return st;
+    }
     const bool has_tokens = p.total_tokens > 0;
     if (has_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
     if (!workspace) return KDA_ERR_WORKSPACE;

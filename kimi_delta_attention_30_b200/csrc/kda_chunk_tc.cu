@@ -1072,7 +1072,9 @@ int sm_count() {
 
 bool tc_available() { return true; }
 
-bool tc_supports(int C) { return C == kC; }
+// Requests for 64- or 128-token chunks are both served with 64-token chunks.
+bool tc_supports(int C) { return C == kC || C == 2 * kC; }
+int tc_chunk() { return kC; }
 
 size_t tc_workspace_bytes(int n_chunks, int H, int C) {
     if (C != kC) return 0;

@@ -22,20 +22,23 @@ def bf16_half_ulp(x):
     return np.where(ax > 0, 2.0 ** (e - 8), 2.0 ** -134)
 
 
-def rel_err(got, ref, stored_as=None) -> float:
+def rel_err(got, ref, stored_as=None, both_stored=False) -> float:
     """max |got - ref| / rms(ref) over the compared elements.
 
     With ``stored_as="bf16"`` the GPU values were rounded once to bf16 when
     they were written (the output dtype follows the inputs); that rounding is
     not an error of the computation, so each |got - ref| is first reduced by
-    the half-ulp the storage may add (and floored at 0)."""
+    the half-ulp the storage may add (and floored at 0).  With
+    ``both_stored=True`` (two stored GPU outputs compared with each other) the
+    half-ulp of each side is allowed."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if got.size == 0:
         return 0.0
     d = np.abs(got - ref)
     if stored_as == "bf16":
-        d = np.maximum(d - bf16_half_ulp(got), 0.0)
+        allow = bf16_half_ulp(got) + (bf16_half_ulp(ref) if both_stored else 0.0)
+        d = np.maximum(d - allow, 0.0)
     rms = np.sqrt(np.mean(ref ** 2))
     if rms == 0.0:
         return float(np.max(d))

@@ -62,6 +62,18 @@ def test_workspace_size_queries():
     assert _ws(B=B, T=T, H=H, dk=d, dv=d, C=C, dtype=1, algo="simt") >= need
 
 
+def test_tensor_core_path_serves_both_chunk_sizes_with_64_token_chunks():
+    # bf16, d = 128: the tensor-core workspace for C = 128 is the one for C = 64
+    for cu in (None, [0, 100, 300, 301]):
+        B, T = (2, 300) if cu is None else (1, 301)
+        w64 = _ws(B=B, T=T, H=3, dk=128, dv=128, C=64, dtype=0, cu=cu, algo="tc")
+        w128 = _ws(B=B, T=T, H=3, dk=128, dv=128, C=128, dtype=0, cu=cu, algo="tc")
+        assert w64 > 0 and w64 == w128
+    # the CUDA-core path keeps the chunk size it is given
+    assert _ws(B=2, T=300, H=3, dk=128, dv=128, C=64, dtype=0, algo="simt") != \
+        _ws(B=2, T=300, H=3, dk=128, dv=128, C=128, dtype=0, algo="simt")
+
+
 def test_simt_offsets_are_disjoint_and_ordered():
     off = kda.simt_offsets(2, 200, 3, 64, 64, 64)
     assert off == sorted(off) and len(set(off)) == 5

@@ -25,3 +25,15 @@ def test_allowance_does_not_hide_real_errors():
     r = torch.tensor(x).to(torch.bfloat16).to(torch.float64).numpy()
     r[500] += 0.1                      # a computation error well above one ulp
     assert rel_err(r, x, stored_as="bf16") > 0.05
+
+
+def test_two_stored_roundings_of_one_value_compare_equal():
+    """Two outputs each rounded once to bf16 from nearby exact values may sit
+    one ulp apart; with both storages allowed they compare as equal."""
+    x = np.array([1.0 + 2.0 ** -8, 3.0 + 2.0 ** -7, -0.75 - 2.0 ** -10])
+    eps = 1e-6
+    to_bf16 = lambda t: torch.tensor(t, dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    a, b = to_bf16(x + eps * np.abs(x)), to_bf16(x - eps * np.abs(x))
+    assert np.any(a != b)
+    assert rel_err(a, b, stored_as="bf16", both_stored=True) == 0.0
+    assert rel_err(a, b, stored_as="bf16") > 0.0

@@ -108,11 +108,13 @@ def test_prefill_tiny_f32(cuda_ok):
     _check_all(inp, o, fs, TOL["f32"])
 
 
-@pytest.mark.parametrize("algo,C", [("auto", 64), ("auto", 128), ("simt", 64), ("simt", 128), ("tc", 64)])
+@pytest.mark.parametrize("algo,C", [("auto", 64), ("auto", 128), ("simt", 64), ("simt", 128), ("tc", 64),
+                                    ("tc", 128)])
 @pytest.mark.parametrize("T", [1, 63, 64, 200, 300])
 def test_prefill_bf16_ragged(cuda_ok, algo, C, T):
     """bf16, d=128, several chunks and a ragged tail, random initial state;
-    the tensor-core path (chunk 64) and the CUDA-core split."""
+    the tensor-core path (64-token chunks, asked for 64 or 128) and the CUDA-core
+    split (the chunk size as given)."""
     inp = _to(make_prefill("prefill", B=2, T=T, H=3, seed=T), DEV)
     o, fs = _run(inp, algo=algo, C=C)
     _check_all(inp, o, fs, TOL["bf16"])
@@ -246,17 +248,28 @@ def test_full_prefill_b4_h16_t4096(cuda_ok):
         assert rel_err(fg, fs_ref) <= 2e-2
 
 
-@pytest.mark.parametrize("C", [64, 128])
-def test_full_prefill_long_t65536(cuda_ok, C):
-    """B=1, H=32, T=65536, bf16; head 0 alpha = 1, head 1 scalar alpha; sampled heads."""
+def test_full_prefill_long_t65536(cuda_ok):
+    """B=1, H=32, T=65536, bf16; head 0 alpha = 1, head 1 scalar alpha; sampled
+    heads.  Chunk independence on the GPU: the tensor-core path (64-token
+    chunks) and the CUDA-core split with 128-token chunks agree with the oracle
+    and with each other."""
     inp = make_prefill("long", device=DEV)
-    o, fs = _run(inp, C=C)
-    assert torch.isfinite(o.float()).all() and torch.isfinite(fs).all()
     o_ref, fs_ref, ti, s_, h_ = oracle_prefill(inp, heads=[0, 1, 20])
-    og, fg = gpu_slices(o, fs, ti, s_, h_)
-    for j in range(3):
-        assert rel_err(og[:, j], o_ref[:, j], stored_as="bf16") <= 2e-2
-        assert rel_err(fg[:, j], fs_ref[:, j]) <= 2e-2
+    got = {}
+    for algo, C in (("tc", 64), ("tc", 128), ("simt", 128)):
+        o, fs = _run(inp, C=C, algo=algo)
+        assert torch.isfinite(o.float()).all() and torch.isfinite(fs).all()
+        og, fg = gpu_slices(o, fs, ti, s_, h_)
+        for j in range(3):
+            assert rel_err(og[:, j], o_ref[:, j], stored_as="bf16") <= 2e-2, (algo, C, j)
+            assert rel_err(fg[:, j], fs_ref[:, j]) <= 2e-2, (algo, C, j)
+        got[(algo, C)] = (og, fg)
+        del o, fs
+    og64, fg64 = got[("tc", 64)]
+    og128, fg128 = got[("simt", 128)]
+    assert rel_err(og64, og128, stored_as="bf16", both_stored=True) <= 2e-2
+    assert rel_err(fg64, fg128) <= 2e-2
+    assert np.array_equal(got[("tc", 128)][0], og64)      # the same 64-token computation
 
 
 def test_full_prefill_varlen_64_seqs(cuda_ok):
