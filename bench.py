@@ -10,7 +10,10 @@ CUDA events on the launching stream.  In the same run: the decode workload
 (256 sequences x 32 heads, d=128, fp32 state, 64 consecutive steps per bench
 step, timed per launch), the end-to-end prefill through the public API with
 pinned host buffers (H2D inputs + D2H outputs inside the timed region), and the
-fp64 oracle on a bounded sample on the host cores (rank 0, N = 1).
+fp64 oracle on a bounded sample on the host cores (rank 0, N = 1).  The
+"prep" object times the same prefill and decode launches on raw inputs with the
+input preprocessing fused in (``kda_chunk_fwd_prep`` / ``kda_decode_step_prep``:
+q/k L2 norm, -softplus gate, sigmoid beta).
 
 With N > 1 (torchrun) every rank runs its own independent batch (weak scaling,
 no collective on the data path); times are the max over ranks.
@@ -46,6 +49,7 @@ def _args():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prep", action="store_true", help="skip the fused-preprocessing timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample length")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="profiling aid: run only one part (the JSON line then lacks the other)")
@@ -169,6 +173,12 @@ def minimal_bytes(B, T, H, dk, dv, in_bytes=2, with_state=True):
     return b
 
 
+def separate_prep_bytes(n_tok_heads, dk, in_bytes=2):
+    """A stand-alone preprocessing pass: read raw q, k, gate (dk each) and beta,
+    write them back processed."""
+    return 2 * n_tok_heads * (3 * dk + 1) * in_bytes
+
+
 def measured_traffic(kernel, B, T, H, C):
     """DRAM bytes per launch of `kernel` on this workload from the committed ncu
     table, or None when there is none or the kernel sources changed since."""
@@ -279,7 +289,7 @@ def main():
     import torch.distributed as dist
 
     import kimi_delta_attention_30_b200 as kda
-    from kda_inputs import make_decode_state, make_decode_token, make_prefill
+    from kda_inputs import RAW_PREP, make_decode_state, make_decode_token, make_prefill
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -306,6 +316,8 @@ def main():
     clocks = ClockSampler(gpu_id if rank == 0 else None)
     value = ms_per_step = roofline = path_roofline = kernel_table = t_wall = None
     kernels, nk = [], 0
+    run_prep = not a.no_prep and a.algo in ("auto", "tc")
+    prep = {} if run_prep else None
     if run_prefill:
         inp = make_prefill("prefill", device=dev, seed=rank, B=B)
         kernels = kda.chunk_kernels(B, T, H, dk, dv, C, torch.bfloat16, algo=a.algo)
@@ -361,6 +373,44 @@ def main():
         path_roofline = {"minimal_bytes": min_b, "time_min_us": min_b / (pk["hbm_gbs"] * 1e9) * 1e6,
                          "frac_of_hbm_bound": (min_b / (pk["hbm_gbs"] * 1e9)) / (ms_per_step / 1e3)}
 
+        # ------------------------------------------------ prefill, preprocessing fused
+        if run_prep:
+            raw = make_prefill("prefill_raw", device=dev, seed=rank, B=B)
+
+            def prep_step(evs=None):
+                if evs is not None:
+                    kda.set_timing_events(evs)
+                kda.chunk_fwd(raw.q, raw.k, raw.v, raw.log_alpha, raw.beta, init_state=raw.init_state, C=C, o=o,
+                              final_state=fs, workspace=ws, algo=a.algo, prep=RAW_PREP)
+
+            for _ in range(a.warmup):
+                flush.zero_()
+                prep_step()
+            pev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(a.steps)]
+            for row in pev:
+                for e in row:
+                    e.record(stream)
+            barrier()
+            torch.cuda.synchronize()
+            for i in range(a.steps):
+                flush.zero_()
+                prep_step(pev[i])
+            torch.cuda.synchronize()
+            barrier()
+            p_total = max_over_ranks(sum(pev[i][0].elapsed_time(pev[i][nk]) for i in range(a.steps)))
+            pk_avg = [statistics.mean(pev[i][j].elapsed_time(pev[i][j + 1]) for i in range(a.steps))
+                      for j in range(nk)]
+            sep = separate_prep_bytes(tokens * H, dk)
+            prep["prefill"] = {
+                "value": job_throughput(world, tokens, a.steps, p_total), "unit": "tokens/s",
+                "ms_per_step": p_total / a.steps, "added_ms_vs_plain": p_total / a.steps - ms_per_step,
+                "kernel_times": {kernels[j]: {"avg_us": pk_avg[j] * 1e3} for j in range(nk)},
+                "separate_pass_bytes": sep, "separate_pass_min_ms": sep / (pk["hbm_gbs"] * 1e9) * 1e3,
+                "config": {"workload": f"prefill B={B} H={H} T={T} d={dk} C={C} bf16, raw q/k (unnormalised), "
+                           "gate logits, beta logits; flags QK_L2NORM|GATE_SOFTPLUS|BETA_SIGMOID",
+                           "l2": "flushed before every timed step (256 MiB write)"}}
+            del raw
+
     # ---------------------------------------------------------------- decode
     decode = None
     if run_decode:
@@ -369,27 +419,29 @@ def main():
         toks = [make_decode_token("decode", step=s, device=dev, seed=rank, N=d["N"]) for s in range(d["steps"])]
         od = torch.empty((d["N"], d["H"], d["dv"]), dtype=torch.bfloat16, device=dev)
 
-        def decode_round(evs=None):
+        def decode_round(evs=None, tk=toks, flags=0):
             for s in range(d["steps"]):
-                t = toks[s]
+                t = tk[s]
                 if evs is not None:
                     evs[s][0].record(stream)
-                kda.decode_step(t.q, t.k, t.v, t.log_alpha, t.beta, state, o=od)
+                kda.decode_step(t.q, t.k, t.v, t.log_alpha, t.beta, state, o=od, prep=flags)
                 if evs is not None:
                     evs[s][1].record(stream)
 
-        for _ in range(a.warmup):
-            decode_round()
-        dev_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(d["steps"])]
-                  for _ in range(a.steps)]
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(a.steps):
-            decode_round(dev_ev[i])
-        torch.cuda.synchronize()
-        barrier()
-        per_launch = [e[0].elapsed_time(e[1]) for r in dev_ev for e in r]
-        dtot = max_over_ranks(sum(per_launch))
+        def timed_rounds(**kw):
+            for _ in range(a.warmup):
+                decode_round(**kw)
+            dev_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(d["steps"])]
+                      for _ in range(a.steps)]
+            barrier()
+            torch.cuda.synchronize()
+            for i in range(a.steps):
+                decode_round(dev_ev[i], **kw)
+            torch.cuda.synchronize()
+            barrier()
+            return max_over_ranks(sum(e[0].elapsed_time(e[1]) for r in dev_ev for e in r))
+
+        dtot = timed_rounds()
         n_launch = a.steps * d["steps"]
         us = dtot / n_launch * 1e3
         st_bytes = d["N"] * d["H"] * d["dk"] * d["dv"] * 4
@@ -404,7 +456,19 @@ def main():
                   "config": {"workload": f"decode N={d['N']} H={d['H']} d={d['dk']} fp32 state, bf16 tokens, "
                              f"{d['steps']} consecutive steps", "l2": "state 512 MiB > L2"},
                   "gpu_launches": n_launch}
-        del state, toks
+        if run_prep:
+            del toks
+            raw_toks = [make_decode_token("decode_raw", step=s, device=dev, seed=rank, N=d["N"])
+                        for s in range(d["steps"])]
+            ptot = timed_rounds(tk=raw_toks, flags=RAW_PREP)
+            pus = ptot / n_launch * 1e3
+            prep["decode"] = {"value": job_throughput(world, d["N"], n_launch, ptot), "unit": "tokens/s",
+                              "us_per_step": pus, "hbm_gbs": alg / (pus * 1e-6) / 1e9,
+                              "added_us_vs_plain": pus - us,
+                              "config": {"workload": f"decode N={d['N']} H={d['H']} d={d['dk']} raw bf16 tokens, "
+                                         "flags QK_L2NORM|GATE_SOFTPLUS|BETA_SIGMOID"}}
+            del raw_toks
+        del state
 
     clk = clocks.stop() if rank == 0 else None
 
@@ -459,7 +523,8 @@ def main():
                            "kernels": kernels, "l2": "flushed before every timed step (256 MiB write)",
                            "parallelism": f"replicas x{world} (independent sequences per GPU)"},
                 "roofline": roofline, "path_roofline": path_roofline, "kernel_times": kernel_table,
-                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "e2e": e2e, "cpu_baseline": cpu,
+                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "prep": prep,
+                "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clk, "wall_s_timed": t_wall, "gpu": props.name}
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -236,6 +236,52 @@ KDA_API kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            float* state, int N, int H, int dk, int dv, void* o,
                            void* stream);
 
+/*
+ * Input preprocessing fused into the kernels (the gate and the key/query
+ * normalisation that usually run as separate passes before the operator).
+ * The per-channel decay comes from an "alpha projection" with alpha between 0
+ * and 1 ("22580倍参数量级" article, tahou.com/article/213680821660188677,
+ * sections on Gated DeltaNet and on the Kimi Linear architecture), but the pages
+ * do not fix the gate's parametrisation; this library reads it as
+ *   KDA_PREP_QK_L2NORM     : q and k are divided by their L2 norm over d_k
+ *                            (per token and head; an all-zero vector stays 0)
+ *   KDA_PREP_GATE_SOFTPLUS : the log_alpha argument holds raw gate logits a,
+ *                            log alpha = -softplus(a) = -log(1 + e^a)
+ *   KDA_PREP_BETA_SIGMOID  : the beta argument holds raw logits b,
+ *                            beta = 1 / (1 + e^-b)
+ * Flags combine with |.  With no flag the calls below are kda_chunk_fwd and
+ * kda_decode_step.
+ */
+typedef enum {
+    KDA_PREP_NONE = 0,
+    KDA_PREP_QK_L2NORM = 1,
+    KDA_PREP_GATE_SOFTPLUS = 2,
+    KDA_PREP_BETA_SIGMOID = 4
+} kda_prep;
+
+/*
+ * kda_chunk_fwd with the inputs preprocessed inside the tensor-core kernels
+ * (same arguments, layouts, workspace and errors; `prep` is a kda_prep mask).
+ * The preprocessing is fused into the tensor-core path only: with prep != 0,
+ * problems that path does not take (fp32, dk or dv of 64) are rejected with
+ * KDA_ERR_SHAPE, as is a mask with unknown bits.
+ */
+KDA_API kda_status kda_chunk_fwd_prep(const void* q, const void* k, const void* v,
+                                      const void* log_alpha, const void* beta, kda_dtype dtype,
+                                      unsigned int prep, const float* init_state,
+                                      const int32_t* cu_seqlens_host, int n_seqs,
+                                      int B, int T, int H, int dk, int dv, int C,
+                                      void* o, float* final_state,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* kda_decode_step with the inputs preprocessed inside the decode kernel (all
+ * shapes and dtypes of kda_decode_step; unknown bits: KDA_ERR_SHAPE). */
+KDA_API kda_status kda_decode_step_prep(const void* q, const void* k, const void* v,
+                                        const void* log_alpha, const void* beta, kda_dtype dtype,
+                                        unsigned int prep, float* state, int N, int H, int dk, int dv,
+                                        void* o, void* stream);
+
+
 #ifdef __cplusplus
 }
 #endif

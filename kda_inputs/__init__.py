@@ -20,10 +20,16 @@ Workloads (sizes and value distributions):
   depends on the head index mod 3: near one (log alpha ~ U(-1e-3, 0)), near
   zero (log alpha ~ U(-16, -8)), mixed (log alpha = -softplus(N(0, 2))).
 
+* ``prefill_raw`` / ``decode_raw`` -- the ``prefill`` / ``decode`` sizes with
+  raw (un-preprocessed) inputs: q, k ~ N(0,1) * 2 NOT normalised, the gate
+  argument holds logits a ~ N(0,1) + 3 (so -softplus(a) has the ``prefill``
+  gate's distribution) and beta holds logits ~ N(0,1).
+
 Common to all: q, k ~ N(0,1), L2-normalised over d_k (in fp64), v ~ N(0,1),
 beta = sigmoid(N(0,1)) unless stated; every value is drawn in fp32/fp64 and
 rounded once (round-to-nearest-even) to the input dtype.  N(mu, s^2) is
-variance notation.
+variance notation.  The logistic and softplus maps used here only shape the
+draws' distributions.
 """
 from __future__ import annotations
 
@@ -51,6 +57,7 @@ class Workload:
     n_seqs: int = 0                 # varlen: number of packed sequences
     len_range: tuple = (0, 0)       # varlen: inclusive length range
     steps: int = 0                  # decode: number of steps
+    raw: bool = False               # raw q/k, gate logits and beta logits
     extra: dict = field(default_factory=dict)
 
 
@@ -62,7 +69,14 @@ WORKLOADS = {
     "decode": Workload("decode", B=256, H=32, T=1, dk=128, dv=128, dtype="bf16", init_std=0.02, steps=64),
     "varlen": Workload("varlen", H=32, dk=128, dv=128, C=64, dtype="bf16", gate="regimes",
                        beta_dist="uniform", init_std=0.02, n_seqs=64, len_range=(512, 32768)),
+    "prefill_raw": Workload("prefill_raw", B=4, H=16, T=4096, dk=128, dv=128, C=64, dtype="bf16",
+                            init_std=0.02, raw=True),
+    "decode_raw": Workload("decode_raw", B=256, H=32, T=1, dk=128, dv=128, dtype="bf16", init_std=0.02,
+                           steps=64, raw=True),
 }
+
+# Raw workloads pass these kda_prep flags (QK_L2NORM | GATE_SOFTPLUS | BETA_SIGMOID).
+RAW_PREP = 1 | 2 | 4
 
 
 def torch_dtype(name: str):
@@ -97,9 +111,20 @@ def _unit_rows(shape, gen, device):
     return x / torch.linalg.vector_norm(x, dim=-1, keepdim=True)
 
 
+def _qk(shape, wl: Workload, gen, device):
+    if wl.raw:
+        return _normal(shape, gen, device) * 2.0
+    return _unit_rows(shape, gen, device)
+
+
 def _gate(shape, wl: Workload, gen, device, head_offset: int = 0):
-    """log alpha of the given shape [..., H, dk] (fp32, before rounding)."""
+    """log alpha of the given shape [..., H, dk] (fp32, before rounding); for a
+    raw workload the gate logits."""
     H, dk = shape[-2], shape[-1]
+    if wl.raw:
+        if wl.gate not in ("softplus2", "softplus3") or wl.special_heads:
+            raise ValueError("raw workloads draw softplus gate logits only")
+        return _normal(shape, gen, device) + (2.0 if wl.gate == "softplus2" else 3.0)
     if wl.gate in ("softplus2", "softplus3"):
         shift = 2.0 if wl.gate == "softplus2" else 3.0
         la = -torch.nn.functional.softplus(_normal(shape, gen, device) + shift)
@@ -121,6 +146,8 @@ def _gate(shape, wl: Workload, gen, device, head_offset: int = 0):
 
 
 def _beta(shape, wl: Workload, gen, device):
+    if wl.raw:
+        return _normal(shape, gen, device)
     if wl.beta_dist == "sigmoid":
         return torch.sigmoid(_normal(shape, gen, device))
     return torch.rand(shape, generator=gen, device=device)
@@ -186,8 +213,8 @@ def make_prefill(wl: Workload | str, device="cpu", seed: int = 0, *, B=None, T=N
             t1 = min(Tx, t0 + step)
             g = _gen(device, seed, 1 + b * 100003 + s)
             n = t1 - t0
-            q[b, t0:t1] = _unit_rows((n, H, dk), g, device).to(dt)
-            k[b, t0:t1] = _unit_rows((n, H, dk), g, device).to(dt)
+            q[b, t0:t1] = _qk((n, H, dk), wl, g, device).to(dt)
+            k[b, t0:t1] = _qk((n, H, dk), wl, g, device).to(dt)
             v[b, t0:t1] = _normal((n, H, dv), g, device).to(dt)
             la[b, t0:t1] = _gate((n, H, dk), wl, g, device).to(dt)
             beta[b, t0:t1] = _beta((n, H), wl, g, device).to(dt)
@@ -228,8 +255,8 @@ def make_decode_token(wl: Workload | str = "decode", step: int = 0, device="cpu"
     H = wl.H if H is None else H
     dt = torch_dtype(wl.dtype)
     g = _gen(device, seed, 7_000_001 + step)
-    q = _unit_rows((N, H, wl.dk), g, device).to(dt)
-    k = _unit_rows((N, H, wl.dk), g, device).to(dt)
+    q = _qk((N, H, wl.dk), wl, g, device).to(dt)
+    k = _qk((N, H, wl.dk), wl, g, device).to(dt)
     v = _normal((N, H, wl.dv), g, device).to(dt)
     la = _gate((N, H, wl.dk), wl, g, device).to(dt)
     beta = _beta((N, H), wl, g, device).to(dt)

@@ -10,6 +10,10 @@ Calls:
 * :func:`chunk_fwd` -- chunkwise prefill (``kda_chunk_fwd``).
 * :func:`decode_step` -- one recurrent step, state updated in place
   (``kda_decode_step``).
+
+Both take ``prep`` (a bitwise OR of the ``PREP_*`` flags): raw q/k, gate
+logits and beta logits are then normalised / activated inside the kernels
+(``kda_chunk_fwd_prep``, ``kda_decode_step_prep``).
 """
 from __future__ import annotations
 
@@ -26,6 +30,9 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 KDA_BF16, KDA_F32 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tc": 2}
 _DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
+# kda_prep flags (include/kda.h)
+PREP_NONE, PREP_QK_L2NORM, PREP_GATE_SOFTPLUS, PREP_BETA_SIGMOID = 0, 1, 2, 4
+PREP_ALL = PREP_QK_L2NORM | PREP_GATE_SOFTPLUS | PREP_BETA_SIGMOID
 
 
 class KdaError(RuntimeError):
@@ -58,6 +65,11 @@ def _declare(lib):
     lib.kda_chunk_simt_offsets.restype = c_int
     lib.kda_decode_step.argtypes = [vp] * 5 + [c_int, vp] + [c_int] * 4 + [vp, vp]
     lib.kda_decode_step.restype = c_int
+    lib.kda_chunk_fwd_prep.argtypes = [vp] * 5 + [c_int, ctypes.c_uint, vp, i32p, c_int] + [c_int] * 6 + \
+        [vp, vp, vp, c_size, vp]
+    lib.kda_chunk_fwd_prep.restype = c_int
+    lib.kda_decode_step_prep.argtypes = [vp] * 5 + [c_int, ctypes.c_uint, vp] + [c_int] * 4 + [vp, vp]
+    lib.kda_decode_step_prep.restype = c_int
     lib.kda_set_timing_events.argtypes = [ctypes.POINTER(vp), c_int]
     lib.kda_set_timing_events.restype = c_int
     lib.kda_chunk_fwd_kernels.argtypes = [c_int] * 7 + [i32p, c_int, c_int, ctypes.POINTER(ctypes.c_char_p), c_int]
@@ -95,7 +107,7 @@ def exported_symbols():
     return ["kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
             "kda_chunk_fwd_workspace_size_ex", "kda_chunk_fwd", "kda_chunk_fwd_ex",
             "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
-            "kda_chunk_fwd_noalloc"]
+            "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep"]
 
 
 def _ptr(t):
@@ -166,14 +178,17 @@ def set_timing_events(events):
 
 def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int = 64,
               output_final_state: bool = True, o=None, final_state=None, workspace=None,
-              algo: str = "auto", stream=None):
+              algo: str = "auto", stream=None, prep: int = 0):
     """Chunkwise KDA prefill.
 
     q, k, log_alpha ``[B, T, H, dk]``; v ``[B, T, H, dv]``; beta ``[B, T, H]``;
     all one dtype (bf16 or fp32), contiguous, on one CUDA device.  ``cu_seqlens``
     (host sequence, N + 1 offsets) selects packed varlen mode with B = 1.
     ``init_state`` ``[N, H, dk, dv]`` fp32 or None.  Returns ``(o, final_state)``
-    (final_state is None when ``output_final_state`` is False).
+    (final_state is None when ``output_final_state`` is False).  ``prep`` != 0
+    calls ``kda_chunk_fwd_prep`` (tensor-core shapes only; ``algo`` must be
+    "auto" or "tc"): log_alpha then holds gate logits and beta beta logits when
+    the matching flag is set.
     """
     dt = q.dtype
     if dt not in _DTYPES:
@@ -195,6 +210,16 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
     if workspace is None:
         workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
     _check_cuda("workspace", workspace)
+    if prep:
+        if algo not in ("auto", "tc"):
+            raise ValueError("prep is fused into the tensor-core path only")
+        st = lib().kda_chunk_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], prep,
+                                      _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o),
+                                      _ptr(final_state), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        if st != 0:
+            raise KdaError(st, "kda_chunk_fwd_prep")
+        return o, final_state
     st = lib().kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
                                 _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o), _ptr(final_state),
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -238,10 +263,11 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None
     return o, final_state
 
 
-def decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
+def decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None, prep: int = 0):
     """One KDA decode step for N sequences; ``state`` ``[N, H, dk, dv]`` fp32 is
     updated in place.  q, k, log_alpha ``[N, H, dk]``, v ``[N, H, dv]``, beta
-    ``[N, H]``.  Returns o ``[N, H, dv]``."""
+    ``[N, H]``.  Returns o ``[N, H, dv]``.  ``prep`` != 0 calls
+    ``kda_decode_step_prep`` (raw inputs normalised / activated in the kernel)."""
     dt = q.dtype
     if dt not in _DTYPES:
         raise ValueError(f"unsupported dtype {dt}")
@@ -253,6 +279,12 @@ def decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None):
     if o is None:
         o = torch.empty((N, H, dv), dtype=dt, device=q.device)
     _check_cuda("o", o, dt)
+    if prep:
+        st = lib().kda_decode_step_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], prep,
+                                        _ptr(state), N, H, dk, dv, _ptr(o), _stream_handle(stream))
+        if st != 0:
+            raise KdaError(st, "kda_decode_step_prep")
+        return o
     st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], _ptr(state),
                                N, H, dk, dv, _ptr(o), _stream_handle(stream))
     if st != 0:

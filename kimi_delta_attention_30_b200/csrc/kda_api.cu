@@ -13,7 +13,7 @@ namespace kda {
 cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                               const float* init_state, void* o, float* final_state, const ChunkMap& cmap,
                               const SeqMap& smap, int n_chunks, int n_seqs, int H, int C, void* tc_ws,
-                              cudaStream_t stream);
+                              unsigned prep, cudaStream_t stream);
 size_t tc_workspace_bytes(int n_chunks, int H, int C);
 bool tc_available();
 bool tc_supports(int C);
@@ -192,17 +192,25 @@ kda_status kda_chunk_simt_offsets(int B, int T, int H, int dk, int dv, int C, co
     return KDA_OK;
 }
 
-kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
-                            kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs,
-                            int B, int T, int H, int dk, int dv, int C, void* o, float* final_state,
-                            void* workspace, size_t workspace_bytes, void* stream, kda_algo algo) {
+}  // extern "C"
+
+namespace {
+
+constexpr unsigned kPrepAll = KDA_PREP_QK_L2NORM | KDA_PREP_GATE_SOFTPLUS | KDA_PREP_BETA_SIGMOID;
+
+kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                          kda_dtype dtype, unsigned prep, const float* init_state, const int32_t* cu_seqlens_host,
+                          int n_seqs, int B, int T, int H, int dk, int dv, int C, void* o, float* final_state,
+                          void* workspace, size_t workspace_bytes, void* stream, kda_algo algo) {
     if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
     if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_SHAPE;
+    if (prep & ~kPrepAll) return KDA_ERR_SHAPE;
     Plan p;
     kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
     if (st != KDA_OK) return st;
     algo = resolve(algo, dtype, dk, dv, C);
     if (algo == KDA_ALGO_TC && !tc_shape(dtype, dk, dv, C)) return KDA_ERR_SHAPE;
+    if (prep != 0 && algo != KDA_ALGO_TC) return KDA_ERR_SHAPE;   // preprocessing is fused into the TC kernels
     if (algo == KDA_ALGO_TC && C != tc_chunk()) {
         // the tensor-core kernels tile by 64 tokens; the chunk form gives the
         // same result for either chunk length
@@ -243,10 +251,49 @@ kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const v
                                   p.n_chunks, p.n_seqs, H, dk, dv, C, w, s);
     } else {
         err = launch_tc_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap, p.n_chunks,
-                                p.n_seqs, H, C, ws + table_bytes(p), s);
+                                p.n_seqs, H, C, ws + table_bytes(p), prep, s);
     }
     timing_hook().n = 0;
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status decode_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                       kda_dtype dtype, unsigned prep, float* state, int N, int H, int dk, int dv, void* o,
+                       void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (prep & ~kPrepAll) return KDA_ERR_SHAPE;
+    if (N < 0 || H <= 0 || !((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_SHAPE;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    if (N == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_NULL;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, state, o};
+    for (const void* ptr : ptrs)
+        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
+    kda_status st = check_device();
+    if (st != KDA_OK) return st;
+    cudaError_t err =
+        launch_decode(dtype, q, k, v, log_alpha, beta, state, N, H, dk, dv, o, prep, (cudaStream_t)stream);
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                            kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs,
+                            int B, int T, int H, int dk, int dv, int C, void* o, float* final_state,
+                            void* workspace, size_t workspace_bytes, void* stream, kda_algo algo) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, dtype, 0u, init_state, cu_seqlens_host, n_seqs, B, T, H, dk, dv,
+                          C, o, final_state, workspace, workspace_bytes, stream, algo);
+}
+
+kda_status kda_chunk_fwd_prep(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              kda_dtype dtype, unsigned int prep, const float* init_state,
+                              const int32_t* cu_seqlens_host, int n_seqs, int B, int T, int H, int dk, int dv, int C,
+                              void* o, float* final_state, void* workspace, size_t workspace_bytes, void* stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, dtype, prep, init_state, cu_seqlens_host, n_seqs, B, T, H, dk,
+                          dv, C, o, final_state, workspace, workspace_bytes, stream, KDA_ALGO_AUTO);
 }
 
 kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
@@ -282,18 +329,13 @@ int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype 
 
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                            kda_dtype dtype, float* state, int N, int H, int dk, int dv, void* o, void* stream) {
-    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
-    if (N < 0 || H <= 0 || !((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_SHAPE;
-    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_SHAPE;
-    if (N == 0) return KDA_OK;
-    if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_NULL;
-    const void* ptrs[] = {q, k, v, log_alpha, beta, state, o};
-    for (const void* ptr : ptrs)
-        if (!aligned16(ptr)) return KDA_ERR_ALIGN;
-    kda_status st = check_device();
-    if (st != KDA_OK) return st;
-    cudaError_t err = launch_decode(dtype, q, k, v, log_alpha, beta, state, N, H, dk, dv, o, (cudaStream_t)stream);
-    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return decode_impl(q, k, v, log_alpha, beta, dtype, 0u, state, N, H, dk, dv, o, stream);
+}
+
+kda_status kda_decode_step_prep(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                                kda_dtype dtype, unsigned int prep, float* state, int N, int H, int dk, int dv,
+                                void* o, void* stream) {
+    return decode_impl(q, k, v, log_alpha, beta, dtype, prep, state, N, H, dk, dv, o, stream);
 }
 
 }  // extern "C"

@@ -99,7 +99,7 @@ constexpr uint32_t kXh = 0;
 constexpr uint32_t kXl = 32768;
 constexpr uint32_t kTab = 98304;         // tables
 constexpr int kNumTab = 18;              // tau[4], sigma[6], exp(gb)[4], exp(g_C - gb[b+1])[4]
-constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 64 * 4 + 64;
+constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 3 * 64 * 4 + 64;
 constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
 constexpr int kAS = 65;                  // row stride of As (floats)
 constexpr int kTS = 68;                  // row stride of Ts (floats; rows 16-byte aligned)
@@ -198,17 +198,22 @@ __device__ __forceinline__ void tsolve_cols(const float* As, float* Ts, float* Y
 // ============================================================================
 // tc_intra
 // ============================================================================
+template <bool PREP>
 __global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
-         int H) {
+         int H, unsigned prep_flags) {
+    // PREP = false is the plain operator: no preprocessing code is compiled in
+    const unsigned prep = PREP ? prep_flags : 0u;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* tab = reinterpret_cast<float*>(sm + kTab);                 // [18][128]
     float* gb = tab + kNumTab * 128;                                  // [5][128]
     float* sbeta = gb + 5 * 128;                                      // [64]
-    uint32_t* sflags = reinterpret_cast<uint32_t*>(sbeta + 64);       // [0] fallback mask, [1] abort, [2] tmem base
+    float* inv_nk = sbeta + 64;                                       // [64] 1 / ||k_r|| (1 without normalisation)
+    float* inv_nq = inv_nk + 64;                                      // [64] 1 / ||q_r||
+    uint32_t* sflags = reinterpret_cast<uint32_t*>(inv_nq + 64);      // [0] fallback mask, [1] abort, [2] tmem base
     __shared__ uint64_t mbar;    // tensor-core products, in issue order
     __shared__ uint64_t mbar_k;  // the second half of the last product
     __shared__ uint64_t mbar_la; // log alpha rows landed
@@ -249,8 +254,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             mbar_arrive(&mbar_la);
         }
     }
-    const float beta_t = (tid < len && tid < 64) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
-
+    const float beta_t =
+        (tid < len && tid < 64) ? prep_beta(__bfloat162float(beta[(size_t)(tok0 + tid) * H + h]), prep) : 0.f;
     // ---- log alpha of 8 rows x 4 channels; k, q, v prefetched into L2 ---------
     // (k and q of a channel half are read one phase before the round that uses
     // them, v at the end; holding them in registers through the chunk would push
@@ -279,6 +284,27 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         }
     }
     load_kq(0);
+    // key / query normalisation factors: thread t < 64 takes row t of k, 64 <= t < 128 row t - 64 of q
+    float inv_t = 1.f;
+    if (PREP && (prep & KDA_PREP_QK_L2NORM) && tid < 128) {
+        const int r = tid & 63;
+        inv_t = 0.f;
+        if (r < len) {
+            const uint4* row = reinterpret_cast<const uint4*>((tid < 64 ? k : q) + ((size_t)(tok0 + r) * H + h) * kD);
+            float ss = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                float f[8];
+                const uint4 u = row[x];
+                f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+                f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+            }
+            inv_t = inv_norm_from_sq(ss);
+        }
+    }
+
     if (!mbar_wait(&mbar_la, 0)) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
@@ -290,11 +316,12 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         for (int hh = 0; hh < 2; ++hh) {
             uint32_t a = 0u;
             if (r < len) a = *reinterpret_cast<const uint32_t*>(sm + kLaStage + r * 256 + (64 * hh + kc) * 2);
-            g[j][2 * hh] = (r < len) ? fmaxf(bf16_lo(a), kLogAlphaFloor) : 0.f;
-            g[j][2 * hh + 1] = (r < len) ? fmaxf(bf16_hi(a), kLogAlphaFloor) : 0.f;
+            g[j][2 * hh] = (r < len) ? prep_log_alpha(bf16_lo(a), prep) : 0.f;
+            g[j][2 * hh + 1] = (r < len) ? prep_log_alpha(bf16_hi(a), prep) : 0.f;
         }
     }
     if (tid < 64) sbeta[tid] = beta_t;
+    if (PREP && tid < 128) inv_nk[tid] = inv_t;   // inv_nk [0, 64) and inv_nq [64, 128) are adjacent
     // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
     for (int j = 1; j < 8; ++j)
@@ -380,7 +407,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             const int r = r0 + j;
             const float2 gj = make_float2(g[j][2 * hr], g[j][2 * hr + 1]);
             const float2 e = exp_diff2(gj, gref), f = exp_diff2(glast, gj);
-            const float2 k2 = unpack_bf16x2(kv[j]), q2 = unpack_bf16x2(qv[j]);
+            float2 k2 = unpack_bf16x2(kv[j]), q2 = unpack_bf16x2(qv[j]);
+            if (PREP) {
+                k2 = mul2(k2, make_float2(inv_nk[r], inv_nk[r]));
+                q2 = mul2(q2, make_float2(inv_nq[r], inv_nq[r]));
+            }
             const float2 ke = mul2(k2, e), qe = mul2(q2, e), kf = mul2(k2, f);
             store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(r, kc, 128), ke.x, ke.y);
             store2_split(sm + kAKQh, sm + kAKQl, sw128_offset(64 + r, kc, 128), qe.x, qe.y);
@@ -493,8 +524,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             float* sh = scr;   // [16][128] block-local cumulative log decay
             for (int e = tid; e < 16 * 128; e += kIntraThreads) {
                 const int rr = e >> 7, c = e & 127, row = 16 * R + rr;
-                sh[e] = (row < len) ? fmaxf(__bfloat162float(la[((size_t)(tok0 + row) * H + h) * kD + c]),
-                                            kLogAlphaFloor)
+                sh[e] = (row < len) ? prep_log_alpha(__bfloat162float(la[((size_t)(tok0 + row) * H + h) * kD + c]),
+                                                     prep)
                                     : 0.f;
             }
             __syncthreads();
@@ -510,9 +541,12 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 if (row < len) {
                     const size_t ro = ((size_t)(tok0 + row) * H + h) * kD, io = ((size_t)(tok0 + col) * H + h) * kD;
                     for (int c = lane; c < 128; c += 32) {
-                        const float kdv = __bfloat162float(k[io + c]) * __expf(sh[rr * 128 + c] - sh[ii * 128 + c]);
-                        sa += __bfloat162float(k[ro + c]) * kdv;
-                        spq += __bfloat162float(q[ro + c]) * kdv;
+                        const float sk_c = PREP ? inv_nk[col] : 1.f, sk_r = PREP ? inv_nk[row] : 1.f;
+                        const float sq_r = PREP ? inv_nq[row] : 1.f;
+                        const float kdv = __bfloat162float(k[io + c]) * sk_c *
+                                          __expf(sh[rr * 128 + c] - sh[ii * 128 + c]);
+                        sa += __bfloat162float(k[ro + c]) * sk_r * kdv;
+                        spq += __bfloat162float(q[ro + c]) * sq_r * kdv;
                     }
                 }
 #pragma unroll
@@ -653,9 +687,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 if (r < len)
-                    a2[hh] = __fadd2_rn(a2[hh], make_float2(fmaxf(bf16_lo(lv[j][hh]), kLogAlphaFloor),
-                                                            fmaxf(bf16_hi(lv[j][hh]), kLogAlphaFloor)));
-                const float2 kb = mul2(mul2(b2, unpack_bf16x2(kx[j][hh])), exp_diff2(a2[hh], zero2));
+                    a2[hh] = __fadd2_rn(a2[hh], make_float2(prep_log_alpha(bf16_lo(lv[j][hh]), prep),
+                                                            prep_log_alpha(bf16_hi(lv[j][hh]), prep)));
+                float2 kn = unpack_bf16x2(kx[j][hh]);
+                if (PREP) kn = mul2(kn, make_float2(inv_nk[r], inv_nk[r]));
+                const float2 kb = mul2(mul2(b2, kn), exp_diff2(a2[hh], zero2));
                 store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + 64 * hh + kc, 64), kb.x, kb.y);
             }
         }
@@ -1084,18 +1120,19 @@ size_t tc_workspace_bytes(int n_chunks, int H, int C) {
 cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                               const float* init_state, void* o, float* final_state, const ChunkMap& cmap,
                               const SeqMap& smap, int n_chunks, int n_seqs, int H, int C, void* tc_ws,
-                              cudaStream_t stream) {
+                              unsigned prep, cudaStream_t stream) {
     if (C != kC) return cudaErrorNotSupported;
     int* err = reinterpret_cast<int*>(tc_ws);
     uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     if (n_chunks > 0) {
-        e = cudaFuncSetAttribute(tc_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIntraAlloc);
+        auto kern = prep ? tc_intra<true> : tc_intra<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIntraAlloc);
         if (e != cudaSuccess) return e;
-        tc_intra<<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
+        kern<<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, prep);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -9,6 +9,9 @@
 // KDA" explainer (pwwt.cn/news/3787313), section 15; order decay -> read ->
 // error -> write: same page, section 8; per-channel alpha: section 9.
 //
+// With kda_prep flags the kernel also normalises q and k, turns raw gate
+// logits into log alpha = -softplus(a) and raw beta logits into sigmoid(b).
+//
 // The step is bound by HBM bandwidth: every state element is loaded once and
 // stored once.  One 256-thread block owns one (sequence, head) state; a warp
 // reads whole rows with 128-bit loads (coalesced), every thread keeps its
@@ -25,7 +28,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
               const Tin* __restrict__ la, const Tin* __restrict__ beta, float* __restrict__ state,
-              Tin* __restrict__ o) {
+              Tin* __restrict__ o, unsigned prep) {
     constexpr int V4 = DV / 4;          // float4 per state row
     constexpr int RPP = kThreads / V4;  // rows covered by one pass of the block
     constexpr int NR = DK / RPP;        // rows held by each thread
@@ -33,7 +36,7 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     __shared__ float sk[DK], sq[DK], sa[DK], sv[DV], su[DV];
     __shared__ __align__(16) float red_r[RPP][DV];
     __shared__ __align__(16) float red_p[RPP][DV];
-    __shared__ float s_kq;
+    __shared__ float s_kq, s_inv_k, s_inv_q;
 
     const int nh = blockIdx.x;
     const int tid = threadIdx.x, col4 = tid % V4, rg = tid / V4;
@@ -46,11 +49,28 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     for (int c = tid; c < DK; c += kThreads) {
         sk[c] = to_f32(k[(size_t)nh * DK + c]);
         sq[c] = to_f32(q[(size_t)nh * DK + c]);
-        sa[c] = expf(fmaxf(to_f32(la[(size_t)nh * DK + c]), kLogAlphaFloor));
+        sa[c] = expf(prep_log_alpha(to_f32(la[(size_t)nh * DK + c]), prep));
     }
     for (int j = tid; j < DV; j += kThreads) sv[j] = to_f32(v[(size_t)nh * DV + j]);
     __syncthreads();
 
+    if (prep & KDA_PREP_QK_L2NORM) {
+        // k and q divided by their norms (fused key/query normalisation)
+        if (tid < 32) {
+            float nk = 0.f, nq = 0.f;
+            for (int c = tid; c < DK; c += 32) { nk += sk[c] * sk[c]; nq += sq[c] * sq[c]; }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+                nq += __shfl_xor_sync(0xffffffffu, nq, off);
+            }
+            if (tid == 0) { s_inv_k = inv_norm_from_sq(nk); s_inv_q = inv_norm_from_sq(nq); }
+        }
+        __syncthreads();
+        const float ik = s_inv_k, iq = s_inv_q;
+        for (int c = tid; c < DK; c += kThreads) { sk[c] *= ik; sq[c] *= iq; }
+        __syncthreads();
+    }
     if (tid < 32) {
         float acc = 0.f;
         for (int c = tid; c < DK; c += 32) acc += sk[c] * sq[c];
@@ -71,7 +91,7 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     reinterpret_cast<float4*>(&red_p[rg][0])[col4] = pacc;
     __syncthreads();
 
-    const float b = to_f32(beta[nh]);
+    const float b = prep_beta(to_f32(beta[nh]), prep);
     for (int j = tid; j < DV; j += kThreads) {
         float r = 0.f, p = 0.f;
 #pragma unroll
@@ -93,24 +113,28 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
 
 template <typename Tin>
 cudaError_t run(const void* q, const void* k, const void* v, const void* la, const void* beta, float* state, int N,
-                int H, int dk, int dv, void* o, cudaStream_t stream) {
+                int H, int dk, int dv, void* o, unsigned prep, cudaStream_t stream) {
     const dim3 grid((unsigned)N * (unsigned)H);
     const Tin *Q = (const Tin*)q, *K = (const Tin*)k, *V = (const Tin*)v, *LA = (const Tin*)la, *BE = (const Tin*)beta;
     Tin* O = (Tin*)o;
-    if (dk == 128 && dv == 128) decode_kernel<Tin, 128, 128><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O);
-    else if (dk == 128 && dv == 64) decode_kernel<Tin, 128, 64><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O);
-    else if (dk == 64 && dv == 128) decode_kernel<Tin, 64, 128><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O);
-    else decode_kernel<Tin, 64, 64><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O);
+    if (dk == 128 && dv == 128)
+        decode_kernel<Tin, 128, 128><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O, prep);
+    else if (dk == 128 && dv == 64)
+        decode_kernel<Tin, 128, 64><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O, prep);
+    else if (dk == 64 && dv == 128)
+        decode_kernel<Tin, 64, 128><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O, prep);
+    else
+        decode_kernel<Tin, 64, 64><<<grid, kThreads, 0, stream>>>(Q, K, V, LA, BE, state, O, prep);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(kda_dtype dtype, const void* q, const void* k, const void* v, const void* log_alpha,
-                          const void* beta, float* state, int N, int H, int dk, int dv, void* o,
+                          const void* beta, float* state, int N, int H, int dk, int dv, void* o, unsigned prep,
                           cudaStream_t stream) {
-    if (dtype == KDA_F32) return run<float>(q, k, v, log_alpha, beta, state, N, H, dk, dv, o, stream);
-    return run<__nv_bfloat16>(q, k, v, log_alpha, beta, state, N, H, dk, dv, o, stream);
+    if (dtype == KDA_F32) return run<float>(q, k, v, log_alpha, beta, state, N, H, dk, dv, o, prep, stream);
+    return run<__nv_bfloat16>(q, k, v, log_alpha, beta, state, N, H, dk, dv, o, prep, stream);
 }
 
 }  // namespace kda

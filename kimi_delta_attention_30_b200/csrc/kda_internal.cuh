@@ -83,6 +83,44 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // keeping cumulative sums finite when alpha = 0 (log alpha = -inf).
 constexpr float kLogAlphaFloor = -100.0f;
 
+// 2^x and log2(x) on the special-function unit (PTX ex2.approx / lg2.approx:
+// about 22 correct bits; subnormal results flush to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---- fused input preprocessing (kda_prep flags) --------------------------------
+// -softplus(a) = -log(1 + e^a), split as max(a, 0) + log(1 + e^-|a|) so that
+// nothing overflows; the second term lies in (0, ln 2] and takes one 2^x and one
+// log2 on the SFU.  When e^-|a| < 2^-24 the sum 1 + e^-|a| rounds to 1 and the
+// term (below 6e-8) is dropped: an absolute error in log alpha of that size,
+// i.e. a relative error of alpha below 6e-8.
+__device__ __forceinline__ float neg_softplus(float a) {
+    const float t = ex2_approx(-fabsf(a) * kLog2e);
+    return -fmaf(lg2_approx(1.f + t), kLn2, fmaxf(a, 0.f));
+}
+// log alpha from the log_alpha argument: as given, or -softplus of a raw gate
+// logit; then the floor every kernel applies.
+__device__ __forceinline__ float prep_log_alpha(float x, unsigned prep) {
+    if (prep & KDA_PREP_GATE_SOFTPLUS) x = neg_softplus(x);
+    return fmaxf(x, kLogAlphaFloor);
+}
+// beta from the beta argument: as given, or the logistic function of a raw logit.
+__device__ __forceinline__ float prep_beta(float x, unsigned prep) {
+    return (prep & KDA_PREP_BETA_SIGMOID) ? 1.f / (1.f + expf(-x)) : x;
+}
+// 1 / ||x|| for the key/query normalisation (0 for an all-zero vector).
+__device__ __forceinline__ float inv_norm_from_sq(float sum_sq) { return sum_sq > 0.f ? rsqrtf(sum_sq) : 0.f; }
+
 // ---- optional per-kernel timing hook (see kda_set_timing_events) -----------
 
 struct TimingHook {
@@ -115,6 +153,6 @@ cudaError_t launch_simt_prefill(kda_dtype dtype, const void* q, const void* k, c
 
 cudaError_t launch_decode(kda_dtype dtype, const void* q, const void* k, const void* v,
                           const void* log_alpha, const void* beta, float* state, int N, int H,
-                          int dk, int dv, void* o, cudaStream_t stream);
+                          int dk, int dv, void* o, unsigned prep, cudaStream_t stream);
 
 }  // namespace kda

@@ -250,16 +250,9 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-// 2^x on the special-function unit (approximate, flushes subnormal results to 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-// exp(a - b) for a pair, as 2^((a - b) log2 e).  The difference is formed first
-// (exact when a and b are close, as cumulative decays within a block are), so
-// large |a|, |b| cost no accuracy.
-constexpr float kLog2e = 1.4426950408889634f;
+// exp(a - b) for a pair, as 2^((a - b) log2 e) (ex2_approx: kda_internal.cuh).
+// The difference is formed first (exact when a and b are close, as cumulative
+// decays within a block are), so large |a|, |b| cost no accuracy.
 __device__ __forceinline__ float2 exp_diff2(float2 a, float2 b) {
     const float2 t = __fmul2_rn(__ffma2_rn(b, make_float2(-1.f, -1.f), a), make_float2(kLog2e, kLog2e));
     return make_float2(ex2_approx(t.x), ex2_approx(t.y));

@@ -17,6 +17,9 @@ All arrays are numpy fp64, token-major: q, k, log_alpha ``[n_tokens, H, dk]``,
 v ``[n_tokens, H, dv]``, beta ``[n_tokens, H]``; sequences are contiguous token
 ranges given by ``seq_start`` (``[n_seqs + 1]`` offsets starting at 0).
 States are ``[n_seqs, H, dk, dv]``.
+
+:mod:`oracle.prep` (numpy) maps raw q / k, gate logits and beta logits to the
+operator's inputs (L2 norm, -softplus, sigmoid).
 """
 from __future__ import annotations
 
@@ -26,6 +29,8 @@ import subprocess
 import threading
 
 import numpy as np
+
+from . import prep  # noqa: F401  (re-exported: oracle.prep.preprocess)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kda_oracle.c")

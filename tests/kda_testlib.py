@@ -45,9 +45,10 @@ def rel_err(got, ref, stored_as=None, both_stored=False) -> float:
     return float(np.max(d) / rms)
 
 
-def oracle_prefill(inp, heads=None, seqs=None, n_threads=0):
+def oracle_prefill(inp, heads=None, seqs=None, n_threads=0, prep=0):
     """Oracle o / final_state for the given heads and sequences of a PrefillInputs.
 
+    ``prep`` (kda_prep flags) runs the inputs through ``oracle.prep`` first.
     Returns (o_ref [n_tok_sel, n_heads, dv], fs_ref [n_seq_sel, n_heads, dk, dv],
     token index array, seq list, head list)."""
     H = inp.q.shape[2]
@@ -68,8 +69,8 @@ def oracle_prefill(inp, heads=None, seqs=None, n_threads=0):
     if inp.init_state is not None:
         si = torch.as_tensor(seqs, device=inp.q.device, dtype=torch.long)
         s0 = to_f64(inp.init_state.index_select(0, si).index_select(1, hi))
-    o, fs = oracle.forward(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.log_alpha), pick(inp.beta),
-                           sub_start, init_state=s0, n_threads=n_threads)
+    q, k, la, beta = oracle.prep.preprocess(pick(inp.q), pick(inp.k), pick(inp.log_alpha), pick(inp.beta), prep)
+    o, fs = oracle.forward(q, k, pick(inp.v), la, beta, sub_start, init_state=s0, n_threads=n_threads)
     return o, fs, tok_idx, seqs, heads
 
 

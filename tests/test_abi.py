@@ -129,6 +129,42 @@ def test_decode_rejects_before_launch():
     assert lib.kda_decode_step(*args, 0, vp(0x70000), 0, 2, 64, 64, vp(0x80000), None) == OK   # N = 0: no work
 
 
+def _call_prep(prep, dtype=0, dk=128, dv=128, C=64, ws=0x100000):
+    lib = kda.lib()
+    vp = ctypes.c_void_p
+    return lib.kda_chunk_fwd_prep(vp(0x10000), vp(0x20000), vp(0x30000), vp(0x40000), vp(0x50000), dtype, prep,
+                                  None, None, 0, 1, 256, 2, dk, dv, C, vp(0x60000), None, vp(ws), 1 << 40, None)
+
+
+def test_prep_entry_points_reject_before_launch():
+    assert _call_prep(8) == E_SHAPE                       # unknown flag
+    assert _call_prep(1 << 31) == E_SHAPE
+    assert _call_prep(7, dtype=1) == E_SHAPE              # fp32: not the tensor-core path
+    assert _call_prep(1, dk=64, dv=64) == E_SHAPE         # d = 64: not the tensor-core path
+    assert _call_prep(7, dtype=5) == E_DTYPE
+    assert _call_prep(7, C=32) == E_CHUNK
+    assert _call_prep(7, ws=0) == E_WS
+    assert _call_prep(7, ws=0x100010) == E_ALIGN
+    lib = kda.lib()
+    vp = ctypes.c_void_p
+    args = [vp(0x10000)] * 5
+    assert lib.kda_decode_step_prep(*args, 0, 8, vp(0x70000), 4, 2, 64, 64, vp(0x80000), None) == E_SHAPE
+    assert lib.kda_decode_step_prep(*args, 3, 7, vp(0x70000), 4, 2, 64, 64, vp(0x80000), None) == E_DTYPE
+    assert lib.kda_decode_step_prep(*args, 0, 7, None, 4, 2, 64, 64, vp(0x80000), None) == E_NULL
+    assert lib.kda_decode_step_prep(*args, 1, 7, vp(0x70000), 0, 2, 64, 64, vp(0x80000), None) == OK   # N = 0
+
+
+def test_prep_flags_match_the_header():
+    text = open(HEADER).read()
+    for name, val in (("KDA_PREP_NONE", kda.PREP_NONE), ("KDA_PREP_QK_L2NORM", kda.PREP_QK_L2NORM),
+                      ("KDA_PREP_GATE_SOFTPLUS", kda.PREP_GATE_SOFTPLUS),
+                      ("KDA_PREP_BETA_SIGMOID", kda.PREP_BETA_SIGMOID)):
+        assert re.search(rf"{name}\s*=\s*{val}\b", text), name
+    import oracle.prep as op
+    assert (op.QK_L2NORM, op.GATE_SOFTPLUS, op.BETA_SIGMOID) == (kda.PREP_QK_L2NORM, kda.PREP_GATE_SOFTPLUS,
+                                                                 kda.PREP_BETA_SIGMOID)
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 4, 1, 64)

@@ -309,3 +309,106 @@ def test_decode_step_is_one_token():
                                   init_state=s0[n:n + 1])
         np.testing.assert_array_equal(o[n], o_n[0])
         np.testing.assert_array_equal(s1[n], f_n[0])
+
+
+# ---------------------------------------------------------- input preprocessing
+# tahou -- "22580倍参数量级" article, tahou.com/article/213680821660188677
+# (alpha between 0 and 1 from an "alpha projection"; alpha = 1 is the delta
+# rule, alpha = 0 clears the memory).  The -softplus / sigmoid / L2-norm maps
+# are this library's reading of how raw projections reach those ranges.
+
+from oracle import prep  # noqa: E402
+
+
+def test_l2_normalize_closed_forms():
+    np.testing.assert_allclose(prep.l2_normalize([3.0, 4.0]), [0.6, 0.8], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(prep.l2_normalize([[0.0, -2.0, 0.0]]), [[0.0, -1.0, 0.0]], atol=0)
+    x = np.random.default_rng(3).standard_normal((4, 3, 7))
+    x[1, 2] = 0.0                                           # all-zero row stays zero, no NaN
+    y = prep.l2_normalize(x)
+    n = np.linalg.norm(y, axis=-1)
+    np.testing.assert_allclose(np.delete(n.reshape(-1), 5), 1.0, atol=1e-14)   # over the last axis
+    assert np.all(y[1, 2] == 0.0)
+    np.testing.assert_allclose(np.linalg.norm(x, axis=-1, keepdims=True) * y, x, atol=1e-14)
+    c = np.random.default_rng(4).uniform(0.1, 10.0, size=(4, 3, 1))
+    np.testing.assert_allclose(prep.l2_normalize(c * x), y, atol=1e-14)       # positive scale invariance
+    np.testing.assert_allclose(prep.l2_normalize(-x), -y, atol=0)
+
+
+def test_gate_softplus_closed_forms():
+    ln3 = np.log(3.0)
+    np.testing.assert_allclose(prep.log_alpha_from_gate([0.0, ln3, -ln3]),
+                               [-np.log(2.0), -np.log(4.0), -np.log(4.0 / 3.0)], rtol=1e-15)
+    np.testing.assert_allclose(np.exp(prep.log_alpha_from_gate(ln3)), 0.25, rtol=1e-15)   # alpha = 1/(1+3)
+    a = np.random.default_rng(5).standard_normal(1000) * 6.0
+    la = prep.log_alpha_from_gate(a)
+    assert np.all(la < 0.0)                                                # alpha in (0, 1)
+    np.testing.assert_allclose(prep.log_alpha_from_gate(-a) - la, a, atol=1e-12)   # sp(x) - sp(-x) = x
+    np.testing.assert_allclose(prep.log_alpha_from_gate(50.0), -50.0, rtol=1e-15)
+    np.testing.assert_allclose(prep.log_alpha_from_gate(-50.0), -np.exp(-50.0), rtol=1e-12)
+    assert prep.log_alpha_from_gate(-800.0) == 0.0                         # alpha = 1: delta rule
+    assert np.exp(prep.log_alpha_from_gate(800.0)) == 0.0                  # alpha = 0: clear
+    h = 1e-5                                                               # d/da softplus = sigmoid
+    d = -(prep.log_alpha_from_gate(a + h) - prep.log_alpha_from_gate(a - h)) / (2 * h)
+    np.testing.assert_allclose(d, prep.beta_from_logit(a), atol=1e-9)
+
+
+def test_beta_sigmoid_closed_forms():
+    ln3 = np.log(3.0)
+    np.testing.assert_allclose(prep.beta_from_logit([0.0, ln3, -ln3]), [0.5, 0.75, 0.25], rtol=1e-15)
+    b = np.random.default_rng(6).standard_normal(1000) * 8.0
+    s = prep.beta_from_logit(b)
+    assert np.all((s > 0.0) & (s < 1.0))
+    np.testing.assert_allclose(s + prep.beta_from_logit(-b), 1.0, atol=1e-15)
+    assert prep.beta_from_logit(-1000.0) == 0.0 and prep.beta_from_logit(1000.0) == 1.0
+    assert np.all(np.diff(prep.beta_from_logit(np.sort(b))) >= 0.0)       # increasing
+
+
+def test_preprocess_flags_select_their_inputs():
+    rng = np.random.default_rng(7)
+    q, k, g = (rng.standard_normal((5, 2, 4)) * 3 for _ in range(3))
+    b = rng.standard_normal((5, 2))
+    for flags in range(8):
+        q2, k2, g2, b2 = prep.preprocess(q, k, g, b, flags)
+        same = lambda x, y: np.array_equal(x, y)
+        assert same(q2, q) != bool(flags & prep.QK_L2NORM)
+        assert same(k2, k) != bool(flags & prep.QK_L2NORM)
+        assert same(g2, g) != bool(flags & prep.GATE_SOFTPLUS)
+        assert same(b2, b) != bool(flags & prep.BETA_SIGMOID)
+        if flags & prep.QK_L2NORM:
+            np.testing.assert_allclose(np.linalg.norm(k2, axis=-1), 1.0, atol=1e-14)
+            np.testing.assert_allclose(np.linalg.norm(q2, axis=-1), 1.0, atol=1e-14)
+
+
+def test_prep_forward_scale_invariance_and_gate_limits():
+    """With the L2 norm, rescaling any token's raw q or k by a positive number
+    changes nothing; gate logits of -800 / +800 give the delta rule / a cleared
+    memory (tahou, Gated DeltaNet section)."""
+    rng = np.random.default_rng(8)
+    T, H, dk, dv = 19, 2, 6, 5
+    q, k, g = (rng.standard_normal((T, H, dk)) for _ in range(3))
+    v = rng.standard_normal((T, H, dv))
+    b = rng.standard_normal((T, H))
+    s0 = rng.standard_normal((1, H, dk, dv))
+    allf = prep.QK_L2NORM | prep.GATE_SOFTPLUS | prep.BETA_SIGMOID
+    o1, f1 = oracle.forward(*_order(prep.preprocess(q, k, g, b, allf), v), [0, T], init_state=s0)
+    cq, ck = rng.uniform(0.05, 20.0, (T, H, 1)), rng.uniform(0.05, 20.0, (T, H, 1))
+    o2, f2 = oracle.forward(*_order(prep.preprocess(cq * q, ck * k, g, b, allf), v), [0, T], init_state=s0)
+    np.testing.assert_allclose(o2, o1, atol=1e-12)
+    np.testing.assert_allclose(f2, f1, atol=1e-12)
+    # all logits -800: alpha = 1 exactly, the delta rule (log alpha = 0)
+    qn, kn, la0, bn = prep.preprocess(q, k, np.full_like(g, -800.0), b, allf)
+    assert np.all(la0 == 0.0)
+    # token 7 with logits +800: alpha = 0, the memory before it is cleared
+    gc = g.copy()
+    gc[7] = 800.0
+    oc, fc = oracle.forward(*_order(prep.preprocess(q, k, gc, b, allf), v), [0, T], init_state=s0)
+    qn, kn, la, bn = prep.preprocess(q, k, gc, b, allf)
+    of, ff = oracle.forward(qn[7:], kn[7:], v[7:], la[7:], bn[7:], [0, T - 7], init_state=np.zeros_like(s0))
+    np.testing.assert_allclose(oc[7:], of, atol=1e-12)
+    np.testing.assert_allclose(fc, ff, atol=1e-12)
+
+
+def _order(pre, v):
+    q, k, la, b = pre
+    return q, k, v, la, b
