@@ -179,7 +179,7 @@ def separate_prep_bytes(n_tok_heads, dk, in_bytes=2):
     return 2 * n_tok_heads * (3 * dk + 1) * in_bytes
 
 
-def measured_traffic(kernel, B, T, H, C):
+def measured_traffic(kernel, B, T, H, C, workload="prefill"):
     """DRAM bytes per launch of `kernel` on this workload from the committed ncu
     table, or None when there is none or the kernel sources changed since."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
@@ -191,7 +191,7 @@ def measured_traffic(kernel, B, T, H, C):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     digest = h.hexdigest()[:16]
-    want = f"prefill_b{B}_h{H}_t{T}_c{C}"
+    want = f"{workload}_b{B}_h{H}_t{T}_c{C}"
     for line in open(path):
         f = line.split()
         if len(f) == 5 and not line.startswith("#") and f[0] == kernel and f[1] == want and f[4] == digest:
@@ -213,7 +213,8 @@ def peaks():
 class OracleSample:
     """The fp64 oracle timed on whole prefill sequences (T = 4096) of the prefill
     workload: one (sequence, head) pair per host thread, as many pairs as fit
-    about `seconds` of wall time (at most the workload's 64 pairs).  Inputs are
+    about `seconds` of wall time (at most the workload's 64 pairs); when all 64
+    take less than that, the whole workload is repeated to fill it.  Inputs are
     drawn once; each call of :meth:`time` reruns the oracle on them."""
 
     def __init__(self, seconds: float, seed: int = 0):
@@ -228,26 +229,30 @@ class OracleSample:
         self.full = (f(inp.q), f(inp.k), f(inp.v), f(inp.log_alpha), to_f64(inp.beta).reshape(T, 64),
                      to_f64(inp.init_state))
         self.seq = inp.seq_start
-        self.n_pairs = 1
+        self.n_pairs, self.reps = 1, 1
         t1 = self.time()
         n = max(1, min(64, int(self.threads * max(1.0, seconds / max(t1, 1e-3)))))
         if n > self.threads:
             n -= n % self.threads              # whole waves of threads
         self.n_pairs = n
+        if n == 64:
+            self.reps = max(1, int(round(seconds / max(self.time(), 1e-3))))
 
     def time(self) -> float:
         n = self.n_pairs
         q, k, v, la, beta, s0 = self.full
         args = (q[:, :n], k[:, :n], v[:, :n], la[:, :n], beta[:, :n])
         t0 = time.perf_counter()
-        self.oracle.forward(*args, self.seq, init_state=s0[:, :n], n_threads=self.threads)
+        for _ in range(self.reps):
+            self.oracle.forward(*args, self.seq, init_state=s0[:, :n], n_threads=self.threads)
         return time.perf_counter() - t0
 
     def tokens(self) -> float:
-        return self.n_pairs * self.T / self.H      # a token carries all H heads
+        return self.reps * self.n_pairs * self.T / self.H      # a token carries all H heads
 
     def describe(self, dt: float) -> str:
-        return (f"{self.n_pairs} (sequence, head) pairs x {self.T} tokens of the prefill workload "
+        return (f"{self.n_pairs} (sequence, head) pairs x {self.T} tokens of the prefill workload"
+                f"{f', {self.reps} passes' if self.reps > 1 else ''} "
                 f"(= {self.tokens():.0f} full {self.H}-head tokens), fp64 token recurrence, "
                 f"{self.threads} threads, {dt:.1f} s")
 
@@ -400,12 +405,42 @@ def main():
             p_total = max_over_ranks(sum(pev[i][0].elapsed_time(pev[i][nk]) for i in range(a.steps)))
             pk_avg = [statistics.mean(pev[i][j].elapsed_time(pev[i][j + 1]) for i in range(a.steps))
                       for j in range(nk)]
+            # the unfused alternative: torch kernels preprocess into bf16 buffers, then the plain operator
+            F = torch.nn.functional
+            qn, kn, lan, bn = (torch.empty_like(t) for t in (raw.q, raw.k, raw.log_alpha, raw.beta))
+
+            def unfused_step():
+                qn.copy_(F.normalize(raw.q.float(), dim=-1))
+                kn.copy_(F.normalize(raw.k.float(), dim=-1))
+                lan.copy_(-F.softplus(raw.log_alpha.float()))
+                bn.copy_(torch.sigmoid(raw.beta.float()))
+                kda.chunk_fwd(qn, kn, raw.v, lan, bn, init_state=raw.init_state, C=C, o=o, final_state=fs,
+                              workspace=ws, algo=a.algo)
+
+            for _ in range(a.warmup):
+                flush.zero_()
+                unfused_step()
+            uev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
+            barrier()
+            torch.cuda.synchronize()
+            for i in range(a.steps):
+                flush.zero_()
+                uev[i][0].record(stream)
+                unfused_step()
+                uev[i][1].record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            u_total = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in uev))
+            del qn, kn, lan, bn
             sep = separate_prep_bytes(tokens * H, dk)
             prep["prefill"] = {
                 "value": job_throughput(world, tokens, a.steps, p_total), "unit": "tokens/s",
                 "ms_per_step": p_total / a.steps, "added_ms_vs_plain": p_total / a.steps - ms_per_step,
-                "kernel_times": {kernels[j]: {"avg_us": pk_avg[j] * 1e3} for j in range(nk)},
+                "kernel_times": {kernels[j]: {"avg_us": pk_avg[j] * 1e3,
+                                              "traffic": measured_traffic(kernels[j], B, T, H, C, "prefill_raw")}
+                                 for j in range(nk)},
                 "separate_pass_bytes": sep, "separate_pass_min_ms": sep / (pk["hbm_gbs"] * 1e9) * 1e3,
+                "unfused_torch_ms_per_step": u_total / a.steps,
                 "config": {"workload": f"prefill B={B} H={H} T={T} d={dk} C={C} bf16, raw q/k (unnormalised), "
                            "gate logits, beta logits; flags QK_L2NORM|GATE_SOFTPLUS|BETA_SIGMOID",
                            "l2": "flushed before every timed step (256 MiB write)"}}

@@ -101,6 +101,7 @@ constexpr uint32_t kTab = 98304;         // tables
 constexpr int kNumTab = 18;              // tau[4], sigma[6], exp(gb)[4], exp(g_C - gb[b+1])[4]
 constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 3 * 64 * 4 + 64;
 constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
+constexpr int kGCol = 192;               // TMEM columns 192-255 hold g until the last product
 constexpr int kAS = 65;                  // row stride of As (floats)
 constexpr int kTS = 68;                  // row stride of Ts (floats; rows 16-byte aligned)
 
@@ -254,8 +255,23 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             mbar_arrive(&mbar_la);
         }
     }
-    const float beta_t =
-        (tid < len && tid < 64) ? prep_beta(__bfloat162float(beta[(size_t)(tok0 + tid) * H + h]), prep) : 0.f;
+    // key / query rows for the normalisation, read row-wise (coalesced) before anything
+    // waits: warp w takes rows 16 (w % 4) .. + 15 of k (w < 4) or q (w >= 4), lane l
+    // channels 4l .. 4l + 3
+    uint2 nu[16];
+    if (PREP && (prep & KDA_PREP_QK_L2NORM)) {
+        const __nv_bfloat16* src = warp < 4 ? k : q;
+        const int rb = 16 * (warp & 3);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            nu[i] = make_uint2(0u, 0u);
+            if (rb + i < len)
+                nu[i] = *reinterpret_cast<const uint2*>(src + ((size_t)(tok0 + rb + i) * H + h) * kD + 4 * lane);
+        }
+    }
+    // beta stays as raw bits until it is stored, so that nothing waits for this load
+    const unsigned short beta_raw =
+        (tid < len && tid < 64) ? reinterpret_cast<const unsigned short*>(beta)[(size_t)(tok0 + tid) * H + h] : 0;
     // ---- log alpha of 8 rows x 4 channels; k, q, v prefetched into L2 ---------
     // (k and q of a channel half are read one phase before the round that uses
     // them, v at the end; holding them in registers through the chunk would push
@@ -284,27 +300,32 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         }
     }
     load_kq(0);
-    // key / query normalisation factors: thread t < 64 takes row t of k, 64 <= t < 128 row t - 64 of q
-    float inv_t = 1.f;
-    if (PREP && (prep & KDA_PREP_QK_L2NORM) && tid < 128) {
-        const int r = tid & 63;
-        inv_t = 0.f;
-        if (r < len) {
-            const uint4* row = reinterpret_cast<const uint4*>((tid < 64 ? k : q) + ((size_t)(tok0 + r) * H + h) * kD);
-            float ss = 0.f;
+    // key / query normalisation factors: the sums of squares are formed here, from
+    // the rows loaded at the start
+    if (PREP && (prep & KDA_PREP_QK_L2NORM)) {
+        float ss[16];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                float f[8];
-                const uint4 u = row[x];
-                f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x); f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
-                f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-            }
-            inv_t = inv_norm_from_sq(ss);
+        for (int i = 0; i < 16; ++i) {
+            const float a = bf16_lo(nu[i].x), b = bf16_hi(nu[i].x), c = bf16_lo(nu[i].y), d = bf16_hi(nu[i].y);
+            ss[i] = fmaf(a, a, fmaf(b, b, fmaf(c, c, d * d)));
         }
+        // halving exchanges (distance 16, 8, 4, 2: each keeps the half of the rows that
+        // the lane's bit selects), then the pair (2m, 2m + 1) adds its two halves of row m
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1) {
+            const bool up = (lane & (2 * w)) != 0;
+#pragma unroll
+            for (int m = 0; m < w; ++m) {
+                const float keep = up ? ss[m + w] : ss[m];
+                const float give = up ? ss[m] : ss[m + w];
+                ss[m] = keep + __shfl_xor_sync(0xffffffffu, give, 2 * w);
+            }
+        }
+        const float tot = ss[0] + __shfl_xor_sync(0xffffffffu, ss[0], 1);
+        if ((lane & 1) == 0) inv_nk[(warp < 4 ? 0 : 64) + 16 * (warp & 3) + (lane >> 1)] = inv_norm_from_sq(tot);
+    } else if (PREP && tid < 128) {
+        inv_nk[tid] = 1.f;   // inv_nk [0, 64) and inv_nq [64, 128) are adjacent
     }
-
     if (!mbar_wait(&mbar_la, 0)) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
@@ -316,12 +337,12 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         for (int hh = 0; hh < 2; ++hh) {
             uint32_t a = 0u;
             if (r < len) a = *reinterpret_cast<const uint32_t*>(sm + kLaStage + r * 256 + (64 * hh + kc) * 2);
-            g[j][2 * hh] = (r < len) ? prep_log_alpha(bf16_lo(a), prep) : 0.f;
-            g[j][2 * hh + 1] = (r < len) ? prep_log_alpha(bf16_hi(a), prep) : 0.f;
+            const float2 l2 = prep_log_alpha2(unpack_bf16x2(a), prep);
+            g[j][2 * hh] = (r < len) ? l2.x : 0.f;
+            g[j][2 * hh + 1] = (r < len) ? l2.y : 0.f;
         }
     }
-    if (tid < 64) sbeta[tid] = beta_t;
-    if (PREP && tid < 128) inv_nk[tid] = inv_t;   // inv_nk [0, 64) and inv_nq [64, 128) are adjacent
+    if (tid < 64) sbeta[tid] = (tid < len) ? prep_beta(__uint_as_float((uint32_t)beta_raw << 16), prep) : 0.f;
     // ---- cumulative log decay (row a1): local prefix, then carries ----------
 #pragma unroll
     for (int j = 1; j < 8; ++j)
@@ -339,6 +360,20 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     for (int j = 0; j < 8; ++j)
 #pragma unroll
         for (int x = 0; x < 4; ++x) g[j][x] += carry[x];
+    // g is kept for the [beta V | beta K exp(g)] operand in TMEM columns 192-255, which no
+    // product writes before that operand is built: warp w stores its 8 rows x 4 channels
+    // in its own sub-partition (lane = its lane), 32 columns from 192 + 32 (w / 4)
+    const uint32_t tbase = sflags[2];
+    const uint32_t t_g = tmem_addr(tbase, 32 * (warp & 3), kGCol + 32 * (warp >> 2));
+    {
+        float gs[16];
+#pragma unroll
+        for (int hj = 0; hj < 2; ++hj) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) gs[i] = g[4 * hj + (i >> 2)][i & 3];
+            tmem_st16(t_g + 16 * hj, gs);
+        }
+    }
     if (tid < 128) gb[tid] = 0.f;
     if (warp & 1) {
 #pragma unroll
@@ -376,7 +411,6 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
     if (tid < 128) reinterpret_cast<float*>(out + kOffGam)[tid] = __expf(gb[4 * 128 + tid]);
 
-    const uint32_t tbase = sflags[2];
     uint32_t phase = 0;
     bool abort = false;
 
@@ -575,21 +609,20 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         bulk_s2g(out + kOffPl, sm + kPl, 8192);
         bulk_commit();
     }
-    // v, k and log alpha for the [beta V | beta K exp(g)] operand are read again
-    // (from L2) while T is solved; g is rebuilt from the carries, so that no
-    // per-row state stays in registers through the middle of the kernel.
-    uint32_t vv[8][2], kx[8][2], lv[8][2];
+    // v and k for the [beta V | beta K exp(g)] operand are read again (from L2)
+    // while T is solved, and g comes back from TMEM, so that no per-row state stays
+    // in registers through the middle of the kernel.
+    uint32_t vv[8][2], kx[8][2];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const int r = r0 + j;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-            vv[j][hh] = kx[j][hh] = lv[j][hh] = 0u;
+            vv[j][hh] = kx[j][hh] = 0u;
             if (r < len && !abort) {
                 const size_t off = ((size_t)(tok0 + r) * H + h) * kD + 64 * hh + kc;
                 vv[j][hh] = *reinterpret_cast<const uint32_t*>(v + off);
                 kx[j][hh] = *reinterpret_cast<const uint32_t*>(k + off);
-                lv[j][hh] = *reinterpret_cast<const uint32_t*>(la + off);
             }
         }
     }
@@ -678,7 +711,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         mma_commit(&mbar);
     }
     if (!abort) {
-        float2 a2[2] = {make_float2(carry[0], carry[1]), make_float2(carry[2], carry[3])};
+        float gs[2][16];
+        tmem_st_wait();
+        tmem_ld16(t_g, gs[0]);
+        tmem_ld16(t_g + 16, gs[1]);
+        tmem_ld_wait();
         const float2 zero2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -686,12 +723,10 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             const float2 b2 = make_float2(sbeta[r], sbeta[r]);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                if (r < len)
-                    a2[hh] = __fadd2_rn(a2[hh], make_float2(prep_log_alpha(bf16_lo(lv[j][hh]), prep),
-                                                            prep_log_alpha(bf16_hi(lv[j][hh]), prep)));
+                const float2 gj = make_float2(gs[j >> 2][4 * (j & 3) + 2 * hh], gs[j >> 2][4 * (j & 3) + 2 * hh + 1]);
                 float2 kn = unpack_bf16x2(kx[j][hh]);
                 if (PREP) kn = mul2(kn, make_float2(inv_nk[r], inv_nk[r]));
-                const float2 kb = mul2(mul2(b2, kn), exp_diff2(a2[hh], zero2));
+                const float2 kb = mul2(mul2(b2, kn), exp_diff2(gj, zero2));
                 store2_split(sm + kXh, sm + kXl, mn_offset(r, 128 + 64 * hh + kc, 64), kb.x, kb.y);
             }
         }
@@ -770,6 +805,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             bulk_wait_read_all();                // shared memory stays valid until read
         }
     }
+    tmem_st_wait();   // the g stash has landed (returns at once unless the kernel aborted early)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

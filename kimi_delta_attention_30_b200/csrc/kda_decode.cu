@@ -54,29 +54,30 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     for (int j = tid; j < DV; j += kThreads) sv[j] = to_f32(v[(size_t)nh * DV + j]);
     __syncthreads();
 
-    if (prep & KDA_PREP_QK_L2NORM) {
-        // k and q divided by their norms (fused key/query normalisation)
-        if (tid < 32) {
-            float nk = 0.f, nq = 0.f;
-            for (int c = tid; c < DK; c += 32) { nk += sk[c] * sk[c]; nq += sq[c] * sq[c]; }
+    // With the key/query normalisation the vectors stay raw: 1/||k|| and 1/||q|| scale
+    // the reduced results (S^T k, S^T q, k.q) and the write, and come out of the same
+    // warp-0 pass as k.q, so the normalisation adds no barrier.
+    const bool l2 = (prep & KDA_PREP_QK_L2NORM) != 0;
+    if (tid < 32) {
+        float acc = 0.f, nk = 0.f, nq = 0.f;
+        for (int c = tid; c < DK; c += 32) {
+            acc += sk[c] * sq[c];
+            if (l2) { nk += sk[c] * sk[c]; nq += sq[c] * sq[c]; }
+        }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
+        for (int off = 16; off > 0; off >>= 1) {
+            acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (l2) {
                 nk += __shfl_xor_sync(0xffffffffu, nk, off);
                 nq += __shfl_xor_sync(0xffffffffu, nq, off);
             }
-            if (tid == 0) { s_inv_k = inv_norm_from_sq(nk); s_inv_q = inv_norm_from_sq(nq); }
         }
-        __syncthreads();
-        const float ik = s_inv_k, iq = s_inv_q;
-        for (int c = tid; c < DK; c += kThreads) { sk[c] *= ik; sq[c] *= iq; }
-        __syncthreads();
-    }
-    if (tid < 32) {
-        float acc = 0.f;
-        for (int c = tid; c < DK; c += 32) acc += sk[c] * sq[c];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (tid == 0) s_kq = acc;
+        if (tid == 0) {
+            const float ik = l2 ? inv_norm_from_sq(nk) : 1.f, iq = l2 ? inv_norm_from_sq(nq) : 1.f;
+            s_inv_k = ik;
+            s_inv_q = iq;
+            s_kq = acc * ik * iq;
+        }
     }
     float4 racc = make_float4(0.f, 0.f, 0.f, 0.f), pacc = racc;
 #pragma unroll
@@ -92,10 +93,13 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     __syncthreads();
 
     const float b = prep_beta(to_f32(beta[nh]), prep);
+    const float ik = s_inv_k, iq = s_inv_q;
     for (int j = tid; j < DV; j += kThreads) {
         float r = 0.f, p = 0.f;
 #pragma unroll
         for (int g = 0; g < RPP; ++g) { r += red_r[g][j]; p += red_p[g][j]; }
+        r *= ik;
+        p *= iq;
         const float u = sv[j] - r;
         su[j] = u;
         o[(size_t)nh * DV + j] = from_f32<Tin>(p + b * s_kq * u);
@@ -105,7 +109,7 @@ decode_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* _
     const float4 u4 = reinterpret_cast<const float4*>(su)[col4];
 #pragma unroll
     for (int i = 0; i < NR; ++i) {
-        const float bk = b * sk[rg + i * RPP];
+        const float bk = b * ik * sk[rg + i * RPP];
         s[i].x += bk * u4.x; s[i].y += bk * u4.y; s[i].z += bk * u4.z; s[i].w += bk * u4.w;
         S4[(rg + i * RPP) * V4 + col4] = s[i];
     }

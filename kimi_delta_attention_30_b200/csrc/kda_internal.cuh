@@ -83,30 +83,36 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // keeping cumulative sums finite when alpha = 0 (log alpha = -inf).
 constexpr float kLogAlphaFloor = -100.0f;
 
-// 2^x and log2(x) on the special-function unit (PTX ex2.approx / lg2.approx:
-// about 22 correct bits; subnormal results flush to 0).
+// 2^x on the special-function unit (PTX ex2.approx: about 22 correct bits;
+// subnormal results flush to 0).
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float lg2_approx(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 // ---- fused input preprocessing (kda_prep flags) --------------------------------
+// log(1 + u) for u in [0, 1] as u q(u): q of degree 8 is the Chebyshev interpolant
+// of log(1 + u) / u at 400 Chebyshev nodes of [0, 1], rewritten in powers of u.
+// In fp32 with fused multiply-adds the absolute error is at most 1.2e-7 (relative
+// 2e-7, and relative 1e-7 as u -> 0), checked in fp64 at 2e6 points.  It runs on
+// the FMA pipe, leaving the special-function unit one 2^x per gate value.
+__host__ __device__ constexpr float l1p_coef(int i) {
+    return i == 0 ? 1.000000000e+00f : i == 1 ? -4.999950230e-01f : i == 2 ? 3.331927061e-01f
+         : i == 3 ? -2.484436929e-01f : i == 4 ? 1.911143064e-01f : i == 5 ? -1.367477030e-01f
+         : i == 6 ? 7.836166769e-02f : i == 7 ? -2.958850749e-02f : 5.253457930e-03f;
+}
+__device__ __forceinline__ float log1p_unit(float u) {
+    float p = l1p_coef(8);
+#pragma unroll
+    for (int i = 7; i >= 0; --i) p = fmaf(p, u, l1p_coef(i));
+    return p * u;
+}
 // -softplus(a) = -log(1 + e^a), split as max(a, 0) + log(1 + e^-|a|) so that
-// nothing overflows; the second term lies in (0, ln 2] and takes one 2^x and one
-// log2 on the SFU.  When e^-|a| < 2^-24 the sum 1 + e^-|a| rounds to 1 and the
-// term (below 6e-8) is dropped: an absolute error in log alpha of that size,
-// i.e. a relative error of alpha below 6e-8.
+// nothing overflows (e^-|a| in (0, 1]).
 __device__ __forceinline__ float neg_softplus(float a) {
-    const float t = ex2_approx(-fabsf(a) * kLog2e);
-    return -fmaf(lg2_approx(1.f + t), kLn2, fmaxf(a, 0.f));
+    return -(fmaxf(a, 0.f) + log1p_unit(ex2_approx(-fabsf(a) * kLog2e)));
 }
 // log alpha from the log_alpha argument: as given, or -softplus of a raw gate
 // logit; then the floor every kernel applies.

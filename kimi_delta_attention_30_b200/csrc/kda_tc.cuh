@@ -258,6 +258,20 @@ __device__ __forceinline__ float2 exp_diff2(float2 a, float2 b) {
     return make_float2(ex2_approx(t.x), ex2_approx(t.y));
 }
 
+// prep_log_alpha (kda_internal.cuh) for a pair, the softplus polynomial as packed
+// fused multiply-adds.
+__device__ __forceinline__ float2 prep_log_alpha2(float2 x, unsigned prep) {
+    if (prep & KDA_PREP_GATE_SOFTPLUS) {
+        const float2 u = make_float2(ex2_approx(-fabsf(x.x) * kLog2e), ex2_approx(-fabsf(x.y) * kLog2e));
+        float2 p = make_float2(l1p_coef(8), l1p_coef(8));
+#pragma unroll
+        for (int i = 7; i >= 0; --i) p = __ffma2_rn(p, u, make_float2(l1p_coef(i), l1p_coef(i)));
+        p = __fmul2_rn(p, u);
+        x = make_float2(-(fmaxf(x.x, 0.f) + p.x), -(fmaxf(x.y, 0.f) + p.y));
+    }
+    return make_float2(fmaxf(x.x, kLogAlphaFloor), fmaxf(x.y, kLogAlphaFloor));
+}
+
 __device__ __forceinline__ void split1(float a, __nv_bfloat16& hi, __nv_bfloat16& lo) {
     hi = __float2bfloat16_rn(a);
     lo = __float2bfloat16_rn(a - __bfloat162float(hi));
