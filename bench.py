@@ -50,6 +50,7 @@ def _args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prep", action="store_true", help="skip the fused-preprocessing timings")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample length")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="profiling aid: run only one part (the JSON line then lacks the other)")
@@ -164,6 +165,12 @@ def kernel_bytes(name, B, T, H, dk, dv, C, in_bytes=2):
     return table.get(name)
 
 
+def algorithmic_flops(B, T, H, dk, dv, C):
+    """FLOPs of the chunk algorithm per call, masked work counted once:
+    6 dk dv + C (3 dk + 2 dv) + C^2 / 3 per token-head."""
+    return B * T * H * (6 * dk * dv + C * (3 * dk + 2 * dv) + C * C / 3)
+
+
 def minimal_bytes(B, T, H, dk, dv, in_bytes=2, with_state=True):
     """q, k, v, log alpha, beta in; o out; initial and final state."""
     tok = B * T * H
@@ -250,6 +257,16 @@ class OracleSample:
     def tokens(self) -> float:
         return self.reps * self.n_pairs * self.T / self.H      # a token carries all H heads
 
+    def single_core(self) -> dict:
+        """One (sequence, head) pair on one thread (tokens/s in full H-head tokens)."""
+        q, k, v, la, beta, s0 = self.full
+        t0 = time.perf_counter()
+        self.oracle.forward(q[:, :1], k[:, :1], v[:, :1], la[:, :1], beta[:, :1], self.seq, init_state=s0[:, :1],
+                            n_threads=1)
+        dt = time.perf_counter() - t0
+        return {"value": self.T / self.H / dt, "unit": "tokens/s", "cores": 1,
+                "sample": f"1 (sequence, head) pair x {self.T} tokens, {dt:.2f} s"}
+
     def describe(self, dt: float) -> str:
         return (f"{self.n_pairs} (sequence, head) pairs x {self.T} tokens of the prefill workload"
                 f"{f', {self.reps} passes' if self.reps > 1 else ''} "
@@ -294,7 +311,7 @@ def main():
     import torch.distributed as dist
 
     import kimi_delta_attention_30_b200 as kda
-    from kda_inputs import RAW_PREP, make_decode_state, make_decode_token, make_prefill
+    from kda_inputs import RAW_PREP, make_decode_state, make_decode_token, make_grad_outputs, make_prefill
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -375,8 +392,14 @@ def main():
                         "algorithmic_bytes": dom_bytes,
                         "peak_source": pk["source"]}
         min_b = minimal_bytes(B, T, H, dk, dv)
-        path_roofline = {"minimal_bytes": min_b, "time_min_us": min_b / (pk["hbm_gbs"] * 1e9) * 1e6,
-                         "frac_of_hbm_bound": (min_b / (pk["hbm_gbs"] * 1e9)) / (ms_per_step / 1e3)}
+        flops = algorithmic_flops(B, T, H, dk, dv, C)
+        t_hbm = min_b / (pk["hbm_gbs"] * 1e9)
+        t_tc = flops / (pk["bf16_tflops"] * 1e12)
+        path_roofline = {"minimal_bytes": min_b, "time_min_us": max(t_hbm, t_tc) * 1e6,
+                         "frac_of_hbm_bound": t_hbm / (ms_per_step / 1e3),
+                         "algorithmic_flops": flops, "tflops": flops / (ms_per_step / 1e3) / 1e12,
+                         "frac_of_tensor_peak": flops / (ms_per_step / 1e3) / (pk["bf16_tflops"] * 1e12),
+                         "time_min_over_time": max(t_hbm, t_tc) / (ms_per_step / 1e3)}
 
         # ------------------------------------------------ prefill, preprocessing fused
         if run_prep:
@@ -445,6 +468,54 @@ def main():
                            "gate logits, beta logits; flags QK_L2NORM|GATE_SOFTPLUS|BETA_SIGMOID",
                            "l2": "flushed before every timed step (256 MiB write)"}}
             del raw
+
+    # ---------------------------------------------------------------- backward
+    bwd = None
+    if run_prefill and not a.no_bwd:
+        d_o, dfs = make_grad_outputs(inp, seed=rank)
+        grads = (torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v),
+                 torch.empty_like(inp.log_alpha), torch.empty_like(inp.beta), torch.empty_like(inp.init_state))
+        bws = torch.empty(kda.bwd_workspace_size(B, T, H, dk, dv, C), dtype=torch.uint8, device=dev)
+        nb = len(kda.BWD_TIMED)
+
+        def bwd_step(evs=None):
+            if evs is not None:
+                kda.set_timing_events(evs)
+            kda.chunk_bwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, d_o, init_state=inp.init_state,
+                          d_final_state=dfs, C=C, grads=grads, workspace=bws)
+
+        for _ in range(a.warmup):
+            flush.zero_()
+            bwd_step()
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(nb + 1)] for _ in range(a.steps)]
+        for row in bev:
+            for e in row:
+                e.record(stream)
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(a.steps):
+            flush.zero_()
+            bwd_step(bev[i])
+        torch.cuda.synchronize()
+        barrier()
+        b_total = max_over_ranks(sum(bev[i][0].elapsed_time(bev[i][nb]) for i in range(a.steps)))
+        b_avg = [statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(a.steps)) for j in range(nb)]
+        # minimal traffic of a backward pass: the forward's inputs and d_o in, five gradients out, plus the
+        # initial state, the final-state gradient and the initial-state gradient
+        tok_h = tokens * H
+        min_bwd = tok_h * ((3 * dk + dv + 1) * 2 + dv * 2 + (3 * dk + dv + 1) * 2) + 3 * B * H * dk * dv * 4
+        b_ms = b_total / a.steps
+        bwd = {"value": job_throughput(world, tokens, a.steps, b_total), "unit": "tokens/s", "ms_per_step": b_ms,
+               "kernel_times": {kda.BWD_TIMED[j]: {"avg_us": b_avg[j] * 1e3, "share": b_avg[j] / max(sum(b_avg), 1e-12)}
+                                for j in range(nb)},
+               "path_roofline": {"minimal_bytes": min_bwd,
+                                 "time_min_us": min_bwd / (pk["hbm_gbs"] * 1e9) * 1e6,
+                                 "frac_of_hbm_bound": min_bwd / (pk["hbm_gbs"] * 1e9) / (b_ms / 1e3)},
+               "gpu_launches": (len(kda.BWD_KERNELS)) * a.steps,
+               "config": {"workload": f"backward of the prefill workload (B={B} H={H} T={T} d={dk}), d_o ~ N(0,1) "
+                                      "bf16, d_final_state ~ N(0, 0.1^2); fp32 CUDA-core kernels, 64-token chunks",
+                          "l2": "flushed before every timed step (256 MiB write)"}}
+        del grads, bws, d_o, dfs
 
     # ---------------------------------------------------------------- decode
     decode = None
@@ -547,7 +618,7 @@ def main():
         smp = OracleSample(a.cpu_seconds)
         dt = smp.time()
         cpu = {"value": smp.tokens() / dt, "unit": "tokens/s", "cores": smp.threads, "kind": "oracle",
-               "sample": smp.describe(dt)}
+               "sample": smp.describe(dt), "single_core": smp.single_core()}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
@@ -558,7 +629,7 @@ def main():
                            "kernels": kernels, "l2": "flushed before every timed step (256 MiB write)",
                            "parallelism": f"replicas x{world} (independent sequences per GPU)"},
                 "roofline": roofline, "path_roofline": path_roofline, "kernel_times": kernel_table,
-                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "prep": prep,
+                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "prep": prep, "backward": bwd,
                 "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clk, "wall_s_timed": t_wall, "gpu": props.name}
         print(json.dumps(line), flush=True)

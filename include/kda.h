@@ -282,6 +282,46 @@ KDA_API kda_status kda_decode_step_prep(const void* q, const void* k, const void
                                         void* o, void* stream);
 
 
+/*
+ * Chunkwise backward pass (training): the gradients of
+ *   L = sum(d_o * o) + sum(d_final_state * final_state)
+ * where o and final_state are what kda_chunk_fwd computes from the same
+ * inputs.  The pages say training needs the chunkwise parallel form ("From
+ * GPT-2 to Kimi K3" essay, pwwt.cn/news/3716252, chunkwise paragraph) but
+ * derive no backward pass; this one is the chain rule applied to that form.
+ *
+ *   q, k, v, log_alpha, beta, init_state, cu_seqlens_host, n_seqs, B, T, H,
+ *   dk, dv, C       : the forward call's arguments (same meaning and layout)
+ *   d_o             : device [B, T, H, dv], dtype `dtype`
+ *   d_final_state   : device [N, H, dk, dv] fp32, or NULL (zero)
+ *   dq, dk, dlog_alpha : device [B, T, H, dk], dtype `dtype` (written)
+ *   dv              : device [B, T, H, dv], dtype `dtype` (written)
+ *   dbeta           : device [B, T, H], dtype `dtype` (written)
+ *   d_init_state    : device [N, H, dk, dv] fp32, or NULL (not written); the
+ *                     gradient for init_state (for a zero initial state when
+ *                     init_state is NULL)
+ *   workspace       : >= kda_chunk_bwd_workspace_size(...) bytes, 256-byte
+ *                     aligned, caller-owned, not read before it is written
+ *
+ * The forward intermediates are recomputed inside the call (on CUDA cores, in
+ * fp32, with 64-token chunks whatever C asks for: the chunk form does not
+ * depend on the chunk length).  dlog_alpha is zero where log_alpha is below
+ * the kernels' floor of -100 (log alpha = -inf included).  Errors as
+ * kda_chunk_fwd; all output pointers must be distinct from the inputs.
+ */
+KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
+                                            const int32_t* cu_seqlens_host, int n_seqs);
+
+KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, kda_dtype dtype,
+                                 const float* init_state, const int32_t* cu_seqlens_host,
+                                 int n_seqs, int B, int T, int H, int dk, int dv, int C,
+                                 const void* d_o, const float* d_final_state,
+                                 void* dq, void* dk_out, void* dv_out, void* dlog_alpha,
+                                 void* dbeta, float* d_init_state,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+
 #ifdef __cplusplus
 }
 #endif

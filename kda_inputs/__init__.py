@@ -263,6 +263,20 @@ def make_decode_token(wl: Workload | str = "decode", step: int = 0, device="cpu"
     return DecodeInputs(q, k, v, la, beta)
 
 
+def make_grad_outputs(inp: PrefillInputs, seed: int = 0, final: bool = True):
+    """Upstream gradients for a prefill batch: d_o ~ N(0,1) in the input dtype,
+    shaped like o, and (if ``final``) d_final_state ~ N(0, 0.1^2) fp32 shaped like
+    the states."""
+    dev = inp.q.device
+    B, T, H, _ = inp.q.shape
+    dv = inp.v.shape[-1]
+    dk = inp.q.shape[-1]
+    g = _gen(dev, seed, 9_000_001)
+    d_o = _normal((B, T, H, dv), g, dev).to(inp.q.dtype)
+    dfs = _normal((inp.n_seqs, H, dk, dv), g, dev) * 0.1 if final else None
+    return d_o, dfs
+
+
 def to_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a (bf16 / fp32) tensor to a host fp64 array."""
     return t.detach().to("cpu").to(torch.float64).numpy()

@@ -10,6 +10,7 @@ Calls:
 * :func:`chunk_fwd` -- chunkwise prefill (``kda_chunk_fwd``).
 * :func:`decode_step` -- one recurrent step, state updated in place
   (``kda_decode_step``).
+* :func:`chunk_bwd` -- gradients of the prefill for training (``kda_chunk_bwd``).
 
 Both take ``prep`` (a bitwise OR of the ``PREP_*`` flags): raw q/k, gate
 logits and beta logits are then normalised / activated inside the kernels
@@ -70,6 +71,11 @@ def _declare(lib):
     lib.kda_chunk_fwd_prep.restype = c_int
     lib.kda_decode_step_prep.argtypes = [vp] * 5 + [c_int, ctypes.c_uint, vp] + [c_int] * 4 + [vp, vp]
     lib.kda_decode_step_prep.restype = c_int
+    lib.kda_chunk_bwd_workspace_size.argtypes = [c_int] * 6 + [i32p, c_int]
+    lib.kda_chunk_bwd_workspace_size.restype = c_size
+    lib.kda_chunk_bwd.argtypes = [vp] * 5 + [c_int, vp, i32p, c_int] + [c_int] * 6 + [vp, vp] + [vp] * 6 + \
+        [vp, c_size, vp]
+    lib.kda_chunk_bwd.restype = c_int
     lib.kda_set_timing_events.argtypes = [ctypes.POINTER(vp), c_int]
     lib.kda_set_timing_events.restype = c_int
     lib.kda_chunk_fwd_kernels.argtypes = [c_int] * 7 + [i32p, c_int, c_int, ctypes.POINTER(ctypes.c_char_p), c_int]
@@ -107,7 +113,8 @@ def exported_symbols():
     return ["kda_status_string", "kda_version", "kda_chunk_fwd_workspace_size",
             "kda_chunk_fwd_workspace_size_ex", "kda_chunk_fwd", "kda_chunk_fwd_ex",
             "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
-            "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep"]
+            "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep", "kda_chunk_bwd_workspace_size",
+            "kda_chunk_bwd"]
 
 
 def _ptr(t):
@@ -227,6 +234,55 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
     if st != 0:
         raise KdaError(st, "kda_chunk_fwd")
     return o, final_state
+
+
+BWD_KERNELS = ["k1_cumsum", "k2_wy", "k3_state", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
+# the timing hook's marks of kda_chunk_bwd: start, k1..k3 recompute, kb_p, kb_chain, kb_a, kb_b, kb_c
+BWD_TIMED = ["recompute (k1-k3)", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
+
+
+def bwd_workspace_size(B, T, H, dk, dv, C=64, cu_seqlens=None) -> int:
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    return int(lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, C, cu, n))
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, d_o, init_state=None, d_final_state=None, cu_seqlens=None, C: int = 64,
+              need_d_init_state: bool = True, grads=None, workspace=None, stream=None):
+    """Gradients of ``sum(d_o * o) + sum(d_final_state * final_state)`` for the
+    prefill :func:`chunk_fwd` computes from the same inputs.  Returns
+    ``(dq, dk, dv, dlog_alpha, dbeta, d_init_state)`` (the first five in the
+    input dtype, ``d_init_state`` fp32 ``[N, H, dk, dv]`` or None).  ``grads``
+    may pass preallocated output tensors in that order."""
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta), ("d_o", d_o)):
+        _check_cuda(name, t, dt)
+    _check_cuda("init_state", init_state, torch.float32)
+    _check_cuda("d_final_state", d_final_state, torch.float32)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu, n_seqs, _keep = _cu_arg(cu_seqlens)
+    N = n_seqs if cu_seqlens is not None else B
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_alpha),
+                 torch.empty_like(beta),
+                 torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if need_d_init_state else None)
+    dq, dk_, dv_, dla, dbeta, dinit = grads
+    for name, t in (("dq", dq), ("dk", dk_), ("dv", dv_), ("dlog_alpha", dla), ("dbeta", dbeta)):
+        _check_cuda(name, t, dt)
+    _check_cuda("d_init_state", dinit, torch.float32)
+    need = lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, C, cu, n_seqs)
+    if workspace is None:
+        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
+    _check_cuda("workspace", workspace)
+    st = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], _ptr(init_state),
+                             cu, n_seqs, B, T, H, dk, dv, C, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk_),
+                             _ptr(dv_), _ptr(dla), _ptr(dbeta), _ptr(dinit), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != 0:
+        raise KdaError(st, "kda_chunk_bwd")
+    return dq, dk_, dv_, dla, dbeta, dinit
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20   # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h

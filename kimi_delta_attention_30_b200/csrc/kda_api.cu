@@ -83,7 +83,7 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, int C, const int32_t* 
 size_t table_bytes(const Plan& p) { return p.varlen ? align_up(2 * sizeof(SeqInfo) * (size_t)p.n_seqs) : 0; }
 
 struct SimtLayout {
-    size_t off[5];
+    size_t off[6];
     size_t total;
 };
 
@@ -96,9 +96,35 @@ SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
     L.off[2] = o; o = align_up(o + tok * dk * sizeof(float));               // Wk
     L.off[3] = o; o = align_up(o + tok * dv * sizeof(float));               // W
     L.off[4] = o; o = align_up(o + (size_t)p.n_chunks * H * dk * dv * sizeof(float));  // S_chunk
+    L.off[5] = o; o = align_up(o + tok * dk * sizeof(float));               // g, low part
     L.total = o;
     return L;
 }
+
+// Backward workspace: the CUDA-core forward's scratch, then the gradient scratch.
+struct BwdLayout {
+    SimtLayout fwd;
+    size_t off[9];
+    size_t total;
+};
+
+BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C) {
+    BwdLayout L;
+    L.fwd = simt_layout(p, H, dk, dv);
+    size_t o = L.fwd.total;
+    const size_t tok = (size_t)p.total_tokens * H;
+    const size_t ch = (size_t)p.n_chunks * H;
+    const size_t sizes[9] = {ch * dk * dv, tok * dv, ch * C * C, tok * dk, tok * dk, tok * dk, tok * dk,
+                             ch * dk, ch * C * C};   // dS_chunk dW P dQg dKd dWk dKg dGam dAt
+    for (int i = 0; i < 9; ++i) {
+        L.off[i] = o;
+        o = align_up(o + sizes[i] * sizeof(float));
+    }
+    L.total = o;
+    return L;
+}
+
+constexpr int kBwdChunk = 64;   // the backward kernels tile by 64 tokens
 
 bool tc_shape(kda_dtype dtype, int dk, int dv, int C) {
     return dtype == KDA_BF16 && dk == 128 && dv == 128 && tc_supports(C);
@@ -245,8 +271,8 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
     cudaError_t err;
     if (algo == KDA_ALGO_SIMT) {
         SimtLayout L = simt_layout(p, H, dk, dv);
-        SimtWorkspace w{(float*)(ws + L.off[0]), (float*)(ws + L.off[1]), (float*)(ws + L.off[2]),
-                        (float*)(ws + L.off[3]), (float*)(ws + L.off[4])};
+        SimtWorkspace w{(float*)(ws + L.off[0]), (float*)(ws + L.off[5]), (float*)(ws + L.off[1]),
+                        (float*)(ws + L.off[2]), (float*)(ws + L.off[3]), (float*)(ws + L.off[4])};
         err = launch_simt_prefill(dtype, q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap,
                                   p.n_chunks, p.n_seqs, H, dk, dv, C, w, s);
     } else {
@@ -325,6 +351,74 @@ int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype 
     const int n = (algo == KDA_ALGO_TC) ? kTcKernelCount : 4;
     for (int i = 0; names && i < n && i < max_names; ++i) names[i] = list[i];
     return n;
+}
+
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C, const int32_t* cu_seqlens_host,
+                                    int n_seqs) {
+    Plan p;
+    if (C != 64 && C != 128) return 0;
+    if (make_plan(B, T, H, dk, dv, kBwdChunk, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
+    return bwd_layout(p, H, dk, dv, kBwdChunk).total;
+}
+
+kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                         kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs, int B,
+                         int T, int H, int dk, int dv, int C, const void* d_o, const float* d_final_state, void* dq,
+                         void* dk_out, void* dv_out, void* dlog_alpha, void* dbeta, float* d_init_state,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (C != 64 && C != 128) return KDA_ERR_CHUNK;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, kBwdChunk, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    const bool has_tokens = p.total_tokens > 0;
+    if (has_tokens && (!q || !k || !v || !log_alpha || !beta || !d_o || !dq || !dk_out || !dv_out || !dlog_alpha ||
+                       !dbeta))
+        return KDA_ERR_NULL;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq, dk_out, dv_out,
+                          dlog_alpha, dbeta, d_init_state};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return KDA_ERR_ALIGN;
+    const BwdLayout L = bwd_layout(p, H, dk, dv, kBwdChunk);
+    if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+    if ((st = check_device()) != KDA_OK) return st;
+    if (p.n_seqs == 0) return KDA_OK;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    const int Cb = kBwdChunk;
+    const int ncps = (int)((T + Cb - 1) / Cb);
+    ChunkMap cmap{nullptr, p.n_seqs, T, Cb, ncps};
+    SeqMap smap{nullptr, T, Cb, ncps};
+    if (p.varlen) {
+        std::vector<SeqInfo> both(p.natural);
+        both.insert(both.end(), p.by_len.begin(), p.by_len.end());
+        if (cudaMemcpyAsync(ws, both.data(), both.size() * sizeof(SeqInfo), cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        cmap.seqs = (const SeqInfo*)ws;
+        smap.order = (const SeqInfo*)ws + p.n_seqs;
+    }
+    auto f = [&](size_t off) { return (float*)(ws + off); };
+    BwdWorkspace w;
+    w.fwd = SimtWorkspace{f(L.fwd.off[0]), f(L.fwd.off[5]), f(L.fwd.off[1]), f(L.fwd.off[2]), f(L.fwd.off[3]),
+                          f(L.fwd.off[4])};
+    w.dS_chunk = f(L.off[0]);
+    w.dW = f(L.off[1]);
+    w.P = f(L.off[2]);
+    w.dQg = f(L.off[3]);
+    w.dKd = f(L.off[4]);
+    w.dWk = f(L.off[5]);
+    w.dKg = f(L.off[6]);
+    w.dGam = f(L.off[7]);
+    w.dAt = f(L.off[8]);
+    timing_mark(s, 0);
+    cudaError_t err = launch_simt_backward(dtype, q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq,
+                                           dk_out, dv_out, dlog_alpha, dbeta, d_init_state, cmap, smap, p.n_chunks,
+                                           p.n_seqs, H, dk, dv, Cb, w, s);
+    timing_hook().n = 0;
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,

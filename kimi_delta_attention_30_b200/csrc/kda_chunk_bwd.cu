@@ -1,0 +1,563 @@
+// Chunkwise KDA backward pass (CUDA cores, fp32 arithmetic): the gradients of
+// the loss  L = <dO, O> + <dS_final, S_final>  with respect to q, k, v,
+// log alpha, beta and the initial state.
+//
+// The pages say training needs the chunkwise parallel form ("From GPT-2 to
+// Kimi K3" essay, pwwt.cn/news/3716252, chunkwise paragraph) but derive no
+// backward pass; this one is the chain rule applied to the chunk form that
+// the forward kernels compute.  Per chunk, with start state S, cumulative
+// decay g (rows r = 0..L-1), Gam = exp(g_{L-1}) and
+//   Qg = Q . exp(g),  Kg = K . exp(g),  Kd = K . exp(g_{L-1} - g),
+//   At[r][i] = sum_c k_rc k_ic exp(g_rc - g_ic)   (i < r),  A = Diag(beta) At,
+//   P[r][i]  = sum_c q_rc k_ic exp(g_rc - g_ic)   (i <= r),
+//   U = (I + A)^-1 Diag(beta) V,  Wk = (I + A)^-1 Diag(beta) Kg,  W = U - Wk S,
+//   O = Qg S + P W,   S' = Diag(Gam) S + Kd^T W,
+// the chunk is affine in S, so the state gradient runs backwards over the
+// chunks (kb_chain):
+//   dW = P^T dO + Kd dS',    dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW,
+// and everything else is chunk-parallel (kb_a, kb_b, kb_c):
+//   dQg = dO S^T, dKd = W dS'^T, dWk = -dW S^T, dGam = rowsum(dS' . S),
+//   dP = dO W^T (i <= r),
+//   [Y | Z] = (I + A)^-T [dW | dWk]           (back substitution),
+//   dv = Diag(beta) Y,  dKg = Diag(beta) Z,
+//   dA = -(Y U^T + Z Wk^T) (i < r),  dAt = Diag(beta) dA,
+//   dbeta_r = v_r.Y_r + Kg_r.Z_r + sum_i dA_ri At_ri,
+// then the pairwise terms of At and P give dq and dk (with E = exp(g_r - g_i)),
+// the elementwise factors add theirs, and dlog alpha sums, for each token j,
+// exactly the terms whose decay spans it (see kb_c).
+// Every decay is exp of a non-positive difference, as in the forward split, of
+// cumulative decays held as fp32 (hi, lo) pairs (exp_gdiff, exp_g).
+// The forward intermediates (g, U, Wk, W, chunk start states) are recomputed by
+// the CUDA-core forward kernels.
+#include <algorithm>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kT = 256;
+constexpr int kBV = 32;       // d_v columns per chain block / per tile
+constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
+
+__device__ __forceinline__ float wsum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ size_t tok_off(int t, int H, int h, int d) { return ((size_t)t * H + h) * d; }
+
+// P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic) for i <= r < L, zero elsewhere.
+// One block per (chunk, head); shared Qs, Ks, Gs, GLs [C][dk].
+template <typename Tin>
+__global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                           const float* __restrict__ g, const float* __restrict__ gl,
+                                           float* __restrict__ P, ChunkMap cmap, int H, int dk, int C) {
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    float* Qs = smem;
+    float* Ks = Qs + C * dk;
+    float* Gs = Ks + C * dk;
+    float* GLs = Gs + C * dk;
+    for (int e = tid; e < len * dk; e += kT) {
+        const int r = e / dk, c = e - r * dk;
+        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
+        Qs[e] = to_f32(q[off]);
+        Ks[e] = to_f32(k[off]);
+        Gs[e] = g[off];
+        GLs[e] = gl[off];
+    }
+    __syncthreads();
+    float* Pc = P + ((size_t)blockIdx.x * H + h) * C * C;
+    for (int p = warp; p < C * C; p += kT / 32) {
+        const int r = p / C, i = p - r * C;
+        float s = 0.f;
+        if (r < len && i <= r) {
+            for (int c = lane; c < dk; c += 32)
+                s += Qs[r * dk + c] * Ks[i * dk + c] *
+                     exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
+            s = wsum(s);
+        }
+        if (lane == 0) Pc[p] = s;
+    }
+}
+
+// Reverse chain over one sequence's chunks, one block per (sequence, head,
+// kBV state columns).  Stores each chunk's end-state gradient dS' and dW, and
+// the initial-state gradient.  Shared: dS [dk][kBV], M1 [C][dk] (Kd, then Qg),
+// M2 [C][dk] (Wk), dOs [C][kBV], dWs [C][kBV], Ps [C][C], gC, gCl [dk].
+template <typename Tin>
+__global__ void __launch_bounds__(kT) kb_chain(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                               const float* __restrict__ g, const float* __restrict__ gl,
+                                               const float* __restrict__ Wk,
+                                               const float* __restrict__ P, const Tin* __restrict__ d_o,
+                                               const float* __restrict__ d_final, float* __restrict__ dS_chunk,
+                                               float* __restrict__ dW, float* __restrict__ d_init, SeqMap smap,
+                                               int H, int dk, int dv, int C) {
+    extern __shared__ float smem[];
+    const SeqInfo sq = smap.get(blockIdx.x);
+    const int h = blockIdx.y, j0 = blockIdx.z * kBV, tid = threadIdx.x;
+    float* dS = smem;
+    float* M1 = dS + dk * kBV;
+    float* M2 = M1 + C * dk;
+    float* dOs = M2 + C * dk;
+    float* dWs = dOs + C * kBV;
+    float* Ps = dWs + C * kBV;
+    float* gC = Ps + C * C;
+    float* gCl = gC + dk;
+
+    const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
+    for (int e = tid; e < dk * kBV; e += kT) {
+        const int c = e / kBV, j = e - c * kBV;
+        dS[e] = d_final ? d_final[st_base + (size_t)c * dv + j0 + j] : 0.f;
+    }
+    __syncthreads();
+    const int nch = (sq.len + C - 1) / C;
+    for (int n = nch - 1; n >= 0; --n) {
+        const int t0 = sq.tok0 + n * C;
+        const int L = min(C, sq.len - n * C);
+        const size_t chunk = (size_t)sq.chunk0 + n;
+        const size_t sc_base = (chunk * H + h) * dk * dv;
+        for (int e = tid; e < dk * kBV; e += kT) {
+            const int c = e / kBV, j = e - c * kBV;
+            dS_chunk[sc_base + (size_t)c * dv + j0 + j] = dS[e];
+        }
+        const float* Pc = P + (chunk * H + h) * C * C;
+        for (int e = tid; e < C * C; e += kT) Ps[e] = Pc[e];
+        for (int e = tid; e < L * kBV; e += kT) {
+            const int r = e / kBV, j = e - r * kBV;
+            dOs[e] = to_f32(d_o[tok_off(t0 + r, H, h, dv) + j0 + j]);
+        }
+        for (int c = tid; c < dk; c += kT) {
+            gC[c] = g[tok_off(t0 + L - 1, H, h, dk) + c];
+            gCl[c] = gl[tok_off(t0 + L - 1, H, h, dk) + c];
+        }
+        __syncthreads();
+        for (int e = tid; e < L * dk; e += kT) {
+            const int r = e / dk, c = e - r * dk;
+            const size_t off = tok_off(t0 + r, H, h, dk) + c;
+            M1[e] = to_f32(k[off]) * exp_gdiff(gC[c], gCl[c], g[off], gl[off]);   // Kd
+            M2[e] = Wk[off];
+        }
+        __syncthreads();
+        // dW = P^T dO + Kd dS'
+        for (int e = tid; e < L * kBV; e += kT) {
+            const int i = e / kBV, j = e - i * kBV;
+            float s = 0.f;
+            for (int r = i; r < L; ++r) s += Ps[r * C + i] * dOs[r * kBV + j];
+            for (int c = 0; c < dk; ++c) s += M1[i * dk + c] * dS[c * kBV + j];
+            dWs[e] = s;
+            dW[tok_off(t0 + i, H, h, dv) + j0 + j] = s;
+        }
+        __syncthreads();
+        for (int e = tid; e < L * dk; e += kT) {
+            const int r = e / dk, c = e - r * dk;
+            const size_t off = tok_off(t0 + r, H, h, dk) + c;
+            M1[e] = to_f32(q[off]) * exp_g(g[off], gl[off]);                     // Qg
+        }
+        __syncthreads();
+        // dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW
+        for (int e = tid; e < dk * kBV; e += kT) {
+            const int c = e / kBV, j = e - c * kBV;
+            float s = exp_g(gC[c], gCl[c]) * dS[e];
+            for (int r = 0; r < L; ++r) s += M1[r * dk + c] * dOs[r * kBV + j] - M2[r * dk + c] * dWs[r * kBV + j];
+            dS[e] = s;
+        }
+        __syncthreads();
+    }
+    if (d_init) {
+        for (int e = tid; e < dk * kBV; e += kT) {
+            const int c = e / kBV, j = e - c * kBV;
+            d_init[st_base + (size_t)c * dv + j0 + j] = dS[e];
+        }
+    }
+}
+
+// Per (chunk, head): dQg = dO S^T, dKd = W dS'^T, dWk = -dW S^T (rows x DK),
+// dGam = rowsum(dS' . S), and dP = dO W^T (i <= r, written over P).  d_v is
+// walked in tiles of kBV columns.  Thread t owns channel c = t % DK of rows
+// r = t / DK + m (kT / DK).  Shared: St, dSt [kBV][DK] (transposed tiles),
+// dOs, Ws, dWs [C][kBP].
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const float* __restrict__ W,
+                                           const float* __restrict__ dW, const float* __restrict__ S_chunk,
+                                           const float* __restrict__ dS_chunk, float* __restrict__ dQg,
+                                           float* __restrict__ dKd, float* __restrict__ dWk, float* __restrict__ dGam,
+                                           float* __restrict__ dP, ChunkMap cmap, int H, int dv) {
+    constexpr int C = 64;
+    constexpr int NRG = kT / DK;   // row groups
+    constexpr int MR = C / NRG;    // rows per thread
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, c = tid % DK, rg = tid / DK;
+    float* St = smem;
+    float* dSt = St + kBV * DK;
+    float* dOs = dSt + kBV * DK;
+    float* Ws = dOs + C * kBP;
+    float* dWs = Ws + C * kBP;
+    const size_t chunk = blockIdx.x;
+    const size_t sc_base = (chunk * H + h) * DK * dv;
+    float aQ[MR], aD[MR], aW[MR];
+#pragma unroll
+    for (int m = 0; m < MR; ++m) aQ[m] = aD[m] = aW[m] = 0.f;
+    float gam = 0.f;
+    // dP: thread t owns column i = t % 64 of rows r = t / 64 + 4 m (m < 16)
+    const int pi = tid & 63, pr = tid >> 6;
+    float aP[C / 4];
+#pragma unroll
+    for (int m = 0; m < C / 4; ++m) aP[m] = 0.f;
+    for (int jt = 0; jt < dv; jt += kBV) {
+        for (int e = tid; e < kBV * DK; e += kT) {
+            const int cc = e / kBV, j = e - cc * kBV;
+            St[j * DK + cc] = S_chunk[sc_base + (size_t)cc * dv + jt + j];
+            dSt[j * DK + cc] = dS_chunk[sc_base + (size_t)cc * dv + jt + j];
+        }
+        for (int e = tid; e < C * kBV; e += kT) {
+            const int r = e / kBV, j = e - r * kBV;
+            float a = 0.f, b = 0.f, d = 0.f;
+            if (r < len) {
+                a = to_f32(d_o[tok_off(tok0 + r, H, h, dv) + jt + j]);
+                b = W[tok_off(tok0 + r, H, h, dv) + jt + j];
+                d = dW[tok_off(tok0 + r, H, h, dv) + jt + j];
+            }
+            dOs[r * kBP + j] = a;
+            Ws[r * kBP + j] = b;
+            dWs[r * kBP + j] = d;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < MR; ++m) {
+            const int r = rg + m * NRG;
+#pragma unroll 8
+            for (int j = 0; j < kBV; ++j) {
+                const float s = St[j * DK + c], ds = dSt[j * DK + c];
+                aQ[m] += dOs[r * kBP + j] * s;
+                aD[m] += Ws[r * kBP + j] * ds;
+                aW[m] -= dWs[r * kBP + j] * s;
+            }
+        }
+        if (rg == 0)
+            for (int j = 0; j < kBV; ++j) gam += dSt[j * DK + c] * St[j * DK + c];
+#pragma unroll
+        for (int m = 0; m < C / 4; ++m) {
+            const int r = pr + 4 * m;
+#pragma unroll 8
+            for (int j = 0; j < kBV; ++j) aP[m] += dOs[r * kBP + j] * Ws[pi * kBP + j];
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int m = 0; m < MR; ++m) {
+        const int r = rg + m * NRG;
+        if (r < len) {
+            const size_t off = tok_off(tok0 + r, H, h, DK) + c;
+            dQg[off] = aQ[m];
+            dKd[off] = aD[m];
+            dWk[off] = aW[m];
+        }
+    }
+    if (rg == 0) dGam[(chunk * H + h) * DK + c] = gam;
+    float* dPc = dP + (chunk * H + h) * C * C;
+#pragma unroll
+    for (int m = 0; m < C / 4; ++m) {
+        const int r = pr + 4 * m;
+        dPc[r * C + pi] = (r < len && pi <= r) ? aP[m] : 0.f;
+    }
+}
+
+// Per (chunk, head): At, the back substitution for [Y | Z], dv, dKg, dbeta and
+// dAt.  Shared: At, dA [C][C], bs, db [C], R: Ks, Gs, GLs [C][dk] (phase 1), then
+// X = [Y | Z] [C][dv + dk]; after R (max(3 C dk, C (dv + dk)) floats) UW = [U | Wk]
+// [C][dv + dk].
+template <typename Tin>
+__global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin* __restrict__ v,
+                                           const Tin* __restrict__ beta, const float* __restrict__ g,
+                                           const float* __restrict__ gl,
+                                           const float* __restrict__ U, const float* __restrict__ Wk,
+                                           const float* __restrict__ dW, const float* __restrict__ dWk,
+                                           Tin* __restrict__ dv_out, Tin* __restrict__ dbeta_out,
+                                           float* __restrict__ dKg, float* __restrict__ dAt, ChunkMap cmap, int H,
+                                           int dk, int dv, int C) {
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ncol = dv + dk;
+    float* At = smem;
+    float* dA = At + C * C;
+    float* bs = dA + C * C;
+    float* db = bs + C;
+    float* R = db + C;
+    float* Ks = R;
+    float* Gs = R + C * dk;
+    float* GLs = Gs + C * dk;
+    float* X = R;
+    float* UW = R + max(3 * C * dk, C * ncol);
+
+    for (int e = tid; e < len * dk; e += kT) {
+        const int r = e / dk, c = e - r * dk;
+        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
+        Ks[e] = to_f32(k[off]);
+        Gs[e] = g[off];
+        GLs[e] = gl[off];
+    }
+    for (int r = tid; r < C; r += kT) {
+        bs[r] = r < len ? to_f32(beta[(size_t)(tok0 + r) * H + h]) : 0.f;
+        db[r] = 0.f;
+    }
+    for (int e = tid; e < len * ncol; e += kT) {
+        const int r = e / ncol, j = e - r * ncol;
+        UW[e] = j < dv ? U[tok_off(tok0 + r, H, h, dv) + j] : Wk[tok_off(tok0 + r, H, h, dk) + j - dv];
+    }
+    __syncthreads();
+    for (int p = warp; p < C * C; p += kT / 32) {
+        const int r = p / C, i = p - r * C;
+        float s = 0.f;
+        if (r < len && i < r) {
+            for (int c = lane; c < dk; c += 32)
+                s += Ks[r * dk + c] * Ks[i * dk + c] *
+                     exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
+            s = wsum(s);
+        }
+        if (lane == 0) At[p] = s;
+    }
+    __syncthreads();
+    // (I + A)^T [Y | Z] = [dW | dWk], one column per thread, rows from the last
+    for (int j = tid; j < ncol; j += kT) {
+        for (int r = len - 1; r >= 0; --r) {
+            float s = j < dv ? dW[tok_off(tok0 + r, H, h, dv) + j] : dWk[tok_off(tok0 + r, H, h, dk) + j - dv];
+            for (int i = r + 1; i < len; ++i) s -= bs[i] * At[i * C + r] * X[i * ncol + j];
+            X[r * ncol + j] = s;
+        }
+    }
+    __syncthreads();
+    // dv = beta Y, dKg = beta Z, dbeta_r = v_r . Y_r + Kg_r . Z_r (one warp per row)
+    for (int r = warp; r < len; r += kT / 32) {
+        const float b = bs[r];
+        float s = 0.f;
+        for (int j = lane; j < ncol; j += 32) {
+            const float x = X[r * ncol + j];
+            if (j < dv) {
+                const size_t off = tok_off(tok0 + r, H, h, dv) + j;
+                dv_out[off] = from_f32<Tin>(b * x);
+                s += to_f32(v[off]) * x;
+            } else {
+                const size_t off = tok_off(tok0 + r, H, h, dk) + j - dv;
+                dKg[off] = b * x;
+                s += to_f32(k[off]) * exp_g(g[off], gl[off]) * x;
+            }
+        }
+        s = wsum(s);
+        if (lane == 0) db[r] = s;
+    }
+    // dA = -(Y U^T + Z Wk^T), i < r (one warp per pair)
+    for (int p = warp; p < C * C; p += kT / 32) {
+        const int r = p / C, i = p - r * C;
+        float s = 0.f;
+        if (r < len && i < r) {
+            for (int j = lane; j < ncol; j += 32) s += X[r * ncol + j] * UW[i * ncol + j];
+            s = -wsum(s);
+        }
+        if (lane == 0) dA[p] = s;
+    }
+    __syncthreads();
+    float* dAc = dAt + ((size_t)blockIdx.x * H + h) * C * C;
+    for (int r = tid; r < C; r += kT) {
+        float s = db[r];
+        for (int i = 0; i < r; ++i) s += dA[r * C + i] * At[r * C + i];
+        if (r < len) dbeta_out[(size_t)(tok0 + r) * H + h] = from_f32<Tin>(s);
+    }
+    for (int e = tid; e < C * C; e += kT) dAc[e] = bs[e / C] * dA[e];
+}
+
+// Per (chunk, head): the pairwise terms of At and P, the elementwise factors,
+// and dlog alpha.  A pairwise term T_ri = (dAt_ri k_r + dP_ri q_r) k_i E_ri depends
+// on log alpha_j exactly for i < j <= r, so its share of dlog alpha_j is
+// F(j) = sum_{r >= j} sum_{i < j} T_ri, accumulated from each row's prefix sums
+// over i (no term is added and later cancelled, as a reverse cumulative sum of
+// row minus column sums would do).  Likewise Qg_r, Kg_r depend on log alpha_j for
+// j <= r, Kd_r for r < j, and Gam for every j:
+//   dlog alpha_j = F(j) + sum_{r>=j} (dQg Qg + dKg Kg)_r + sum_{r<j} (dKd Kd)_r + dGam Gam.
+// Phase A (rows): thread t takes channel c = t % DK and rows r = t / DK + m NRG,
+// and leaves its row sums for dk in the dWk buffer (no longer needed); phase B
+// (columns) the same with columns i; phase C one thread per channel.
+// Shared: Qs, Ks, Gs, GLs [C][DK], F [NRG][C][DK], dAs, dPs [C][C], gC, gCl [DK].
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                           const Tin* __restrict__ la, const float* __restrict__ g,
+                                           const float* __restrict__ gl,
+                                           const float* __restrict__ dAt, const float* __restrict__ dP,
+                                           const float* __restrict__ dQg, const float* __restrict__ dKd,
+                                           const float* __restrict__ dKg, const float* __restrict__ dGam,
+                                           float* __restrict__ dKrow, Tin* __restrict__ dq_out,
+                                           Tin* __restrict__ dk_out, Tin* __restrict__ dla_out, ChunkMap cmap,
+                                           int H) {
+    constexpr int C = 64;
+    constexpr int NRG = kT / DK;
+    extern __shared__ float smem[];
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y, tid = threadIdx.x, c = tid % DK, rg = tid / DK;
+    float* Qs = smem;
+    float* Ks = Qs + C * DK;
+    float* Gs = Ks + C * DK;
+    float* GLs = Gs + C * DK;
+    float* F = GLs + C * DK;         // [NRG][C][DK]
+    float* dAs = F + NRG * C * DK;
+    float* dPs = dAs + C * C;
+    float* gC = dPs + C * C;
+    float* gCl = gC + DK;
+    const size_t chunk = blockIdx.x;
+    for (int e = tid; e < len * DK; e += kT) {
+        const int r = e / DK, cc = e - r * DK;
+        const size_t off = tok_off(tok0 + r, H, h, DK) + cc;
+        Qs[e] = to_f32(q[off]);
+        Ks[e] = to_f32(k[off]);
+        Gs[e] = g[off];
+        GLs[e] = gl[off];
+    }
+    for (int e = tid; e < NRG * C * DK; e += kT) F[e] = 0.f;
+    for (int e = tid; e < C * C; e += kT) {
+        dAs[e] = dAt[(chunk * H + h) * C * C + e];
+        dPs[e] = dP[(chunk * H + h) * C * C + e];
+    }
+    __syncthreads();
+    if (rg == 0) {
+        gC[c] = Gs[(len - 1) * DK + c];
+        gCl[c] = GLs[(len - 1) * DK + c];
+    }
+    float* Fm = F + rg * C * DK;
+    // phase A: x1 = sum_{i<r} dAt k_i E, x2 = sum_{i<=r} dP k_i E; prefix sums of T_ri into F
+    for (int r = rg; r < len; r += NRG) {
+        const float gr = Gs[r * DK + c], grl = GLs[r * DK + c];
+        const float qv = Qs[r * DK + c], kv = Ks[r * DK + c];
+        float x1 = 0.f, x2 = 0.f, pre = 0.f;
+        for (int i = 0; i < r; ++i) {
+            const float ke = Ks[i * DK + c] * exp_gdiff(gr, grl, Gs[i * DK + c], GLs[i * DK + c]);
+            const float a = dAs[r * C + i] * ke, b = dPs[r * C + i] * ke;
+            x1 += a;
+            x2 += b;
+            pre += kv * a + qv * b;
+            Fm[(i + 1) * DK + c] += pre;   // T_ri with i < j <= r
+        }
+        x2 += dPs[r * C + r] * kv;         // the diagonal of P (E = 1)
+        const size_t off = tok_off(tok0 + r, H, h, DK) + c;
+        dq_out[off] = from_f32<Tin>(x2 + dQg[off] * exp_g(gr, grl));
+        dKrow[off] = x1;
+    }
+    __syncthreads();
+    // phase B: column sums y = sum_{r>i} dAt k_r E + sum_{r>=i} dP q_r E
+    for (int i = rg; i < len; i += NRG) {
+        const float gi = Gs[i * DK + c], gil = GLs[i * DK + c];
+        float y = 0.f;
+        for (int r = i; r < len; ++r) {
+            const float e = exp_gdiff(Gs[r * DK + c], GLs[r * DK + c], gi, gil);
+            y += (dAs[r * C + i] * Ks[r * DK + c] + dPs[r * C + i] * Qs[r * DK + c]) * e;
+        }
+        const size_t off = tok_off(tok0 + i, H, h, DK) + c;
+        dk_out[off] = from_f32<Tin>(dKrow[off] + y + dKg[off] * exp_g(gi, gil) +
+                                    dKd[off] * exp_gdiff(gC[c], gCl[c], gi, gil));
+    }
+    __syncthreads();
+    // phase C: dlog alpha (zero where the forward's floor on log alpha was active)
+    if (rg == 0) {
+        float pre = 0.f;   // sum_{r<j} dKd Kd, added to F[0][j]
+        for (int j = 0; j < len; ++j) {
+            F[j * DK + c] += pre;
+            const size_t off = tok_off(tok0 + j, H, h, DK) + c;
+            pre += dKd[off] * Ks[j * DK + c] * exp_gdiff(gC[c], gCl[c], Gs[j * DK + c], GLs[j * DK + c]);
+        }
+        const float gam = dGam[(chunk * H + h) * DK + c] * exp_g(gC[c], gCl[c]);
+        float suf = 0.f;   // sum_{r>=j} (dQg Qg + dKg Kg)
+        for (int j = len - 1; j >= 0; --j) {
+            const size_t off = tok_off(tok0 + j, H, h, DK) + c;
+            const float eg = exp_g(Gs[j * DK + c], GLs[j * DK + c]);
+            suf += (dQg[off] * Qs[j * DK + c] + dKg[off] * Ks[j * DK + c]) * eg;
+            float f = 0.f;
+#pragma unroll
+            for (int m = 0; m < NRG; ++m) f += F[(m * C + j) * DK + c];
+            dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? f + suf + gam : 0.f);
+        }
+    }
+}
+
+template <typename Tin, int DK>
+cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const Tin* beta,
+                       const Tin* d_o, Tin* dq, Tin* dk_, Tin* dv_, Tin* dla, Tin* dbeta, const ChunkMap& cmap,
+                       int n_chunks, int H, int dv, const BwdWorkspace& ws, cudaStream_t stream) {
+    constexpr int C = 64;
+    const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * DK + 3 * (size_t)C * kBP);
+    const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + std::max((size_t)3 * C * DK, (size_t)C * (dv + DK)) +
+                                           (size_t)C * (dv + DK));
+    const size_t smem_c = sizeof(float) * ((4 + kT / DK) * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
+    if ((e = cudaFuncSetAttribute(kb_b<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
+    if ((e = cudaFuncSetAttribute(kb_c<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c))) return e;
+    const dim3 grid(n_chunks, H);
+    kb_a<Tin, DK><<<grid, kT, smem_a, stream>>>(d_o, ws.fwd.W, ws.dW, ws.fwd.S_chunk, ws.dS_chunk, ws.dQg, ws.dKd,
+                                               ws.dWk, ws.dGam, ws.P, cmap, H, dv);
+    timing_mark(stream, 4);
+    kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.fwd.U, ws.fwd.Wk, ws.dW, ws.dWk, dv_,
+                                            dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
+    timing_mark(stream, 5);
+    kb_c<Tin, DK><<<grid, kT, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg,
+                                               ws.dGam, ws.dWk, dq, dk_, dla, cmap, H);
+    timing_mark(stream, 6);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const Tin* beta, const float* init_state,
+                    const Tin* d_o, const float* d_final, Tin* dq, Tin* dk_, Tin* dv_, Tin* dla, Tin* dbeta,
+                    float* d_init, const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs, int H, int dk,
+                    int dv, const BwdWorkspace& ws, cudaStream_t stream, kda_dtype dtype) {
+    constexpr int C = 64;
+    cudaError_t e = launch_simt_states(dtype, k, v, la, beta, init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C,
+                                       ws.fwd, stream);
+    if (e != cudaSuccess) return e;
+    timing_mark(stream, 1);
+    const size_t smem_p = sizeof(float) * 4 * (size_t)C * dk;
+    const size_t smem_chain = sizeof(float) * ((size_t)dk * kBV + 2 * (size_t)C * dk + 2 * (size_t)C * kBV +
+                                               (size_t)C * C + 2 * dk);
+    if ((e = cudaFuncSetAttribute(kb_p<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
+    if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
+        return e;
+    if (n_chunks > 0)
+        kb_p<Tin><<<dim3(n_chunks, H), kT, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, cmap, H, dk, C);
+    timing_mark(stream, 2);
+    if (n_seqs > 0)
+        kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kT, smem_chain, stream>>>(
+            q, k, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, H, dk, dv, C);
+    timing_mark(stream, 3);
+    if ((e = cudaGetLastError()) != cudaSuccess || n_chunks == 0) return e;
+    if (dk == 128) return run_bwd_dk<Tin, 128>(q, k, v, la, beta, d_o, dq, dk_, dv_, dla, dbeta, cmap, n_chunks, H, dv,
+                                               ws, stream);
+    return run_bwd_dk<Tin, 64>(q, k, v, la, beta, d_o, dq, dk_, dv_, dla, dbeta, cmap, n_chunks, H, dv, ws, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, const float* init_state,
+                                 const void* d_o, const float* d_final_state, void* dq, void* dk, void* dv,
+                                 void* dlog_alpha, void* dbeta, float* d_init_state, const ChunkMap& cmap,
+                                 const SeqMap& smap, int n_chunks, int n_seqs, int H, int dkk, int dvv, int C,
+                                 const BwdWorkspace& ws, cudaStream_t stream) {
+    if (C != 64) return cudaErrorNotSupported;
+    if (dtype == KDA_F32)
+        return run_bwd<float>((const float*)q, (const float*)k, (const float*)v, (const float*)log_alpha,
+                              (const float*)beta, init_state, (const float*)d_o, d_final_state, (float*)dq,
+                              (float*)dk, (float*)dv, (float*)dlog_alpha, (float*)dbeta, d_init_state, cmap, smap,
+                              n_chunks, n_seqs, H, dkk, dvv, ws, stream, dtype);
+    using bf = __nv_bfloat16;
+    return run_bwd<bf>((const bf*)q, (const bf*)k, (const bf*)v, (const bf*)log_alpha, (const bf*)beta, init_state,
+                       (const bf*)d_o, d_final_state, (bf*)dq, (bf*)dk, (bf*)dv, (bf*)dlog_alpha, (bf*)dbeta,
+                       d_init_state, cmap, smap, n_chunks, n_seqs, H, dkk, dvv, ws, stream, dtype);
+}
+
+}  // namespace kda

@@ -16,8 +16,9 @@
 // chunks); WY / DPLR restructuring: "我终于看懂了 KDA" explainer
 // (pwwt.cn/news/3787313), sections 16-17.  This path evaluates every decay
 // as exp of a non-positive difference g_r - g_i (r >= i), so it is exact for
-// any decay range; it serves the fp32 inputs and is the CUDA-core reference
-// for the tensor-core path.
+// any decay range, with g summed in fp64 and kept as an fp32 (hi, lo) pair so
+// that the difference keeps its accuracy when g itself is large; it serves the
+// fp32 inputs and is the CUDA-core reference for the tensor-core path.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -35,25 +36,30 @@ __device__ __forceinline__ float warp_sum(float x) {
 // K1: one block per (chunk, head), one thread per key channel.
 template <typename Tin>
 __global__ void __launch_bounds__(128) k1_cumsum(const Tin* __restrict__ la, float* __restrict__ g,
-                                                 ChunkMap cmap, int H, int dk) {
+                                                 float* __restrict__ gl, ChunkMap cmap, int H, int dk) {
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
     const int h = blockIdx.y, c = threadIdx.x;
-    float acc = 0.f;
+    double acc = 0.0;
     for (int r = 0; r < len; ++r) {
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
-        acc += fmaxf(to_f32(la[off]), kLogAlphaFloor);
-        g[off] = acc;
+        acc += (double)fmaxf(to_f32(la[off]), kLogAlphaFloor);
+        const float hi = (float)acc;
+        g[off] = hi;
+        gl[off] = (float)(acc - (double)hi);
     }
 }
 
 // K2: one block per (chunk, head).  Dynamic shared memory:
-//   A [C][C] | phase 1: Ks [C][dk], Gs [C][dk]  / phase 2: X [C][dk + dv]
+//   A [C][C] | phase 1: Ks, Gs [C][dk], GLs [C][dk] (bf16)  / phase 2: X [C][dk + dv]
+// (the low part of g is staged in bf16: |lo| <= ulp(g) / 2, so bf16 keeps it to
+// ulp(g) 2^-10, below 3e-8 for |g| < 256, and 128-token chunks fit at d = 128)
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                                   const Tin* __restrict__ beta, const float* __restrict__ g,
-                                                  float* __restrict__ U, float* __restrict__ Wk, ChunkMap cmap,
-                                                  int H, int dk, int dv, int C) {
+                                                  const float* __restrict__ gl, float* __restrict__ U,
+                                                  float* __restrict__ Wk, ChunkMap cmap, int H, int dk, int dv,
+                                                  int C) {
     extern __shared__ float smem[];
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
@@ -61,12 +67,14 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
     float* A = smem;
     float* Ks = A + C * C;
     float* Gs = Ks + C * dk;
+    __nv_bfloat16* GLs = reinterpret_cast<__nv_bfloat16*>(Gs + C * dk);
 
     for (int e = tid; e < len * dk; e += kThreads) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         Ks[r * dk + c] = to_f32(k[off]);
         Gs[r * dk + c] = g[off];
+        GLs[r * dk + c] = __float2bfloat16_rn(gl[off]);
     }
     __syncthreads();
     // A, one warp per (r, i) pair, lanes over channels
@@ -75,7 +83,9 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
         float s = 0.f;
         if (i < r) {
             for (int c = lane; c < dk; c += 32)
-                s += Ks[r * dk + c] * Ks[i * dk + c] * expf(Gs[r * dk + c] - Gs[i * dk + c]);
+                s += Ks[r * dk + c] * Ks[i * dk + c] *
+                     exp_gdiff(Gs[r * dk + c], __bfloat162float(GLs[r * dk + c]), Gs[i * dk + c],
+                               __bfloat162float(GLs[i * dk + c]));
             s = warp_sum(s) * to_f32(beta[(size_t)(tok0 + r) * H + h]);
         }
         if (lane == 0) A[r * C + i] = s;
@@ -93,7 +103,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
                 s = br * to_f32(v[tok * dv + j]);
             } else {
                 const int c = j - dv;
-                s = br * to_f32(k[tok * dk + c]) * expf(g[tok * dk + c]);
+                s = br * to_f32(k[tok * dk + c]) * exp_g(g[tok * dk + c], gl[tok * dk + c]);
             }
             for (int i = 0; i < r; ++i) s -= A[r * C + i] * X[i * ncol + j];
             X[r * ncol + j] = s;
@@ -105,9 +115,10 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
 
 // K3: one block per (sequence, head, d_v tile of kBV columns), sequential over
 // the sequence's chunks.  Shared: S [dk][kBV], M [C][dk] (Wk, then K . decay),
-// Ws [C][kBV], gC [dk].
+// Ws [C][kBV], gC, gCl [dk].
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
+                                                     const float* __restrict__ gl,
                                                      const float* __restrict__ U, const float* __restrict__ Wkg,
                                                      float* __restrict__ Wg, float* __restrict__ S_chunk,
                                                      const float* __restrict__ init_state,
@@ -120,6 +131,7 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
     float* M = S + dk * kBV;
     float* Ws = M + C * dk;
     float* gC = Ws + C * kBV;
+    float* gCl = gC + dk;
 
     const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
     for (int e = tid; e < dk * kBV; e += kThreads) {
@@ -150,18 +162,21 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
             Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = s;
         }
         __syncthreads();
-        for (int c = tid; c < dk; c += kThreads) gC[c] = g[((size_t)(t0 + L - 1) * H + h) * dk + c];
+        for (int c = tid; c < dk; c += kThreads) {
+            gC[c] = g[((size_t)(t0 + L - 1) * H + h) * dk + c];
+            gCl[c] = gl[((size_t)(t0 + L - 1) * H + h) * dk + c];
+        }
         __syncthreads();
         for (int e = tid; e < L * dk; e += kThreads) {
             int r = e / dk, c = e - r * dk;
             size_t off = ((size_t)(t0 + r) * H + h) * dk + c;
-            M[e] = to_f32(k[off]) * expf(gC[c] - g[off]);
+            M[e] = to_f32(k[off]) * exp_gdiff(gC[c], gCl[c], g[off], gl[off]);
         }
         __syncthreads();
         // S <- Diag(exp(g_C)) S + (K . exp(g_C - g))^T W
         for (int e = tid; e < dk * kBV; e += kThreads) {
             int c = e / kBV, j = e - c * kBV;
-            float s = expf(gC[c]) * S[e];
+            float s = exp_g(gC[c], gCl[c]) * S[e];
             for (int r = 0; r < L; ++r) s += M[r * dk + c] * Ws[r * kBV + j];
             S[e] = s;
         }
@@ -176,10 +191,11 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
 }
 
 // K4: one block per (chunk, head).  Shared: Ks [C][dk] (then Q . exp(g)),
-// Gs [C][dk], P [C][C].
+// Gs [C][dk], P [C][C], GLs [C][dk] (bf16, as in K2).
 template <typename Tin>
 __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                                                      const float* __restrict__ g, const float* __restrict__ Wg,
+                                                      const float* __restrict__ g, const float* __restrict__ gl,
+                                                      const float* __restrict__ Wg,
                                                       const float* __restrict__ S_chunk, Tin* __restrict__ o,
                                                       ChunkMap cmap, int H, int dk, int dv, int C) {
     extern __shared__ float smem[];
@@ -189,11 +205,13 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
     float* Ks = smem;
     float* Gs = Ks + C * dk;
     float* P = Gs + C * dk;
+    __nv_bfloat16* GLs = reinterpret_cast<__nv_bfloat16*>(P + C * C);
     for (int e = tid; e < len * dk; e += kThreads) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         Ks[e] = to_f32(k[off]);
         Gs[e] = g[off];
+        GLs[e] = __float2bfloat16_rn(gl[off]);
     }
     __syncthreads();
     // P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic), i <= r (inclusive mask)
@@ -203,7 +221,9 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
         if (i <= r) {
             const size_t qoff = ((size_t)(tok0 + r) * H + h) * dk;
             for (int c = lane; c < dk; c += 32)
-                s += to_f32(q[qoff + c]) * Ks[i * dk + c] * expf(Gs[r * dk + c] - Gs[i * dk + c]);
+                s += to_f32(q[qoff + c]) * Ks[i * dk + c] *
+                     exp_gdiff(Gs[r * dk + c], __bfloat162float(GLs[r * dk + c]), Gs[i * dk + c],
+                               __bfloat162float(GLs[i * dk + c]));
             s = warp_sum(s);
         }
         if (lane == 0) P[r * C + i] = s;
@@ -212,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
     for (int e = tid; e < len * dk; e += kThreads) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
-        Ks[e] = to_f32(q[off]) * expf(Gs[e]);
+        Ks[e] = to_f32(q[off]) * exp_g(Gs[e], __bfloat162float(GLs[e]));
     }
     __syncthreads();
     const size_t sc_base = ((size_t)blockIdx.x * H + h) * dk * dv;
@@ -225,35 +245,76 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
     }
 }
 
+// K2's shared memory: A, then the larger of (Ks, Gs fp32 + GLs bf16) and X.
+size_t k2_smem(int C, int dk, int dv) {
+    const size_t phase1 = sizeof(float) * 2 * (size_t)C * dk + sizeof(__nv_bfloat16) * (size_t)C * dk;
+    const size_t phase2 = sizeof(float) * (size_t)C * (dk + dv);
+    return sizeof(float) * (size_t)C * C + (phase1 > phase2 ? phase1 : phase2);
+}
+
 template <typename Tin>
 cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const Tin* beta, const float* init_state,
                 Tin* o, float* final_state, const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs,
                 int H, int dk, int dv, int C, const SimtWorkspace& ws, cudaStream_t stream) {
-    const size_t smem2 = sizeof(float) * ((size_t)C * C + (size_t)C * (size_t)((2 * dk > dk + dv) ? 2 * dk : dk + dv));
-    const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + dk);
-    const size_t smem4 = sizeof(float) * (2 * (size_t)C * dk + (size_t)C * C);
+    const size_t smem2 = k2_smem(C, dk, dv);
+    const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + 2 * dk);
+    const size_t smem4 = sizeof(float) * (2 * (size_t)C * dk + (size_t)C * C) + sizeof(__nv_bfloat16) * (size_t)C * dk;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
     if ((e = cudaFuncSetAttribute(k3_state<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
     if ((e = cudaFuncSetAttribute(k4_output<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4))) return e;
-    if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, cmap, H, dk);
+    if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
     timing_mark(stream, 1);
     if (n_chunks > 0)
-        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.U, ws.Wk, cmap, H, dk, dv, C);
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk, dv,
+                                                                 C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
-        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.U, ws.Wk, ws.W, ws.S_chunk,
-                                                                            init_state, final_state, smap, H, dk,
-                                                                            dv, C);
+        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W,
+                                                                            ws.S_chunk, init_state, final_state,
+                                                                            smap, H, dk, dv, C);
     timing_mark(stream, 3);
     if (n_chunks > 0)
-        k4_output<Tin><<<dim3(n_chunks, H), kThreads, smem4, stream>>>(q, k, ws.g, ws.W, ws.S_chunk, o, cmap, H, dk,
-                                                                     dv, C);
+        k4_output<Tin><<<dim3(n_chunks, H), kThreads, smem4, stream>>>(q, k, ws.g, ws.gl, ws.W, ws.S_chunk, o, cmap,
+                                                                     H, dk, dv, C);
     timing_mark(stream, 4);
     return cudaGetLastError();
 }
 
+template <typename Tin>
+cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* beta, const float* init_state,
+                       const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs, int H, int dk, int dv,
+                       int C, const SimtWorkspace& ws, cudaStream_t stream) {
+    const size_t smem2 = k2_smem(C, dk, dv);
+    const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + 2 * dk);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
+    if ((e = cudaFuncSetAttribute(k3_state<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
+    if (n_chunks > 0) {
+        k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk, dv,
+                                                                 C);
+    }
+    if (n_seqs > 0)
+        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W,
+                                                                            ws.S_chunk, init_state, nullptr, smap, H,
+                                                                            dk, dv, C);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_simt_states(kda_dtype dtype, const void* k, const void* v, const void* log_alpha,
+                               const void* beta, const float* init_state, const ChunkMap& cmap, const SeqMap& smap,
+                               int n_chunks, int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws,
+                               cudaStream_t stream) {
+    if (dtype == KDA_F32)
+        return run_states<float>((const float*)k, (const float*)v, (const float*)log_alpha, (const float*)beta,
+                                 init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws, stream);
+    return run_states<__nv_bfloat16>((const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                     (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, init_state, cmap,
+                                     smap, n_chunks, n_seqs, H, dk, dv, C, ws, stream);
+}
 
 cudaError_t launch_simt_prefill(kda_dtype dtype, const void* q, const void* k, const void* v, const void* log_alpha,
                                 const void* beta, const float* init_state, void* o, float* final_state,

@@ -127,6 +127,17 @@ __device__ __forceinline__ float prep_beta(float x, unsigned prep) {
 // 1 / ||x|| for the key/query normalisation (0 for an all-zero vector).
 __device__ __forceinline__ float inv_norm_from_sq(float sum_sq) { return sum_sq > 0.f ? rsqrtf(sum_sq) : 0.f; }
 
+// ---- cumulative decays as fp32 (hi, lo) pairs -------------------------------
+// Within a chunk g reaches -100 and beyond, where one fp32 ulp is ~1e-5; a decay
+// exp(g_a - g_b) formed from two rounded g would carry that as a relative error.
+// The CUDA-core kernels therefore keep g as hi + lo (the fp64 cumulative sum split
+// in two floats) and form differences as (hi_a - hi_b) + (lo_a - lo_b).
+__device__ __forceinline__ float exp_gdiff(float ah, float al, float bh, float bl) {
+    return expf((ah - bh) + (al - bl));
+}
+// exp(g) for g = hi + lo, |lo| <= ulp(hi) / 2: exp(hi) (1 + lo) to second order.
+__device__ __forceinline__ float exp_g(float h, float l) { return expf(h) * (1.f + l); }
+
 // ---- optional per-kernel timing hook (see kda_set_timing_events) -----------
 
 struct TimingHook {
@@ -144,7 +155,8 @@ inline void timing_mark(cudaStream_t s, int i) {
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 
 struct SimtWorkspace {
-    float* g;
+    float* g;        // cumulative log decay, high part (fp32 rounding of the fp64 sum)
+    float* gl;       // low part: g = g + gl to about 48 bits
     float* U;
     float* Wk;
     float* W;
@@ -156,6 +168,35 @@ cudaError_t launch_simt_prefill(kda_dtype dtype, const void* q, const void* k, c
                                 void* o, float* final_state, const ChunkMap& cmap, const SeqMap& smap,
                                 int n_chunks, int n_seqs, int H, int dk, int dv, int C,
                                 const SimtWorkspace& ws, cudaStream_t stream);
+
+// The CUDA-core forward without the output kernel: g, U, Wk, W and every
+// chunk's start state into `ws` (for the backward pass).
+cudaError_t launch_simt_states(kda_dtype dtype, const void* k, const void* v, const void* log_alpha,
+                               const void* beta, const float* init_state, const ChunkMap& cmap, const SeqMap& smap,
+                               int n_chunks, int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws,
+                               cudaStream_t stream);
+
+// Backward scratch (fp32): the forward intermediates plus the gradients the
+// backward kernels hand to one another.
+struct BwdWorkspace {
+    SimtWorkspace fwd;  // g, U, Wk, W [tokens, H, d]; S_chunk [chunks, H, dk, dv]
+    float* dS_chunk;    // [chunks, H, dk, dv] gradient w.r.t. each chunk's end state
+    float* dW;          // [tokens, H, dv]
+    float* P;           // [chunks, H, C, C] decayed causal scores
+    float* dQg;         // [tokens, H, dk]
+    float* dKd;         // [tokens, H, dk]
+    float* dWk;         // [tokens, H, dk]
+    float* dKg;         // [tokens, H, dk]
+    float* dGam;        // [chunks, H, dk]
+    float* dAt;         // [chunks, H, C, C] gradient w.r.t. the unscaled key products
+};
+
+cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, const float* init_state,
+                                 const void* d_o, const float* d_final_state, void* dq, void* dk, void* dv,
+                                 void* dlog_alpha, void* dbeta, float* d_init_state, const ChunkMap& cmap,
+                                 const SeqMap& smap, int n_chunks, int n_seqs, int H, int dkk, int dvv, int C,
+                                 const BwdWorkspace& ws, cudaStream_t stream);
 
 cudaError_t launch_decode(kda_dtype dtype, const void* q, const void* k, const void* v,
                           const void* log_alpha, const void* beta, float* state, int N, int H,

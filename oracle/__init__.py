@@ -4,10 +4,13 @@ Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The CUDA library and its Python binding
 never import it, and it imports nothing from them.
 
-Two implementations of the same operator, both in plain C (``kda_oracle.c``):
+Two implementations of the same operator and its gradient, in plain C
+(``kda_oracle.c``):
 
 * :func:`forward` -- the token-by-token recurrence (decay, read, error, write,
   read-out), the definition of KDA.
+* :func:`backward` -- the reverse-mode gradient of the token recurrence
+  (for training), states recomputed from copies kept every 64 tokens.
 * :func:`chunkform` -- the chunkwise form with the WY/UT triangular solve,
   written with pairwise decay products; it also returns the intermediates that
   the GPU kernels materialise (cumulative log decay, U, Wk, W and the start
@@ -63,6 +66,10 @@ def _load():
                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp, dp, dp,
                                                   dp, dp, dp, ctypes.c_int]
             lib.kda_ref_chunkform_f64.restype = ctypes.c_int
+            lib.kda_ref_backward_f64.argtypes = [dp, dp, dp, dp, dp, dp, i64p, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_int, dp, dp, dp, dp, dp, dp, dp, dp,
+                                                 ctypes.c_int]
+            lib.kda_ref_backward_f64.restype = ctypes.c_int
             lib.kda_ref_max_threads.argtypes = []
             lib.kda_ref_max_threads.restype = ctypes.c_int
             _lib = lib
@@ -139,6 +146,34 @@ def chunkform(q, k, v, log_alpha, beta, seq_start, C: int, init_state=None,
         _ptr(out.get("w")), _ptr(out.get("s_chunk")), int(n_threads))
     if rc != 0:
         raise RuntimeError(f"kda_ref_chunkform_f64 failed ({rc})")
+    return out
+
+
+def backward(q, k, v, log_alpha, beta, seq_start, d_o, d_final_state=None, init_state=None,
+             n_threads: int = 0):
+    """Reverse-mode gradient of :func:`forward` (O3) for the loss
+    ``sum(d_o * o) + sum(d_final_state * final_state)``.  Returns a dict with
+    ``dq, dk, dv, dlog_alpha, dbeta, d_init_state`` shaped like the inputs
+    (``d_init_state`` ``[N,H,dk,dv]``, the gradient for a zero initial state when
+    ``init_state`` is None)."""
+    q, k, v, log_alpha, beta, seq_start, n_tok, H, dk, dv = _check(q, k, v, log_alpha, beta, seq_start)
+    n_seqs = len(seq_start) - 1
+    s0 = None if init_state is None else _f64(init_state)
+    d_o = _f64(d_o)
+    assert d_o.shape == (n_tok, H, dv)
+    dfs = None if d_final_state is None else _f64(d_final_state)
+    if dfs is not None:
+        assert dfs.shape == (n_seqs, H, dk, dv)
+    out = {"dq": np.zeros((n_tok, H, dk)), "dk": np.zeros((n_tok, H, dk)), "dv": np.zeros((n_tok, H, dv)),
+           "dlog_alpha": np.zeros((n_tok, H, dk)), "dbeta": np.zeros((n_tok, H)),
+           "d_init_state": np.zeros((n_seqs, H, dk, dv))}
+    rc = _load().kda_ref_backward_f64(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(s0),
+        seq_start.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n_seqs, H, dk, dv, _ptr(d_o), _ptr(dfs),
+        _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]),
+        _ptr(out["d_init_state"]), int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"kda_ref_backward_f64 failed ({rc})")
     return out
 
 

@@ -307,6 +307,172 @@ int kda_ref_chunkform_f64(const double* q, const double* k, const double* v,
     return failed ? -2 : 0;
 }
 
+/* ------------------------------------------------------------------------
+ * O3: reverse-mode gradient of O1 (the token recurrence), for training.
+ *
+ * The pages say training needs the chunkwise parallel form but derive no
+ * backward pass; this is the chain rule applied to O1's steps, in reverse
+ * token order.  For token t, with S_prev the state before it and G the
+ * gradient with respect to the state after it:
+ *   dq_t   = S_t do_t                    (o_t = S_t^T q_t)
+ *   G     += q_t do_t^T
+ *   Sd     = Diag(alpha_t) S_prev,  u = v_t - Sd^T k_t
+ *   dbeta_t = k_t^T G u
+ *   du     = beta_t G^T k_t,  dv_t = du
+ *   dk_t   = beta_t G u - Sd du
+ *   dSd    = G - k_t du^T
+ *   dlog_alpha_t[c] = sum_j dSd[c][j] Sd[c][j]
+ *   G      = Diag(alpha_t) dSd           (gradient with respect to S_prev)
+ * and d init_state = G after the first token.  The loss is
+ *   L = sum(do * o) + sum(d_final_state * final_state).
+ * States are recomputed forward from a copy kept every 64 tokens (the same
+ * values as one forward pass; the copies only bound the memory).
+ * ------------------------------------------------------------------------ */
+int kda_ref_backward_f64(const double* q, const double* k, const double* v,
+                         const double* log_alpha, const double* beta,
+                         const double* init_state, const int64_t* seq_start,
+                         int n_seqs, int H, int dk, int dv,
+                         const double* d_o, const double* d_final_state,
+                         double* dq, double* dkk, double* dvv, double* dla, double* dbeta,
+                         double* d_init_state, int n_threads)
+{
+    enum { KB = 64 };
+    if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    const size_t sz = (size_t)dk * dv;
+    long n_pairs = (long)n_seqs * H;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < n_pairs; ++p) {
+        int n = (int)(p / H), h = (int)(p % H);
+        int64_t t_begin = seq_start[n], t_end = seq_start[n + 1], len = t_end - t_begin;
+        int64_t n_blk = (len + KB - 1) / KB;
+        double* ckpt = (double*)malloc(sizeof(double) * sz * (size_t)(n_blk > 0 ? n_blk : 1));
+        double* st = (double*)malloc(sizeof(double) * sz * (KB + 1));   /* states of one block */
+        double* G = (double*)malloc(sizeof(double) * sz);
+        double* dSd = (double*)malloc(sizeof(double) * sz);
+        double* a = (double*)malloc(sizeof(double) * (size_t)dk);
+        double* r = (double*)malloc(sizeof(double) * (size_t)(dv > dk ? dv : dk));
+        double* u = (double*)malloc(sizeof(double) * (size_t)dv);
+        double* du = (double*)malloc(sizeof(double) * (size_t)dv);
+        double* Gu = (double*)malloc(sizeof(double) * (size_t)dk);
+        if (!ckpt || !st || !G || !dSd || !a || !r || !u || !du || !Gu) {
+            free(ckpt); free(st); free(G); free(dSd); free(a); free(r); free(u); free(du); free(Gu);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        /* one step of O1: S (in place) from the state before token t */
+#define STEP(S, t)                                                                          \
+        do {                                                                                \
+            const double* kt_ = k + ((size_t)(t) * H + h) * dk;                             \
+            const double* vt_ = v + ((size_t)(t) * H + h) * dv;                             \
+            const double* lat_ = log_alpha + ((size_t)(t) * H + h) * dk;                    \
+            double bt_ = beta[(size_t)(t) * H + h];                                         \
+            for (int c = 0; c < dk; ++c) a[c] = exp(lat_[c]);                               \
+            for (int c = 0; c < dk; ++c)                                                    \
+                for (int j = 0; j < dv; ++j) (S)[(size_t)c * dv + j] *= a[c];               \
+            for (int j = 0; j < dv; ++j) r[j] = 0.0;                                        \
+            for (int c = 0; c < dk; ++c)                                                    \
+                for (int j = 0; j < dv; ++j) r[j] += (S)[(size_t)c * dv + j] * kt_[c];      \
+            for (int c = 0; c < dk; ++c)                                                    \
+                for (int j = 0; j < dv; ++j) (S)[(size_t)c * dv + j] += bt_ * kt_[c] * (vt_[j] - r[j]); \
+        } while (0)
+
+        /* forward: the state at the start of every block of KB tokens */
+        if (init_state) memcpy(st, init_state + ((size_t)n * H + h) * sz, sizeof(double) * sz);
+        else memset(st, 0, sizeof(double) * sz);
+        for (int64_t b = 0; b < n_blk; ++b) {
+            memcpy(ckpt + (size_t)b * sz, st, sizeof(double) * sz);
+            int64_t t0 = t_begin + b * KB, t1 = t0 + KB < t_end ? t0 + KB : t_end;
+            for (int64_t t = t0; t < t1; ++t) STEP(st, t);
+        }
+        /* G = gradient with respect to the final state */
+        if (d_final_state) memcpy(G, d_final_state + ((size_t)n * H + h) * sz, sizeof(double) * sz);
+        else memset(G, 0, sizeof(double) * sz);
+        for (int64_t b = n_blk - 1; b >= 0; --b) {
+            int64_t t0 = t_begin + b * KB, t1 = t0 + KB < t_end ? t0 + KB : t_end;
+            /* st[i] = state after i tokens of the block */
+            memcpy(st, ckpt + (size_t)b * sz, sizeof(double) * sz);
+            for (int64_t t = t0; t < t1; ++t) {
+                double* nx = st + (size_t)(t - t0 + 1) * sz;
+                memcpy(nx, nx - sz, sizeof(double) * sz);
+                STEP(nx, t);
+            }
+            for (int64_t t = t1 - 1; t >= t0; --t) {
+                const double* Sprev = st + (size_t)(t - t0) * sz;
+                const double* St = Sprev + sz;
+                const double* qt = q + ((size_t)t * H + h) * dk;
+                const double* kt = k + ((size_t)t * H + h) * dk;
+                const double* vt = v + ((size_t)t * H + h) * dv;
+                const double* lat = log_alpha + ((size_t)t * H + h) * dk;
+                const double* dot = d_o + ((size_t)t * H + h) * dv;
+                double bt = beta[(size_t)t * H + h];
+                double* dqt = dq + ((size_t)t * H + h) * dk;
+                double* dkt = dkk + ((size_t)t * H + h) * dk;
+                double* dvt = dvv + ((size_t)t * H + h) * dv;
+                double* dlat = dla + ((size_t)t * H + h) * dk;
+                /* output: dq_t = S_t do_t, G += q_t do_t^T */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += St[(size_t)c * dv + j] * dot[j];
+                    dqt[c] = acc;
+                }
+                for (int c = 0; c < dk; ++c)
+                    for (int j = 0; j < dv; ++j) G[(size_t)c * dv + j] += qt[c] * dot[j];
+                /* Sd = Diag(alpha) S_prev (kept in dSd for now), u = v - Sd^T k */
+                for (int c = 0; c < dk; ++c) a[c] = exp(lat[c]);
+                for (int c = 0; c < dk; ++c)
+                    for (int j = 0; j < dv; ++j) dSd[(size_t)c * dv + j] = a[c] * Sprev[(size_t)c * dv + j];
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk; ++c) acc += dSd[(size_t)c * dv + j] * kt[c];
+                    u[j] = vt[j] - acc;
+                }
+                /* Gu = G u, r = G^T k */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += G[(size_t)c * dv + j] * u[j];
+                    Gu[c] = acc;
+                }
+                for (int j = 0; j < dv; ++j) {
+                    double acc = 0.0;
+                    for (int c = 0; c < dk; ++c) acc += G[(size_t)c * dv + j] * kt[c];
+                    r[j] = acc;
+                }
+                double db = 0.0;
+                for (int c = 0; c < dk; ++c) db += kt[c] * Gu[c];
+                dbeta[(size_t)t * H + h] = db;
+                for (int j = 0; j < dv; ++j) { du[j] = bt * r[j]; dvt[j] = du[j]; }
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += dSd[(size_t)c * dv + j] * du[j];
+                    dkt[c] = bt * Gu[c] - acc;
+                }
+                /* dSd = G - k du^T; dlog_alpha = rowsum(dSd . Sd); G = Diag(alpha) dSd */
+                for (int c = 0; c < dk; ++c) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) {
+                        double sd = dSd[(size_t)c * dv + j];
+                        double g = G[(size_t)c * dv + j] - kt[c] * du[j];
+                        acc += g * sd;
+                        G[(size_t)c * dv + j] = a[c] * g;
+                    }
+                    dlat[c] = acc;
+                }
+            }
+        }
+#undef STEP
+        if (d_init_state) memcpy(d_init_state + ((size_t)n * H + h) * sz, G, sizeof(double) * sz);
+        free(ckpt); free(st); free(G); free(dSd); free(a); free(r); free(u); free(du); free(Gu);
+    }
+    return failed ? -2 : 0;
+}
+
 /* Number of threads the OpenMP runtime would use (1 without OpenMP). */
 int kda_ref_max_threads(void)
 {

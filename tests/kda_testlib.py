@@ -74,6 +74,50 @@ def oracle_prefill(inp, heads=None, seqs=None, n_threads=0, prep=0):
     return o, fs, tok_idx, seqs, heads
 
 
+def oracle_backward(inp, d_o, d_final=None, heads=None, seqs=None, n_threads=0):
+    """Oracle gradients (dict of fp64 arrays, token-major over the selected
+    sequences, heads on axis 1) for the given heads and sequences."""
+    H = inp.q.shape[2]
+    heads = list(range(H)) if heads is None else list(heads)
+    ss = inp.seq_start
+    seqs = list(range(len(ss) - 1)) if seqs is None else list(seqs)
+    flat = lambda t: t.reshape(-1, *t.shape[2:])
+    tok_idx = np.concatenate([np.arange(ss[s], ss[s + 1]) for s in seqs]) if seqs else np.zeros(0, np.int64)
+    lens = [int(ss[s + 1] - ss[s]) for s in seqs]
+    sub_start = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    ti = torch.as_tensor(tok_idx, device=inp.q.device, dtype=torch.long)
+    hi = torch.as_tensor(heads, device=inp.q.device, dtype=torch.long)
+    si = torch.as_tensor(seqs, device=inp.q.device, dtype=torch.long)
+
+    def pick(t):
+        return to_f64(flat(t).index_select(0, ti).index_select(1, hi))
+
+    pick_s = lambda t: None if t is None else to_f64(t.index_select(0, si).index_select(1, hi))
+    g = oracle.backward(pick(inp.q), pick(inp.k), pick(inp.v), pick(inp.log_alpha), pick(inp.beta), sub_start,
+                        pick(d_o), d_final_state=pick_s(d_final), init_state=pick_s(inp.init_state),
+                        n_threads=n_threads)
+    return g, tok_idx, seqs, heads
+
+
+def gpu_grad_slices(grads, tok_idx, seqs, heads):
+    """The same slices of the GPU gradients (dq, dk, dv, dlog_alpha, dbeta,
+    d_init_state) as a dict of host fp64 arrays."""
+    names = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "d_init_state")
+    out = {}
+    for name, t in zip(names, grads):
+        if t is None:
+            continue
+        dev = t.device
+        hi = torch.as_tensor(heads, device=dev, dtype=torch.long)
+        if name == "d_init_state":
+            si = torch.as_tensor(seqs, device=dev, dtype=torch.long)
+            out[name] = to_f64(t.index_select(0, si).index_select(1, hi))
+        else:
+            ti = torch.as_tensor(tok_idx, device=dev, dtype=torch.long)
+            out[name] = to_f64(t.reshape(-1, *t.shape[2:]).index_select(0, ti).index_select(1, hi))
+    return out
+
+
 def gpu_slices(o_gpu, fs_gpu, tok_idx, seqs, heads):
     """The same slices of the GPU outputs as host fp64 arrays."""
     dev = o_gpu.device

@@ -165,6 +165,54 @@ def test_prep_flags_match_the_header():
                                                                  kda.PREP_BETA_SIGMOID)
 
 
+def _call_bwd(**kw):
+    """kda_chunk_bwd with fake (never dereferenced) device pointers."""
+    lib = kda.lib()
+    a = dict(q=0x10000, k=0x20000, v=0x30000, la=0x40000, beta=0x50000, dtype=1, s0=None, cu=None, n=0,
+             B=1, T=256, H=2, dk=64, dv=64, C=64, do=0x60000, dfs=None, dq=0x70000, dk_=0x80000, dv_=0x90000,
+             dla=0xa0000, db=0xb0000, ds0=None, ws=0x100000, wsb=1 << 40)
+    a.update(kw)
+    cu = None
+    keep = None
+    if a["cu"] is not None:
+        keep = (ctypes.c_int32 * len(a["cu"]))(*a["cu"])
+        cu = ctypes.cast(keep, ctypes.POINTER(ctypes.c_int32))
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.kda_chunk_bwd(vp(a["q"]), vp(a["k"]), vp(a["v"]), vp(a["la"]), vp(a["beta"]), a["dtype"],
+                             vp(a["s0"]), cu, a["n"], a["B"], a["T"], a["H"], a["dk"], a["dv"], a["C"], vp(a["do"]),
+                             vp(a["dfs"]), vp(a["dq"]), vp(a["dk_"]), vp(a["dv_"]), vp(a["dla"]), vp(a["db"]),
+                             vp(a["ds0"]), vp(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dtype=5), E_DTYPE),
+    (dict(C=32), E_CHUNK),
+    (dict(dk=96), E_SHAPE),
+    (dict(H=0), E_SHAPE),
+    (dict(do=None), E_NULL),
+    (dict(dla=None), E_NULL),
+    (dict(db=None), E_NULL),
+    (dict(ws=None), E_WS),
+    (dict(wsb=16), E_WS),
+    (dict(dq=0x70004), E_ALIGN),
+    (dict(ds0=0x110008), E_ALIGN),
+    (dict(ws=0x100010), E_ALIGN),
+    (dict(cu=[0, 100, 50, 256], n=3), E_SEQ),
+])
+def test_chunk_bwd_rejects_before_launch(kw, code):
+    assert _call_bwd(**kw) == code
+
+
+def test_bwd_workspace_size():
+    B, T, H, d = 2, 200, 3, 64
+    w = kda.bwd_workspace_size(B, T, H, d, d, 64)
+    assert w > kda.workspace_size(B, T, H, d, d, 64, 1, algo="simt")   # holds the CUDA-core forward's scratch
+    assert w == kda.bwd_workspace_size(B, T, H, d, d, 128)           # 64-token chunks either way
+    assert kda.bwd_workspace_size(B, T, H, d, d, 32) == 0
+    assert kda.bwd_workspace_size(1, 10, H, d, d, 64, cu_seqlens=[0, 4, 10]) > 0
+    assert kda.bwd_workspace_size(1, 10, H, d, d, 64, cu_seqlens=[0, 6, 4, 10]) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 4, 1, 64)

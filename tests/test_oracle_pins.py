@@ -412,3 +412,94 @@ def test_prep_forward_scale_invariance_and_gate_limits():
 def _order(pre, v):
     q, k, la, b = pre
     return q, k, v, la, b
+
+
+# ------------------------------------------------------------- backward (O3)
+# The pages give no backward derivation (training is only said to need the
+# parallel form); O3 is pinned to the forward oracle, which is pinned above, by
+# finite differences and by exact identities of the recurrence.
+
+def _loss_inputs(seed, lens=(5, 0, 4), H=2, dk=3, dv=2):
+    seq = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    T = int(seq[-1])
+    q, k, v, la, beta = _rand_inputs(T, H, dk, dv, seed)
+    rng = np.random.default_rng(seed + 1)
+    s0 = rng.standard_normal((len(lens), H, dk, dv))
+    do = rng.standard_normal((T, H, dv))
+    dfs = rng.standard_normal((len(lens), H, dk, dv))
+    return seq, q, k, v, la, beta, s0, do, dfs
+
+
+def _loss(seq, q, k, v, la, beta, s0, do, dfs):
+    o, fs = oracle.forward(q, k, v, la, beta, seq, init_state=s0)
+    return float(np.sum(o * do) + np.sum(fs * dfs))
+
+
+def test_backward_matches_central_differences():
+    """Every gradient entry (q, k, v, log alpha, beta, initial state) against a
+    central difference of the fp64 forward; sequences of length 5, 0 and 4."""
+    seq, q, k, v, la, beta, s0, do, dfs = _loss_inputs(51)
+    g = oracle.backward(q, k, v, la, beta, seq, do, d_final_state=dfs, init_state=s0)
+    args = {"q": q, "k": k, "v": v, "la": la, "beta": beta, "s0": s0}
+    names = {"q": "dq", "k": "dk", "v": "dv", "la": "dlog_alpha", "beta": "dbeta", "s0": "d_init_state"}
+    h = 1e-6
+    for name, x in args.items():
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            lp = _loss(seq, args["q"], args["k"], args["v"], args["la"], args["beta"], args["s0"], do, dfs)
+            x[idx] = old - h
+            lm = _loss(seq, args["q"], args["k"], args["v"], args["la"], args["beta"], args["s0"], do, dfs)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[names[name]], fd, atol=2e-7, rtol=1e-6, err_msg=name)
+
+
+def test_backward_homogeneity_identities():
+    """o and the final state are jointly linear in (V, S0), and o is linear in
+    q (the final state does not depend on q), so by Euler's identity
+    <dV, V> + <dS0, S0> = L and <dq, q> = <do, o> exactly (up to rounding)."""
+    seq, q, k, v, la, beta, s0, do, dfs = _loss_inputs(52, lens=(37, 1, 70), H=3, dk=8, dv=5)
+    g = oracle.backward(q, k, v, la, beta, seq, do, d_final_state=dfs, init_state=s0)
+    o, fs = oracle.forward(q, k, v, la, beta, seq, init_state=s0)
+    L = np.sum(o * do) + np.sum(fs * dfs)
+    np.testing.assert_allclose(np.sum(g["dv"] * v) + np.sum(g["d_init_state"] * s0), L, rtol=1e-10)
+    np.testing.assert_allclose(np.sum(g["dq"] * q), np.sum(o * do), rtol=1e-10)
+
+
+def test_backward_alpha_zero_cuts_the_gradient():
+    """alpha = 0 at token 40 clears the memory (tahou, Gated DeltaNet section):
+    outputs from token 40 on do not depend on anything before it, so changing
+    their upstream gradients leaves the gradients of tokens 0..39 and of S0
+    unchanged, and log alpha at token 40 gets zero gradient (the decayed state
+    is zero)."""
+    seq, q, k, v, la, beta, s0, do, dfs = _loss_inputs(53, lens=(90,), H=2, dk=6, dv=4)
+    la[40] = -np.inf
+    g1 = oracle.backward(q, k, v, la, beta, seq, do, d_final_state=dfs, init_state=s0)
+    do2 = do.copy()
+    do2[40:] = np.random.default_rng(9).standard_normal(do2[40:].shape)
+    g2 = oracle.backward(q, k, v, la, beta, seq, do2, d_final_state=2 * dfs, init_state=s0)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        np.testing.assert_array_equal(g1[name][:40], g2[name][:40], err_msg=name)
+    np.testing.assert_array_equal(g1["d_init_state"], g2["d_init_state"])
+    assert np.all(g1["dlog_alpha"][40] == 0.0)
+    assert not np.allclose(g1["dv"][40:], g2["dv"][40:])
+
+
+def test_backward_long_sequence_crosses_checkpoints():
+    """A 200-token sequence (checkpoint copies every 64 tokens) gives the same
+    gradients as the same tokens run as one forward/backward with the state
+    handed over at token 130 (two sequences chained through the initial
+    state and its gradient)."""
+    seq, q, k, v, la, beta, s0, do, dfs = _loss_inputs(54, lens=(200,), H=1, dk=5, dv=3)
+    g = oracle.backward(q, k, v, la, beta, seq, do, d_final_state=dfs, init_state=s0)
+    a, b = slice(0, 130), slice(130, 200)
+    _, s_mid = oracle.forward(q[a], k[a], v[a], la[a], beta[a], [0, 130], init_state=s0)
+    g2 = oracle.backward(q[b], k[b], v[b], la[b], beta[b], [0, 70], do[b], d_final_state=dfs, init_state=s_mid)
+    g1 = oracle.backward(q[a], k[a], v[a], la[a], beta[a], [0, 130], do[a], d_final_state=g2["d_init_state"],
+                         init_state=s0)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta"):
+        np.testing.assert_allclose(np.concatenate([g1[name], g2[name]]), g[name], rtol=1e-9, atol=1e-12,
+                                   err_msg=name)
+    np.testing.assert_allclose(g1["d_init_state"], g["d_init_state"], rtol=1e-9, atol=1e-12)

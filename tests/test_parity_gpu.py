@@ -175,6 +175,26 @@ def test_prefill_empty_and_no_final_state(cuda_ok):
     torch.testing.assert_close(o1, o2, rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("algo", ["tc", "simt"])
+def test_prefill_final_state_may_alias_init_state(cuda_ok, algo):
+    """final_state may be the init_state buffer (updated in place): same o and
+    state, bit for bit, as with separate buffers; also through the no-alloc call."""
+    inp = _to(make_prefill("prefill", lengths=[130, 0, 64, 200], H=3, seed=77), DEV)
+    o1, f1 = _run(inp, algo=algo)
+    st = inp.init_state.clone()
+    o2, f2 = kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, init_state=st, final_state=st,
+                           cu_seqlens=inp.cu_seqlens, C=64, algo=algo)
+    torch.cuda.synchronize()
+    assert f2 is st
+    assert torch.equal(o2, o1) and torch.equal(st, f1)
+    if algo == "tc":
+        st = inp.init_state.clone()
+        o3, _ = kda.chunk_fwd_noalloc(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, init_state=st, final_state=st,
+                                      cu_seqlens=inp.cu_seqlens, C=64)
+        torch.cuda.synchronize()
+        assert torch.equal(o3, o1) and torch.equal(st, f1)
+
+
 def test_prefill_resume_and_handoff(cuda_ok):
     """Prefill of x[:t1] then x[t1:] from the carried state equals one prefill;
     prefill of T tokens then decode steps equals prefill of T + m tokens."""
