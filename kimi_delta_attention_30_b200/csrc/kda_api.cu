@@ -104,7 +104,7 @@ SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
 // Backward workspace: the CUDA-core forward's scratch, then the gradient scratch.
 struct BwdLayout {
     SimtLayout fwd;
-    size_t off[9];
+    size_t off[12];
     size_t total;
 };
 
@@ -114,9 +114,10 @@ BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C) {
     size_t o = L.fwd.total;
     const size_t tok = (size_t)p.total_tokens * H;
     const size_t ch = (size_t)p.n_chunks * H;
-    const size_t sizes[9] = {ch * dk * dv, tok * dv, ch * C * C, tok * dk, tok * dk, tok * dk, tok * dk,
-                             ch * dk, ch * C * C};   // dS_chunk dW P dQg dKd dWk dKg dGam dAt
-    for (int i = 0; i < 9; ++i) {
+    const size_t sizes[12] = {ch * dk * dv, tok * dv, ch * C * C, tok * dk, tok * dk, tok * dk, tok * dk,
+                              ch * dk, ch * C * C, ch * C * C, tok * dk, tok * dk};
+    // dS_chunk dW P dQg dKd dWk dKg dGam dAt At Qg Kd
+    for (int i = 0; i < 12; ++i) {
         L.off[i] = o;
         o = align_up(o + sizes[i] * sizeof(float));
     }
@@ -413,6 +414,9 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     w.dKg = f(L.off[6]);
     w.dGam = f(L.off[7]);
     w.dAt = f(L.off[8]);
+    w.At = f(L.off[9]);
+    w.Qg = f(L.off[10]);
+    w.Kd = f(L.off[11]);
     timing_mark(s, 0);
     cudaError_t err = launch_simt_backward(dtype, q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq,
                                            dk_out, dv_out, dlog_alpha, dbeta, d_init_state, cmap, smap, p.n_chunks,

@@ -39,6 +39,8 @@ namespace {
 constexpr int kT = 256;
 constexpr int kBV = 32;       // d_v columns per chain block / per tile
 constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
+constexpr int kMaxDK = 128;
+constexpr int kBwdC = 64;     // the backward kernels tile by 64 tokens
 
 __device__ __forceinline__ float wsum(float x) {
 #pragma unroll
@@ -48,12 +50,15 @@ __device__ __forceinline__ float wsum(float x) {
 
 __device__ __forceinline__ size_t tok_off(int t, int H, int h, int d) { return ((size_t)t * H + h) * d; }
 
-// P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic) for i <= r < L, zero elsewhere.
+// P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic) for i <= r < L and At[r][i] (the same
+// with k_r, i < r), zero elsewhere, from one exponential per (r, i, c); and the
+// elementwise Qg = q exp(g), Kd = k exp(g_C - g) the chain and the later kernels read.
 // One block per (chunk, head); shared Qs, Ks, Gs, GLs [C][dk].
 template <typename Tin>
 __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                            const float* __restrict__ g, const float* __restrict__ gl,
-                                           float* __restrict__ P, ChunkMap cmap, int H, int dk, int C) {
+                                           float* __restrict__ P, float* __restrict__ At, float* __restrict__ Qg,
+                                           float* __restrict__ Kd, ChunkMap cmap, int H, int dk, int C) {
     extern __shared__ float smem[];
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
@@ -72,16 +77,31 @@ __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin*
     }
     __syncthreads();
     float* Pc = P + ((size_t)blockIdx.x * H + h) * C * C;
+    float* Ac = At + ((size_t)blockIdx.x * H + h) * C * C;
     for (int p = warp; p < C * C; p += kT / 32) {
         const int r = p / C, i = p - r * C;
-        float s = 0.f;
+        float s = 0.f, a = 0.f;
         if (r < len && i <= r) {
-            for (int c = lane; c < dk; c += 32)
-                s += Qs[r * dk + c] * Ks[i * dk + c] *
-                     exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
+            for (int c = lane; c < dk; c += 32) {
+                const float ke = Ks[i * dk + c] *
+                                 exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
+                s += Qs[r * dk + c] * ke;
+                a += Ks[r * dk + c] * ke;
+            }
             s = wsum(s);
+            a = wsum(a);
         }
-        if (lane == 0) Pc[p] = s;
+        if (lane == 0) {
+            Pc[p] = s;
+            Ac[p] = (i < r) ? a : 0.f;
+        }
+    }
+    for (int e = tid; e < len * dk; e += kT) {
+        const int r = e / dk, c = e - r * dk;
+        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
+        const int l = (len - 1) * dk + c;
+        Qg[off] = Qs[e] * exp_g(Gs[e], GLs[e]);
+        Kd[off] = Ks[e] * exp_gdiff(Gs[l], GLs[l], Gs[e], GLs[e]);
     }
 }
 
@@ -90,7 +110,7 @@ __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin*
 // the initial-state gradient.  Shared: dS [dk][kBV], M1 [C][dk] (Kd, then Qg),
 // M2 [C][dk] (Wk), dOs [C][kBV], dWs [C][kBV], Ps [C][C], gC, gCl [dk].
 template <typename Tin>
-__global__ void __launch_bounds__(kT) kb_chain(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, const float* __restrict__ Kd,
                                                const float* __restrict__ g, const float* __restrict__ gl,
                                                const float* __restrict__ Wk,
                                                const float* __restrict__ P, const Tin* __restrict__ d_o,
@@ -139,32 +159,66 @@ __global__ void __launch_bounds__(kT) kb_chain(const Tin* __restrict__ q, const 
         for (int e = tid; e < L * dk; e += kT) {
             const int r = e / dk, c = e - r * dk;
             const size_t off = tok_off(t0 + r, H, h, dk) + c;
-            M1[e] = to_f32(k[off]) * exp_gdiff(gC[c], gCl[c], g[off], gl[off]);   // Kd
+            M1[e] = Kd[off];
             M2[e] = Wk[off];
         }
         __syncthreads();
-        // dW = P^T dO + Kd dS'
-        for (int e = tid; e < L * kBV; e += kT) {
-            const int i = e / kBV, j = e - i * kBV;
-            float s = 0.f;
-            for (int r = i; r < L; ++r) s += Ps[r * C + i] * dOs[r * kBV + j];
-            for (int c = 0; c < dk; ++c) s += M1[i * dk + c] * dS[c * kBV + j];
-            dWs[e] = s;
-            dW[tok_off(t0 + i, H, h, dv) + j0 + j] = s;
+        // dW = P^T dO + Kd dS' (P is zero above its diagonal): thread t forms column
+        // t % 32 of rows t / 32 + 8 m
+        {
+            const int j = tid & 31, i0 = tid >> 5;
+            float acc[kBwdC / 8];
+#pragma unroll
+            for (int m = 0; m < kBwdC / 8; ++m) acc[m] = 0.f;
+            for (int r = 0; r < L; ++r) {
+                const float o = dOs[r * kBV + j];
+#pragma unroll
+                for (int m = 0; m < kBwdC / 8; ++m) acc[m] = fmaf(Ps[r * C + i0 + 8 * m], o, acc[m]);
+            }
+            for (int c = 0; c < dk; ++c) {
+                const float ds = dS[c * kBV + j];
+#pragma unroll
+                for (int m = 0; m < kBwdC / 8; ++m) acc[m] = fmaf(M1[(i0 + 8 * m) * dk + c], ds, acc[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < kBwdC / 8; ++m) {
+                const int i = i0 + 8 * m;
+                if (i < L) {
+                    dWs[i * kBV + j] = acc[m];
+                    dW[tok_off(t0 + i, H, h, dv) + j0 + j] = acc[m];
+                }
+            }
         }
         __syncthreads();
         for (int e = tid; e < L * dk; e += kT) {
             const int r = e / dk, c = e - r * dk;
             const size_t off = tok_off(t0 + r, H, h, dk) + c;
-            M1[e] = to_f32(q[off]) * exp_g(g[off], gl[off]);                     // Qg
+            M1[e] = Qg[off];
         }
         __syncthreads();
-        // dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW
-        for (int e = tid; e < dk * kBV; e += kT) {
-            const int c = e / kBV, j = e - c * kBV;
-            float s = exp_g(gC[c], gCl[c]) * dS[e];
-            for (int r = 0; r < L; ++r) s += M1[r * dk + c] * dOs[r * kBV + j] - M2[r * dk + c] * dWs[r * kBV + j];
-            dS[e] = s;
+        // dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW: thread t forms column t % 32 of
+        // rows t / 32 + 8 m (each element is read and written by its own thread)
+        {
+            const int j = tid & 31, c0 = tid >> 5;
+            float acc[kMaxDK / 8];
+#pragma unroll
+            for (int m = 0; m < kMaxDK / 8; ++m) {
+                const int c = c0 + 8 * m;
+                acc[m] = c < dk ? exp_g(gC[c], gCl[c]) * dS[c * kBV + j] : 0.f;
+            }
+            for (int r = 0; r < L; ++r) {
+                const float o = dOs[r * kBV + j], w = dWs[r * kBV + j];
+#pragma unroll
+                for (int m = 0; m < kMaxDK / 8; ++m) {
+                    const int c = c0 + 8 * m;
+                    if (c < dk) acc[m] += M1[r * dk + c] * o - M2[r * dk + c] * w;
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < kMaxDK / 8; ++m) {
+                const int c = c0 + 8 * m;
+                if (c < dk) dS[c * kBV + j] = acc[m];
+            }
         }
         __syncthreads();
     }
@@ -179,7 +233,7 @@ __global__ void __launch_bounds__(kT) kb_chain(const Tin* __restrict__ q, const 
 // Per (chunk, head): dQg = dO S^T, dKd = W dS'^T, dWk = -dW S^T (rows x DK),
 // dGam = rowsum(dS' . S), and dP = dO W^T (i <= r, written over P).  d_v is
 // walked in tiles of kBV columns.  Thread t owns channel c = t % DK of rows
-// r = t / DK + m (kT / DK).  Shared: St, dSt [kBV][DK] (transposed tiles),
+// r = t / DK + m (kT / DK).  Shared: St, dSt [kBV][DK + 1] (transposed tiles),
 // dOs, Ws, dWs [C][kBP].
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const float* __restrict__ W,
@@ -194,9 +248,10 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
     const int h = blockIdx.y, tid = threadIdx.x, c = tid % DK, rg = tid / DK;
+    constexpr int SP = DK + 1;     // padded row stride of the transposed state tiles
     float* St = smem;
-    float* dSt = St + kBV * DK;
-    float* dOs = dSt + kBV * DK;
+    float* dSt = St + kBV * SP;
+    float* dOs = dSt + kBV * SP;
     float* Ws = dOs + C * kBP;
     float* dWs = Ws + C * kBP;
     const size_t chunk = blockIdx.x;
@@ -213,8 +268,8 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
     for (int jt = 0; jt < dv; jt += kBV) {
         for (int e = tid; e < kBV * DK; e += kT) {
             const int cc = e / kBV, j = e - cc * kBV;
-            St[j * DK + cc] = S_chunk[sc_base + (size_t)cc * dv + jt + j];
-            dSt[j * DK + cc] = dS_chunk[sc_base + (size_t)cc * dv + jt + j];
+            St[j * SP + cc] = S_chunk[sc_base + (size_t)cc * dv + jt + j];
+            dSt[j * SP + cc] = dS_chunk[sc_base + (size_t)cc * dv + jt + j];
         }
         for (int e = tid; e < C * kBV; e += kT) {
             const int r = e / kBV, j = e - r * kBV;
@@ -234,14 +289,14 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
             const int r = rg + m * NRG;
 #pragma unroll 8
             for (int j = 0; j < kBV; ++j) {
-                const float s = St[j * DK + c], ds = dSt[j * DK + c];
+                const float s = St[j * SP + c], ds = dSt[j * SP + c];
                 aQ[m] += dOs[r * kBP + j] * s;
                 aD[m] += Ws[r * kBP + j] * ds;
                 aW[m] -= dWs[r * kBP + j] * s;
             }
         }
         if (rg == 0)
-            for (int j = 0; j < kBV; ++j) gam += dSt[j * DK + c] * St[j * DK + c];
+            for (int j = 0; j < kBV; ++j) gam += dSt[j * SP + c] * St[j * SP + c];
 #pragma unroll
         for (int m = 0; m < C / 4; ++m) {
             const int r = pr + 4 * m;
@@ -270,13 +325,12 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
 }
 
 // Per (chunk, head): At, the back substitution for [Y | Z], dv, dKg, dbeta and
-// dAt.  Shared: At, dA [C][C], bs, db [C], R: Ks, Gs, GLs [C][dk] (phase 1), then
-// X = [Y | Z] [C][dv + dk]; after R (max(3 C dk, C (dv + dk)) floats) UW = [U | Wk]
-// [C][dv + dk].
+// dAt.  Shared: At, dA [C][C], bs, db [C], X = [Y | Z] [C][dv + dk + 1], UW =
+// [U | Wk] [C][dv + dk + 1] (rows padded by one float against bank conflicts).
 template <typename Tin>
 __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                            const Tin* __restrict__ beta, const float* __restrict__ g,
-                                           const float* __restrict__ gl,
+                                           const float* __restrict__ gl, const float* __restrict__ Atg,
                                            const float* __restrict__ U, const float* __restrict__ Wk,
                                            const float* __restrict__ dW, const float* __restrict__ dWk,
                                            Tin* __restrict__ dv_out, Tin* __restrict__ dbeta_out,
@@ -286,52 +340,39 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
     const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ncol = dv + dk;
+    const int ncol = dv + dk, xs = ncol + 1;
     float* At = smem;
     float* dA = At + C * C;
     float* bs = dA + C * C;
     float* db = bs + C;
-    float* R = db + C;
-    float* Ks = R;
-    float* Gs = R + C * dk;
-    float* GLs = Gs + C * dk;
-    float* X = R;
-    float* UW = R + max(3 * C * dk, C * ncol);
+    float* X = db + C;
+    float* UW = X + C * xs;
 
-    for (int e = tid; e < len * dk; e += kT) {
-        const int r = e / dk, c = e - r * dk;
-        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
-        Ks[e] = to_f32(k[off]);
-        Gs[e] = g[off];
-        GLs[e] = gl[off];
-    }
+    for (int e = tid; e < C * C; e += kT) At[e] = Atg[((size_t)blockIdx.x * H + h) * C * C + e];
     for (int r = tid; r < C; r += kT) {
         bs[r] = r < len ? to_f32(beta[(size_t)(tok0 + r) * H + h]) : 0.f;
         db[r] = 0.f;
     }
     for (int e = tid; e < len * ncol; e += kT) {
         const int r = e / ncol, j = e - r * ncol;
-        UW[e] = j < dv ? U[tok_off(tok0 + r, H, h, dv) + j] : Wk[tok_off(tok0 + r, H, h, dk) + j - dv];
+        UW[r * xs + j] = j < dv ? U[tok_off(tok0 + r, H, h, dv) + j] : Wk[tok_off(tok0 + r, H, h, dk) + j - dv];
     }
+    for (int e = len * xs + tid; e < C * xs; e += kT) UW[e] = 0.f;
     __syncthreads();
-    for (int p = warp; p < C * C; p += kT / 32) {
-        const int r = p / C, i = p - r * C;
-        float s = 0.f;
-        if (r < len && i < r) {
-            for (int c = lane; c < dk; c += 32)
-                s += Ks[r * dk + c] * Ks[i * dk + c] *
-                     exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
-            s = wsum(s);
-        }
-        if (lane == 0) At[p] = s;
+    // (I + A)^T [Y | Z] = [dW | dWk]: right-hand sides loaded whole, then one
+    // column per thread, rows from the last (A_ir = beta_i At_ir scaled once)
+    for (int e = tid; e < len * ncol; e += kT) {
+        const int r = e / ncol, j = e - r * ncol;
+        X[r * xs + j] = j < dv ? dW[tok_off(tok0 + r, H, h, dv) + j] : dWk[tok_off(tok0 + r, H, h, dk) + j - dv];
     }
+    for (int e = len * xs + tid; e < C * xs; e += kT) X[e] = 0.f;
+    for (int e = tid; e < C * C; e += kT) dA[e] = bs[e / C] * At[e];   // A, until dA is formed
     __syncthreads();
-    // (I + A)^T [Y | Z] = [dW | dWk], one column per thread, rows from the last
     for (int j = tid; j < ncol; j += kT) {
         for (int r = len - 1; r >= 0; --r) {
-            float s = j < dv ? dW[tok_off(tok0 + r, H, h, dv) + j] : dWk[tok_off(tok0 + r, H, h, dk) + j - dv];
-            for (int i = r + 1; i < len; ++i) s -= bs[i] * At[i * C + r] * X[i * ncol + j];
-            X[r * ncol + j] = s;
+            float s = X[r * xs + j];
+            for (int i = r + 1; i < len; ++i) s -= dA[i * C + r] * X[i * xs + j];
+            X[r * xs + j] = s;
         }
     }
     __syncthreads();
@@ -340,7 +381,7 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
         const float b = bs[r];
         float s = 0.f;
         for (int j = lane; j < ncol; j += 32) {
-            const float x = X[r * ncol + j];
+            const float x = X[r * xs + j];
             if (j < dv) {
                 const size_t off = tok_off(tok0 + r, H, h, dv) + j;
                 dv_out[off] = from_f32<Tin>(b * x);
@@ -354,15 +395,33 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
         s = wsum(s);
         if (lane == 0) db[r] = s;
     }
-    // dA = -(Y U^T + Z Wk^T), i < r (one warp per pair)
-    for (int p = warp; p < C * C; p += kT / 32) {
-        const int r = p / C, i = p - r * C;
-        float s = 0.f;
-        if (r < len && i < r) {
-            for (int j = lane; j < ncol; j += 32) s += X[r * ncol + j] * UW[i * ncol + j];
-            s = -wsum(s);
+    __syncthreads();   // the rows of X are read by other threads below (and dA is overwritten)
+    // dA = -(Y U^T + Z Wk^T), i < r: thread t forms rows t / 16 + 16 m, columns t % 16 + 16 n
+    {
+        const int rb = tid >> 4, ib = tid & 15;
+        float acc[4][4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
+        for (int j = 0; j < ncol; ++j) {
+            float xr[4], ui[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) xr[m] = X[(rb + 16 * m) * xs + j];
+#pragma unroll
+            for (int n = 0; n < 4; ++n) ui[n] = UW[(ib + 16 * n) * xs + j];
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int n = 0; n < 4; ++n) acc[m][n] = fmaf(xr[m], ui[n], acc[m][n]);
         }
-        if (lane == 0) dA[p] = s;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int r = rb + 16 * m, i = ib + 16 * n;
+                dA[r * C + i] = (r < len && i < r) ? -acc[m][n] : 0.f;
+            }
     }
     __syncthreads();
     float* dAc = dAt + ((size_t)blockIdx.x * H + h) * C * C;
@@ -490,9 +549,8 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
                        const Tin* d_o, Tin* dq, Tin* dk_, Tin* dv_, Tin* dla, Tin* dbeta, const ChunkMap& cmap,
                        int n_chunks, int H, int dv, const BwdWorkspace& ws, cudaStream_t stream) {
     constexpr int C = 64;
-    const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * DK + 3 * (size_t)C * kBP);
-    const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + std::max((size_t)3 * C * DK, (size_t)C * (dv + DK)) +
-                                           (size_t)C * (dv + DK));
+    const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * (DK + 1) + 3 * (size_t)C * kBP);
+    const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + 2 * (size_t)C * (dv + DK + 1));
     const size_t smem_c = sizeof(float) * ((4 + kT / DK) * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
@@ -502,8 +560,8 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     kb_a<Tin, DK><<<grid, kT, smem_a, stream>>>(d_o, ws.fwd.W, ws.dW, ws.fwd.S_chunk, ws.dS_chunk, ws.dQg, ws.dKd,
                                                ws.dWk, ws.dGam, ws.P, cmap, H, dv);
     timing_mark(stream, 4);
-    kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.fwd.U, ws.fwd.Wk, ws.dW, ws.dWk, dv_,
-                                            dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
+    kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
+                                            ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
     timing_mark(stream, 5);
     kb_c<Tin, DK><<<grid, kT, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg,
                                                ws.dGam, ws.dWk, dq, dk_, dla, cmap, H);
@@ -528,11 +586,13 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
     if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
         return e;
     if (n_chunks > 0)
-        kb_p<Tin><<<dim3(n_chunks, H), kT, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, cmap, H, dk, C);
+        kb_p<Tin><<<dim3(n_chunks, H), kT, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg, ws.Kd,
+                                                             cmap, H, dk, C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
         kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kT, smem_chain, stream>>>(
-            q, k, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, H, dk, dv, C);
+            ws.Qg, ws.Kd, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, H, dk,
+            dv, C);
     timing_mark(stream, 3);
     if ((e = cudaGetLastError()) != cudaSuccess || n_chunks == 0) return e;
     if (dk == 128) return run_bwd_dk<Tin, 128>(q, k, v, la, beta, d_o, dq, dk_, dv_, dla, dbeta, cmap, n_chunks, H, dv,

@@ -26,6 +26,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kBV = 32;   // d_v columns per state-carry block
+constexpr int kMaxDK = 128;
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -91,32 +92,42 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
         if (lane == 0) A[r * C + i] = s;
     }
     __syncthreads();
-    // forward substitution, one column per thread; X reuses the Ks/Gs region
+    // forward substitution: the right-hand sides [beta V | beta K exp(g)] are loaded
+    // whole (X reuses the Ks/Gs region), then one column per thread, in place
     float* X = Ks;
     const int ncol = dk + dv;
+    for (int e = tid; e < len * ncol; e += kThreads) {
+        const int r = e / ncol, j = e - r * ncol;
+        const size_t tok = (size_t)(tok0 + r) * H + h;
+        const float br = to_f32(beta[tok]);
+        if (j < dv) {
+            X[e] = br * to_f32(v[tok * dv + j]);
+        } else {
+            const int c = j - dv;
+            X[e] = br * to_f32(k[tok * dk + c]) * exp_g(g[tok * dk + c], gl[tok * dk + c]);
+        }
+    }
+    __syncthreads();
     for (int j = tid; j < ncol; j += kThreads) {
-        for (int r = 0; r < len; ++r) {
-            const size_t tok = (size_t)(tok0 + r) * H + h;
-            const float br = to_f32(beta[tok]);
-            float s;
-            if (j < dv) {
-                s = br * to_f32(v[tok * dv + j]);
-            } else {
-                const int c = j - dv;
-                s = br * to_f32(k[tok * dk + c]) * exp_g(g[tok * dk + c], gl[tok * dk + c]);
-            }
+        for (int r = 1; r < len; ++r) {
+            float s = X[r * ncol + j];
             for (int i = 0; i < r; ++i) s -= A[r * C + i] * X[i * ncol + j];
             X[r * ncol + j] = s;
-            if (j < dv) U[tok * dv + j] = s;
-            else Wk[tok * dk + (j - dv)] = s;
         }
+    }
+    __syncthreads();
+    for (int e = tid; e < len * ncol; e += kThreads) {
+        const int r = e / ncol, j = e - r * ncol;
+        const size_t tok = (size_t)(tok0 + r) * H + h;
+        if (j < dv) U[tok * dv + j] = X[e];
+        else Wk[tok * dk + (j - dv)] = X[e];
     }
 }
 
 // K3: one block per (sequence, head, d_v tile of kBV columns), sequential over
 // the sequence's chunks.  Shared: S [dk][kBV], M [C][dk] (Wk, then K . decay),
 // Ws [C][kBV], gC, gCl [dk].
-template <typename Tin>
+template <typename Tin, int CC>
 __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
                                                      const float* __restrict__ gl,
                                                      const float* __restrict__ U, const float* __restrict__ Wkg,
@@ -153,13 +164,28 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
             M[e] = Wkg[((size_t)(t0 + r) * H + h) * dk + c];
         }
         __syncthreads();
-        // W = U - Wk S
-        for (int e = tid; e < L * kBV; e += kThreads) {
-            int r = e / kBV, j = e - r * kBV;
-            float s = U[((size_t)(t0 + r) * H + h) * dv + j0 + j];
-            for (int c = 0; c < dk; ++c) s -= M[r * dk + c] * S[c * kBV + j];
-            Ws[e] = s;
-            Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = s;
+        // W = U - Wk S: thread t forms column t % 32 of rows t / 32 + 8 m
+        {
+            const int j = tid & 31, r0 = tid >> 5;
+            float acc[CC / 8];
+#pragma unroll
+            for (int m = 0; m < CC / 8; ++m) {
+                const int r = r0 + 8 * m;
+                acc[m] = r < L ? U[((size_t)(t0 + r) * H + h) * dv + j0 + j] : 0.f;
+            }
+            for (int c = 0; c < dk; ++c) {
+                const float sv = S[c * kBV + j];
+#pragma unroll
+                for (int m = 0; m < CC / 8; ++m) acc[m] -= M[(r0 + 8 * m) * dk + c] * sv;   // rows >= L unused
+            }
+#pragma unroll
+            for (int m = 0; m < CC / 8; ++m) {
+                const int r = r0 + 8 * m;
+                if (r < L) {
+                    Ws[r * kBV + j] = acc[m];
+                    Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = acc[m];
+                }
+            }
         }
         __syncthreads();
         for (int c = tid; c < dk; c += kThreads) {
@@ -173,12 +199,27 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
             M[e] = to_f32(k[off]) * exp_gdiff(gC[c], gCl[c], g[off], gl[off]);
         }
         __syncthreads();
-        // S <- Diag(exp(g_C)) S + (K . exp(g_C - g))^T W
-        for (int e = tid; e < dk * kBV; e += kThreads) {
-            int c = e / kBV, j = e - c * kBV;
-            float s = exp_g(gC[c], gCl[c]) * S[e];
-            for (int r = 0; r < L; ++r) s += M[r * dk + c] * Ws[r * kBV + j];
-            S[e] = s;
+        // S <- Diag(exp(g_C)) S + (K . exp(g_C - g))^T W: thread t forms column t % 32
+        // of rows t / 32 + 8 m (each element is read and written by its own thread)
+        {
+            const int j = tid & 31, c0 = tid >> 5;
+            float acc[kMaxDK / 8];
+#pragma unroll
+            for (int m = 0; m < kMaxDK / 8; ++m) {
+                const int c = c0 + 8 * m;
+                acc[m] = c < dk ? exp_g(gC[c], gCl[c]) * S[c * kBV + j] : 0.f;
+            }
+            for (int r = 0; r < L; ++r) {
+                const float w = Ws[r * kBV + j];
+#pragma unroll
+                for (int m = 0; m < kMaxDK / 8; ++m)
+                    if (c0 + 8 * m < dk) acc[m] += M[r * dk + c0 + 8 * m] * w;
+            }
+#pragma unroll
+            for (int m = 0; m < kMaxDK / 8; ++m) {
+                const int c = c0 + 8 * m;
+                if (c < dk) S[c * kBV + j] = acc[m];
+            }
         }
         __syncthreads();
     }
@@ -261,7 +302,8 @@ cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const T
     const size_t smem4 = sizeof(float) * (2 * (size_t)C * dk + (size_t)C * C) + sizeof(__nv_bfloat16) * (size_t)C * dk;
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
-    if ((e = cudaFuncSetAttribute(k3_state<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
+    auto k3 = C == 128 ? k3_state<Tin, 128> : k3_state<Tin, 64>;
+    if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
     if ((e = cudaFuncSetAttribute(k4_output<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem4))) return e;
     if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
     timing_mark(stream, 1);
@@ -270,9 +312,8 @@ cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const T
                                                                  C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
-        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W,
-                                                                            ws.S_chunk, init_state, final_state,
-                                                                            smap, H, dk, dv, C);
+        k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
+                                                                 init_state, final_state, smap, H, dk, dv, C);
     timing_mark(stream, 3);
     if (n_chunks > 0)
         k4_output<Tin><<<dim3(n_chunks, H), kThreads, smem4, stream>>>(q, k, ws.g, ws.gl, ws.W, ws.S_chunk, o, cmap,
@@ -289,16 +330,16 @@ cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* bet
     const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + 2 * dk);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
-    if ((e = cudaFuncSetAttribute(k3_state<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
+    auto k3 = C == 128 ? k3_state<Tin, 128> : k3_state<Tin, 64>;
+    if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
     if (n_chunks > 0) {
         k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
         k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk, dv,
                                                                  C);
     }
     if (n_seqs > 0)
-        k3_state<Tin><<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W,
-                                                                            ws.S_chunk, init_state, nullptr, smap, H,
-                                                                            dk, dv, C);
+        k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
+                                                                 init_state, nullptr, smap, H, dk, dv, C);
     return cudaGetLastError();
 }
 

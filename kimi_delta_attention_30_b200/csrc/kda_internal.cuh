@@ -132,11 +132,13 @@ __device__ __forceinline__ float inv_norm_from_sq(float sum_sq) { return sum_sq 
 // exp(g_a - g_b) formed from two rounded g would carry that as a relative error.
 // The CUDA-core kernels therefore keep g as hi + lo (the fp64 cumulative sum split
 // in two floats) and form differences as (hi_a - hi_b) + (lo_a - lo_b).
+// Both use 2^x on the SFU: a relative error near 2^-22, plus the rounding of the
+// exponent times log2 e (3e-7 relative at |exponent| = 5, where terms still count).
 __device__ __forceinline__ float exp_gdiff(float ah, float al, float bh, float bl) {
-    return expf((ah - bh) + (al - bl));
+    return ex2_approx(((ah - bh) + (al - bl)) * kLog2e);
 }
 // exp(g) for g = hi + lo, |lo| <= ulp(hi) / 2: exp(hi) (1 + lo) to second order.
-__device__ __forceinline__ float exp_g(float h, float l) { return expf(h) * (1.f + l); }
+__device__ __forceinline__ float exp_g(float h, float l) { return ex2_approx(h * kLog2e) * (1.f + l); }
 
 // ---- optional per-kernel timing hook (see kda_set_timing_events) -----------
 
@@ -189,6 +191,9 @@ struct BwdWorkspace {
     float* dKg;         // [tokens, H, dk]
     float* dGam;        // [chunks, H, dk]
     float* dAt;         // [chunks, H, C, C] gradient w.r.t. the unscaled key products
+    float* At;          // [chunks, H, C, C] the unscaled key products (strictly lower)
+    float* Qg;          // [tokens, H, dk] q . exp(g)
+    float* Kd;          // [tokens, H, dk] k . exp(g_C - g)
 };
 
 cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
