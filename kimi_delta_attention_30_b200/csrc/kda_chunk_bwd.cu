@@ -37,6 +37,7 @@ namespace kda {
 namespace {
 
 constexpr int kT = 256;
+constexpr int kTW = 512;      // the pairwise kernels (kb_p, kb_c): more warps to hide latency
 constexpr int kBV = 32;       // d_v columns per chain block / per tile
 constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
 constexpr int kMaxDK = 128;
@@ -55,7 +56,7 @@ __device__ __forceinline__ size_t tok_off(int t, int H, int h, int d) { return (
 // elementwise Qg = q exp(g), Kd = k exp(g_C - g) the chain and the later kernels read.
 // One block per (chunk, head); shared Qs, Ks, Gs, GLs [C][dk].
 template <typename Tin>
-__global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(kTW) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                            const float* __restrict__ g, const float* __restrict__ gl,
                                            float* __restrict__ P, float* __restrict__ At, float* __restrict__ Qg,
                                            float* __restrict__ Kd, ChunkMap cmap, int H, int dk, int C) {
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin*
     float* Ks = Qs + C * dk;
     float* Gs = Ks + C * dk;
     float* GLs = Gs + C * dk;
-    for (int e = tid; e < len * dk; e += kT) {
+    for (int e = tid; e < len * dk; e += kTW) {
         const int r = e / dk, c = e - r * dk;
         const size_t off = tok_off(tok0 + r, H, h, dk) + c;
         Qs[e] = to_f32(q[off]);
@@ -78,7 +79,7 @@ __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin*
     __syncthreads();
     float* Pc = P + ((size_t)blockIdx.x * H + h) * C * C;
     float* Ac = At + ((size_t)blockIdx.x * H + h) * C * C;
-    for (int p = warp; p < C * C; p += kT / 32) {
+    for (int p = warp; p < C * C; p += kTW / 32) {
         const int r = p / C, i = p - r * C;
         float s = 0.f, a = 0.f;
         if (r < len && i <= r) {
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kT) kb_p(const Tin* __restrict__ q, const Tin*
             Ac[p] = (i < r) ? a : 0.f;
         }
     }
-    for (int e = tid; e < len * dk; e += kT) {
+    for (int e = tid; e < len * dk; e += kTW) {
         const int r = e / dk, c = e - r * dk;
         const size_t off = tok_off(tok0 + r, H, h, dk) + c;
         const int l = (len - 1) * dk + c;
@@ -444,9 +445,9 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
 // Phase A (rows): thread t takes channel c = t % DK and rows r = t / DK + m NRG,
 // and leaves its row sums for dk in the dWk buffer (no longer needed); phase B
 // (columns) the same with columns i; phase C one thread per channel.
-// Shared: Qs, Ks, Gs, GLs [C][DK], F [NRG][C][DK], dAs, dPs [C][C], gC, gCl [DK].
+// Shared: Qs, Ks, Gs, GLs, F [C][DK], dAs, dPs [C][C], gC, gCl [DK].
 template <typename Tin, int DK>
-__global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(kTW) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                            const Tin* __restrict__ la, const float* __restrict__ g,
                                            const float* __restrict__ gl,
                                            const float* __restrict__ dAt, const float* __restrict__ dP,
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
                                            Tin* __restrict__ dk_out, Tin* __restrict__ dla_out, ChunkMap cmap,
                                            int H) {
     constexpr int C = 64;
-    constexpr int NRG = kT / DK;
+    constexpr int NRG = kTW / DK;
     extern __shared__ float smem[];
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
@@ -465,13 +466,13 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
     float* Ks = Qs + C * DK;
     float* Gs = Ks + C * DK;
     float* GLs = Gs + C * DK;
-    float* F = GLs + C * DK;         // [NRG][C][DK]
-    float* dAs = F + NRG * C * DK;
+    float* F = GLs + C * DK;         // [C][DK], added to by the row groups with shared atomics
+    float* dAs = F + C * DK;
     float* dPs = dAs + C * C;
     float* gC = dPs + C * C;
     float* gCl = gC + DK;
     const size_t chunk = blockIdx.x;
-    for (int e = tid; e < len * DK; e += kT) {
+    for (int e = tid; e < len * DK; e += kTW) {
         const int r = e / DK, cc = e - r * DK;
         const size_t off = tok_off(tok0 + r, H, h, DK) + cc;
         Qs[e] = to_f32(q[off]);
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
         Gs[e] = g[off];
         GLs[e] = gl[off];
     }
-    for (int e = tid; e < NRG * C * DK; e += kT) F[e] = 0.f;
-    for (int e = tid; e < C * C; e += kT) {
+    for (int e = tid; e < C * DK; e += kTW) F[e] = 0.f;
+    for (int e = tid; e < C * C; e += kTW) {
         dAs[e] = dAt[(chunk * H + h) * C * C + e];
         dPs[e] = dP[(chunk * H + h) * C * C + e];
     }
@@ -489,7 +490,6 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
         gC[c] = Gs[(len - 1) * DK + c];
         gCl[c] = GLs[(len - 1) * DK + c];
     }
-    float* Fm = F + rg * C * DK;
     // phase A: x1 = sum_{i<r} dAt k_i E, x2 = sum_{i<=r} dP k_i E; prefix sums of T_ri into F
     for (int r = rg; r < len; r += NRG) {
         const float gr = Gs[r * DK + c], grl = GLs[r * DK + c];
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
             x1 += a;
             x2 += b;
             pre += kv * a + qv * b;
-            Fm[(i + 1) * DK + c] += pre;   // T_ri with i < j <= r
+            atomicAdd(&F[(i + 1) * DK + c], pre);   // T_ri with i < j <= r
         }
         x2 += dPs[r * C + r] * kv;         // the diagonal of P (E = 1)
         const size_t off = tok_off(tok0 + r, H, h, DK) + c;
@@ -536,9 +536,7 @@ __global__ void __launch_bounds__(kT) kb_c(const Tin* __restrict__ q, const Tin*
             const size_t off = tok_off(tok0 + j, H, h, DK) + c;
             const float eg = exp_g(Gs[j * DK + c], GLs[j * DK + c]);
             suf += (dQg[off] * Qs[j * DK + c] + dKg[off] * Ks[j * DK + c]) * eg;
-            float f = 0.f;
-#pragma unroll
-            for (int m = 0; m < NRG; ++m) f += F[(m * C + j) * DK + c];
+            const float f = F[j * DK + c];
             dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? f + suf + gam : 0.f);
         }
     }
@@ -551,7 +549,7 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     constexpr int C = 64;
     const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * (DK + 1) + 3 * (size_t)C * kBP);
     const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + 2 * (size_t)C * (dv + DK + 1));
-    const size_t smem_c = sizeof(float) * ((4 + kT / DK) * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
+    const size_t smem_c = sizeof(float) * (5 * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
     if ((e = cudaFuncSetAttribute(kb_b<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
@@ -563,7 +561,7 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
                                             ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
     timing_mark(stream, 5);
-    kb_c<Tin, DK><<<grid, kT, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg,
+    kb_c<Tin, DK><<<grid, kTW, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg,
                                                ws.dGam, ws.dWk, dq, dk_, dla, cmap, H);
     timing_mark(stream, 6);
     return cudaGetLastError();
@@ -585,8 +583,10 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
     if ((e = cudaFuncSetAttribute(kb_p<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
     if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
         return e;
+    // two chain blocks per SM (115,712 bytes each at d = 128) need the whole shared-memory carveout
+    if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100))) return e;
     if (n_chunks > 0)
-        kb_p<Tin><<<dim3(n_chunks, H), kT, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg, ws.Kd,
+        kb_p<Tin><<<dim3(n_chunks, H), kTW, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg, ws.Kd,
                                                              cmap, H, dk, C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
