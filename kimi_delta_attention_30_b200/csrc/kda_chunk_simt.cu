@@ -25,6 +25,7 @@ namespace kda {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kThreadsW = 512;   // K2 and K4: their pairwise loops are latency bound at one block per SM
 constexpr int kBV = 32;   // d_v columns per state-carry block
 constexpr int kMaxDK = 128;
 
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(128) k1_cumsum(const Tin* __restrict__ la, flo
 // (the low part of g is staged in bf16: |lo| <= ulp(g) / 2, so bf16 keeps it to
 // ulp(g) 2^-10, below 3e-8 for |g| < 256, and 128-token chunks fit at d = 128)
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, const Tin* __restrict__ v,
+__global__ void __launch_bounds__(kThreadsW) k2_wy(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                                   const Tin* __restrict__ beta, const float* __restrict__ g,
                                                   const float* __restrict__ gl, float* __restrict__ U,
                                                   float* __restrict__ Wk, ChunkMap cmap, int H, int dk, int dv,
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
     float* Gs = Ks + C * dk;
     __nv_bfloat16* GLs = reinterpret_cast<__nv_bfloat16*>(Gs + C * dk);
 
-    for (int e = tid; e < len * dk; e += kThreads) {
+    for (int e = tid; e < len * dk; e += kThreadsW) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         Ks[r * dk + c] = to_f32(k[off]);
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
     }
     __syncthreads();
     // A, one warp per (r, i) pair, lanes over channels
-    for (int p = warp; p < len * len; p += kThreads / 32) {
+    for (int p = warp; p < len * len; p += kThreadsW / 32) {
         int r = p / len, i = p - r * len;
         float s = 0.f;
         if (i < r) {
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
     // whole (X reuses the Ks/Gs region), then one column per thread, in place
     float* X = Ks;
     const int ncol = dk + dv;
-    for (int e = tid; e < len * ncol; e += kThreads) {
+    for (int e = tid; e < len * ncol; e += kThreadsW) {
         const int r = e / ncol, j = e - r * ncol;
         const size_t tok = (size_t)(tok0 + r) * H + h;
         const float br = to_f32(beta[tok]);
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
         }
     }
     __syncthreads();
-    for (int j = tid; j < ncol; j += kThreads) {
+    for (int j = tid; j < ncol; j += kThreadsW) {
         for (int r = 1; r < len; ++r) {
             float s = X[r * ncol + j];
             for (int i = 0; i < r; ++i) s -= A[r * C + i] * X[i * ncol + j];
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) k2_wy(const Tin* __restrict__ k, con
         }
     }
     __syncthreads();
-    for (int e = tid; e < len * ncol; e += kThreads) {
+    for (int e = tid; e < len * ncol; e += kThreadsW) {
         const int r = e / ncol, j = e - r * ncol;
         const size_t tok = (size_t)(tok0 + r) * H + h;
         if (j < dv) U[tok * dv + j] = X[e];
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
 // K4: one block per (chunk, head).  Shared: Ks [C][dk] (then Q . exp(g)),
 // Gs [C][dk], P [C][C], GLs [C][dk] (bf16, as in K2).
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q, const Tin* __restrict__ k,
+__global__ void __launch_bounds__(kThreadsW) k4_output(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                       const float* __restrict__ g, const float* __restrict__ gl,
                                                       const float* __restrict__ Wg,
                                                       const float* __restrict__ S_chunk, Tin* __restrict__ o,
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
     float* Gs = Ks + C * dk;
     float* P = Gs + C * dk;
     __nv_bfloat16* GLs = reinterpret_cast<__nv_bfloat16*>(P + C * C);
-    for (int e = tid; e < len * dk; e += kThreads) {
+    for (int e = tid; e < len * dk; e += kThreadsW) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         Ks[e] = to_f32(k[off]);
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
     }
     __syncthreads();
     // P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic), i <= r (inclusive mask)
-    for (int p = warp; p < len * len; p += kThreads / 32) {
+    for (int p = warp; p < len * len; p += kThreadsW / 32) {
         int r = p / len, i = p - r * len;
         float s = 0.f;
         if (i <= r) {
@@ -270,14 +271,14 @@ __global__ void __launch_bounds__(kThreads) k4_output(const Tin* __restrict__ q,
         if (lane == 0) P[r * C + i] = s;
     }
     __syncthreads();
-    for (int e = tid; e < len * dk; e += kThreads) {
+    for (int e = tid; e < len * dk; e += kThreadsW) {
         int r = e / dk, c = e - r * dk;
         size_t off = ((size_t)(tok0 + r) * H + h) * dk + c;
         Ks[e] = to_f32(q[off]) * exp_g(Gs[e], __bfloat162float(GLs[e]));
     }
     __syncthreads();
     const size_t sc_base = ((size_t)blockIdx.x * H + h) * dk * dv;
-    for (int e = tid; e < len * dv; e += kThreads) {
+    for (int e = tid; e < len * dv; e += kThreadsW) {
         int r = e / dv, j = e - r * dv;
         float s = 0.f;
         for (int c = 0; c < dk; ++c) s += Ks[r * dk + c] * S_chunk[sc_base + (size_t)c * dv + j];
@@ -308,15 +309,15 @@ cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const T
     if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
     timing_mark(stream, 1);
     if (n_chunks > 0)
-        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk, dv,
-                                                                 C);
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreadsW, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk,
+                                                                  dv, C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
         k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
                                                                  init_state, final_state, smap, H, dk, dv, C);
     timing_mark(stream, 3);
     if (n_chunks > 0)
-        k4_output<Tin><<<dim3(n_chunks, H), kThreads, smem4, stream>>>(q, k, ws.g, ws.gl, ws.W, ws.S_chunk, o, cmap,
+        k4_output<Tin><<<dim3(n_chunks, H), kThreadsW, smem4, stream>>>(q, k, ws.g, ws.gl, ws.W, ws.S_chunk, o, cmap,
                                                                      H, dk, dv, C);
     timing_mark(stream, 4);
     return cudaGetLastError();
@@ -334,8 +335,8 @@ cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* bet
     if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
     if (n_chunks > 0) {
         k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
-        k2_wy<Tin><<<dim3(n_chunks, H), kThreads, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk, dv,
-                                                                 C);
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreadsW, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk,
+                                                                  dv, C);
     }
     if (n_seqs > 0)
         k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
