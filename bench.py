@@ -51,6 +51,7 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prep", action="store_true", help="skip the fused-preprocessing timings")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass timings")
+    ap.add_argument("--no-seqpar", action="store_true", help="skip the sequence-parallel timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample length")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="profiling aid: run only one part (the JSON line then lacks the other)")
@@ -517,6 +518,55 @@ def main():
                           "l2": "flushed before every timed step (256 MiB write)"}}
         del grads, bws, d_o, dfs
 
+    # ---------------------------------------------------------------- sequence parallelism
+    # one 65,536-token sequence (H = 32, d = 128, bf16) split into contiguous segments, one per
+    # rank, start states exchanged by one all-gather of per-segment affine maps (seqpar.py).
+    # With N > 1 ranks this is measured; on one GPU the per-rank critical path of an 8-way split
+    # (maps of one segment, then its prefill from the start state) is timed and reported as a
+    # projection beside the single-GPU prefill of the whole sequence.
+    seqp = None
+    if run_prefill and not a.no_seqpar:
+        from kimi_delta_attention_30_b200 import seqpar
+        Tl, Hl = 65536, 32
+        nseg = world if world > 1 else 8
+        seg = Tl // nseg
+        sin = make_prefill("prefill", device=dev, seed=rank, B=1, T=seg, H=Hl)
+        args5 = (sin.q, sin.k, sin.v, sin.log_alpha, sin.beta)
+
+        def timed(fn, n):
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            for _ in range(a.warmup):
+                flush.zero_()
+                fn()
+            barrier()
+            torch.cuda.synchronize()
+            for e0, e1 in evs:
+                flush.zero_()
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in evs)) / n
+
+        if world > 1:
+            ms = timed(lambda: seqpar.seqpar_forward(*args5, init_state=sin.init_state[:1]), a.steps)
+            seqp = {"value": Tl / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "measured": True}
+        else:
+            s0 = sin.init_state[:1].contiguous()
+            ms_maps = timed(lambda: seqpar.segment_maps(*args5), a.steps)
+            ms_pass = timed(lambda: kda.chunk_fwd(*args5, init_state=s0), a.steps)
+            full = make_prefill("prefill", device=dev, seed=rank, B=1, T=Tl, H=Hl)
+            ms_full = timed(lambda: kda.chunk_fwd(full.q, full.k, full.v, full.log_alpha, full.beta,
+                                                  init_state=full.init_state[:1]), a.steps)
+            del full
+            seqp = {"measured": False, "projected_ranks": nseg, "ms_maps_one_segment": ms_maps,
+                    "ms_prefill_one_segment": ms_pass, "projected_ms_per_rank": ms_maps + ms_pass,
+                    "single_gpu_ms": ms_full, "projected_speedup": ms_full / (ms_maps + ms_pass),
+                    "note": "per-rank critical path without the all-gather (2 MiB per rank)"}
+        seqp["config"] = {"workload": f"one sequence T={Tl} H={Hl} d=128 bf16 split into {nseg} segments"}
+        del sin
+
     # ---------------------------------------------------------------- decode
     decode = None
     if run_decode:
@@ -629,7 +679,7 @@ def main():
                            "kernels": kernels, "l2": "flushed before every timed step (256 MiB write)",
                            "parallelism": f"replicas x{world} (independent sequences per GPU)"},
                 "roofline": roofline, "path_roofline": path_roofline, "kernel_times": kernel_table,
-                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "prep": prep, "backward": bwd,
+                "gpu_launches": nk * a.steps if run_prefill else None, "decode": decode, "prep": prep, "backward": bwd, "seqpar": seqp,
                 "e2e": e2e, "cpu_baseline": cpu,
                 "clocks": clk, "wall_s_timed": t_wall, "gpu": props.name}
         print(json.dumps(line), flush=True)
