@@ -52,6 +52,8 @@ def _args():
     ap.add_argument("--no-prep", action="store_true", help="skip the fused-preprocessing timings")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward-pass timings")
     ap.add_argument("--no-seqpar", action="store_true", help="skip the sequence-parallel timings")
+    ap.add_argument("--seqpar", action="store_true",
+                    help="with N > 1 ranks, also time one long sequence split over the ranks (NCCL all-gather)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample length")
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="profiling aid: run only one part (the JSON line then lacks the other)")
@@ -521,11 +523,12 @@ def main():
     # ---------------------------------------------------------------- sequence parallelism
     # one 65,536-token sequence (H = 32, d = 128, bf16) split into contiguous segments, one per
     # rank, start states exchanged by one all-gather of per-segment affine maps (seqpar.py).
-    # With N > 1 ranks this is measured; on one GPU the per-rank critical path of an 8-way split
+    # With N > 1 ranks this is measured when --seqpar is given (the replicas' scaling line does not
+    # depend on it); on one GPU the per-rank critical path of an 8-way split
     # (maps of one segment, then its prefill from the start state) is timed and reported as a
     # projection beside the single-GPU prefill of the whole sequence.
     seqp = None
-    if run_prefill and not a.no_seqpar:
+    if run_prefill and not a.no_seqpar and (world == 1 or a.seqpar):
         from kimi_delta_attention_30_b200 import seqpar
         Tl, Hl = 65536, 32
         nseg = world if world > 1 else 8
