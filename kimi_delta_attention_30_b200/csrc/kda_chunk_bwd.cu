@@ -233,9 +233,11 @@ __global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, con
 
 // Per (chunk, head): dQg = dO S^T, dKd = W dS'^T, dWk = -dW S^T (rows x DK),
 // dGam = rowsum(dS' . S), and dP = dO W^T (i <= r, written over P).  d_v is
-// walked in tiles of kBV columns.  Thread t owns channel c = t % DK of rows
-// r = t / DK + m (kT / DK).  Shared: St, dSt [kBV][DK + 1] (transposed tiles),
-// dOs, Ws, dWs [C][kBP].
+// walked in tiles of kBV columns.  Register tiles: thread t forms rows
+// t / 16 + 16 m (m < 4) and channels t % 16 + 16 n (n < DK / 16) of the three
+// products, and rows t / 16 + 16 m, columns t % 16 + 16 n (n < 4) of dP, so a
+// shared-memory load feeds several multiply-adds and a warp's loads spread over
+// the banks.  Shared: St, dSt [kBV][DK + 1] (transposed tiles), dOs, Ws, dWs [C][kBP].
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const float* __restrict__ W,
                                            const float* __restrict__ dW, const float* __restrict__ S_chunk,
@@ -243,12 +245,12 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
                                            float* __restrict__ dKd, float* __restrict__ dWk, float* __restrict__ dGam,
                                            float* __restrict__ dP, ChunkMap cmap, int H, int dv) {
     constexpr int C = 64;
-    constexpr int NRG = kT / DK;   // row groups
-    constexpr int MR = C / NRG;    // rows per thread
+    constexpr int NC = DK / 16;    // channels per thread
+    static_assert(kT == 256, "tiles of 16 x 16 threads");
     extern __shared__ float smem[];
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
-    const int h = blockIdx.y, tid = threadIdx.x, c = tid % DK, rg = tid / DK;
+    const int h = blockIdx.y, tid = threadIdx.x, rb = tid >> 4, cb = tid & 15;
     constexpr int SP = DK + 1;     // padded row stride of the transposed state tiles
     float* St = smem;
     float* dSt = St + kBV * SP;
@@ -257,15 +259,17 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
     float* dWs = Ws + C * kBP;
     const size_t chunk = blockIdx.x;
     const size_t sc_base = (chunk * H + h) * DK * dv;
-    float aQ[MR], aD[MR], aW[MR];
+    float aQ[4][NC], aD[4][NC], aW[4][NC], aP[4][4];
 #pragma unroll
-    for (int m = 0; m < MR; ++m) aQ[m] = aD[m] = aW[m] = 0.f;
-    float gam = 0.f;
-    // dP: thread t owns column i = t % 64 of rows r = t / 64 + 4 m (m < 16)
-    const int pi = tid & 63, pr = tid >> 6;
-    float aP[C / 4];
+    for (int m = 0; m < 4; ++m) {
 #pragma unroll
-    for (int m = 0; m < C / 4; ++m) aP[m] = 0.f;
+        for (int n = 0; n < NC; ++n) aQ[m][n] = aD[m][n] = aW[m][n] = 0.f;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) aP[m][n] = 0.f;
+    }
+    float gam[NC];
+#pragma unroll
+    for (int n = 0; n < NC; ++n) gam[n] = 0.f;
     for (int jt = 0; jt < dv; jt += kBV) {
         for (int e = tid; e < kBV * DK; e += kT) {
             const int cc = e / kBV, j = e - cc * kBV;
@@ -285,43 +289,66 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
             dWs[r * kBP + j] = d;
         }
         __syncthreads();
+#pragma unroll 4
+        for (int j = 0; j < kBV; ++j) {
+            float o[4], w[4], dw[4], s[NC], ds[NC], wp[4];
 #pragma unroll
-        for (int m = 0; m < MR; ++m) {
-            const int r = rg + m * NRG;
-#pragma unroll 8
-            for (int j = 0; j < kBV; ++j) {
-                const float s = St[j * SP + c], ds = dSt[j * SP + c];
-                aQ[m] += dOs[r * kBP + j] * s;
-                aD[m] += Ws[r * kBP + j] * ds;
-                aW[m] -= dWs[r * kBP + j] * s;
+            for (int m = 0; m < 4; ++m) {
+                const int r = rb + 16 * m;
+                o[m] = dOs[r * kBP + j];
+                w[m] = Ws[r * kBP + j];
+                dw[m] = dWs[r * kBP + j];
+                wp[m] = Ws[(cb + 16 * m) * kBP + j];
             }
-        }
-        if (rg == 0)
-            for (int j = 0; j < kBV; ++j) gam += dSt[j * SP + c] * St[j * SP + c];
 #pragma unroll
-        for (int m = 0; m < C / 4; ++m) {
-            const int r = pr + 4 * m;
-#pragma unroll 8
-            for (int j = 0; j < kBV; ++j) aP[m] += dOs[r * kBP + j] * Ws[pi * kBP + j];
+            for (int n = 0; n < NC; ++n) {
+                s[n] = St[j * SP + cb + 16 * n];
+                ds[n] = dSt[j * SP + cb + 16 * n];
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                for (int n = 0; n < NC; ++n) {
+                    aQ[m][n] = fmaf(o[m], s[n], aQ[m][n]);
+                    aD[m][n] = fmaf(w[m], ds[n], aD[m][n]);
+                    aW[m][n] = fmaf(-dw[m], s[n], aW[m][n]);
+                }
+#pragma unroll
+                for (int n = 0; n < 4; ++n) aP[m][n] = fmaf(o[m], wp[n], aP[m][n]);
+            }
+            if (rb == 0) {
+#pragma unroll
+                for (int n = 0; n < NC; ++n) gam[n] = fmaf(ds[n], s[n], gam[n]);
+            }
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int m = 0; m < MR; ++m) {
-        const int r = rg + m * NRG;
+    for (int m = 0; m < 4; ++m) {
+        const int r = rb + 16 * m;
         if (r < len) {
-            const size_t off = tok_off(tok0 + r, H, h, DK) + c;
-            dQg[off] = aQ[m];
-            dKd[off] = aD[m];
-            dWk[off] = aW[m];
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                const size_t off = tok_off(tok0 + r, H, h, DK) + cb + 16 * n;
+                dQg[off] = aQ[m][n];
+                dKd[off] = aD[m][n];
+                dWk[off] = aW[m][n];
+            }
         }
     }
-    if (rg == 0) dGam[(chunk * H + h) * DK + c] = gam;
+    if (rb == 0) {
+#pragma unroll
+        for (int n = 0; n < NC; ++n) dGam[(chunk * H + h) * DK + cb + 16 * n] = gam[n];
+    }
     float* dPc = dP + (chunk * H + h) * C * C;
 #pragma unroll
-    for (int m = 0; m < C / 4; ++m) {
-        const int r = pr + 4 * m;
-        dPc[r * C + pi] = (r < len && pi <= r) ? aP[m] : 0.f;
+    for (int m = 0; m < 4; ++m) {
+        const int r = rb + 16 * m;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int i = cb + 16 * n;
+            dPc[r * C + i] = (r < len && i <= r) ? aP[m][n] : 0.f;
+        }
     }
 }
 
