@@ -306,7 +306,9 @@ KDA_API kda_status kda_decode_step_prep(const void* q, const void* k, const void
  * The forward intermediates are recomputed inside the call (on CUDA cores, in
  * fp32, with 64-token chunks whatever C asks for: the chunk form does not
  * depend on the chunk length).  dlog_alpha is zero where log_alpha is below
- * the kernels' floor of -100 (log alpha = -inf included).  Errors as
+ * the kernels' floor of -100 (log alpha = -inf included).  dlog_alpha sums
+ * per-row contributions with shared-memory atomics, so repeated calls may
+ * differ in its last bits; the other gradients are reproducible.  Errors as
  * kda_chunk_fwd; all output pointers must be distinct from the inputs.
  */
 KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,
