@@ -106,12 +106,12 @@ __global__ void __launch_bounds__(kTW) kb_p(const Tin* __restrict__ q, const Tin
     }
 }
 
-// Reverse chain over one sequence's chunks, one block per (sequence, head,
-// kBV state columns).  Stores each chunk's end-state gradient dS' and dW, and
+// Reverse chain over one sequence's chunks, one block of kTW threads per
+// (sequence, head, kBV state columns), two blocks per SM (its loads are latency bound).  Stores each chunk's end-state gradient dS' and dW, and
 // the initial-state gradient.  Shared: dS [dk][kBV], M1 [C][dk] (Kd, then Qg),
 // M2 [C][dk] (Wk), dOs [C][kBV], dWs [C][kBV], Ps [C][C], gC, gCl [dk].
 template <typename Tin>
-__global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, const float* __restrict__ Kd,
+__global__ void __launch_bounds__(kTW, 2) kb_chain(const float* __restrict__ Qg, const float* __restrict__ Kd,
                                                const float* __restrict__ g, const float* __restrict__ gl,
                                                const float* __restrict__ Wk,
                                                const float* __restrict__ P, const Tin* __restrict__ d_o,
@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, con
     float* gCl = gC + dk;
 
     const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
-    for (int e = tid; e < dk * kBV; e += kT) {
+    for (int e = tid; e < dk * kBV; e += kTW) {
         const int c = e / kBV, j = e - c * kBV;
         dS[e] = d_final ? d_final[st_base + (size_t)c * dv + j0 + j] : 0.f;
     }
@@ -142,22 +142,22 @@ __global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, con
         const int L = min(C, sq.len - n * C);
         const size_t chunk = (size_t)sq.chunk0 + n;
         const size_t sc_base = (chunk * H + h) * dk * dv;
-        for (int e = tid; e < dk * kBV; e += kT) {
+        for (int e = tid; e < dk * kBV; e += kTW) {
             const int c = e / kBV, j = e - c * kBV;
             dS_chunk[sc_base + (size_t)c * dv + j0 + j] = dS[e];
         }
         const float* Pc = P + (chunk * H + h) * C * C;
-        for (int e = tid; e < C * C; e += kT) Ps[e] = Pc[e];
-        for (int e = tid; e < L * kBV; e += kT) {
+        for (int e = tid; e < C * C; e += kTW) Ps[e] = Pc[e];
+        for (int e = tid; e < L * kBV; e += kTW) {
             const int r = e / kBV, j = e - r * kBV;
             dOs[e] = to_f32(d_o[tok_off(t0 + r, H, h, dv) + j0 + j]);
         }
-        for (int c = tid; c < dk; c += kT) {
+        for (int c = tid; c < dk; c += kTW) {
             gC[c] = g[tok_off(t0 + L - 1, H, h, dk) + c];
             gCl[c] = gl[tok_off(t0 + L - 1, H, h, dk) + c];
         }
         __syncthreads();
-        for (int e = tid; e < L * dk; e += kT) {
+        for (int e = tid; e < L * dk; e += kTW) {
             const int r = e / dk, c = e - r * dk;
             const size_t off = tok_off(t0 + r, H, h, dk) + c;
             M1[e] = Kd[off];
@@ -165,25 +165,25 @@ __global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, con
         }
         __syncthreads();
         // dW = P^T dO + Kd dS' (P is zero above its diagonal): thread t forms column
-        // t % 32 of rows t / 32 + 8 m
+        // t % 32 of rows t / 32 + 16 m
         {
             const int j = tid & 31, i0 = tid >> 5;
-            float acc[kBwdC / 8];
+            float acc[kBwdC / 16];
 #pragma unroll
-            for (int m = 0; m < kBwdC / 8; ++m) acc[m] = 0.f;
+            for (int m = 0; m < kBwdC / 16; ++m) acc[m] = 0.f;
             for (int r = 0; r < L; ++r) {
                 const float o = dOs[r * kBV + j];
 #pragma unroll
-                for (int m = 0; m < kBwdC / 8; ++m) acc[m] = fmaf(Ps[r * C + i0 + 8 * m], o, acc[m]);
+                for (int m = 0; m < kBwdC / 16; ++m) acc[m] = fmaf(Ps[r * C + i0 + 16 * m], o, acc[m]);
             }
             for (int c = 0; c < dk; ++c) {
                 const float ds = dS[c * kBV + j];
 #pragma unroll
-                for (int m = 0; m < kBwdC / 8; ++m) acc[m] = fmaf(M1[(i0 + 8 * m) * dk + c], ds, acc[m]);
+                for (int m = 0; m < kBwdC / 16; ++m) acc[m] = fmaf(M1[(i0 + 16 * m) * dk + c], ds, acc[m]);
             }
 #pragma unroll
-            for (int m = 0; m < kBwdC / 8; ++m) {
-                const int i = i0 + 8 * m;
+            for (int m = 0; m < kBwdC / 16; ++m) {
+                const int i = i0 + 16 * m;
                 if (i < L) {
                     dWs[i * kBV + j] = acc[m];
                     dW[tok_off(t0 + i, H, h, dv) + j0 + j] = acc[m];
@@ -191,40 +191,40 @@ __global__ void __launch_bounds__(kT) kb_chain(const float* __restrict__ Qg, con
             }
         }
         __syncthreads();
-        for (int e = tid; e < L * dk; e += kT) {
+        for (int e = tid; e < L * dk; e += kTW) {
             const int r = e / dk, c = e - r * dk;
             const size_t off = tok_off(t0 + r, H, h, dk) + c;
             M1[e] = Qg[off];
         }
         __syncthreads();
         // dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW: thread t forms column t % 32 of
-        // rows t / 32 + 8 m (each element is read and written by its own thread)
+        // rows t / 32 + 16 m (each element is read and written by its own thread)
         {
             const int j = tid & 31, c0 = tid >> 5;
-            float acc[kMaxDK / 8];
+            float acc[kMaxDK / 16];
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 8; ++m) {
-                const int c = c0 + 8 * m;
+            for (int m = 0; m < kMaxDK / 16; ++m) {
+                const int c = c0 + 16 * m;
                 acc[m] = c < dk ? exp_g(gC[c], gCl[c]) * dS[c * kBV + j] : 0.f;
             }
             for (int r = 0; r < L; ++r) {
                 const float o = dOs[r * kBV + j], w = dWs[r * kBV + j];
 #pragma unroll
-                for (int m = 0; m < kMaxDK / 8; ++m) {
-                    const int c = c0 + 8 * m;
+                for (int m = 0; m < kMaxDK / 16; ++m) {
+                    const int c = c0 + 16 * m;
                     if (c < dk) acc[m] += M1[r * dk + c] * o - M2[r * dk + c] * w;
                 }
             }
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 8; ++m) {
-                const int c = c0 + 8 * m;
+            for (int m = 0; m < kMaxDK / 16; ++m) {
+                const int c = c0 + 16 * m;
                 if (c < dk) dS[c * kBV + j] = acc[m];
             }
         }
         __syncthreads();
     }
     if (d_init) {
-        for (int e = tid; e < dk * kBV; e += kT) {
+        for (int e = tid; e < dk * kBV; e += kTW) {
             const int c = e / kBV, j = e - c * kBV;
             d_init[st_base + (size_t)c * dv + j0 + j] = dS[e];
         }
@@ -353,8 +353,9 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
 }
 
 // Per (chunk, head): At, the back substitution for [Y | Z], dv, dKg, dbeta and
-// dAt.  Shared: At, dA [C][C], bs, db [C], X = [Y | Z] [C][dv + dk + 1], UW =
-// [U | Wk] [C][dv + dk + 1] (rows padded by one float against bank conflicts).
+// dAt.  Shared: At, dA [C][C], bs, db [C], X = [Y | Z] [C][dv + dk + 1] (rows padded
+// by one float against bank conflicts); U and Wk are read through L1 (98 KB of
+// shared memory at d = 128, so two blocks share an SM).
 template <typename Tin>
 __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                            const Tin* __restrict__ beta, const float* __restrict__ g,
@@ -374,18 +375,12 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
     float* bs = dA + C * C;
     float* db = bs + C;
     float* X = db + C;
-    float* UW = X + C * xs;
 
     for (int e = tid; e < C * C; e += kT) At[e] = Atg[((size_t)blockIdx.x * H + h) * C * C + e];
     for (int r = tid; r < C; r += kT) {
         bs[r] = r < len ? to_f32(beta[(size_t)(tok0 + r) * H + h]) : 0.f;
         db[r] = 0.f;
     }
-    for (int e = tid; e < len * ncol; e += kT) {
-        const int r = e / ncol, j = e - r * ncol;
-        UW[r * xs + j] = j < dv ? U[tok_off(tok0 + r, H, h, dv) + j] : Wk[tok_off(tok0 + r, H, h, dk) + j - dv];
-    }
-    for (int e = len * xs + tid; e < C * xs; e += kT) UW[e] = 0.f;
     __syncthreads();
     // (I + A)^T [Y | Z] = [dW | dWk]: right-hand sides loaded whole, then one
     // column per thread, rows from the last (A_ir = beta_i At_ir scaled once)
@@ -432,12 +427,22 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
         for (int m = 0; m < 4; ++m)
 #pragma unroll
             for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
+        // rows i >= len of U, Wk are read as zero
+        const float* urow[4];
+        const float* wrow[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int i = ib + 16 * n;
+            urow[n] = i < len ? U + tok_off(tok0 + i, H, h, dv) : nullptr;
+            wrow[n] = i < len ? Wk + tok_off(tok0 + i, H, h, dk) : nullptr;
+        }
         for (int j = 0; j < ncol; ++j) {
             float xr[4], ui[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) xr[m] = X[(rb + 16 * m) * xs + j];
 #pragma unroll
-            for (int n = 0; n < 4; ++n) ui[n] = UW[(ib + 16 * n) * xs + j];
+            for (int n = 0; n < 4; ++n)
+                ui[n] = urow[n] ? (j < dv ? __ldg(urow[n] + j) : __ldg(wrow[n] + j - dv)) : 0.f;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
 #pragma unroll
@@ -575,7 +580,7 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
                        int n_chunks, int H, int dv, const BwdWorkspace& ws, cudaStream_t stream) {
     constexpr int C = 64;
     const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * (DK + 1) + 3 * (size_t)C * kBP);
-    const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + 2 * (size_t)C * (dv + DK + 1));
+    const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + (size_t)C * (dv + DK + 1));
     const size_t smem_c = sizeof(float) * (5 * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
@@ -617,7 +622,7 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
                                                              cmap, H, dk, C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
-        kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kT, smem_chain, stream>>>(
+        kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kTW, smem_chain, stream>>>(
             ws.Qg, ws.Kd, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, H, dk,
             dv, C);
     timing_mark(stream, 3);

@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kThreadsW) k2_wy(const Tin* __restrict__ k, co
 // the sequence's chunks.  Shared: S [dk][kBV], M [C][dk] (Wk, then K . decay),
 // Ws [C][kBV], gC, gCl [dk].
 template <typename Tin, int CC>
-__global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
+__global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
                                                      const float* __restrict__ gl,
                                                      const float* __restrict__ U, const float* __restrict__ Wkg,
                                                      float* __restrict__ Wg, float* __restrict__ S_chunk,
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
     float* gCl = gC + dk;
 
     const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
-    for (int e = tid; e < dk * kBV; e += kThreads) {
+    for (int e = tid; e < dk * kBV; e += kThreadsW) {
         int c = e / kBV, j = e - c * kBV;
         S[e] = init_state ? init_state[st_base + (size_t)c * dv + j0 + j] : 0.f;
     }
@@ -156,32 +156,32 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
         const int t0 = sq.tok0 + n * C;
         const int L = min(C, sq.len - n * C);
         const size_t sc_base = ((size_t)(sq.chunk0 + n) * H + h) * dk * dv;
-        for (int e = tid; e < dk * kBV; e += kThreads) {
+        for (int e = tid; e < dk * kBV; e += kThreadsW) {
             int c = e / kBV, j = e - c * kBV;
             S_chunk[sc_base + (size_t)c * dv + j0 + j] = S[e];
         }
-        for (int e = tid; e < L * dk; e += kThreads) {
+        for (int e = tid; e < L * dk; e += kThreadsW) {
             int r = e / dk, c = e - r * dk;
             M[e] = Wkg[((size_t)(t0 + r) * H + h) * dk + c];
         }
         __syncthreads();
-        // W = U - Wk S: thread t forms column t % 32 of rows t / 32 + 8 m
+        // W = U - Wk S: thread t forms column t % 32 of rows t / 32 + 16 m
         {
             const int j = tid & 31, r0 = tid >> 5;
-            float acc[CC / 8];
+            float acc[CC / 16];
 #pragma unroll
-            for (int m = 0; m < CC / 8; ++m) {
-                const int r = r0 + 8 * m;
+            for (int m = 0; m < CC / 16; ++m) {
+                const int r = r0 + 16 * m;
                 acc[m] = r < L ? U[((size_t)(t0 + r) * H + h) * dv + j0 + j] : 0.f;
             }
             for (int c = 0; c < dk; ++c) {
                 const float sv = S[c * kBV + j];
 #pragma unroll
-                for (int m = 0; m < CC / 8; ++m) acc[m] -= M[(r0 + 8 * m) * dk + c] * sv;   // rows >= L unused
+                for (int m = 0; m < CC / 16; ++m) acc[m] -= M[(r0 + 16 * m) * dk + c] * sv;   // rows >= L unused
             }
 #pragma unroll
-            for (int m = 0; m < CC / 8; ++m) {
-                const int r = r0 + 8 * m;
+            for (int m = 0; m < CC / 16; ++m) {
+                const int r = r0 + 16 * m;
                 if (r < L) {
                     Ws[r * kBV + j] = acc[m];
                     Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = acc[m];
@@ -189,43 +189,43 @@ __global__ void __launch_bounds__(kThreads) k3_state(const Tin* __restrict__ k, 
             }
         }
         __syncthreads();
-        for (int c = tid; c < dk; c += kThreads) {
+        for (int c = tid; c < dk; c += kThreadsW) {
             gC[c] = g[((size_t)(t0 + L - 1) * H + h) * dk + c];
             gCl[c] = gl[((size_t)(t0 + L - 1) * H + h) * dk + c];
         }
         __syncthreads();
-        for (int e = tid; e < L * dk; e += kThreads) {
+        for (int e = tid; e < L * dk; e += kThreadsW) {
             int r = e / dk, c = e - r * dk;
             size_t off = ((size_t)(t0 + r) * H + h) * dk + c;
             M[e] = to_f32(k[off]) * exp_gdiff(gC[c], gCl[c], g[off], gl[off]);
         }
         __syncthreads();
         // S <- Diag(exp(g_C)) S + (K . exp(g_C - g))^T W: thread t forms column t % 32
-        // of rows t / 32 + 8 m (each element is read and written by its own thread)
+        // of rows t / 32 + 16 m (each element is read and written by its own thread)
         {
             const int j = tid & 31, c0 = tid >> 5;
-            float acc[kMaxDK / 8];
+            float acc[kMaxDK / 16];
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 8; ++m) {
-                const int c = c0 + 8 * m;
+            for (int m = 0; m < kMaxDK / 16; ++m) {
+                const int c = c0 + 16 * m;
                 acc[m] = c < dk ? exp_g(gC[c], gCl[c]) * S[c * kBV + j] : 0.f;
             }
             for (int r = 0; r < L; ++r) {
                 const float w = Ws[r * kBV + j];
 #pragma unroll
-                for (int m = 0; m < kMaxDK / 8; ++m)
-                    if (c0 + 8 * m < dk) acc[m] += M[r * dk + c0 + 8 * m] * w;
+                for (int m = 0; m < kMaxDK / 16; ++m)
+                    if (c0 + 16 * m < dk) acc[m] += M[r * dk + c0 + 16 * m] * w;
             }
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 8; ++m) {
-                const int c = c0 + 8 * m;
+            for (int m = 0; m < kMaxDK / 16; ++m) {
+                const int c = c0 + 16 * m;
                 if (c < dk) S[c * kBV + j] = acc[m];
             }
         }
         __syncthreads();
     }
     if (final_state) {
-        for (int e = tid; e < dk * kBV; e += kThreads) {
+        for (int e = tid; e < dk * kBV; e += kThreadsW) {
             int c = e / kBV, j = e - c * kBV;
             final_state[st_base + (size_t)c * dv + j0 + j] = S[e];
         }
@@ -313,7 +313,7 @@ cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const T
                                                                   dv, C);
     timing_mark(stream, 2);
     if (n_seqs > 0)
-        k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
+        k3<<<dim3(n_seqs, H, dv / kBV), kThreadsW, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
                                                                  init_state, final_state, smap, H, dk, dv, C);
     timing_mark(stream, 3);
     if (n_chunks > 0)
@@ -339,7 +339,7 @@ cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* bet
                                                                   dv, C);
     }
     if (n_seqs > 0)
-        k3<<<dim3(n_seqs, H, dv / kBV), kThreads, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
+        k3<<<dim3(n_seqs, H, dv / kBV), kThreadsW, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
                                                                  init_state, nullptr, smap, H, dk, dv, C);
     return cudaGetLastError();
 }
