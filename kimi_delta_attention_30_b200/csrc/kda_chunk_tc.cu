@@ -19,8 +19,8 @@
 //       W   = U - D[0:64]                         per-token corrections
 //       S  <- Diag(Gamma_C) S + Kd^T W            M = 128 MMA accumulating in TMEM (row a3)
 //       D  += [0 ; P] W,  O = D[64:128]           outputs (row a4), read during the next chunk
-//     The next chunk's operands stream in by 1-D bulk copies (TMA engine, no
-//     multicast) while the current chunk is processed.
+//     The next chunk's operands stream in by 1-D bulk copies (TMA engine, each
+//     into this CTA's own shared memory) while the current chunk is processed.
 //
 // Derivation (ours; the oracle's chunk form checks it against the token
 // recurrence): with Gamma_r = exp(g_r) the per-token corrections W solve
