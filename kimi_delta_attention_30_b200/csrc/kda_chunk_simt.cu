@@ -24,8 +24,7 @@
 namespace kda {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kThreadsW = 512;   // K2 and K4: their pairwise loops are latency bound at one block per SM
+constexpr int kThreadsW = 512;   // threads per block: the kernels' loops are latency bound
 constexpr int kBV = 32;   // d_v columns per state-carry block
 constexpr int kMaxDK = 128;
 
