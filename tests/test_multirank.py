@@ -75,3 +75,21 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
         steps, warmup = 2, 3
     assert bench.run_reference(Args(), world=2, rank=1) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_its_json_line(capsys):
+    """bench.py --impl reference on rank 0: one JSON line with the keys the
+    contract reads (the fp64 oracle timed on the host cores, a bounded sample)."""
+    import json
+
+    class Args:
+        steps, warmup, gpus = 1, 0, 1
+    bench.run_reference(Args(), world=1, rank=0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert line["config"]["workload"].startswith("prefill B=4 H=16 T=4096")
