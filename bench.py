@@ -514,9 +514,10 @@ def main():
                "path_roofline": {"minimal_bytes": min_bwd,
                                  "time_min_us": min_bwd / (pk["hbm_gbs"] * 1e9) * 1e6,
                                  "frac_of_hbm_bound": min_bwd / (pk["hbm_gbs"] * 1e9) / (b_ms / 1e3)},
-               "gpu_launches": (len(kda.BWD_KERNELS)) * a.steps,
+               "gpu_launches": len(kda.bwd_kernels(torch.bfloat16, dk, dv)) * a.steps,
                "config": {"workload": f"backward of the prefill workload (B={B} H={H} T={T} d={dk}), d_o ~ N(0,1) "
-                                      "bf16, d_final_state ~ N(0, 0.1^2); fp32 CUDA-core kernels, 64-token chunks",
+                                      "bf16, d_final_state ~ N(0, 0.1^2); recompute on the tensor-core forward, "
+                                      "gradient kernels fp32 on CUDA cores, 64-token chunks",
                           "l2": "flushed before every timed step (256 MiB write)"}}
         del grads, bws, d_o, dfs
 

@@ -236,9 +236,17 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
     return o, final_state
 
 
+# kernels of one kda_chunk_bwd call: the recompute (bf16 with d = 128: k1 and the tensor-core
+# forward with its states stored; otherwise the CUDA-core k1-k3), then the gradient kernels
+BWD_KERNELS_TC = ["k1_cumsum", "tc_intra", "tc_unpack_u_wk", "tc_recur", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
 BWD_KERNELS = ["k1_cumsum", "k2_wy", "k3_state", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
-# the timing hook's marks of kda_chunk_bwd: start, k1..k3 recompute, kb_p, kb_chain, kb_a, kb_b, kb_c
-BWD_TIMED = ["recompute (k1-k3)", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
+# the timing hook's marks of kda_chunk_bwd: start, recompute, kb_p, kb_chain, kb_a, kb_b, kb_c
+BWD_TIMED = ["recompute", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
+
+
+def bwd_kernels(dtype, dk, dv):
+    """The kernels one kda_chunk_bwd call launches for this problem."""
+    return BWD_KERNELS_TC if (dtype == torch.bfloat16 and dk == 128 and dv == 128) else BWD_KERNELS
 
 
 def bwd_workspace_size(B, T, H, dk, dv, C=64, cu_seqlens=None) -> int:

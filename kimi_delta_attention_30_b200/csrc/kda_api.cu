@@ -105,10 +105,13 @@ SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
 struct BwdLayout {
     SimtLayout fwd;
     size_t off[12];
+    size_t tc = 0, o_scratch = 0;   // tensor-core recompute (0: not used)
     size_t total;
 };
 
-BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C) {
+bool tc_shape(kda_dtype dtype, int dk, int dv, int C);
+
+BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C, bool tc = false) {
     BwdLayout L;
     L.fwd = simt_layout(p, H, dk, dv);
     size_t o = L.fwd.total;
@@ -120,6 +123,12 @@ BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C) {
     for (int i = 0; i < 12; ++i) {
         L.off[i] = o;
         o = align_up(o + sizes[i] * sizeof(float));
+    }
+    if (tc) {
+        L.tc = o;
+        o = align_up(o + tc_workspace_bytes(p.n_chunks, H, C));
+        L.o_scratch = o;
+        o = align_up(o + tok * dv * sizeof(uint16_t));
     }
     L.total = o;
     return L;
@@ -359,7 +368,8 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C, 
     Plan p;
     if (C != 64 && C != 128) return 0;
     if (make_plan(B, T, H, dk, dv, kBwdChunk, cu_seqlens_host, n_seqs, p) != KDA_OK) return 0;
-    return bwd_layout(p, H, dk, dv, kBwdChunk).total;
+    // sized for the tensor-core recompute whenever the shape allows it (bf16 is not known here)
+    return bwd_layout(p, H, dk, dv, kBwdChunk, dk == 128 && dv == 128).total;
 }
 
 kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
@@ -382,7 +392,8 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     for (const void* ptr : ptrs)
         if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return KDA_ERR_ALIGN;
-    const BwdLayout L = bwd_layout(p, H, dk, dv, kBwdChunk);
+    const bool use_tc = tc_available() && tc_shape(dtype, dk, dv, kBwdChunk);
+    const BwdLayout L = bwd_layout(p, H, dk, dv, kBwdChunk, use_tc);
     if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
     if ((st = check_device()) != KDA_OK) return st;
     if (p.n_seqs == 0) return KDA_OK;
@@ -417,6 +428,8 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     w.At = f(L.off[9]);
     w.Qg = f(L.off[10]);
     w.Kd = f(L.off[11]);
+    w.tc_ws = use_tc ? (void*)(ws + L.tc) : nullptr;
+    w.o_scratch = use_tc ? (void*)(ws + L.o_scratch) : nullptr;
     timing_mark(s, 0);
     cudaError_t err = launch_simt_backward(dtype, q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq,
                                            dk_out, dv_out, dlog_alpha, dbeta, d_init_state, cmap, smap, p.n_chunks,

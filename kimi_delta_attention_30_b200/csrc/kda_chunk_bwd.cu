@@ -28,7 +28,8 @@
 // Every decay is exp of a non-positive difference, as in the forward split, of
 // cumulative decays held as fp32 (hi, lo) pairs (exp_gdiff, exp_g).
 // The forward intermediates (g, U, Wk, W, chunk start states) are recomputed by
-// the CUDA-core forward kernels.
+// the tensor-core forward (bf16, d = 128; g by the CUDA-core K1) or by the
+// CUDA-core forward kernels.
 #include <algorithm>
 
 #include "kda_internal.cuh"
@@ -605,8 +606,16 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
                     float* d_init, const ChunkMap& cmap, const SeqMap& smap, int n_chunks, int n_seqs, int H, int dk,
                     int dv, const BwdWorkspace& ws, cudaStream_t stream, kda_dtype dtype) {
     constexpr int C = 64;
-    cudaError_t e = launch_simt_states(dtype, k, v, la, beta, init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C,
-                                       ws.fwd, stream);
+    cudaError_t e;
+    if (ws.tc_ws) {
+        // bf16, d = 128: the tensor-core forward recomputes U, Wk, W and the chunk start states
+        if ((e = launch_simt_g(dtype, la, cmap, n_chunks, H, dk, ws.fwd, stream)) != cudaSuccess) return e;
+        e = launch_tc_states(q, k, v, la, beta, init_state, ws.o_scratch, cmap, smap, n_chunks, n_seqs, H, ws.tc_ws,
+                             ws.fwd.S_chunk, ws.fwd.W, ws.fwd.U, ws.fwd.Wk, stream);
+    } else {
+        e = launch_simt_states(dtype, k, v, la, beta, init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws.fwd,
+                               stream);
+    }
     if (e != cudaSuccess) return e;
     timing_mark(stream, 1);
     const size_t smem_p = sizeof(float) * 4 * (size_t)C * dk;

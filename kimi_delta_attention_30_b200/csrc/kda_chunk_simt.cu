@@ -345,6 +345,17 @@ cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* bet
 
 }  // namespace
 
+cudaError_t launch_simt_g(kda_dtype dtype, const void* log_alpha, const ChunkMap& cmap, int n_chunks, int H, int dk,
+                          const SimtWorkspace& ws, cudaStream_t stream) {
+    if (n_chunks == 0) return cudaSuccess;
+    if (dtype == KDA_F32)
+        k1_cumsum<float><<<dim3(n_chunks, H), dk, 0, stream>>>((const float*)log_alpha, ws.g, ws.gl, cmap, H, dk);
+    else
+        k1_cumsum<__nv_bfloat16><<<dim3(n_chunks, H), dk, 0, stream>>>((const __nv_bfloat16*)log_alpha, ws.g, ws.gl,
+                                                                        cmap, H, dk);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_simt_states(kda_dtype dtype, const void* k, const void* v, const void* log_alpha,
                                const void* beta, const float* init_state, const ChunkMap& cmap, const SeqMap& smap,
                                int n_chunks, int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws,

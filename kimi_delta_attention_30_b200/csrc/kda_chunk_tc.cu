@@ -840,10 +840,13 @@ struct RecurLayout {
     static constexpr uint32_t kTmemCols = (3 * BV <= 32) ? 32 : (3 * BV <= 64) ? 64 : (3 * BV <= 128) ? 128 : 256;
 };
 
-template <int BV>
+// STORE (for the backward pass): every chunk's start state S_n goes to s_store
+// [chunks, H, 128, 128] and W_n to w_store [tokens, H, 128], both fp32.
+template <int BV, bool STORE>
 __global__ void __launch_bounds__(kRecurThreads, 1)
 tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, float* __restrict__ final_state,
-         __nv_bfloat16* __restrict__ o, int* __restrict__ err, SeqMap smap, int H) {
+         __nv_bfloat16* __restrict__ o, int* __restrict__ err, SeqMap smap, int H, float* __restrict__ s_store,
+         float* __restrict__ w_store) {
     using Lay = RecurLayout<BV>;
     constexpr int HB = BV / 2;          // state columns per thread
     constexpr int NG = HB / 16;         // 16-column TMEM groups per thread
@@ -987,6 +990,12 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         const uint8_t* uu = sm + Lay::kUU + stage * Lay::kUStage;
         const uint32_t par = (uint32_t)n & 1u;
         const uint32_t t_d = tbase + (uint32_t)(BV * (n & 1));
+        if (STORE) {
+            float* dst = s_store + ((((size_t)sq.chunk0 + n) * H + h) * kD + c) * kD + j0 + cq;
+#pragma unroll
+            for (int j = 0; j < HB; j += 4)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+        }
         // S_n as the MN-major B operand (K = channel row c, N = columns)
 #pragma unroll
         for (int j = 0; j < HB; j += 8) store8_split(s_h, s_l, mn_chunk(c, cq + j, 128), s + j);
@@ -1040,6 +1049,12 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 }
                 store8_split(w_h, w_h + 8192, mn_chunk(r, jb, 64), d[g]);
                 store8_split(w_h, w_h + 8192, mn_chunk(r, jb + 8, 64), d[g] + 8);
+                if (STORE && r < min(kC, sq.len - n * kC)) {
+                    float* dst = w_store + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + jb;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) = make_float4(d[g][e], d[g][e + 1], d[g][e + 2], d[g][e + 3]);
+                }
             }
             fence_async_smem();
             tc_fence_before();
@@ -1116,15 +1131,36 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     if (warp == 0) tmem_dealloc(tbase, Lay::kTmemCols);
 }
 
-template <int BV>
+template <int BV, bool STORE = false>
 cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* final_state, __nv_bfloat16* o, int* err,
-                         const SeqMap& smap, int n_seqs, int H, cudaStream_t stream) {
+                         const SeqMap& smap, int n_seqs, int H, cudaStream_t stream, float* s_store = nullptr,
+                         float* w_store = nullptr) {
     using Lay = RecurLayout<BV>;
-    cudaError_t e = cudaFuncSetAttribute(tc_recur<BV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
+    cudaError_t e =
+        cudaFuncSetAttribute(tc_recur<BV, STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    tc_recur<BV><<<dim3(n_seqs, H, kD / BV), kRecurThreads, Lay::kAlloc, stream>>>(ws, init_state, final_state, o,
-                                                                                   err, smap, H);
+    tc_recur<BV, STORE><<<dim3(n_seqs, H, kD / BV), kRecurThreads, Lay::kAlloc, stream>>>(
+        ws, init_state, final_state, o, err, smap, H, s_store, w_store);
     return cudaGetLastError();
+}
+
+// U (fp32, row-swizzled) and Wk (rows 0-63 of the [Wk ; Q exp(g)] hi/lo images) of
+// every chunk-head as plain token-major fp32 arrays [tokens, H, 128].
+__global__ void __launch_bounds__(256) tc_unpack_u_wk(const uint8_t* __restrict__ ws, float* __restrict__ U,
+                                                      float* __restrict__ Wk, ChunkMap cmap, int H) {
+    int seq, tok0, len, idx;
+    cmap.locate(blockIdx.x, seq, tok0, len, idx);
+    const int h = blockIdx.y;
+    const uint8_t* src = ws + ((size_t)blockIdx.x * H + h) * kChunkBytes;
+    const float* uo = reinterpret_cast<const float*>(src + kOffU);
+    for (int e = threadIdx.x; e < len * kD; e += 256) {
+        const int r = e >> 7, j = e & 127;
+        const size_t off = ((size_t)(tok0 + r) * H + h) * kD + j;
+        U[off] = uo[u_index(r, j & ~3) + (j & 3)];
+        const uint32_t b = sw128_offset(r, j, 128);
+        Wk[off] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(src + kOffWkQh + b)) +
+                  __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(src + kOffWkQl + b));
+    }
 }
 
 // multiprocessors of the current device, looked up once per device
@@ -1183,6 +1219,38 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
     }
     timing_mark(stream, 2);
     return cudaSuccess;
+}
+
+// The forward intermediates the backward pass needs, from the tensor-core path:
+// every chunk's start state and W (fp32, from the state carry) and U, Wk (fp32,
+// unpacked from the per-chunk workspace).  o_scratch receives the outputs.
+cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
+                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
+                             float* Wk, cudaStream_t stream) {
+    int* err = reinterpret_cast<int*>(tc_ws);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+    if (n_chunks > 0) {
+        e = cudaFuncSetAttribute(tc_intra<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIntraAlloc);
+        if (e != cudaSuccess) return e;
+        tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        tc_unpack_u_wk<<<dim3(n_chunks, H), 256, 0, stream>>>(ws, U, Wk, cmap, H);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (n_seqs > 0) {
+        if ((long)n_seqs * H * 4 <= sm_count())
+            e = launch_recur<32, true>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
+                                       S_chunk, W);
+        else
+            e = launch_recur<64, true>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
+                                       S_chunk, W);
+    }
+    return e;
 }
 
 }  // namespace kda

@@ -194,7 +194,20 @@ struct BwdWorkspace {
     float* At;          // [chunks, H, C, C] the unscaled key products (strictly lower)
     float* Qg;          // [tokens, H, dk] q . exp(g)
     float* Kd;          // [tokens, H, dk] k . exp(g_C - g)
+    void* tc_ws;        // tensor-core workspace for the recompute (bf16, d = 128), or null
+    void* o_scratch;    // outputs of that recompute [tokens, H, dv] bf16 (unused)
 };
+
+// g only (the CUDA-core K1), into ws.g / ws.gl.
+cudaError_t launch_simt_g(kda_dtype dtype, const void* log_alpha, const ChunkMap& cmap, int n_chunks, int H, int dk,
+                          const SimtWorkspace& ws, cudaStream_t stream);
+
+// Tensor-core recompute for the backward pass (bf16, d = 128): chunk start
+// states and W from the state carry, U and Wk unpacked from the workspace.
+cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                             const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
+                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
+                             float* Wk, cudaStream_t stream);
 
 cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
                                  const void* log_alpha, const void* beta, const float* init_state,
