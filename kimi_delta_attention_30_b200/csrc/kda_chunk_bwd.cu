@@ -555,20 +555,29 @@ __global__ void __launch_bounds__(kTW) kb_c(const Tin* __restrict__ q, const Tin
                                     dKd[off] * exp_gdiff(gC[c], gCl[c], gi, gil));
     }
     __syncthreads();
-    // phase C: dlog alpha (zero where the forward's floor on log alpha was active)
+    // phase C: the per-(row, channel) terms are formed by every thread first (the
+    // dAt / dP tiles are free now, and Q is replaced in place), so the two
+    // sequential sums below read shared memory only
+    float* tkd = dAs;   // [C][DK] (the dAt and dP tiles together): dKd Kd
+    for (int e = tid; e < len * DK; e += kTW) {
+        const int j = e / DK, cc = e - j * DK;
+        const size_t off = tok_off(tok0 + j, H, h, DK) + cc;
+        tkd[e] = dKd[off] * Ks[e] * exp_gdiff(gC[cc], gCl[cc], Gs[e], GLs[e]);
+        Qs[e] = (dQg[off] * Qs[e] + dKg[off] * Ks[e]) * exp_g(Gs[e], GLs[e]);   // dQg Qg + dKg Kg
+    }
+    __syncthreads();
+    // dlog alpha (zero where the forward's floor on log alpha was active)
     if (rg == 0) {
-        float pre = 0.f;   // sum_{r<j} dKd Kd, added to F[0][j]
+        float pre = 0.f;   // sum_{r<j} dKd Kd, added to F[j]
         for (int j = 0; j < len; ++j) {
             F[j * DK + c] += pre;
-            const size_t off = tok_off(tok0 + j, H, h, DK) + c;
-            pre += dKd[off] * Ks[j * DK + c] * exp_gdiff(gC[c], gCl[c], Gs[j * DK + c], GLs[j * DK + c]);
+            pre += tkd[j * DK + c];
         }
         const float gam = dGam[(chunk * H + h) * DK + c] * exp_g(gC[c], gCl[c]);
         float suf = 0.f;   // sum_{r>=j} (dQg Qg + dKg Kg)
         for (int j = len - 1; j >= 0; --j) {
             const size_t off = tok_off(tok0 + j, H, h, DK) + c;
-            const float eg = exp_g(Gs[j * DK + c], GLs[j * DK + c]);
-            suf += (dQg[off] * Qs[j * DK + c] + dKg[off] * Ks[j * DK + c]) * eg;
+            suf += Qs[j * DK + c];
             const float f = F[j * DK + c];
             dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? f + suf + gam : 0.f);
         }
