@@ -71,6 +71,15 @@ def test_bwd_bf16_ragged(cuda_ok, C, T):
     _check(inp, _bwd(inp, d_o, dfs, C=C), d_o, dfs, TOL["bf16"])
 
 
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_bwd_bf16_small_heads(cuda_ok, dk, dv):
+    """bf16 with d_k or d_v of 64 (CUDA-core recompute), ragged tail."""
+    wl = replace(WORKLOADS["prefill"], dk=dk, dv=dv)
+    inp = _to(make_prefill(wl, B=2, T=150, H=2, seed=13), DEV)
+    d_o, dfs = make_grad_outputs(inp, seed=13)
+    _check(inp, _bwd(inp, d_o, dfs), d_o, dfs, TOL["bf16"])
+
+
 def test_bwd_varlen_with_empty_and_tiny_sequences(cuda_ok):
     inp = _to(make_prefill("prefill", lengths=[0, 1, 70, 0, 129, 5], H=2, seed=4), DEV)
     d_o, dfs = make_grad_outputs(inp, seed=4)
