@@ -1,0 +1,103 @@
+"""The chunkwise backward algebra the CUDA kernels implement, checked in fp64
+against the oracle's token-level reverse mode (O3) on the CPU.
+
+The pages give no backward pass; the kernels use a derivation of their own
+(the chunk map is affine in its start state, T = (I + A)^-1 is applied
+transposed by back substitution, dA = -(Y U^T + Z Wk^T), and dlog alpha_j sums
+exactly the terms whose decay spans token j).  This test writes those
+formulas out with numpy on small inputs, chunk by chunk, and requires the
+gradients of O3 to 1e-10: a wrong sign, transpose or index in the derivation
+fails it without a GPU.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def chunk_backward(q, k, v, la, beta, s0, do, dfs, C):
+    """One sequence, one head: q, k, la [T, dk], v [T, dv], beta [T], s0, dfs
+    [dk, dv], do [T, dv].  Returns dq, dk, dv, dla, dbeta, ds0."""
+    T, dk = q.shape
+    chunks = [(c0, min(C, T - c0)) for c0 in range(0, T, C)]
+    # forward, keeping what the backward reads
+    S = s0.copy()
+    saved = []
+    for c0, L in chunks:
+        sl = slice(c0, c0 + L)
+        qq, kk, vv, b, g = q[sl], k[sl], v[sl], beta[sl], np.cumsum(la[sl], axis=0)
+        E = np.exp(np.minimum(g[:, None, :] - g[None, :, :], 0.0))        # [r, i, c], used for i <= r
+        low, inc = np.tril(np.ones((L, L)), -1), np.tril(np.ones((L, L)))
+        At = np.einsum('rc,ic,ric->ri', kk, kk, E) * low
+        P = np.einsum('rc,ic,ric->ri', qq, kk, E) * inc
+        Tm = np.linalg.inv(np.eye(L) + b[:, None] * At)
+        Kg, Qg, Kd = kk * np.exp(g), qq * np.exp(g), kk * np.exp(g[-1] - g)
+        U, Wk = Tm @ (b[:, None] * vv), Tm @ (b[:, None] * Kg)
+        W = U - Wk @ S
+        saved.append(dict(sl=sl, g=g, E=E, At=At, P=P, Tm=Tm, Kg=Kg, Qg=Qg, Kd=Kd, U=U, Wk=Wk, W=W, S=S.copy(),
+                          b=b, low=low, inc=inc, kk=kk, qq=qq, vv=vv))
+        S = np.exp(g[-1])[:, None] * S + Kd.T @ W
+    # reverse chain: dW = P^T dO + Kd dS', dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW
+    dS = dfs.copy()
+    out = {n: np.zeros_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dla", la), ("dbeta", beta))}
+    for s in reversed(saved):
+        dOc = do[s["sl"]]
+        dSe = dS
+        dW = s["P"].T @ dOc + s["Kd"] @ dSe
+        dS = np.exp(s["g"][-1])[:, None] * dSe + s["Qg"].T @ dOc - s["Wk"].T @ dW
+        # chunk-parallel part
+        dQg = dOc @ s["S"].T
+        dKd = s["W"] @ dSe.T
+        dWk = -dW @ s["S"].T
+        dGam = np.sum(dSe * s["S"], axis=1)
+        dP = (dOc @ s["W"].T) * s["inc"]
+        Y = s["Tm"].T @ dW                       # (I + A)^T Y = dW
+        Z = s["Tm"].T @ dWk
+        b = s["b"]
+        dA = -(Y @ s["U"].T + Z @ s["Wk"].T) * s["low"]
+        dAt = b[:, None] * dA
+        out["dv"][s["sl"]] = b[:, None] * Y
+        dKg = b[:, None] * Z
+        out["dbeta"][s["sl"]] = np.sum(s["vv"] * Y, 1) + np.sum(s["Kg"] * Z, 1) + np.sum(dA * s["At"], 1)
+        kk, qq, E, g = s["kk"], s["qq"], s["E"], s["g"]
+        L = len(b)
+        x1 = np.einsum('ri,ic,ric->rc', dAt, kk, E)
+        x2 = np.einsum('ri,ic,ric->rc', dP, kk, E)
+        y = np.einsum('ri,rc,ric->ic', dAt, kk, E) + np.einsum('ri,rc,ric->ic', dP, qq, E)
+        out["dq"][s["sl"]] = x2 + dQg * np.exp(g)
+        out["dk"][s["sl"]] = x1 + y + dKg * np.exp(g) + dKd * np.exp(g[-1] - g)
+        # dlog alpha_j: pairwise terms with i < j <= r, Qg/Kg terms of rows r >= j,
+        # Kd terms of rows r < j, and the Gamma term
+        Tp = (dAt[:, :, None] * kk[:, None, :] + dP[:, :, None] * qq[:, None, :]) * kk[None, :, :] * E
+        dla = np.zeros((L, dk))
+        for j in range(L):
+            dla[j] = Tp[j:, :j].sum(axis=(0, 1))
+            dla[j] += ((dQg * s["Qg"] + dKg * s["Kg"])[j:]).sum(axis=0)
+            dla[j] += ((dKd * s["Kd"])[:j]).sum(axis=0)
+            dla[j] += dGam * np.exp(g[-1])
+        out["dla"][s["sl"]] = dla
+    out["ds0"] = dS
+    return out
+
+
+@pytest.mark.parametrize("T,C", [(23, 8), (40, 16), (7, 64)])
+def test_chunk_backward_algebra_matches_token_reverse_mode(T, C):
+    rng = np.random.default_rng(T * 100 + C)
+    dk, dv = 6, 5
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((T, dv))
+    la = -np.logaddexp(0.0, rng.standard_normal((T, dk)) + 1.0)
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal(T)))
+    s0 = rng.standard_normal((dk, dv))
+    do = rng.standard_normal((T, dv))
+    dfs = rng.standard_normal((dk, dv))
+    got = chunk_backward(q, k, v, la, beta, s0, do, dfs, C)
+    ref = oracle.backward(q[:, None], k[:, None], v[:, None], la[:, None], beta[:, None], [0, T], do[:, None],
+                          d_final_state=dfs[None, None], init_state=s0[None, None])
+    pairs = (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dla", "dlog_alpha"), ("dbeta", "dbeta"))
+    for mine, theirs in pairs:
+        np.testing.assert_allclose(got[mine], ref[theirs][:, 0], rtol=1e-9, atol=1e-10, err_msg=mine)
+    np.testing.assert_allclose(got["ds0"], ref["d_init_state"][0, 0], rtol=1e-9, atol=1e-10)
