@@ -147,6 +147,27 @@ __global__ void __launch_bounds__(kTW, 2) kb_chain(const float* __restrict__ Qg,
             const int c = e / kBV, j = e - c * kBV;
             dS_chunk[sc_base + (size_t)c * dv + j0 + j] = dS[e];
         }
+        if (n > 0) {
+            // the previous chunk (next in this walk) into L2 while this one is worked on:
+            // its Kd, Qg, Wk rows (4 lines of 128 bytes each), P (128 lines) and dO tile
+            const int tp = t0 - C;
+            for (int e = tid; e < 3 * C * (dk / 32) + (C * C) / 32 + C; e += kTW) {
+                const char* a = nullptr;
+                if (e < 3 * C * (dk / 32)) {
+                    const int mtx = e / (C * (dk / 32)), rem = e - mtx * (C * (dk / 32));
+                    const int r = rem / (dk / 32), ln = rem - r * (dk / 32);
+                    const float* base = mtx == 0 ? Kd : mtx == 1 ? Qg : Wk;
+                    a = reinterpret_cast<const char*>(base + tok_off(tp + r, H, h, dk) + 32 * ln);
+                } else if (e < 3 * C * (dk / 32) + (C * C) / 32) {
+                    a = reinterpret_cast<const char*>(P + (((size_t)chunk - 1) * H + h) * C * C +
+                                                      32 * (e - 3 * C * (dk / 32)));
+                } else {
+                    const int r = e - 3 * C * (dk / 32) - (C * C) / 32;
+                    a = reinterpret_cast<const char*>(d_o + tok_off(tp + r, H, h, dv) + j0);
+                }
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+            }
+        }
         const float* Pc = P + (chunk * H + h) * C * C;
         for (int e = tid; e < C * C; e += kTW) Ps[e] = Pc[e];
         for (int e = tid; e < L * kBV; e += kTW) {
