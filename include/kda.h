@@ -303,9 +303,10 @@ KDA_API kda_status kda_decode_step_prep(const void* q, const void* k, const void
  *   workspace       : >= kda_chunk_bwd_workspace_size(...) bytes, 256-byte
  *                     aligned, caller-owned, not read before it is written
  *
- * The forward intermediates are recomputed inside the call (on CUDA cores, in
- * fp32, with 64-token chunks whatever C asks for: the chunk form does not
- * depend on the chunk length).  dlog_alpha is zero where log_alpha is below
+ * The forward intermediates are recomputed inside the call, with 64-token
+ * chunks whatever C asks for (the chunk form does not depend on the chunk
+ * length): by the tensor-core forward for bf16 with dk = dv = 128, by the
+ * fp32 CUDA-core kernels otherwise; the gradient kernels run in fp32.  dlog_alpha is zero where log_alpha is below
  * the kernels' floor of -100 (log alpha = -inf included).  dlog_alpha sums
  * per-row contributions with shared-memory atomics, so repeated calls may
  * differ in its last bits; the other gradients are reproducible.  Errors as
