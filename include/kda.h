@@ -325,6 +325,33 @@ KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 
+/*
+ * Device-side status of a finished call.  The tensor-core kernels bound every
+ * wait on the device (2 s); if one expires they stop, leave their outputs
+ * undefined and record KDA_ERR_TIMEOUT in an error word inside the workspace
+ * (cleared at the start of each call).  These two calls synchronise `stream`
+ * and return KDA_OK or the recorded error for the last kda_chunk_fwd[_ex|_prep]
+ * / kda_chunk_bwd call that used `workspace` with the same size arguments.
+ * For problems on the CUDA-core path they return KDA_OK without touching the
+ * device (those kernels do not wait on the device).  Errors: KDA_ERR_NULL for a
+ * NULL workspace, the size errors of the calls themselves, KDA_ERR_CUDA if the
+ * copy or the synchronisation fails.
+ */
+KDA_API kda_status kda_chunk_fwd_device_status(const void* workspace, kda_dtype dtype,
+                                               const int32_t* cu_seqlens_host, int n_seqs,
+                                               int B, int T, int H, int dk, int dv, int C,
+                                               kda_algo algo, void* stream);
+KDA_API kda_status kda_chunk_bwd_device_status(const void* workspace, kda_dtype dtype,
+                                               const int32_t* cu_seqlens_host, int n_seqs,
+                                               int B, int T, int H, int dk, int dv, int C,
+                                               void* stream);
+/* The same for the last kda_chunk_fwd_noalloc call on the current device
+ * (its scratch is the library's own array). */
+KDA_API kda_status kda_chunk_fwd_noalloc_device_status(kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                                       int n_seqs, int B, int T, int H, int dk, int dv,
+                                                       int C, void* stream);
+
+
 #ifdef __cplusplus
 }
 #endif

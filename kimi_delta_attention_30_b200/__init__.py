@@ -30,6 +30,7 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_BF16, KDA_F32 = 0, 1
 ALGOS = {"auto": 0, "simt": 1, "tc": 2}
+KDA_ERR_TIMEOUT = -9   # a bounded device-side wait gave up (kda_status in include/kda.h)
 _DTYPES = {torch.bfloat16: KDA_BF16, torch.float32: KDA_F32}
 # kda_prep flags (include/kda.h)
 PREP_NONE, PREP_QK_L2NORM, PREP_GATE_SOFTPLUS, PREP_BETA_SIGMOID = 0, 1, 2, 4
@@ -82,6 +83,12 @@ def _declare(lib):
     lib.kda_chunk_fwd_kernels.restype = c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [vp] * 5 + [c_int, vp, i32p, c_int] + [c_int] * 6 + [vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = c_int
+    lib.kda_chunk_fwd_device_status.argtypes = [vp, c_int, i32p, c_int] + [c_int] * 6 + [c_int, vp]
+    lib.kda_chunk_fwd_device_status.restype = c_int
+    lib.kda_chunk_bwd_device_status.argtypes = [vp, c_int, i32p, c_int] + [c_int] * 6 + [vp]
+    lib.kda_chunk_bwd_device_status.restype = c_int
+    lib.kda_chunk_fwd_noalloc_device_status.argtypes = [c_int, i32p, c_int] + [c_int] * 6 + [vp]
+    lib.kda_chunk_fwd_noalloc_device_status.restype = c_int
     return lib
 
 
@@ -114,7 +121,8 @@ def exported_symbols():
             "kda_chunk_fwd_workspace_size_ex", "kda_chunk_fwd", "kda_chunk_fwd_ex",
             "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
             "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep", "kda_chunk_bwd_workspace_size",
-            "kda_chunk_bwd"]
+            "kda_chunk_bwd", "kda_chunk_fwd_device_status", "kda_chunk_bwd_device_status",
+            "kda_chunk_fwd_noalloc_device_status"]
 
 
 def _ptr(t):
@@ -291,6 +299,27 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, init_state=None, d_final_state=None
     if st != 0:
         raise KdaError(st, "kda_chunk_bwd")
     return dq, dk_, dv_, dla, dbeta, dinit
+
+
+def device_status(kind, workspace, dtype, B, T, H, dk, dv, C=64, cu_seqlens=None, algo="auto", stream=None):
+    """Synchronise ``stream`` and return the device-side status (0 or
+    KDA_ERR_TIMEOUT) of the last call of ``kind`` ("fwd", "bwd" or "noalloc")
+    that used ``workspace`` (ignored for "noalloc") with these sizes.  Raises
+    KdaError for invalid arguments or a failed copy."""
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    d = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    h = _stream_handle(stream)
+    if kind == "fwd":
+        st = lib().kda_chunk_fwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, ALGOS[algo], h)
+    elif kind == "bwd":
+        st = lib().kda_chunk_bwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, h)
+    elif kind == "noalloc":
+        st = lib().kda_chunk_fwd_noalloc_device_status(d, cu, n, B, T, H, dk, dv, C, h)
+    else:
+        raise ValueError(f"unknown kind {kind!r}")
+    if st not in (0, KDA_ERR_TIMEOUT):
+        raise KdaError(st, f"device status ({kind})")
+    return int(st)
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20   # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h

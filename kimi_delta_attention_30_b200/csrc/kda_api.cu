@@ -438,6 +438,50 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Copy the error word at `offset` of the workspace to the host after `stream` finishes.
+kda_status read_error_word(const void* workspace, size_t offset, void* stream) {
+    int word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(&word, (const char*)workspace + offset, sizeof(int), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    return word == 0 ? KDA_OK : (kda_status)word;
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd_device_status(const void* workspace, kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                       int n_seqs, int B, int T, int H, int dk, int dv, int C, kda_algo algo,
+                                       void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (algo != KDA_ALGO_AUTO && algo != KDA_ALGO_SIMT && algo != KDA_ALGO_TC) return KDA_ERR_SHAPE;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    if (!workspace) return KDA_ERR_NULL;
+    if (p.n_seqs == 0 || resolve(algo, dtype, dk, dv, C) != KDA_ALGO_TC) return KDA_OK;   // nothing waited
+    return read_error_word(workspace, table_bytes(p), stream);   // the tensor-core scratch starts with it
+}
+
+kda_status kda_chunk_bwd_device_status(const void* workspace, kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                       int n_seqs, int B, int T, int H, int dk, int dv, int C, void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (C != 64 && C != 128) return KDA_ERR_CHUNK;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, kBwdChunk, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    if (!workspace) return KDA_ERR_NULL;
+    if (p.n_seqs == 0 || !(tc_available() && tc_shape(dtype, dk, dv, kBwdChunk))) return KDA_OK;
+    return read_error_word(workspace, bwd_layout(p, H, dk, dv, kBwdChunk, true).tc, stream);
+}
+
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                            kda_dtype dtype, float* state, int N, int H, int dk, int dv, void* o, void* stream) {
     return decode_impl(q, k, v, log_alpha, beta, dtype, 0u, state, N, H, dk, dv, o, stream);

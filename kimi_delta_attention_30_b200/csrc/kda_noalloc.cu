@@ -64,3 +64,12 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const void* q, const void* k, const 
     return kda_chunk_fwd(q, k, v, log_alpha, beta, dtype, init_state, cu_seqlens_host, n_seqs, B, T, H, dk, dv, C,
                          o, final_state, scratch, (size_t)KDA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" kda_status kda_chunk_fwd_noalloc_device_status(kda_dtype dtype, const int32_t* cu_seqlens_host, int n_seqs,
+                                                          int B, int T, int H, int dk, int dv, int C, void* stream) {
+    void* scratch = nullptr;
+    kda_status st = scratch_address(&scratch);
+    if (st != KDA_OK) return st;
+    return kda_chunk_fwd_device_status(scratch, dtype, cu_seqlens_host, n_seqs, B, T, H, dk, dv, C, KDA_ALGO_AUTO,
+                                       stream);
+}

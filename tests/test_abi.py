@@ -218,3 +218,36 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         kda.chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def _status_fwd(ws=0x100000, dtype=1, cu=None, B=1, T=256, H=2, dk=64, dv=64, C=64, algo=0):
+    lib = kda.lib()
+    cu_p, n, _keep = kda._cu_arg(cu)
+    return lib.kda_chunk_fwd_device_status(None if ws is None else ctypes.c_void_p(ws), dtype, cu_p, n, B, T, H,
+                                           dk, dv, C, algo, None)
+
+
+def _status_bwd(ws=0x100000, dtype=1, cu=None, B=1, T=256, H=2, dk=64, dv=64, C=64):
+    lib = kda.lib()
+    cu_p, n, _keep = kda._cu_arg(cu)
+    return lib.kda_chunk_bwd_device_status(None if ws is None else ctypes.c_void_p(ws), dtype, cu_p, n, B, T, H,
+                                           dk, dv, C, None)
+
+
+def test_device_status_validates_on_the_host():
+    # invalid arguments are rejected before anything touches the device
+    assert _status_fwd(ws=None) == E_NULL
+    assert _status_fwd(dtype=5) == E_DTYPE
+    assert _status_fwd(algo=9) == E_SHAPE
+    assert _status_fwd(dk=96) == E_SHAPE
+    assert _status_fwd(cu=[0, 100, 50, 256]) == E_SEQ
+    assert _status_bwd(ws=None) == E_NULL
+    assert _status_bwd(C=32) == E_CHUNK
+    assert _status_bwd(dtype=5) == E_DTYPE
+    # the CUDA-core path never waits on the device: OK without reading the (fake) workspace
+    assert _status_fwd(dk=64, dv=64) == OK
+    assert _status_fwd(dk=128, dv=128, algo=kda.ALGOS["simt"]) == OK
+    assert _status_bwd(dk=64, dv=64, dtype=1) == OK
+    # zero sequences launch nothing, on either path
+    assert _status_bwd(dtype=0, dk=128, dv=128, B=0) == OK
+    assert _status_fwd(dtype=0, dk=128, dv=128, B=0) == OK

@@ -195,6 +195,21 @@ def test_prefill_final_state_may_alias_init_state(cuda_ok, algo):
         assert torch.equal(o3, o1) and torch.equal(st, f1)
 
 
+def test_device_status_after_tensor_core_calls(cuda_ok):
+    """The error word of the bounded device-side waits reads 0 after calls that
+    finished normally (forward, fused-prep forward and backward)."""
+    inp = _to(make_prefill("prefill", B=2, T=200, H=4, seed=77), DEV)
+    B, T, H, dk = inp.q.shape
+    ws = torch.empty(kda.workspace_size(B, T, H, dk, dk, 64, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, C=64, workspace=ws)
+    assert kda.device_status("fwd", ws, torch.bfloat16, B, T, H, dk, dk, 64) == 0
+    kda.chunk_fwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, C=64, workspace=ws, prep=kda.PREP_QK_L2NORM)
+    assert kda.device_status("fwd", ws, torch.bfloat16, B, T, H, dk, dk, 64) == 0
+    wsb = torch.empty(kda.bwd_workspace_size(B, T, H, dk, dk, 64), dtype=torch.uint8, device=DEV)
+    kda.chunk_bwd(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, torch.randn_like(inp.v), C=64, workspace=wsb)
+    assert kda.device_status("bwd", wsb, torch.bfloat16, B, T, H, dk, dk, 64) == 0
+
+
 def test_prefill_resume_and_handoff(cuda_ok):
     """Prefill of x[:t1] then x[t1:] from the carried state equals one prefill;
     prefill of T tokens then decode steps equals prefill of T + m tokens."""

@@ -58,5 +58,7 @@ def test_noalloc_matches_workspace_entry_point(cuda_ok):
     # the first problem again, after the second one used the array
     o_again, fs_again = kda.chunk_fwd_noalloc(*_args(cases[0]), init_state=cases[0].init_state, C=cases[0].C)
     torch.cuda.synchronize()
+    B, T, H = cases[0].q.shape[:3]
+    assert kda.device_status("noalloc", None, torch.bfloat16, B, T, H, 128, 128, cases[0].C) == 0
     assert rel_err(to_f64(o_again), to_f64(ref[0][0]), stored_as="bf16") <= 2e-2
     assert rel_err(to_f64(fs_again), to_f64(ref[0][1])) <= 2e-2
