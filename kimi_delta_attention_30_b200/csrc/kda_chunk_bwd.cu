@@ -38,7 +38,7 @@ namespace kda {
 namespace {
 
 constexpr int kT = 256;
-constexpr int kTW = 512;      // the pairwise kernels (kb_p, kb_c): more warps to hide latency
+constexpr int kTW = 512;      // kb_chain and kb_c: more warps to hide latency
 constexpr int kBV = 32;       // d_v columns per chain block / per tile
 constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
 constexpr int kMaxDK = 128;
@@ -52,58 +52,171 @@ __device__ __forceinline__ float wsum(float x) {
 
 __device__ __forceinline__ size_t tok_off(int t, int H, int h, int d) { return ((size_t)t * H + h) * d; }
 
+// Four consecutive elements as fp32 (8 bytes of bf16 or 16 bytes of fp32, aligned).
+__device__ __forceinline__ void load4(const float* p, float* v) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float* v) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);   // element 0 in the low half of u.x
+    v[0] = __uint_as_float(u.x << 16); v[1] = __uint_as_float(u.x & 0xffff0000u);
+    v[2] = __uint_as_float(u.y << 16); v[3] = __uint_as_float(u.y & 0xffff0000u);
+}
+
+constexpr int kPThreads = 544;   // kb_p: 136 tiles x 4 lanes = 17 warps
+constexpr int kPS = 68;          // row stride of kb_p's channel-major arrays (float4-aligned)
+
 // P[r][i] = sum_c q_rc k_ic exp(g_rc - g_ic) for i <= r < L and At[r][i] (the same
 // with k_r, i < r), zero elsewhere, from one exponential per (r, i, c); and the
 // elementwise Qg = q exp(g), Kd = k exp(g_C - g) the chain and the later kernels read.
-// One block per (chunk, head); shared Qs, Ks, Gs, GLs [C][dk].
-template <typename Tin>
-__global__ void __launch_bounds__(kTW) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                                           const float* __restrict__ g, const float* __restrict__ gl,
-                                           float* __restrict__ P, float* __restrict__ At, float* __restrict__ Qg,
-                                           float* __restrict__ Kd, ChunkMap cmap, int H, int dk, int C) {
-    extern __shared__ float smem[];
+// One block per (chunk, head).  The lower triangle of the 64 x 64 pair grid is
+// cut into 136 tiles of 4 x 4 pairs (rows 4a..4a+3, columns 4b..4b+3, b <= a);
+// four adjacent lanes share a tile, lane s summing the channels s, s + 4, ...,
+// and two shuffles add their partial sums.  Shared memory holds q, k, g and its
+// low part channel-major ([c][r], row stride kPS), so a lane reads the four rows
+// (or columns) of its tile for one channel as one float4.  Rows past the end of
+// a short chunk hold q = k = 0 and the last row's g, which keeps every exponent
+// of a pair i <= r non-positive; their outputs are written as zero, as are the
+// pairs i > r of the diagonal tiles (computed, then discarded).
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kPThreads, 1) kb_p(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                     const float* __restrict__ g, const float* __restrict__ gl,
+                                                     float* __restrict__ P, float* __restrict__ At,
+                                                     float* __restrict__ Qg, float* __restrict__ Kd, ChunkMap cmap,
+                                                     int H) {
+    constexpr int C = kBwdC;
+    extern __shared__ __align__(16) float smem[];
+    float* Qt = smem;
+    float* Kt = Qt + DK * kPS;
+    float* Gt = Kt + DK * kPS;
+    float* GLt = Gt + DK * kPS;
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
-    const int h = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    float* Qs = smem;
-    float* Ks = Qs + C * dk;
-    float* Gs = Ks + C * dk;
-    float* GLs = Gs + C * dk;
-    for (int e = tid; e < len * dk; e += kTW) {
-        const int r = e / dk, c = e - r * dk;
-        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
-        Qs[e] = to_f32(q[off]);
-        Ks[e] = to_f32(k[off]);
-        Gs[e] = g[off];
-        GLs[e] = gl[off];
+    const int h = blockIdx.y, tid = threadIdx.x;
+
+    // Staging in groups of 4 channels.  A warp covers 16 rows x 2 groups, so the
+    // transposed shared stores of its lanes fall in 32 different banks.
+    const size_t last = tok_off(tok0 + len - 1, H, h, DK);
+    for (int e4 = tid; e4 < C * DK / 4; e4 += kPThreads) {
+        const int w = e4 >> 5, ln = e4 & 31;
+        const int r = (ln & 15) + 16 * (w & 3);
+        const int c = 4 * (2 * (w >> 2) + (ln >> 4));
+        float gL[4], lL[4], gv[4], lv[4], qv[4] = {0.f, 0.f, 0.f, 0.f}, kv[4] = {0.f, 0.f, 0.f, 0.f};
+        load4(g + last + c, gL);
+        load4(gl + last + c, lL);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            gv[u] = gL[u];
+            lv[u] = lL[u];
+        }
+        if (r < len) {
+            const size_t off = tok_off(tok0 + r, H, h, DK) + c;
+            load4(q + off, qv);
+            load4(k + off, kv);
+            load4(g + off, gv);
+            load4(gl + off, lv);
+            float4 qg, kd;
+            qg.x = qv[0] * exp_g(gv[0], lv[0]);
+            qg.y = qv[1] * exp_g(gv[1], lv[1]);
+            qg.z = qv[2] * exp_g(gv[2], lv[2]);
+            qg.w = qv[3] * exp_g(gv[3], lv[3]);
+            kd.x = kv[0] * exp_gdiff(gL[0], lL[0], gv[0], lv[0]);
+            kd.y = kv[1] * exp_gdiff(gL[1], lL[1], gv[1], lv[1]);
+            kd.z = kv[2] * exp_gdiff(gL[2], lL[2], gv[2], lv[2]);
+            kd.w = kv[3] * exp_gdiff(gL[3], lL[3], gv[3], lv[3]);
+            *reinterpret_cast<float4*>(Qg + off) = qg;
+            *reinterpret_cast<float4*>(Kd + off) = kd;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            Qt[(c + u) * kPS + r] = qv[u];
+            Kt[(c + u) * kPS + r] = kv[u];
+            Gt[(c + u) * kPS + r] = gv[u];
+            GLt[(c + u) * kPS + r] = lv[u];
+        }
     }
     __syncthreads();
+
+    const int t = tid >> 2, s = tid & 3;   // tile t of the lower triangle, channel phase s
+    int a = 0;
+    while ((a + 1) * (a + 2) / 2 <= t) ++a;
+    const int b = t - a * (a + 1) / 2;
+    float pa[4][4], aa[4][4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) pa[x][y] = aa[x][y] = 0.f;
+#pragma unroll 2
+    for (int j = 0; j < DK / 4; ++j) {
+        const int row = (4 * j + s) * kPS;
+        const float4 qr = *reinterpret_cast<const float4*>(Qt + row + 4 * a);
+        const float4 kr = *reinterpret_cast<const float4*>(Kt + row + 4 * a);
+        const float4 gr = *reinterpret_cast<const float4*>(Gt + row + 4 * a);
+        const float4 lr = *reinterpret_cast<const float4*>(GLt + row + 4 * a);
+        const float4 ki = *reinterpret_cast<const float4*>(Kt + row + 4 * b);
+        const float4 gi = *reinterpret_cast<const float4*>(Gt + row + 4 * b);
+        const float4 li = *reinterpret_cast<const float4*>(GLt + row + 4 * b);
+        const float qx[4] = {qr.x, qr.y, qr.z, qr.w}, kx[4] = {kr.x, kr.y, kr.z, kr.w};
+        const float gx[4] = {gr.x, gr.y, gr.z, gr.w}, lx[4] = {lr.x, lr.y, lr.z, lr.w};
+        const float ky[4] = {ki.x, ki.y, ki.z, ki.w}, gy[4] = {gi.x, gi.y, gi.z, gi.w};
+        const float ly[4] = {li.x, li.y, li.z, li.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                const float ke = ky[y] * exp_gdiff(gx[x], lx[x], gy[y], ly[y]);
+                pa[x][y] = fmaf(qx[x], ke, pa[x][y]);
+                aa[x][y] = fmaf(kx[x], ke, aa[x][y]);
+            }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            pa[x][y] += __shfl_xor_sync(0xffffffffu, pa[x][y], 1);
+            aa[x][y] += __shfl_xor_sync(0xffffffffu, aa[x][y], 1);
+            pa[x][y] += __shfl_xor_sync(0xffffffffu, pa[x][y], 2);
+            aa[x][y] += __shfl_xor_sync(0xffffffffu, aa[x][y], 2);
+        }
+    // lane s of the quad writes row 4a + s of the tile
+    float pr[4], ar[4];
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+        pr[y] = pa[0][y];
+        ar[y] = aa[0][y];
+    }
+#pragma unroll
+    for (int x = 1; x < 4; ++x)
+        if (s == x) {
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                pr[y] = pa[x][y];
+                ar[y] = aa[x][y];
+            }
+        }
+    const int r = 4 * a + s, i0 = 4 * b;
+    const bool live = r < len;
     float* Pc = P + ((size_t)blockIdx.x * H + h) * C * C;
     float* Ac = At + ((size_t)blockIdx.x * H + h) * C * C;
-    for (int p = warp; p < C * C; p += kTW / 32) {
-        const int r = p / C, i = p - r * C;
-        float s = 0.f, a = 0.f;
-        if (r < len && i <= r) {
-            for (int c = lane; c < dk; c += 32) {
-                const float ke = Ks[i * dk + c] *
-                                 exp_gdiff(Gs[r * dk + c], GLs[r * dk + c], Gs[i * dk + c], GLs[i * dk + c]);
-                s += Qs[r * dk + c] * ke;
-                a += Ks[r * dk + c] * ke;
-            }
-            s = wsum(s);
-            a = wsum(a);
+    float4 po, ao;
+    po.x = (live && i0 <= r) ? pr[0] : 0.f;
+    po.y = (live && i0 + 1 <= r) ? pr[1] : 0.f;
+    po.z = (live && i0 + 2 <= r) ? pr[2] : 0.f;
+    po.w = (live && i0 + 3 <= r) ? pr[3] : 0.f;
+    ao.x = (live && i0 < r) ? ar[0] : 0.f;
+    ao.y = (live && i0 + 1 < r) ? ar[1] : 0.f;
+    ao.z = (live && i0 + 2 < r) ? ar[2] : 0.f;
+    ao.w = (live && i0 + 3 < r) ? ar[3] : 0.f;
+    *reinterpret_cast<float4*>(Pc + r * C + i0) = po;
+    *reinterpret_cast<float4*>(Ac + r * C + i0) = ao;
+    // the tiles above the diagonal
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e4 = tid; e4 < C * C / 4; e4 += kPThreads) {
+        const int rr = e4 >> 4, bb = e4 & 15;
+        if (bb > (rr >> 2)) {
+            *reinterpret_cast<float4*>(Pc + rr * C + 4 * bb) = zero;
+            *reinterpret_cast<float4*>(Ac + rr * C + 4 * bb) = zero;
         }
-        if (lane == 0) {
-            Pc[p] = s;
-            Ac[p] = (i < r) ? a : 0.f;
-        }
-    }
-    for (int e = tid; e < len * dk; e += kTW) {
-        const int r = e / dk, c = e - r * dk;
-        const size_t off = tok_off(tok0 + r, H, h, dk) + c;
-        const int l = (len - 1) * dk + c;
-        Qg[off] = Qs[e] * exp_g(Gs[e], GLs[e]);
-        Kd[off] = Ks[e] * exp_gdiff(Gs[l], GLs[l], Gs[e], GLs[e]);
     }
 }
 
@@ -648,17 +761,18 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
     }
     if (e != cudaSuccess) return e;
     timing_mark(stream, 1);
-    const size_t smem_p = sizeof(float) * 4 * (size_t)C * dk;
+    const size_t smem_p = sizeof(float) * 4 * (size_t)kPS * dk;
     const size_t smem_chain = sizeof(float) * ((size_t)dk * kBV + 2 * (size_t)C * dk + 2 * (size_t)C * kBV +
                                                (size_t)C * C + 2 * dk);
-    if ((e = cudaFuncSetAttribute(kb_p<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
+    auto kern_p = dk == 128 ? kb_p<Tin, 128> : kb_p<Tin, 64>;
+    if ((e = cudaFuncSetAttribute(kern_p, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
     if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
         return e;
     // two chain blocks per SM (115,712 bytes each at d = 128) need the whole shared-memory carveout
     if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100))) return e;
     if (n_chunks > 0)
-        kb_p<Tin><<<dim3(n_chunks, H), kTW, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg, ws.Kd,
-                                                             cmap, H, dk, C);
+        kern_p<<<dim3(n_chunks, H), kPThreads, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg,
+                                                                 ws.Kd, cmap, H);
     timing_mark(stream, 2);
     if (n_seqs > 0)
         kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kTW, smem_chain, stream>>>(
