@@ -307,9 +307,9 @@ KDA_API kda_status kda_decode_step_prep(const void* q, const void* k, const void
  * chunks whatever C asks for (the chunk form does not depend on the chunk
  * length): by the tensor-core forward for bf16 with dk = dv = 128, by the
  * fp32 CUDA-core kernels otherwise; the gradient kernels run in fp32.  dlog_alpha is zero where log_alpha is below
- * the kernels' floor of -100 (log alpha = -inf included).  dlog_alpha sums
- * per-row contributions with shared-memory atomics, so repeated calls may
- * differ in its last bits; the other gradients are reproducible.  Errors as
+ * the kernels' floor of -100 (log alpha = -inf included).  dlog_alpha and dk
+ * add per-tile contributions with shared-memory atomics, so repeated calls may
+ * differ in their last bits; dq, dv, dbeta and d_init_state are reproducible.  Errors as
  * kda_chunk_fwd; all output pointers must be distinct from the inputs.
  */
 KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C,

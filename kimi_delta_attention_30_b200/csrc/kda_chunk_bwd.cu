@@ -38,7 +38,7 @@ namespace kda {
 namespace {
 
 constexpr int kT = 256;
-constexpr int kTW = 512;      // kb_chain and kb_c: more warps to hide latency
+constexpr int kTW = 512;      // kb_chain: more warps to hide latency
 constexpr int kBV = 32;       // d_v columns per chain block / per tile
 constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
 constexpr int kMaxDK = 128;
@@ -601,119 +601,232 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
     for (int e = tid; e < C * C; e += kT) dAc[e] = bs[e / C] * dA[e];
 }
 
+constexpr int kCThreads = 512;   // kb_c: 8 pairs of row blocks x 64 channels
+constexpr int kCH = 64;          // kb_c: channels per pass
+
 // Per (chunk, head): the pairwise terms of At and P, the elementwise factors,
 // and dlog alpha.  A pairwise term T_ri = (dAt_ri k_r + dP_ri q_r) k_i E_ri depends
 // on log alpha_j exactly for i < j <= r, so its share of dlog alpha_j is
-// F(j) = sum_{r >= j} sum_{i < j} T_ri, accumulated from each row's prefix sums
-// over i (no term is added and later cancelled, as a reverse cumulative sum of
-// row minus column sums would do).  Likewise Qg_r, Kg_r depend on log alpha_j for
-// j <= r, Kd_r for r < j, and Gam for every j:
+// F(j) = sum_{r >= j} sum_{i < j} T_ri.  Likewise Qg_r, Kg_r depend on log alpha_j
+// for j <= r, Kd_r for r < j, and Gam for every j:
 //   dlog alpha_j = F(j) + sum_{r>=j} (dQg Qg + dKg Kg)_r + sum_{r<j} (dKd Kd)_r + dGam Gam.
-// Phase A (rows): thread t takes channel c = t % DK and rows r = t / DK + m NRG,
-// and leaves its row sums for dk in the dWk buffer (no longer needed); phase B
-// (columns) the same with columns i; phase C one thread per channel.
-// Shared: Qs, Ks, Gs, GLs, F [C][DK], dAs, dPs [C][C], gC, gCl [DK].
+// The pair grid is cut into 4 x 4 tiles (rows of block a: 4a..4a+3, columns of
+// block b: 4b..4b+3, b <= a).  A thread owns one channel and the row blocks a and
+// 15 - a (17 tiles), so each exponential is formed once and the row sums (dq and
+// the row part of dk) stay in registers; the column sums (the rest of dk) are
+// added per tile into shared memory.  F is assembled from tile sums without any
+// term that is added and later cancelled: for j = 4m + u (0 <= u < 4),
+//   F(j) = sum_{a > m} [ sum_{b < m} S_ab + sum_{y < u} colT_am(y) ]   (rows below block m)
+//        + sum_{b < m} sum_{x >= u} rowT_mb(x)                         (rows of block m, u..3)
+//        + sum_{y < u <= x} T_{4m+x, 4m+y}                              (diagonal tile)
+// with S_ab the sum of tile (a, b) and rowT / colT its row and column sums; the
+// thread of row block a adds the first line's terms of tile (a, m) to F(4m + u)
+// and keeps the other two in registers until its row block is done.
+// Channels are processed in passes of 64; q, k, g and its low part are staged
+// channel-major ([c][r], row stride kPS), padded rows as in kb_p.  The dAt and
+// dP tiles are staged with their masks applied (zero for i >= r, resp. i > r, and
+// for rows past the end of the chunk).
+// Shared: Qt, Kt, Gt, GLt [kCH][kPS], dAs, dPs [C][C], Fs, Ys, Xs [C][kCH].
 template <typename Tin, int DK>
-__global__ void __launch_bounds__(kTW) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
-                                           const Tin* __restrict__ la, const float* __restrict__ g,
-                                           const float* __restrict__ gl,
-                                           const float* __restrict__ dAt, const float* __restrict__ dP,
-                                           const float* __restrict__ dQg, const float* __restrict__ dKd,
-                                           const float* __restrict__ dKg, const float* __restrict__ dGam,
-                                           float* __restrict__ dKrow, Tin* __restrict__ dq_out,
-                                           Tin* __restrict__ dk_out, Tin* __restrict__ dla_out, ChunkMap cmap,
-                                           int H) {
-    constexpr int C = 64;
-    constexpr int NRG = kTW / DK;
-    extern __shared__ float smem[];
+__global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
+                                                     const Tin* __restrict__ la, const float* __restrict__ g,
+                                                     const float* __restrict__ gl,
+                                                     const float* __restrict__ dAt, const float* __restrict__ dP,
+                                                     const float* __restrict__ dQg, const float* __restrict__ dKd,
+                                                     const float* __restrict__ dKg, const float* __restrict__ dGam,
+                                                     Tin* __restrict__ dq_out, Tin* __restrict__ dk_out,
+                                                     Tin* __restrict__ dla_out, ChunkMap cmap, int H) {
+    constexpr int C = kBwdC;
+    static_assert(DK % kCH == 0, "whole passes of channels");
+    extern __shared__ __align__(16) float smem[];
+    float* Qt = smem;
+    float* Kt = Qt + kCH * kPS;
+    float* Gt = Kt + kCH * kPS;
+    float* GLt = Gt + kCH * kPS;
+    float* dAs = GLt + kCH * kPS;
+    float* dPs = dAs + C * C;
+    float* Fs = dPs + C * C;
+    float* Ys = Fs + C * kCH;
+    float* Xs = Ys + C * kCH;
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
-    const int h = blockIdx.y, tid = threadIdx.x, c = tid % DK, rg = tid / DK;
-    float* Qs = smem;
-    float* Ks = Qs + C * DK;
-    float* Gs = Ks + C * DK;
-    float* GLs = Gs + C * DK;
-    float* F = GLs + C * DK;         // [C][DK], added to by the row groups with shared atomics
-    float* dAs = F + C * DK;
-    float* dPs = dAs + C * C;
-    float* gC = dPs + C * C;
-    float* gCl = gC + DK;
+    const int h = blockIdx.y, tid = threadIdx.x;
     const size_t chunk = blockIdx.x;
-    for (int e = tid; e < len * DK; e += kTW) {
-        const int r = e / DK, cc = e - r * DK;
-        const size_t off = tok_off(tok0 + r, H, h, DK) + cc;
-        Qs[e] = to_f32(q[off]);
-        Ks[e] = to_f32(k[off]);
-        Gs[e] = g[off];
-        GLs[e] = gl[off];
+    const size_t tbase = (chunk * H + h) * C * C;
+    for (int e4 = tid; e4 < C * C / 4; e4 += kCThreads) {
+        const int r = e4 >> 4, i0 = 4 * (e4 & 15);
+        const bool live = r < len;
+        const float4 av = *reinterpret_cast<const float4*>(dAt + tbase + r * C + i0);
+        const float4 pv = *reinterpret_cast<const float4*>(dP + tbase + r * C + i0);
+        float4 ao, po;
+        ao.x = (live && i0 < r) ? av.x : 0.f;
+        ao.y = (live && i0 + 1 < r) ? av.y : 0.f;
+        ao.z = (live && i0 + 2 < r) ? av.z : 0.f;
+        ao.w = (live && i0 + 3 < r) ? av.w : 0.f;
+        po.x = (live && i0 <= r) ? pv.x : 0.f;
+        po.y = (live && i0 + 1 <= r) ? pv.y : 0.f;
+        po.z = (live && i0 + 2 <= r) ? pv.z : 0.f;
+        po.w = (live && i0 + 3 <= r) ? pv.w : 0.f;
+        *reinterpret_cast<float4*>(dAs + r * C + i0) = ao;
+        *reinterpret_cast<float4*>(dPs + r * C + i0) = po;
     }
-    for (int e = tid; e < C * DK; e += kTW) F[e] = 0.f;
-    for (int e = tid; e < C * C; e += kTW) {
-        dAs[e] = dAt[(chunk * H + h) * C * C + e];
-        dPs[e] = dP[(chunk * H + h) * C * C + e];
-    }
-    __syncthreads();
-    if (rg == 0) {
-        gC[c] = Gs[(len - 1) * DK + c];
-        gCl[c] = GLs[(len - 1) * DK + c];
-    }
-    // phase A: x1 = sum_{i<r} dAt k_i E, x2 = sum_{i<=r} dP k_i E; prefix sums of T_ri into F
-    for (int r = rg; r < len; r += NRG) {
-        const float gr = Gs[r * DK + c], grl = GLs[r * DK + c];
-        const float qv = Qs[r * DK + c], kv = Ks[r * DK + c];
-        float x1 = 0.f, x2 = 0.f, pre = 0.f;
-        for (int i = 0; i < r; ++i) {
-            const float ke = Ks[i * DK + c] * exp_gdiff(gr, grl, Gs[i * DK + c], GLs[i * DK + c]);
-            const float a = dAs[r * C + i] * ke, b = dPs[r * C + i] * ke;
-            x1 += a;
-            x2 += b;
-            pre += kv * a + qv * b;
-            atomicAdd(&F[(i + 1) * DK + c], pre);   // T_ri with i < j <= r
+    const size_t last = tok_off(tok0 + len - 1, H, h, DK);
+    const int c = tid & (kCH - 1), ap = tid / kCH;   // this thread's channel in the pass, row-block pair
+
+    for (int c0 = 0; c0 < DK; c0 += kCH) {
+        if (c0 > 0) __syncthreads();   // the previous pass is done with the shared arrays
+        // staging, groups of 4 channels; a warp covers 16 rows x 2 groups (32 banks)
+        for (int e4 = tid; e4 < C * kCH / 4; e4 += kCThreads) {
+            const int w = e4 >> 5, ln = e4 & 31;
+            const int r = (ln & 15) + 16 * (w & 3);
+            const int cq = 4 * (2 * (w >> 2) + (ln >> 4));
+            float gv[4], lv[4], qv[4] = {0.f, 0.f, 0.f, 0.f}, kv[4] = {0.f, 0.f, 0.f, 0.f};
+            if (r < len) {
+                const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + cq;
+                load4(q + off, qv);
+                load4(k + off, kv);
+                load4(g + off, gv);
+                load4(gl + off, lv);
+            } else {
+                load4(g + last + c0 + cq, gv);
+                load4(gl + last + c0 + cq, lv);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                Qt[(cq + u) * kPS + r] = qv[u];
+                Kt[(cq + u) * kPS + r] = kv[u];
+                Gt[(cq + u) * kPS + r] = gv[u];
+                GLt[(cq + u) * kPS + r] = lv[u];
+            }
         }
-        x2 += dPs[r * C + r] * kv;         // the diagonal of P (E = 1)
-        const size_t off = tok_off(tok0 + r, H, h, DK) + c;
-        dq_out[off] = from_f32<Tin>(x2 + dQg[off] * exp_g(gr, grl));
-        dKrow[off] = x1;
-    }
-    __syncthreads();
-    // phase B: column sums y = sum_{r>i} dAt k_r E + sum_{r>=i} dP q_r E
-    for (int i = rg; i < len; i += NRG) {
-        const float gi = Gs[i * DK + c], gil = GLs[i * DK + c];
-        float y = 0.f;
-        for (int r = i; r < len; ++r) {
-            const float e = exp_gdiff(Gs[r * DK + c], GLs[r * DK + c], gi, gil);
-            y += (dAs[r * C + i] * Ks[r * DK + c] + dPs[r * C + i] * Qs[r * DK + c]) * e;
+        for (int e = tid; e < 2 * C * kCH; e += kCThreads) Fs[e] = 0.f;   // Fs and Ys
+        __syncthreads();
+
+        const float* qc = Qt + c * kPS;
+        const float* kc = Kt + c * kPS;
+        const float* gc = Gt + c * kPS;
+        const float* lc = GLt + c * kPS;
+        for (int half = 0; half < 2; ++half) {
+            const int a = half == 0 ? ap : 15 - ap;
+            float qr[4], kr[4], gr[4], lr[4];
+            {
+                const float4 q4 = *reinterpret_cast<const float4*>(qc + 4 * a);
+                const float4 k4 = *reinterpret_cast<const float4*>(kc + 4 * a);
+                const float4 g4 = *reinterpret_cast<const float4*>(gc + 4 * a);
+                const float4 l4 = *reinterpret_cast<const float4*>(lc + 4 * a);
+                qr[0] = q4.x; qr[1] = q4.y; qr[2] = q4.z; qr[3] = q4.w;
+                kr[0] = k4.x; kr[1] = k4.y; kr[2] = k4.z; kr[3] = k4.w;
+                gr[0] = g4.x; gr[1] = g4.y; gr[2] = g4.z; gr[3] = g4.w;
+                lr[0] = l4.x; lr[1] = l4.y; lr[2] = l4.z; lr[3] = l4.w;
+            }
+            float x1[4] = {0.f, 0.f, 0.f, 0.f}, x2[4] = {0.f, 0.f, 0.f, 0.f};
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};   // F terms of rows 4a + u.. (second and third lines)
+            float pref = 0.f;                      // sum of the tiles (a, b' < b)
+            for (int b = 0; b < a; ++b) {
+                const float4 k4 = *reinterpret_cast<const float4*>(kc + 4 * b);
+                const float4 g4 = *reinterpret_cast<const float4*>(gc + 4 * b);
+                const float4 l4 = *reinterpret_cast<const float4*>(lc + 4 * b);
+                const float ki[4] = {k4.x, k4.y, k4.z, k4.w}, gi[4] = {g4.x, g4.y, g4.z, g4.w};
+                const float li[4] = {l4.x, l4.y, l4.z, l4.w};
+                float colT[4] = {0.f, 0.f, 0.f, 0.f}, yc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(dAs + (4 * a + x) * C + 4 * b);
+                    const float4 p4 = *reinterpret_cast<const float4*>(dPs + (4 * a + x) * C + 4 * b);
+                    const float da[4] = {a4.x, a4.y, a4.z, a4.w}, dp[4] = {p4.x, p4.y, p4.z, p4.w};
+                    float rowT = 0.f;
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const float e = exp_gdiff(gr[x], lr[x], gi[y], li[y]);
+                        const float ke = ki[y] * e;
+                        const float av = da[y] * ke, bv = dp[y] * ke;
+                        x1[x] += av;
+                        x2[x] += bv;
+                        const float t = fmaf(kr[x], av, qr[x] * bv);
+                        rowT += t;
+                        colT[y] += t;
+                        yc[y] = fmaf(fmaf(da[y], kr[x], dp[y] * qr[x]), e, yc[y]);
+                    }
+                    // rows x >= u of this tile count for F(4a + u)
+#pragma unroll
+                    for (int u = 0; u <= x; ++u) rs[u] += rowT;
+                }
+                atomicAdd(&Fs[(4 * b) * kCH + c], pref);
+                atomicAdd(&Fs[(4 * b + 1) * kCH + c], pref + colT[0]);
+                atomicAdd(&Fs[(4 * b + 2) * kCH + c], pref + (colT[0] + colT[1]));
+                atomicAdd(&Fs[(4 * b + 3) * kCH + c], pref + (colT[0] + colT[1] + colT[2]));
+                pref += (colT[0] + colT[1]) + (colT[2] + colT[3]);
+#pragma unroll
+                for (int y = 0; y < 4; ++y) atomicAdd(&Ys[(4 * b + y) * kCH + c], yc[y]);
+            }
+            // the diagonal tile: pairs y <= x (E = 1 on the diagonal)
+            {
+                float yc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(dAs + (4 * a + x) * C + 4 * a);
+                    const float4 p4 = *reinterpret_cast<const float4*>(dPs + (4 * a + x) * C + 4 * a);
+                    const float da[4] = {a4.x, a4.y, a4.z, a4.w}, dp[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+                    for (int y = 0; y <= x; ++y) {
+                        const float e = y == x ? 1.f : exp_gdiff(gr[x], lr[x], gr[y], lr[y]);
+                        const float ke = kr[y] * e;
+                        const float av = da[y] * ke, bv = dp[y] * ke;
+                        x1[x] += av;
+                        x2[x] += bv;
+                        yc[y] = fmaf(fmaf(da[y], kr[x], dp[y] * qr[x]), e, yc[y]);
+                        if (y < x) {
+                            const float t = fmaf(kr[x], av, qr[x] * bv);
+#pragma unroll
+                            for (int u = y + 1; u <= x; ++u) rs[u] += t;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int y = 0; y < 4; ++y) atomicAdd(&Ys[(4 * a + y) * kCH + c], yc[y]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) atomicAdd(&Fs[(4 * a + u) * kCH + c], rs[u]);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int r = 4 * a + x;
+                Xs[r * kCH + c] = x1[x];
+                if (r < len) {
+                    const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + c;
+                    dq_out[off] = from_f32<Tin>(x2[x] + dQg[off] * exp_g(gr[x], lr[x]));
+                }
+            }
         }
-        const size_t off = tok_off(tok0 + i, H, h, DK) + c;
-        dk_out[off] = from_f32<Tin>(dKrow[off] + y + dKg[off] * exp_g(gi, gil) +
-                                    dKd[off] * exp_gdiff(gC[c], gCl[c], gi, gil));
-    }
-    __syncthreads();
-    // phase C: the per-(row, channel) terms are formed by every thread first (the
-    // dAt / dP tiles are free now, and Q is replaced in place), so the two
-    // sequential sums below read shared memory only
-    float* tkd = dAs;   // [C][DK] (the dAt and dP tiles together): dKd Kd
-    for (int e = tid; e < len * DK; e += kTW) {
-        const int j = e / DK, cc = e - j * DK;
-        const size_t off = tok_off(tok0 + j, H, h, DK) + cc;
-        tkd[e] = dKd[off] * Ks[e] * exp_gdiff(gC[cc], gCl[cc], Gs[e], GLs[e]);
-        Qs[e] = (dQg[off] * Qs[e] + dKg[off] * Ks[e]) * exp_g(Gs[e], GLs[e]);   // dQg Qg + dKg Kg
-    }
-    __syncthreads();
-    // dlog alpha (zero where the forward's floor on log alpha was active)
-    if (rg == 0) {
-        float pre = 0.f;   // sum_{r<j} dKd Kd, added to F[j]
-        for (int j = 0; j < len; ++j) {
-            F[j * DK + c] += pre;
-            pre += tkd[j * DK + c];
+        __syncthreads();
+        // dk, and the per-(row, channel) terms of dlog alpha (into Xs and Ys, which
+        // each element's thread has just read)
+        const float gC = Gt[c * kPS + len - 1], gCl = GLt[c * kPS + len - 1];   // used by ap == 0 below
+        for (int e = tid; e < len * kCH; e += kCThreads) {
+            const int r = e / kCH, cc = e - r * kCH;
+            const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + cc;
+            const float gv = Gt[cc * kPS + r], lv = GLt[cc * kPS + r];
+            const float eg = exp_g(gv, lv);
+            const float ed = exp_gdiff(Gt[cc * kPS + len - 1], GLt[cc * kPS + len - 1], gv, lv);
+            const float dkg = dKg[off], dkd = dKd[off];
+            dk_out[off] = from_f32<Tin>(Xs[e] + Ys[e] + dkg * eg + dkd * ed);
+            Xs[e] = dkd * Kt[cc * kPS + r] * ed;                               // dKd Kd
+            Ys[e] = (dQg[off] * Qt[cc * kPS + r] + dkg * Kt[cc * kPS + r]) * eg;   // dQg Qg + dKg Kg
         }
-        const float gam = dGam[(chunk * H + h) * DK + c] * exp_g(gC[c], gCl[c]);
-        float suf = 0.f;   // sum_{r>=j} (dQg Qg + dKg Kg)
-        for (int j = len - 1; j >= 0; --j) {
-            const size_t off = tok_off(tok0 + j, H, h, DK) + c;
-            suf += Qs[j * DK + c];
-            const float f = F[j * DK + c];
-            dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? f + suf + gam : 0.f);
+        __syncthreads();
+        // dlog alpha, one thread per channel (zero where the forward's floor on log alpha was active)
+        if (ap == 0) {
+            float pre = 0.f;   // sum_{r<j} dKd Kd
+            for (int j = 0; j < len; ++j) {
+                Fs[j * kCH + c] += pre;
+                pre += Xs[j * kCH + c];
+            }
+            const float gam = dGam[(chunk * H + h) * DK + c0 + c] * exp_g(gC, gCl);
+            float suf = 0.f;   // sum_{r>=j} (dQg Qg + dKg Kg)
+            for (int j = len - 1; j >= 0; --j) {
+                const size_t off = tok_off(tok0 + j, H, h, DK) + c0 + c;
+                suf += Ys[j * kCH + c];
+                dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? Fs[j * kCH + c] + suf + gam : 0.f);
+            }
         }
     }
 }
@@ -725,7 +838,7 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     constexpr int C = 64;
     const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * (DK + 1) + 3 * (size_t)C * kBP);
     const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + (size_t)C * (dv + DK + 1));
-    const size_t smem_c = sizeof(float) * (5 * (size_t)C * DK + 2 * (size_t)C * C + 2 * DK);
+    const size_t smem_c = sizeof(float) * (4 * (size_t)kCH * kPS + 2 * (size_t)C * C + 3 * (size_t)C * kCH);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
     if ((e = cudaFuncSetAttribute(kb_b<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
@@ -737,8 +850,8 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
                                             ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
     timing_mark(stream, 5);
-    kb_c<Tin, DK><<<grid, kTW, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg,
-                                               ws.dGam, ws.dWk, dq, dk_, dla, cmap, H);
+    kb_c<Tin, DK><<<grid, kCThreads, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd,
+                                                     ws.dKg, ws.dGam, dq, dk_, dla, cmap, H);
     timing_mark(stream, 6);
     return cudaGetLastError();
 }
