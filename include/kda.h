@@ -332,6 +332,9 @@ KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
  * (cleared at the start of each call).  These two calls synchronise `stream`
  * and return KDA_OK or the recorded error for the last kda_chunk_fwd[_ex|_prep]
  * / kda_chunk_bwd call that used `workspace` with the same size arguments.
+ * They copy 4 bytes of the caller-owned workspace to the host and write
+ * nothing.  (No counterpart on the pages: this is part of the library's
+ * failure handling, not of the operation.)
  * For problems on the CUDA-core path they return KDA_OK without touching the
  * device (those kernels do not wait on the device).  Errors: KDA_ERR_NULL for a
  * NULL workspace, the size errors of the calls themselves, KDA_ERR_CUDA if the
