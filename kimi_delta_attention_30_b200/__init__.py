@@ -18,6 +18,7 @@ logits and beta logits are then normalised / activated inside the kernels
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -142,6 +143,31 @@ def _stream_handle(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+@contextlib.contextmanager
+def _launch_on(device, stream, tensors=()):
+    """Run one library call on ``device``: it is made the current device for the
+    duration (the library launches on the current device), and the call's stream
+    is ``stream`` or that device's current stream.  Every tensor must live on
+    ``device``.  Yields ``(stream, allocated)``: tensors the wrapper allocates
+    are appended to ``allocated`` and, when the stream is not the device's
+    current stream, recorded on it afterwards so that the caching allocator does
+    not reuse their memory while the call's kernels may still run."""
+    for name, t in tensors:
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+    with torch.cuda.device(device):
+        cur = torch.cuda.current_stream(device)
+        s = cur if stream is None else stream
+        if s.device != device:
+            raise ValueError(f"stream belongs to {s.device}, the call runs on {device}")
+        allocated = []
+        yield s, allocated
+        if s != cur:
+            for t in allocated:
+                if t is not None:
+                    t.record_stream(s)
+
+
 def _check_cuda(name, t, dtype=None):
     if t is None:
         return
@@ -215,32 +241,38 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
     cu, n_seqs, _keep = _cu_arg(cu_seqlens)
     N = n_seqs if cu_seqlens is not None else B
     _check_cuda("init_state", init_state, torch.float32)
-    if o is None:
-        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
-    if final_state is None and output_final_state:
-        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    _check_cuda("o", o, dt)
-    _check_cuda("final_state", final_state, torch.float32)
-    need = lib().kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, C, _DTYPES[dt], cu, n_seqs, ALGOS[algo])
-    if workspace is None:
-        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
-    _check_cuda("workspace", workspace)
-    if prep:
-        if algo not in ("auto", "tc"):
-            raise ValueError("prep is fused into the tensor-core path only")
-        st = lib().kda_chunk_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], prep,
-                                      _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o),
-                                      _ptr(final_state), _ptr(workspace),
-                                      workspace.numel() * workspace.element_size(), _stream_handle(stream))
-        if st != 0:
-            raise KdaError(st, "kda_chunk_fwd_prep")
-        return o, final_state
-    st = lib().kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
-                                _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o), _ptr(final_state),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                _stream_handle(stream), ALGOS[algo])
+    if prep and algo not in ("auto", "tc"):
+        raise ValueError("prep is fused into the tensor-core path only")
+    dev = q.device
+    with _launch_on(dev, stream, (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta),
+                                  ("init_state", init_state), ("o", o), ("final_state", final_state),
+                                  ("workspace", workspace))) as (s, allocated):
+        if o is None:
+            o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+            allocated.append(o)
+        if final_state is None and output_final_state:
+            final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+            allocated.append(final_state)
+        _check_cuda("o", o, dt)
+        _check_cuda("final_state", final_state, torch.float32)
+        need = lib().kda_chunk_fwd_workspace_size_ex(B, T, H, dk, dv, C, _DTYPES[dt], cu, n_seqs, ALGOS[algo])
+        if workspace is None:
+            workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=dev)
+            allocated.append(workspace)
+        _check_cuda("workspace", workspace)
+        wsb = workspace.numel() * workspace.element_size()
+        if prep:
+            st = lib().kda_chunk_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                          prep, _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o),
+                                          _ptr(final_state), _ptr(workspace), wsb, _stream_handle(s))
+            what = "kda_chunk_fwd_prep"
+        else:
+            st = lib().kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                        _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o),
+                                        _ptr(final_state), _ptr(workspace), wsb, _stream_handle(s), ALGOS[algo])
+            what = "kda_chunk_fwd"
     if st != 0:
-        raise KdaError(st, "kda_chunk_fwd")
+        raise KdaError(st, what)
     return o, final_state
 
 
@@ -280,43 +312,57 @@ def chunk_bwd(q, k, v, log_alpha, beta, d_o, init_state=None, d_final_state=None
     dv = v.shape[-1]
     cu, n_seqs, _keep = _cu_arg(cu_seqlens)
     N = n_seqs if cu_seqlens is not None else B
-    if grads is None:
-        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_alpha),
-                 torch.empty_like(beta),
-                 torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if need_d_init_state else None)
-    dq, dk_, dv_, dla, dbeta, dinit = grads
-    for name, t in (("dq", dq), ("dk", dk_), ("dv", dv_), ("dlog_alpha", dla), ("dbeta", dbeta)):
-        _check_cuda(name, t, dt)
-    _check_cuda("d_init_state", dinit, torch.float32)
-    need = lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, C, cu, n_seqs)
-    if workspace is None:
-        workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=q.device)
-    _check_cuda("workspace", workspace)
-    st = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], _ptr(init_state),
-                             cu, n_seqs, B, T, H, dk, dv, C, _ptr(d_o), _ptr(d_final_state), _ptr(dq), _ptr(dk_),
-                             _ptr(dv_), _ptr(dla), _ptr(dbeta), _ptr(dinit), _ptr(workspace),
-                             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    dev = q.device
+    given = () if grads is None else tuple((f"grads[{i}]", t) for i, t in enumerate(grads))
+    with _launch_on(dev, stream, (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta), ("d_o", d_o),
+                                  ("init_state", init_state), ("d_final_state", d_final_state),
+                                  ("workspace", workspace)) + given) as (s, allocated):
+        if grads is None:
+            grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(log_alpha),
+                     torch.empty_like(beta),
+                     torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if need_d_init_state else None)
+            allocated.extend(grads)
+        dq, dk_, dv_, dla, dbeta, dinit = grads
+        for name, t in (("dq", dq), ("dk", dk_), ("dv", dv_), ("dlog_alpha", dla), ("dbeta", dbeta)):
+            _check_cuda(name, t, dt)
+        _check_cuda("d_init_state", dinit, torch.float32)
+        need = lib().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, C, cu, n_seqs)
+        if workspace is None:
+            workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=dev)
+            allocated.append(workspace)
+        _check_cuda("workspace", workspace)
+        st = lib().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                 _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(d_o), _ptr(d_final_state),
+                                 _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(dbeta), _ptr(dinit),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_handle(s))
     if st != 0:
         raise KdaError(st, "kda_chunk_bwd")
     return dq, dk_, dv_, dla, dbeta, dinit
 
 
-def device_status(kind, workspace, dtype, B, T, H, dk, dv, C=64, cu_seqlens=None, algo="auto", stream=None):
+def device_status(kind, workspace, dtype, B, T, H, dk, dv, C=64, cu_seqlens=None, algo="auto", stream=None,
+                  device=None):
     """Synchronise ``stream`` and return the device-side status (0 or
     KDA_ERR_TIMEOUT) of the last call of ``kind`` ("fwd", "bwd" or "noalloc")
-    that used ``workspace`` (ignored for "noalloc") with these sizes.  Raises
-    KdaError for invalid arguments or a failed copy."""
+    that used ``workspace`` (ignored for "noalloc") with these sizes.  The
+    query runs on the workspace's device (for "noalloc": ``device``, default the
+    current device).  Raises KdaError for invalid arguments or a failed copy."""
     cu, n, _keep = _cu_arg(cu_seqlens)
     d = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
-    h = _stream_handle(stream)
-    if kind == "fwd":
-        st = lib().kda_chunk_fwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, ALGOS[algo], h)
-    elif kind == "bwd":
-        st = lib().kda_chunk_bwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, h)
-    elif kind == "noalloc":
-        st = lib().kda_chunk_fwd_noalloc_device_status(d, cu, n, B, T, H, dk, dv, C, h)
-    else:
+    if kind not in ("fwd", "bwd", "noalloc"):
         raise ValueError(f"unknown kind {kind!r}")
+    if workspace is not None:
+        dev = workspace.device
+    else:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with _launch_on(dev, stream) as (s, _):
+        h = _stream_handle(s)
+        if kind == "fwd":
+            st = lib().kda_chunk_fwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, ALGOS[algo], h)
+        elif kind == "bwd":
+            st = lib().kda_chunk_bwd_device_status(_ptr(workspace), d, cu, n, B, T, H, dk, dv, C, h)
+        else:
+            st = lib().kda_chunk_fwd_noalloc_device_status(d, cu, n, B, T, H, dk, dv, C, h)
     if st not in (0, KDA_ERR_TIMEOUT):
         raise KdaError(st, f"device status ({kind})")
     return int(st)
@@ -342,15 +388,21 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None
     cu, n_seqs, _keep = _cu_arg(cu_seqlens)
     N = n_seqs if cu_seqlens is not None else B
     _check_cuda("init_state", init_state, torch.float32)
-    if o is None:
-        o = torch.empty((B, T, H, dv), dtype=dt, device=q.device)
-    if final_state is None:
-        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
-    _check_cuda("o", o, dt)
-    _check_cuda("final_state", final_state, torch.float32)
-    st = lib().kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
-                                     _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o), _ptr(final_state),
-                                     _stream_handle(stream))
+    dev = q.device
+    with _launch_on(dev, stream, (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta),
+                                  ("init_state", init_state), ("o", o), ("final_state", final_state))) \
+            as (s, allocated):
+        if o is None:
+            o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+            allocated.append(o)
+        if final_state is None:
+            final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+            allocated.append(final_state)
+        _check_cuda("o", o, dt)
+        _check_cuda("final_state", final_state, torch.float32)
+        st = lib().kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                         _ptr(init_state), cu, n_seqs, B, T, H, dk, dv, C, _ptr(o),
+                                         _ptr(final_state), _stream_handle(s))
     if st != 0:
         raise KdaError(st, "kda_chunk_fwd_noalloc")
     return o, final_state
@@ -369,17 +421,21 @@ def decode_step(q, k, v, log_alpha, beta, state, o=None, stream=None, prep: int 
     _check_cuda("state", state, torch.float32)
     N, H, dk = q.shape
     dv = v.shape[-1]
-    if o is None:
-        o = torch.empty((N, H, dv), dtype=dt, device=q.device)
-    _check_cuda("o", o, dt)
-    if prep:
-        st = lib().kda_decode_step_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], prep,
-                                        _ptr(state), N, H, dk, dv, _ptr(o), _stream_handle(stream))
-        if st != 0:
-            raise KdaError(st, "kda_decode_step_prep")
-        return o
-    st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], _ptr(state),
-                               N, H, dk, dv, _ptr(o), _stream_handle(stream))
+    dev = q.device
+    with _launch_on(dev, stream, (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta),
+                                  ("state", state), ("o", o))) as (s, allocated):
+        if o is None:
+            o = torch.empty((N, H, dv), dtype=dt, device=dev)
+            allocated.append(o)
+        _check_cuda("o", o, dt)
+        if prep:
+            st = lib().kda_decode_step_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                            prep, _ptr(state), N, H, dk, dv, _ptr(o), _stream_handle(s))
+            what = "kda_decode_step_prep"
+        else:
+            st = lib().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt],
+                                       _ptr(state), N, H, dk, dv, _ptr(o), _stream_handle(s))
+            what = "kda_decode_step"
     if st != 0:
-        raise KdaError(st, "kda_decode_step")
+        raise KdaError(st, what)
     return o

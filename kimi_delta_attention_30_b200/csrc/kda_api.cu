@@ -20,7 +20,7 @@ bool tc_supports(int C);
 int tc_chunk();
 
 TimingHook& timing_hook() {
-    static thread_local TimingHook hook{{nullptr}, 0};
+    static thread_local TimingHook hook{{nullptr}, 0, 0};
     return hook;
 }
 
@@ -35,6 +35,44 @@ const char* const kSimtKernelNames[] = {"k1_cumsum", "k2_wy", "k3_state", "k4_ou
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Sequence tables reach the device as kernel arguments: the launch copies its
+// parameters when it is issued, so the host neither waits for the stream nor
+// keeps a buffer alive past the call (a copy from pageable host memory would
+// first wait for the stream's earlier work).  One launch carries up to
+// kTableBatch entries (16 KiB of parameters).
+constexpr int kTableBatch = 1024;
+struct TableBatch {
+    SeqInfo e[kTableBatch];
+};
+
+__global__ void __launch_bounds__(256) seq_table_write(SeqInfo* __restrict__ dst, int n, const __grid_constant__ TableBatch b) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = b.e[i];
+}
+
+// natural order then longest first, 2 n_seqs entries at `dst`; returns the number of
+// launches (with `mark`, timing-hook event i follows the i-th of them)
+int upload_tables(SeqInfo* dst, const std::vector<SeqInfo>& natural, const std::vector<SeqInfo>& by_len,
+                  cudaStream_t s, cudaError_t* err, bool mark = false) {
+    const size_t n = natural.size();
+    int launches = 0;
+    TableBatch b;
+    for (size_t i0 = 0; i0 < 2 * n; i0 += kTableBatch) {
+        const int cnt = (int)std::min<size_t>(kTableBatch, 2 * n - i0);
+        for (int i = 0; i < cnt; ++i) {
+            const size_t j = i0 + i;
+            b.e[i] = j < n ? natural[j] : by_len[j - n];
+        }
+        seq_table_write<<<1, 256, 0, s>>>(dst + i0, cnt, b);
+        ++launches;
+        if ((*err = cudaGetLastError()) != cudaSuccess) return launches;
+        if (mark) timing_mark_abs(s, launches);
+    }
+    *err = cudaSuccess;
+    return launches;
+}
+
+int table_launches(size_t n_seqs) { return (int)((2 * n_seqs + kTableBatch - 1) / kTableBatch); }
 
 // Problem geometry shared by the workspace query and the launch.
 struct Plan {
@@ -269,15 +307,18 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
     const int ncps = (int)((T + C - 1) / C);
     ChunkMap cmap{nullptr, p.n_seqs, T, C, ncps};
     SeqMap smap{nullptr, T, C, ncps};
+    timing_mark(s, 0);
     if (p.varlen) {
-        std::vector<SeqInfo> both(p.natural);
-        both.insert(both.end(), p.by_len.begin(), p.by_len.end());
-        if (cudaMemcpyAsync(ws, both.data(), both.size() * sizeof(SeqInfo), cudaMemcpyHostToDevice, s) != cudaSuccess)
+        cudaError_t terr;
+        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr, true);
+        if (terr != cudaSuccess) {
+            timing_hook().n = 0;
+            timing_hook().base = 0;
             return KDA_ERR_CUDA;
+        }
         cmap.seqs = (const SeqInfo*)ws;
         smap.order = (const SeqInfo*)ws + p.n_seqs;
     }
-    timing_mark(s, 0);
     cudaError_t err;
     if (algo == KDA_ALGO_SIMT) {
         SimtLayout L = simt_layout(p, H, dk, dv);
@@ -290,6 +331,7 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
                                 p.n_seqs, H, C, ws + table_bytes(p), prep, s);
     }
     timing_hook().n = 0;
+    timing_hook().base = 0;
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -358,9 +400,10 @@ int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype 
     if (st != KDA_OK) return st;
     algo = resolve(algo, dtype, dk, dv, C);
     const char* const* list = (algo == KDA_ALGO_TC) ? kTcKernelNames : kSimtKernelNames;
+    const int nt = p.varlen ? table_launches(p.natural.size()) : 0;   // sequence-table writes come first
     const int n = (algo == KDA_ALGO_TC) ? kTcKernelCount : 4;
-    for (int i = 0; names && i < n && i < max_names; ++i) names[i] = list[i];
-    return n;
+    for (int i = 0; names && i < nt + n && i < max_names; ++i) names[i] = i < nt ? "seq_table_write" : list[i - nt];
+    return nt + n;
 }
 
 size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int C, const int32_t* cu_seqlens_host,
@@ -405,10 +448,9 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     ChunkMap cmap{nullptr, p.n_seqs, T, Cb, ncps};
     SeqMap smap{nullptr, T, Cb, ncps};
     if (p.varlen) {
-        std::vector<SeqInfo> both(p.natural);
-        both.insert(both.end(), p.by_len.begin(), p.by_len.end());
-        if (cudaMemcpyAsync(ws, both.data(), both.size() * sizeof(SeqInfo), cudaMemcpyHostToDevice, s) != cudaSuccess)
-            return KDA_ERR_CUDA;
+        cudaError_t terr;
+        upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr);
+        if (terr != cudaSuccess) return KDA_ERR_CUDA;
         cmap.seqs = (const SeqInfo*)ws;
         smap.order = (const SeqInfo*)ws + p.n_seqs;
     }

@@ -145,14 +145,17 @@ __device__ __forceinline__ float exp_g(float h, float l) { return ex2_approx(h *
 struct TimingHook {
     void* ev[32];
     int n;
+    int base;   // kernels launched by the call before the algorithm's own (sequence tables)
 };
 TimingHook& timing_hook();   // per host thread
 
-// Record hook event i on `s` if the hook asks for it.
-inline void timing_mark(cudaStream_t s, int i) {
+// Record hook event `i` (counted from the call's first launch) on `s` if the hook asks for it.
+inline void timing_mark_abs(cudaStream_t s, int i) {
     TimingHook& h = timing_hook();
-    if (i < h.n && h.ev[i]) cudaEventRecord((cudaEvent_t)h.ev[i], s);
+    if (i >= 0 && i < h.n && i < 32 && h.ev[i]) cudaEventRecord((cudaEvent_t)h.ev[i], s);
 }
+// The same for the algorithm's own kernels: mark i follows its i-th kernel.
+inline void timing_mark(cudaStream_t s, int i) { timing_mark_abs(s, i == 0 ? 0 : timing_hook().base + i); }
 
 // ---- launchers (return cudaSuccess or the launch error) --------------------
 

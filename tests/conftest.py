@@ -19,3 +19,19 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Parity figures of the GPU tests: the error the bound is judged on (bf16
+    outputs: each |diff| less the half-ulp of the stored value) and the plain
+    max |diff| / rms beside it."""
+    try:
+        from kda_testlib import PARITY_LOG
+    except Exception:  # noqa: BLE001 - nothing to report
+        return
+    if not PARITY_LOG:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "parity: max|d|/rms judged (plain) <= bound")
+    for label, e, raw, tol in PARITY_LOG:
+        tr.write_line(f"{label:60s} {e:.3e} ({raw:.3e}) <= {tol:g}")

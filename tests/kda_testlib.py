@@ -45,6 +45,21 @@ def rel_err(got, ref, stored_as=None, both_stored=False) -> float:
     return float(np.max(d) / rms)
 
 
+# (label, error with the storage allowance, error without it, bound) of every
+# check made through parity(); the session summary prints them
+PARITY_LOG = []
+
+
+def parity(label, got, ref, tol, stored_as=None, both_stored=False) -> float:
+    """rel_err with the bf16 storage allowance (the figure the bound is judged
+    on), logged next to the plain max |got - ref| / rms(ref), which shows how
+    much of the bound the output's own bf16 rounding uses."""
+    e = rel_err(got, ref, stored_as=stored_as, both_stored=both_stored)
+    raw = rel_err(got, ref) if stored_as else e
+    PARITY_LOG.append((label, e, raw, tol))
+    return e
+
+
 def oracle_prefill(inp, heads=None, seqs=None, n_threads=0, prep=0):
     """Oracle o / final_state for the given heads and sequences of a PrefillInputs.
 

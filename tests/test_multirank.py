@@ -92,4 +92,4 @@ def test_reference_arm_prints_its_json_line(capsys):
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
-    assert line["config"]["workload"].startswith("prefill B=4 H=16 T=4096")
+    assert line["config"]["workload"].startswith("packed varlen prefill: 64 sequences")
