@@ -91,6 +91,7 @@ constexpr uint32_t kPh = 17408;          // P 64 x 64 (K-major)
 constexpr uint32_t kPl = 25600;
 constexpr uint32_t kScr = 33792;         // 8 KB scratch
 constexpr uint32_t kTs = 41984;          // T fp32 [64][68]
+constexpr uint32_t kFbStage = 41984;     // before T: rows of a large-range diagonal block (3 x 8 KB)
 // T (64 rows x 64 k, K-major), the A operand of the last product
 constexpr uint32_t kTPh = 65536;
 constexpr uint32_t kTPl = 81920;
@@ -552,48 +553,111 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     __syncthreads();
 
     // ---- diagonal blocks with a large decay range: pairwise on CUDA cores ----------
+    // Block R's 16 rows are staged in shared memory (k and q in fp32, normalised
+    // when asked, and the block-local cumulative log decay times log2 e, so every
+    // factor is 2^(a - b) of two sums over at most 16 tokens).  Warp w forms the
+    // 17 pairs (r, i <= r) of rows w and 15 - w, each lane over 4 channels; the 34
+    // per-lane sums (A and P of each pair) are reduced across the warp by halving
+    // exchanges, after which lane l holds sum number l.
     if (!abort && fbmask) {
+        float* fk = reinterpret_cast<float*>(sm + kFbStage);   // [16][128] k
+        float* fq = fk + 16 * 128;                              // [16][128] q
+        float* fg = fq + 16 * 128;                              // [16][128] block-local g * log2 e
         for (int R = 0; R < 4; ++R) {
             if (!(fbmask & (1u << R))) continue;
-            float* sh = scr;   // [16][128] block-local cumulative log decay
-            for (int e = tid; e < 16 * 128; e += kIntraThreads) {
-                const int rr = e >> 7, c = e & 127, row = 16 * R + rr;
-                sh[e] = (row < len) ? prep_log_alpha(__bfloat162float(la[((size_t)(tok0 + row) * H + h) * kD + c]),
-                                                     prep)
-                                    : 0.f;
+            {
+                // thread: one row, 8 consecutive channels of k, q and log alpha
+                const int row = tid >> 4, c8 = (tid & 15) * 8, rr = 16 * R + row;
+                uint4 k8 = make_uint4(0u, 0u, 0u, 0u), q8 = k8, l8 = k8;
+                if (rr < len) {
+                    const size_t off = ((size_t)(tok0 + rr) * H + h) * kD + c8;
+                    k8 = *reinterpret_cast<const uint4*>(k + off);
+                    q8 = *reinterpret_cast<const uint4*>(q + off);
+                    l8 = *reinterpret_cast<const uint4*>(la + off);
+                }
+                const float2 sk = PREP ? make_float2(inv_nk[rr], inv_nk[rr]) : make_float2(1.f, 1.f);
+                const float2 sq = PREP ? make_float2(inv_nq[rr], inv_nq[rr]) : make_float2(1.f, 1.f);
+                const uint32_t kw[4] = {k8.x, k8.y, k8.z, k8.w}, qw[4] = {q8.x, q8.y, q8.z, q8.w};
+                const uint32_t lw[4] = {l8.x, l8.y, l8.z, l8.w};
+                float* dk_ = fk + row * 128 + c8;
+                float* dq_ = fq + row * 128 + c8;
+                float* dg_ = fg + row * 128 + c8;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    *reinterpret_cast<float2*>(dk_ + 2 * m) = mul2(unpack_bf16x2(kw[m]), sk);
+                    *reinterpret_cast<float2*>(dq_ + 2 * m) = mul2(unpack_bf16x2(qw[m]), sq);
+                    const float2 l2 = prep_log_alpha2(unpack_bf16x2(lw[m]), prep);
+                    *reinterpret_cast<float2*>(dg_ + 2 * m) = (rr < len) ? l2 : make_float2(0.f, 0.f);
+                }
             }
             __syncthreads();
-            if (tid < 128)
-                for (int rr = 1; rr < 16; ++rr) sh[rr * 128 + tid] += sh[(rr - 1) * 128 + tid];
+            if (tid < 128) {
+                float acc = 0.f;
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    acc += fg[rr * 128 + tid];
+                    fg[rr * 128 + tid] = acc * kLog2e;
+                }
+            }
             __syncthreads();
-            for (int p = warp; p < 136; p += kIntraThreads / 32) {
-                int rr = 0;
-                while ((rr + 1) * (rr + 2) / 2 <= p) ++rr;
-                const int ii = p - rr * (rr + 1) / 2;
-                const int row = 16 * R + rr, col = 16 * R + ii;
-                float sa = 0.f, spq = 0.f;
-                if (row < len) {
-                    const size_t ro = ((size_t)(tok0 + row) * H + h) * kD, io = ((size_t)(tok0 + col) * H + h) * kD;
-                    for (int c = lane; c < 128; c += 32) {
-                        const float sk_c = PREP ? inv_nk[col] : 1.f, sk_r = PREP ? inv_nk[row] : 1.f;
-                        const float sq_r = PREP ? inv_nq[row] : 1.f;
-                        const float kdv = __bfloat162float(k[io + c]) * sk_c *
-                                          __expf(sh[rr * 128 + c] - sh[ii * 128 + c]);
-                        sa += __bfloat162float(k[ro + c]) * sk_r * kdv;
-                        spq += __bfloat162float(q[ro + c]) * sq_r * kdv;
+            {
+                const int ra = warp, rb = 15 - warp;
+                float v[34];
+#pragma unroll
+                for (int jj = 0; jj < 17; ++jj) {
+                    const bool first = jj <= ra;
+                    const int r = first ? ra : rb, i = first ? jj : jj - ra - 1;
+                    const float4 gr = *reinterpret_cast<const float4*>(fg + r * 128 + 4 * lane);
+                    const float4 gi = *reinterpret_cast<const float4*>(fg + i * 128 + 4 * lane);
+                    const float4 kr = *reinterpret_cast<const float4*>(fk + r * 128 + 4 * lane);
+                    const float4 qr = *reinterpret_cast<const float4*>(fq + r * 128 + 4 * lane);
+                    const float4 ki = *reinterpret_cast<const float4*>(fk + i * 128 + 4 * lane);
+                    // 2^(g_r - g_i) <= 1 (i <= r)
+                    const float2 d0 = fma2(make_float2(gi.x, gi.y), make_float2(-1.f, -1.f), make_float2(gr.x, gr.y));
+                    const float2 d1 = fma2(make_float2(gi.z, gi.w), make_float2(-1.f, -1.f), make_float2(gr.z, gr.w));
+                    const float2 e0 = make_float2(ex2_approx(d0.x), ex2_approx(d0.y));
+                    const float2 e1 = make_float2(ex2_approx(d1.x), ex2_approx(d1.y));
+                    const float2 ke0 = mul2(make_float2(ki.x, ki.y), e0), ke1 = mul2(make_float2(ki.z, ki.w), e1);
+                    float2 a2 = mul2(make_float2(kr.x, kr.y), ke0), p2 = mul2(make_float2(qr.x, qr.y), ke0);
+                    a2 = fma2(make_float2(kr.z, kr.w), ke1, a2);
+                    p2 = fma2(make_float2(qr.z, qr.w), ke1, p2);
+                    v[2 * jj] = a2.x + a2.y;
+                    v[2 * jj + 1] = p2.x + p2.y;
+                }
+                // values 0-31: halving exchanges (distance 16 .. 1); lane l ends with sum l
+#pragma unroll
+                for (int w = 16; w >= 1; w >>= 1) {
+                    const bool up = (lane & w) != 0;
+#pragma unroll
+                    for (int m = 0; m < w; ++m) {
+                        const float keep = up ? v[m + w] : v[m];
+                        const float give = up ? v[m] : v[m + w];
+                        v[m] = keep + __shfl_xor_sync(0xffffffffu, give, w);
                     }
                 }
+                // values 32, 33 (the last pair: row rb with itself)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
-                    sa += __shfl_xor_sync(0xffffffffu, sa, o);
-                    spq += __shfl_xor_sync(0xffffffffu, spq, o);
+                    v[32] += __shfl_xor_sync(0xffffffffu, v[32], o);
+                    v[33] += __shfl_xor_sync(0xffffffffu, v[33], o);
                 }
+                auto put = [&](int jj, bool is_p, float val) {
+                    const bool first = jj <= ra;
+                    const int r = first ? ra : rb, i = first ? jj : jj - ra - 1;
+                    const int row = 16 * R + r, col = 16 * R + i;
+                    if (!is_p) {
+                        As[row * kAS + col] = (i < r && row < len) ? sbeta[row] * val : 0.f;
+                    } else {
+                        __nv_bfloat16 ph, pl;
+                        split1(row < len ? val : 0.f, ph, pl);
+                        *reinterpret_cast<__nv_bfloat16*>(sm + kPh + sw128_offset(row, col, 64)) = ph;
+                        *reinterpret_cast<__nv_bfloat16*>(sm + kPl + sw128_offset(row, col, 64)) = pl;
+                    }
+                };
+                put(lane >> 1, lane & 1, v[0]);
                 if (lane == 0) {
-                    As[row * kAS + col] = (ii < rr) ? sbeta[row] * sa : 0.f;
-                    __nv_bfloat16 ph, pl;
-                    split1(spq, ph, pl);
-                    *reinterpret_cast<__nv_bfloat16*>(sm + kPh + sw128_offset(row, col, 64)) = ph;
-                    *reinterpret_cast<__nv_bfloat16*>(sm + kPl + sw128_offset(row, col, 64)) = pl;
+                    put(16, false, v[32]);
+                    put(16, true, v[33]);
                 }
             }
             __syncthreads();
@@ -869,9 +933,14 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sp = warp & 3;            // TMEM sub-partition: lanes 32 sp .. 32 sp + 31
     const int cq = (warp >> 2) * HB;    // first state column of this thread (relative to j0)
-    const SeqInfo sq = smap.get(blockIdx.x);
-    const int h = blockIdx.y;
-    const int j0 = blockIdx.z * BV;
+    // grid order: column tile fastest, then head, then sequence (longest first), so
+    // that the tiles of one (sequence, head) run side by side and read its
+    // workspace images from L2 after the first of them has brought them in
+    constexpr int kTiles = kD / BV;
+    const int z = (int)(blockIdx.x % kTiles);
+    const int h = (int)((blockIdx.x / kTiles) % (unsigned)H);
+    const SeqInfo sq = smap.get((int)(blockIdx.x / (kTiles * (unsigned)H)));
+    const int j0 = z * BV;
     const int nch = (sq.len + kC - 1) / kC;
     const int cb0 = j0 / 32;   // first 32-column block of U
 
@@ -1139,7 +1208,7 @@ cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* fina
     cudaError_t e =
         cudaFuncSetAttribute(tc_recur<BV, STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    tc_recur<BV, STORE><<<dim3(n_seqs, H, kD / BV), kRecurThreads, Lay::kAlloc, stream>>>(
+    tc_recur<BV, STORE><<<dim3((unsigned)(n_seqs * H * (kD / BV))), kRecurThreads, Lay::kAlloc, stream>>>(
         ws, init_state, final_state, o, err, smap, H, s_store, w_store);
     return cudaGetLastError();
 }
