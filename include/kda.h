@@ -326,6 +326,51 @@ KDA_API kda_status kda_chunk_bwd(const void* q, const void* k, const void* v,
 
 
 /*
+ * One sequence split over several devices: the affine map of a segment.
+ *
+ * The state carried from chunk to chunk ("From GPT-2 to Kimi K3" essay,
+ * pwwt.cn/news/3716252, chunkwise paragraph) depends affinely on the state a
+ * segment of tokens starts from: for every sequence and head the segment maps
+ * its start state S to
+ *     S_end = M S + F,
+ * M (d_k x d_k) being the segment's final state from the identity with the
+ * values' contribution left out, and F (d_k x d_v) its final state from a zero
+ * start.  A device holding a later segment computes (M, F) of its own segment
+ * in one pass, the maps are exchanged (one all-gather), each device chains the
+ * maps of the segments before it (kda_compose_states) and runs kda_chunk_fwd
+ * from the start state that gives.  (The split is this library's construction,
+ * not a step the pages describe.)
+ *
+ *   q, k, v, log_alpha, beta, dtype, cu_seqlens_host, n_seqs, B, T, H, dk,
+ *   dv, C            : as kda_chunk_fwd (no initial state: it does not enter
+ *                      the map)
+ *   M                : device [N, H, dk, dk] fp32 (written)
+ *   F                : device [N, H, dk, dv] fp32 (written)
+ *   workspace        : >= kda_chunk_fwd_workspace_size(...) bytes, as for
+ *                      kda_chunk_fwd
+ * Errors as kda_chunk_fwd.  Asynchronous on `stream`.  M equals the identity
+ * and F zero for an empty sequence.
+ */
+KDA_API kda_status kda_chunk_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
+                                         const void* beta, kda_dtype dtype, const int32_t* cu_seqlens_host,
+                                         int n_seqs, int B, int T, int H, int dk, int dv, int C, float* M, float* F,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Start states of R consecutive segments chained through their maps:
+ *     states[0] = init_state (or zero),  states[r + 1] = M_r states[r] + F_r
+ * for r = 0 .. R - 1, fp32 on the device.
+ *   M          : device [R, N, H, dk, dk] fp32 (kda_chunk_segment_map's M of each segment)
+ *   F          : device [R, N, H, dk, dv] fp32
+ *   init_state : device [N, H, dk, dv] fp32, or NULL for zero
+ *   states     : device [R + 1, N, H, dk, dv] fp32 (written; may not alias M, F or init_state)
+ * R = 0 copies init_state (or zero) to states[0].  Errors: KDA_ERR_SHAPE (sizes),
+ * KDA_ERR_NULL, KDA_ERR_ALIGN (16 bytes), KDA_ERR_CUDA.  Asynchronous on `stream`.
+ */
+KDA_API kda_status kda_compose_states(const float* M, const float* F, const float* init_state, int R, int N, int H,
+                                      int dk, int dv, float* states, void* stream);
+
+/*
  * Device-side status of a finished call.  The tensor-core kernels bound every
  * wait on the device (2 s); if one expires they stop, leave their outputs
  * undefined and record KDA_ERR_TIMEOUT in an error word inside the workspace

@@ -90,6 +90,10 @@ def _declare(lib):
     lib.kda_chunk_bwd_device_status.restype = c_int
     lib.kda_chunk_fwd_noalloc_device_status.argtypes = [c_int, i32p, c_int] + [c_int] * 6 + [vp]
     lib.kda_chunk_fwd_noalloc_device_status.restype = c_int
+    lib.kda_chunk_segment_map.argtypes = [vp] * 5 + [c_int, i32p, c_int] + [c_int] * 6 + [vp, vp, vp, c_size, vp]
+    lib.kda_chunk_segment_map.restype = c_int
+    lib.kda_compose_states.argtypes = [vp, vp, vp] + [c_int] * 5 + [vp, vp]
+    lib.kda_compose_states.restype = c_int
     return lib
 
 
@@ -123,7 +127,7 @@ def exported_symbols():
             "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
             "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep", "kda_chunk_bwd_workspace_size",
             "kda_chunk_bwd", "kda_chunk_fwd_device_status", "kda_chunk_bwd_device_status",
-            "kda_chunk_fwd_noalloc_device_status"]
+            "kda_chunk_fwd_noalloc_device_status", "kda_chunk_segment_map", "kda_compose_states"]
 
 
 def _ptr(t):
@@ -366,6 +370,67 @@ def device_status(kind, workspace, dtype, B, T, H, dk, dv, C=64, cu_seqlens=None
     if st not in (0, KDA_ERR_TIMEOUT):
         raise KdaError(st, f"device status ({kind})")
     return int(st)
+
+
+def segment_map(q, k, v, log_alpha, beta, cu_seqlens=None, C: int = 64, M=None, F=None, workspace=None,
+                stream=None):
+    """Affine map of a segment (``kda_chunk_segment_map``): for every sequence
+    and head, the segment takes a start state S to ``M S + F``.  Inputs as
+    :func:`chunk_fwd`.  Returns ``(M [N, H, dk, dk], F [N, H, dk, dv])`` fp32."""
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        _check_cuda(name, t, dt)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu, n_seqs, _keep = _cu_arg(cu_seqlens)
+    N = n_seqs if cu_seqlens is not None else B
+    dev = q.device
+    with _launch_on(dev, stream, (("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta), ("M", M),
+                                  ("F", F), ("workspace", workspace))) as (s, allocated):
+        if M is None:
+            M = torch.empty((N, H, dk, dk), dtype=torch.float32, device=dev)
+            allocated.append(M)
+        if F is None:
+            F = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+            allocated.append(F)
+        _check_cuda("M", M, torch.float32)
+        _check_cuda("F", F, torch.float32)
+        need = lib().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, C, _DTYPES[dt], cu, n_seqs)
+        if workspace is None:
+            workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=dev)
+            allocated.append(workspace)
+        _check_cuda("workspace", workspace)
+        st = lib().kda_chunk_segment_map(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _DTYPES[dt], cu,
+                                         n_seqs, B, T, H, dk, dv, C, _ptr(M), _ptr(F), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream_handle(s))
+    if st != 0:
+        raise KdaError(st, "kda_chunk_segment_map")
+    return M, F
+
+
+def compose_states(M, F, init_state=None, out=None, stream=None):
+    """Start states of consecutive segments (``kda_compose_states``): ``M``
+    ``[R, N, H, dk, dk]`` and ``F`` ``[R, N, H, dk, dv]`` (the segments' maps, in
+    order), ``init_state`` ``[N, H, dk, dv]`` or None.  Returns ``[R + 1, N, H,
+    dk, dv]``: entry r is the state segment r starts from, the last one the
+    state after all R segments."""
+    R, N, H, dk, _ = M.shape
+    dv = F.shape[-1]
+    for name, t in (("M", M), ("F", F), ("init_state", init_state)):
+        _check_cuda(name, t, torch.float32)
+    dev = M.device
+    with _launch_on(dev, stream, (("F", F), ("init_state", init_state), ("out", out))) as (s, allocated):
+        if out is None:
+            out = torch.empty((R + 1, N, H, dk, dv), dtype=torch.float32, device=dev)
+            allocated.append(out)
+        _check_cuda("out", out, torch.float32)
+        st = lib().kda_compose_states(_ptr(M), _ptr(F), _ptr(init_state), R, N, H, dk, dv, _ptr(out),
+                                      _stream_handle(s))
+    if st != 0:
+        raise KdaError(st, "kda_compose_states")
+    return out
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20   # KDA_NOALLOC_SCRATCH_BYTES in include/kda.h

@@ -335,6 +335,62 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
     return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+kda_status segment_map_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                            kda_dtype dtype, const int32_t* cu_seqlens_host, int n_seqs, int B, int T, int H, int dk,
+                            int dv, int C, float* M, float* F, void* workspace, size_t workspace_bytes, void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    Plan p;
+    kda_status st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    const kda_algo algo = resolve(KDA_ALGO_AUTO, dtype, dk, dv, C);
+    if (algo == KDA_ALGO_TC && C != tc_chunk()) {
+        C = tc_chunk();
+        if ((st = make_plan(B, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p)) != KDA_OK) return st;
+    }
+    if (!M || !F) return KDA_ERR_NULL;
+    if (p.total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta)) return KDA_ERR_NULL;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, M, F};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return KDA_ERR_ALIGN;
+    if (workspace_bytes < workspace_for(p, H, dk, dv, C, algo)) return KDA_ERR_WORKSPACE;
+    if ((st = check_device()) != KDA_OK) return st;
+    if (p.n_seqs == 0) return KDA_OK;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char* ws = (char*)workspace;
+    const int ncps = (int)((T + C - 1) / C);
+    ChunkMap cmap{nullptr, p.n_seqs, T, C, ncps};
+    SeqMap smap{nullptr, T, C, ncps};
+    timing_mark(s, 0);
+    if (p.varlen) {
+        cudaError_t terr;
+        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr, true);
+        if (terr != cudaSuccess) {
+            timing_hook().n = 0;
+            timing_hook().base = 0;
+            return KDA_ERR_CUDA;
+        }
+        cmap.seqs = (const SeqInfo*)ws;
+        smap.order = (const SeqInfo*)ws + p.n_seqs;
+    }
+    cudaError_t err;
+    if (algo == KDA_ALGO_SIMT) {
+        SimtLayout L = simt_layout(p, H, dk, dv);
+        SimtWorkspace w{(float*)(ws + L.off[0]), (float*)(ws + L.off[5]), (float*)(ws + L.off[1]),
+                        (float*)(ws + L.off[2]), (float*)(ws + L.off[3]), (float*)(ws + L.off[4])};
+        err = launch_simt_segment_map(dtype, k, v, log_alpha, beta, cmap, smap, p.n_chunks, p.n_seqs, H, dk, dv, C, w,
+                                      M, F, s);
+    } else {
+        err = launch_tc_segment_map(q, k, v, log_alpha, beta, cmap, smap, p.n_chunks, p.n_seqs, H,
+                                    ws + table_bytes(p), M, F, s);
+    }
+    timing_hook().n = 0;
+    timing_hook().base = 0;
+    return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status decode_impl(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                        kda_dtype dtype, unsigned prep, float* state, int N, int H, int dk, int dv, void* o,
                        void* stream) {
@@ -522,6 +578,30 @@ kda_status kda_chunk_bwd_device_status(const void* workspace, kda_dtype dtype, c
     if (!workspace) return KDA_ERR_NULL;
     if (p.n_seqs == 0 || !(tc_available() && tc_shape(dtype, dk, dv, kBwdChunk))) return KDA_OK;
     return read_error_word(workspace, bwd_layout(p, H, dk, dv, kBwdChunk, true).tc, stream);
+}
+
+kda_status kda_chunk_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
+                                 const void* beta, kda_dtype dtype, const int32_t* cu_seqlens_host, int n_seqs, int B,
+                                 int T, int H, int dk, int dv, int C, float* M, float* F, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return segment_map_impl(q, k, v, log_alpha, beta, dtype, cu_seqlens_host, n_seqs, B, T, H, dk, dv, C, M, F,
+                            workspace, workspace_bytes, stream);
+}
+
+kda_status kda_compose_states(const float* M, const float* F, const float* init_state, int R, int N, int H, int dk,
+                              int dv, float* states, void* stream) {
+    if (R < 0 || N < 0 || H <= 0 || !((dk == 64 || dk == 128) && (dv == 64 || dv == 128))) return KDA_ERR_SHAPE;
+    if ((long long)N * H > 0x7fffffffLL) return KDA_ERR_SHAPE;
+    if (!states || (R > 0 && (!M || !F))) return KDA_ERR_NULL;
+    const void* ptrs[] = {M, F, init_state, states};
+    for (const void* ptr : ptrs)
+        if (ptr && !aligned16(ptr)) return KDA_ERR_ALIGN;
+    kda_status st = check_device();
+    if (st != KDA_OK) return st;
+    if (N == 0) return KDA_OK;
+    return launch_compose_states(M, F, init_state, R, N, H, dk, dv, states, (cudaStream_t)stream) == cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_CUDA;
 }
 
 kda_status kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,

@@ -127,27 +127,36 @@ __global__ void __launch_bounds__(kThreadsW) k2_wy(const Tin* __restrict__ k, co
 // K3: one block per (sequence, head, d_v tile of kBV columns), sequential over
 // the sequence's chunks.  Shared: S [dk][kBV], M [C][dk] (Wk, then K . decay),
 // Ws [C][kBV], gC, gCl [dk].
-template <typename Tin, int CC>
+// MAP (a segment's affine map S_end = Mmap S_start + F): blockIdx.z < dv / kBV
+// carries the state from zero (F, into final_state [N, H, dk, dv]); the next
+// dk / kBV tiles carry the columns of the identity without the values' term U
+// (Mmap, into map_out [N, H, dk, dk]); nothing else is stored.
+template <typename Tin, int CC, bool MAP = false>
 __global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__ k, const float* __restrict__ g,
                                                      const float* __restrict__ gl,
                                                      const float* __restrict__ U, const float* __restrict__ Wkg,
                                                      float* __restrict__ Wg, float* __restrict__ S_chunk,
                                                      const float* __restrict__ init_state,
                                                      float* __restrict__ final_state, SeqMap smap, int H, int dk,
-                                                     int dv, int C) {
+                                                     int dv, int C, float* __restrict__ map_out) {
     extern __shared__ float smem[];
     const SeqInfo sq = smap.get(blockIdx.x);
-    const int h = blockIdx.y, j0 = blockIdx.z * kBV, tid = threadIdx.x;
+    const bool mcols = MAP && (int)blockIdx.z >= dv / kBV;
+    const int h = blockIdx.y, j0 = (mcols ? (int)blockIdx.z - dv / kBV : (int)blockIdx.z) * kBV, tid = threadIdx.x;
+    const int ld = mcols ? dk : dv;     // row length of this tile's state (F and S: dv; Mmap: dk)
     float* S = smem;
     float* M = S + dk * kBV;
     float* Ws = M + C * dk;
     float* gC = Ws + C * kBV;
     float* gCl = gC + dk;
 
-    const size_t st_base = ((size_t)sq.seq * H + h) * dk * dv;
+    const size_t st_base = ((size_t)sq.seq * H + h) * dk * ld;
     for (int e = tid; e < dk * kBV; e += kThreadsW) {
         int c = e / kBV, j = e - c * kBV;
-        S[e] = init_state ? init_state[st_base + (size_t)c * dv + j0 + j] : 0.f;
+        if (MAP)
+            S[e] = (mcols && c == j0 + j) ? 1.f : 0.f;
+        else
+            S[e] = init_state ? init_state[st_base + (size_t)c * dv + j0 + j] : 0.f;
     }
     __syncthreads();
     const int nch = (sq.len + C - 1) / C;
@@ -155,9 +164,11 @@ __global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__
         const int t0 = sq.tok0 + n * C;
         const int L = min(C, sq.len - n * C);
         const size_t sc_base = ((size_t)(sq.chunk0 + n) * H + h) * dk * dv;
-        for (int e = tid; e < dk * kBV; e += kThreadsW) {
-            int c = e / kBV, j = e - c * kBV;
-            S_chunk[sc_base + (size_t)c * dv + j0 + j] = S[e];
+        if (!MAP) {
+            for (int e = tid; e < dk * kBV; e += kThreadsW) {
+                int c = e / kBV, j = e - c * kBV;
+                S_chunk[sc_base + (size_t)c * dv + j0 + j] = S[e];
+            }
         }
         for (int e = tid; e < L * dk; e += kThreadsW) {
             int r = e / dk, c = e - r * dk;
@@ -171,7 +182,7 @@ __global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__
 #pragma unroll
             for (int m = 0; m < CC / 16; ++m) {
                 const int r = r0 + 16 * m;
-                acc[m] = r < L ? U[((size_t)(t0 + r) * H + h) * dv + j0 + j] : 0.f;
+                acc[m] = (r < L && !mcols) ? U[((size_t)(t0 + r) * H + h) * dv + j0 + j] : 0.f;
             }
             for (int c = 0; c < dk; ++c) {
                 const float sv = S[c * kBV + j];
@@ -183,7 +194,7 @@ __global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__
                 const int r = r0 + 16 * m;
                 if (r < L) {
                     Ws[r * kBV + j] = acc[m];
-                    Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = acc[m];
+                    if (!MAP) Wg[((size_t)(t0 + r) * H + h) * dv + j0 + j] = acc[m];
                 }
             }
         }
@@ -223,10 +234,11 @@ __global__ void __launch_bounds__(kThreadsW, 2) k3_state(const Tin* __restrict__
         }
         __syncthreads();
     }
-    if (final_state) {
+    float* fdst = mcols ? map_out : final_state;
+    if (fdst) {
         for (int e = tid; e < dk * kBV; e += kThreadsW) {
             int c = e / kBV, j = e - c * kBV;
-            final_state[st_base + (size_t)c * dv + j0 + j] = S[e];
+            fdst[st_base + (size_t)c * ld + j0 + j] = S[e];
         }
     }
 }
@@ -313,7 +325,8 @@ cudaError_t run(const Tin* q, const Tin* k, const Tin* v, const Tin* la, const T
     timing_mark(stream, 2);
     if (n_seqs > 0)
         k3<<<dim3(n_seqs, H, dv / kBV), kThreadsW, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
-                                                                 init_state, final_state, smap, H, dk, dv, C);
+                                                                 init_state, final_state, smap, H, dk, dv, C,
+                                                                 nullptr);
     timing_mark(stream, 3);
     if (n_chunks > 0)
         k4_output<Tin><<<dim3(n_chunks, H), kThreadsW, smem4, stream>>>(q, k, ws.g, ws.gl, ws.W, ws.S_chunk, o, cmap,
@@ -339,11 +352,47 @@ cudaError_t run_states(const Tin* k, const Tin* v, const Tin* la, const Tin* bet
     }
     if (n_seqs > 0)
         k3<<<dim3(n_seqs, H, dv / kBV), kThreadsW, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W, ws.S_chunk,
-                                                                 init_state, nullptr, smap, H, dk, dv, C);
+                                                                 init_state, nullptr, smap, H, dk, dv, C, nullptr);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t run_map(const Tin* k, const Tin* v, const Tin* la, const Tin* beta, const ChunkMap& cmap,
+                    const SeqMap& smap, int n_chunks, int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws,
+                    float* Mmap, float* F, cudaStream_t stream) {
+    const size_t smem2 = k2_smem(C, dk, dv);
+    const size_t smem3 = sizeof(float) * ((size_t)dk * kBV + (size_t)C * dk + (size_t)C * kBV + 2 * dk);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k2_wy<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2))) return e;
+    auto k3 = C == 128 ? k3_state<Tin, 128, true> : k3_state<Tin, 64, true>;
+    if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3))) return e;
+    if (n_chunks > 0) k1_cumsum<Tin><<<dim3(n_chunks, H), dk, 0, stream>>>(la, ws.g, ws.gl, cmap, H, dk);
+    timing_mark(stream, 1);
+    if (n_chunks > 0)
+        k2_wy<Tin><<<dim3(n_chunks, H), kThreadsW, smem2, stream>>>(k, v, beta, ws.g, ws.gl, ws.U, ws.Wk, cmap, H, dk,
+                                                                  dv, C);
+    timing_mark(stream, 2);
+    if (n_seqs > 0)
+        k3<<<dim3(n_seqs, H, (dv + dk) / kBV), kThreadsW, smem3, stream>>>(k, ws.g, ws.gl, ws.U, ws.Wk, ws.W,
+                                                                        ws.S_chunk, nullptr, F, smap, H, dk, dv, C,
+                                                                        Mmap);
+    timing_mark(stream, 3);
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_simt_segment_map(kda_dtype dtype, const void* k, const void* v, const void* log_alpha,
+                                    const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,
+                                    int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws, float* Mmap,
+                                    float* F, cudaStream_t stream) {
+    if (dtype == KDA_F32)
+        return run_map<float>((const float*)k, (const float*)v, (const float*)log_alpha, (const float*)beta, cmap,
+                              smap, n_chunks, n_seqs, H, dk, dv, C, ws, Mmap, F, stream);
+    return run_map<__nv_bfloat16>((const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)log_alpha,
+                                  (const __nv_bfloat16*)beta, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws, Mmap, F,
+                                  stream);
+}
 
 cudaError_t launch_simt_g(kda_dtype dtype, const void* log_alpha, const ChunkMap& cmap, int n_chunks, int H, int dk,
                           const SimtWorkspace& ws, cudaStream_t stream) {

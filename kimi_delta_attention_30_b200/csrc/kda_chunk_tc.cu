@@ -100,8 +100,11 @@ constexpr uint32_t kXh = 0;
 constexpr uint32_t kXl = 32768;
 constexpr uint32_t kTab = 98304;         // tables
 constexpr int kNumTab = 18;              // tau[4], sigma[6], exp(gb)[4], exp(g_C - gb[b+1])[4]
-constexpr uint32_t kIntraSmem = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 3 * 64 * 4 + 64;
-constexpr uint32_t kIntraAlloc = kIntraSmem + 1024;
+constexpr uint32_t kIntraBars = kTab + kNumTab * 128 * 4 + 5 * 128 * 4 + 3 * 64 * 4 + 64;   // 3 mbarriers
+constexpr uint32_t kIntraSmem = kIntraBars + 32;
+// no static shared memory: the dynamic region starts at the CTA's (1024-aligned)
+// shared window, so the kernel addresses it without a runtime offset
+constexpr uint32_t kIntraAlloc = kIntraSmem;
 constexpr int kGCol = 192;               // TMEM columns 192-255 hold g until the last product
 constexpr int kAS = 65;                  // row stride of As (floats)
 constexpr int kTS = 68;                  // row stride of Ts (floats; rows 16-byte aligned)
@@ -208,17 +211,24 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
          int H, unsigned prep_flags) {
     // PREP = false is the plain operator: no preprocessing code is compiled in
     const unsigned prep = PREP ? prep_flags : 0u;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // The swizzled operand tiles need a 1024-byte aligned base.  This kernel has no
+    // static shared memory, so its dynamic region starts at the CTA's shared window;
+    // should that ever not be 1024-aligned, the kernel records an error and stops.
+    if (smem_u32(smem_raw) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(err, 0, (int)KDA_ERR_DEVICE);
+        return;
+    }
+    uint8_t* sm = smem_raw;
     float* tab = reinterpret_cast<float*>(sm + kTab);                 // [18][128]
     float* gb = tab + kNumTab * 128;                                  // [5][128]
     float* sbeta = gb + 5 * 128;                                      // [64]
     float* inv_nk = sbeta + 64;                                       // [64] 1 / ||k_r|| (1 without normalisation)
     float* inv_nq = inv_nk + 64;                                      // [64] 1 / ||q_r||
     uint32_t* sflags = reinterpret_cast<uint32_t*>(inv_nq + 64);      // [0] fallback mask, [1] abort, [2] tmem base
-    __shared__ uint64_t mbar;    // tensor-core products, in issue order
-    __shared__ uint64_t mbar_k;  // the second half of the last product
-    __shared__ uint64_t mbar_la; // log alpha rows landed
+    uint64_t& mbar = reinterpret_cast<uint64_t*>(sm + kIntraBars)[0];      // tensor-core products, in issue order
+    uint64_t& mbar_k = reinterpret_cast<uint64_t*>(sm + kIntraBars)[1];    // the second half of the last product
+    uint64_t& mbar_la = reinterpret_cast<uint64_t*>(sm + kIntraBars)[2];   // log alpha rows landed
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this thread: rows [8 w, 8 w + 8) of 16-row block I = w / 2, and channels
@@ -630,8 +640,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                     const bool up = (lane & w) != 0;
 #pragma unroll
                     for (int m = 0; m < w; ++m) {
-                        const float keep = up ? v[m + w] : v[m];
-                        const float give = up ? v[m] : v[m + w];
+                        const float keep = selp(up, v[m + w], v[m]);
+                        const float give = selp(up, v[m], v[m + w]);
                         v[m] = keep + __shfl_xor_sync(0xffffffffu, give, w);
                     }
                 }
@@ -904,18 +914,26 @@ struct RecurLayout {
     static constexpr uint32_t kTmemCols = (3 * BV <= 32) ? 32 : (3 * BV <= 64) ? 64 : (3 * BV <= 128) ? 128 : 256;
 };
 
-// STORE (for the backward pass): every chunk's start state S_n goes to s_store
-// [chunks, H, 128, 128] and W_n to w_store [tokens, H, 128], both fp32.
-template <int BV, bool STORE>
+// MODE 0: the prefill.  MODE 1 (for the backward pass): also every chunk's start
+// state S_n to s_store [chunks, H, 128, 128] and W_n to w_store [tokens, H, 128],
+// both fp32.  MODE 2 (a segment's affine map S_end = M S_start + F, for splitting
+// one sequence over several devices): no outputs; the first 128 / BV column tiles
+// carry the state from zero (F, written to final_state), the next 128 / BV carry
+// the columns of the identity with the values' term U left out (M, written to
+// s_store as [N, H, 128, 128]).
+template <int BV, int MODE>
 __global__ void __launch_bounds__(kRecurThreads, 1)
 tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, float* __restrict__ final_state,
          __nv_bfloat16* __restrict__ o, int* __restrict__ err, SeqMap smap, int H, float* __restrict__ s_store,
          float* __restrict__ w_store) {
+    constexpr bool STORE = MODE == 1, MAP = MODE == 2;
     using Lay = RecurLayout<BV>;
     constexpr int HB = BV / 2;          // state columns per thread
     constexpr int NG = HB / 16;         // 16-column TMEM groups per thread
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, formed as an offset from the shared array so that every
+    // access through it stays a shared-memory access (32-bit addressing)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::kBars);
     uint64_t* wkq_full = bars + 0;
     uint64_t* kdt_full = bars + 1;
@@ -936,11 +954,12 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     // grid order: column tile fastest, then head, then sequence (longest first), so
     // that the tiles of one (sequence, head) run side by side and read its
     // workspace images from L2 after the first of them has brought them in
-    constexpr int kTiles = kD / BV;
+    constexpr int kTiles = (MAP ? 2 : 1) * (kD / BV);
     const int z = (int)(blockIdx.x % kTiles);
     const int h = (int)((blockIdx.x / kTiles) % (unsigned)H);
     const SeqInfo sq = smap.get((int)(blockIdx.x / (kTiles * (unsigned)H)));
-    const int j0 = z * BV;
+    const bool mcols = MAP && z >= kD / BV;      // a tile of M: identity start, no U term
+    const int j0 = (mcols ? z - kD / BV : z) * BV;
     const int nch = (sq.len + kC - 1) / kC;
     const int cb0 = j0 / 32;   // first 32-column block of U
 
@@ -1001,7 +1020,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         load_wkq(0);
         load_kdt(0);
         load_uu(0, 0);
-        load_p(0);
+        if (!MAP) load_p(0);
         if (nch > 1) load_uu(1, 1);
     }
 
@@ -1012,9 +1031,13 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
         for (int j = 0; j < HB; j += 4) {
-            float4 x = init_state ? *reinterpret_cast<const float4*>(init_state + base + j)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 x = (!MAP && init_state) ? *reinterpret_cast<const float4*>(init_state + base + j)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
             s[j] = x.x; s[j + 1] = x.y; s[j + 2] = x.z; s[j + 3] = x.w;
+        }
+        if (mcols) {
+#pragma unroll
+            for (int j = 0; j < HB; ++j) s[j] = (c == j0 + cq + j) ? 1.f : 0.f;
         }
     }
 
@@ -1112,7 +1135,8 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 const int jb = cq + 16 * g;
 #pragma unroll
                 for (int e = 0; e < 16; e += 4) {
-                    const float4 u = *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
+                    const float4 u = mcols ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                           : *reinterpret_cast<const float4*>(ut + u_index(r, jb + e));
                     d[g][e] = u.x - d[g][e]; d[g][e + 1] = u.y - d[g][e + 1];
                     d[g][e + 2] = u.z - d[g][e + 2]; d[g][e + 3] = u.w - d[g][e + 3];
                 }
@@ -1139,7 +1163,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 }
                 mma_commit(bar_s);
             }
-        } else if (n > 0) {
+        } else if (!MAP && n > 0) {
             // outputs of the previous chunk: its product goes in behind this chunk's
             // first one and runs while W is formed; then its P tile may be replaced
             if (tid == 64) {
@@ -1174,18 +1198,19 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     }
     __syncthreads();
     const bool failed = sflags[1] != 0;
-    if (!failed && nch > 0 && sp >= 2) {
+    if (!MAP && !failed && nch > 0 && sp >= 2) {
         // outputs of the last chunk
         if (tid == 64) issue_o(nch - 1);
         if (!mbar_wait(bar_o, (uint32_t)(nch - 1) & 1u)) fail();
         tc_fence_after();
         emit_o(nch - 1);
     }
-    if (!failed && final_state) {
+    float* fdst = mcols ? s_store : final_state;
+    if (!failed && fdst) {
         const size_t base = (((size_t)sq.seq * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
         for (int j = 0; j < HB; j += 4)
-            *reinterpret_cast<float4*>(final_state + base + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+            *reinterpret_cast<float4*>(fdst + base + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
     }
     __syncthreads();
     if (sflags[1] && tid == 0) {
@@ -1200,15 +1225,16 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     if (warp == 0) tmem_dealloc(tbase, Lay::kTmemCols);
 }
 
-template <int BV, bool STORE = false>
+template <int BV, int MODE = 0>
 cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* final_state, __nv_bfloat16* o, int* err,
                          const SeqMap& smap, int n_seqs, int H, cudaStream_t stream, float* s_store = nullptr,
                          float* w_store = nullptr) {
     using Lay = RecurLayout<BV>;
     cudaError_t e =
-        cudaFuncSetAttribute(tc_recur<BV, STORE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
+        cudaFuncSetAttribute(tc_recur<BV, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
     if (e != cudaSuccess) return e;
-    tc_recur<BV, STORE><<<dim3((unsigned)(n_seqs * H * (kD / BV))), kRecurThreads, Lay::kAlloc, stream>>>(
+    const unsigned tiles = (MODE == 2 ? 2u : 1u) * (unsigned)(kD / BV);
+    tc_recur<BV, MODE><<<dim3((unsigned)(n_seqs * H) * tiles), kRecurThreads, Lay::kAlloc, stream>>>(
         ws, init_state, final_state, o, err, smap, H, s_store, w_store);
     return cudaGetLastError();
 }
@@ -1313,13 +1339,43 @@ cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const 
     }
     if (n_seqs > 0) {
         if ((long)n_seqs * H * 4 <= sm_count())
-            e = launch_recur<32, true>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
-                                       S_chunk, W);
+            e = launch_recur<32, 1>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
+                                    S_chunk, W);
         else
-            e = launch_recur<64, true>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
-                                       S_chunk, W);
+            e = launch_recur<64, 1>(ws, init_state, nullptr, (__nv_bfloat16*)o_scratch, err, smap, n_seqs, H, stream,
+                                    S_chunk, W);
     }
     return e;
+}
+
+// A segment's affine map (S_end = M S_start + F per sequence and head): the
+// chunk-local kernel, then the state carry over 2 x 128 columns (F from a zero
+// start, M from the identity without the values' term), no outputs.
+cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
+                                  const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,
+                                  int n_seqs, int H, void* tc_ws, float* M, float* F, cudaStream_t stream) {
+    int* err = reinterpret_cast<int*>(tc_ws);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+    if (n_chunks > 0) {
+        e = cudaFuncSetAttribute(tc_intra<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kIntraAlloc);
+        if (e != cudaSuccess) return e;
+        tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
+            (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    timing_mark(stream, 1);
+    if (n_seqs > 0) {
+        if ((long)n_seqs * H * 8 <= sm_count())
+            e = launch_recur<32, 2>(ws, nullptr, F, nullptr, err, smap, n_seqs, H, stream, M, nullptr);
+        else
+            e = launch_recur<64, 2>(ws, nullptr, F, nullptr, err, smap, n_seqs, H, stream, M, nullptr);
+        if (e != cudaSuccess) return e;
+    }
+    timing_mark(stream, 2);
+    return cudaSuccess;
 }
 
 }  // namespace kda

@@ -219,6 +219,18 @@ cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, 
                                  const SeqMap& smap, int n_chunks, int n_seqs, int H, int dkk, int dvv, int C,
                                  const BwdWorkspace& ws, cudaStream_t stream);
 
+// A segment's affine map S_end = M S_start + F (M [N, H, dk, dk], F [N, H, dk, dv]).
+cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
+                                  const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,
+                                  int n_seqs, int H, void* tc_ws, float* M, float* F, cudaStream_t stream);
+cudaError_t launch_simt_segment_map(kda_dtype dtype, const void* k, const void* v, const void* log_alpha,
+                                    const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,
+                                    int n_seqs, int H, int dk, int dv, int C, const SimtWorkspace& ws, float* Mmap,
+                                    float* F, cudaStream_t stream);
+// states[0] = init (or 0), states[r + 1] = M_r states[r] + F_r, r < R.
+cudaError_t launch_compose_states(const float* M, const float* F, const float* init, int R, int N, int H, int dk,
+                                  int dv, float* out, cudaStream_t stream);
+
 cudaError_t launch_decode(kda_dtype dtype, const void* q, const void* k, const void* v,
                           const void* log_alpha, const void* beta, float* state, int N, int H,
                           int dk, int dv, void* o, unsigned prep, cudaStream_t stream);

@@ -194,12 +194,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Wait for the phase with the given parity to complete; gives up after
 // `limit_ns` nanoseconds and returns false (the caller records the error).
+// The clock is read once per 64 polls (each poll already suspends the thread
+// for a while inside try_wait).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (true) {
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if ((i & 63u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -244,6 +246,16 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
     // x - hi is exact in fp32; one packed fma forms both differences
     const float2 d = __ffma2_rn(unpack_bf16x2(hi), make_float2(-1.f, -1.f), make_float2(a, b));
     lo = pack_bf16(d.x, d.y);
+}
+
+// c ? a : b as one select instruction (keeps the compiler from turning a choice
+// between two elements of a register array into an indexed local-memory load).
+__device__ __forceinline__ float selp(bool c, float a, float b) {
+    float r;
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\tselp.f32 %0, %1, %2, p;\n\t}"
+        : "=f"(r)
+        : "f"(a), "f"(b), "r"((int)c));
+    return r;
 }
 
 // Packed fp32 pair arithmetic (one instruction for both lanes of the pair).

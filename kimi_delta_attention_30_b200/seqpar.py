@@ -10,20 +10,20 @@ its start state:
 
     S_end = M S_start + F
 
-* M  [H, dk, dk]: the segment's final state for the identity as initial state
-  and zero values (with v = 0 the recurrence is linear in S);
-* F  [H, dk, dv]: the segment's final state from a zero initial state.
+* M  [B, H, dk, dk]: the segment's final state from the identity with the
+  values' contribution left out;
+* F  [B, H, dk, dv]: the segment's final state from a zero start.
 
-One all-gather exchanges (M, F) among the ranks (H (dk^2 + dk dv) fp32 per
-rank and sequence: 2 MiB at H = 16, d = 128); rank r then forms its start state
-S_r = M_{r-1} S_{r-1} + F_{r-1} (S_0 is the caller's initial state) with plain
-matrix products, and runs the prefill once more from S_r to produce its
-outputs.  Each rank runs the prefill three times on T / N tokens (rank 0 once),
-against once on T tokens for a single GPU.
+Both come from one library call (``kda_chunk_segment_map``).  One all-gather
+exchanges (M, F) among the ranks (H (dk^2 + dk dv) fp32 per rank and sequence:
+2 MiB at H = 16, d = 128); rank r chains the maps of the ranks before it with
+``kda_compose_states`` and runs the prefill from the start state that gives.
+This module only marshals tensors and calls NCCL; every step of the arithmetic
+runs in the library.
 
-The per-segment prefill is the library's ``chunk_fwd`` (CUDA); ``fwd`` may be
-replaced by another callable with the same signature and return value, which is
-how the exchange logic is tested on CPU ranks.
+``fwd``, ``maps`` and ``compose`` may be replaced by callables with the same
+signatures and results (the CPU tests inject the fp64 oracle and a host
+composition, so the exchange logic runs on gloo ranks without a GPU).
 """
 from __future__ import annotations
 
@@ -36,30 +36,31 @@ def _default_fwd(q, k, v, log_alpha, beta, init_state=None, C=64):
     return chunk_fwd(q, k, v, log_alpha, beta, init_state=init_state, C=C)
 
 
-def segment_maps(q, k, v, log_alpha, beta, C: int = 64, fwd=None):
+def _default_maps(q, k, v, log_alpha, beta, C=64):
+    from . import segment_map
+    return segment_map(q, k, v, log_alpha, beta, C=C)
+
+
+def _default_compose(Ms, Fs, init_state=None):
+    from . import compose_states
+    return compose_states(Ms, Fs, init_state=init_state)
+
+
+def segment_maps(q, k, v, log_alpha, beta, C: int = 64, maps=None):
     """(M, F) of one segment: q, k, log_alpha [B, T, H, dk], v [B, T, H, dv],
     beta [B, T, H].  Returns M [B, H, dk, dk] and F [B, H, dk, dv] (fp32)."""
-    fwd = fwd or _default_fwd
-    B, _, H, dk = q.shape
-    eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(B, H, dk, dk).contiguous()
-    v0 = torch.zeros(q.shape, dtype=v.dtype, device=v.device)
-    _, M = fwd(q, k, v0, log_alpha, beta, init_state=eye, C=C)
-    _, F = fwd(q, k, v, log_alpha, beta, init_state=None, C=C)
-    return M, F
+    return (maps or _default_maps)(q, k, v, log_alpha, beta, C=C)
 
 
-def start_states(Ms, Fs, init_state=None):
-    """Start state of every segment from the gathered maps: S_0 = init_state (or
-    zero), S_{r+1} = M_r S_r + F_r.  Returns the list [S_0, ..., S_{N-1}]."""
-    S = torch.zeros_like(Fs[0]) if init_state is None else init_state.to(Fs[0].dtype)
-    out = [S]
-    for r in range(len(Ms) - 1):
-        S = torch.matmul(Ms[r], S) + Fs[r]
-        out.append(S)
-    return out
+def start_states(Ms, Fs, init_state=None, compose=None):
+    """States the segments start from, given the maps of segments 0 .. R-1 as
+    [R, B, H, dk, dk] and [R, B, H, dk, dv] tensors: S_0 = init_state (or zero),
+    S_{r+1} = M_r S_r + F_r.  Returns [R + 1, B, H, dk, dv]."""
+    return (compose or _default_compose)(Ms.contiguous(), Fs.contiguous(), init_state)
 
 
-def seqpar_forward(q, k, v, log_alpha, beta, init_state=None, C: int = 64, group=None, fwd=None):
+def seqpar_forward(q, k, v, log_alpha, beta, init_state=None, C: int = 64, group=None, fwd=None, maps=None,
+                   compose=None):
     """Prefill of this rank's segment of the sequences (every rank holds the same
     B sequences, segment ``rank`` of each, in rank order).  Returns this rank's
     (o, final_state); the last rank's final_state is the sequences' final state.
@@ -71,18 +72,18 @@ def seqpar_forward(q, k, v, log_alpha, beta, init_state=None, C: int = 64, group
         return fwd(q, k, v, log_alpha, beta, init_state=init_state, C=C)
     if rank == 0:
         o, fs = fwd(q, k, v, log_alpha, beta, init_state=init_state, C=C)
+        # rank 0's entry is (0, its end state), so the chain below starts from its true end state
         M = torch.zeros(q.shape[0], q.shape[2], q.shape[3], q.shape[3], dtype=fs.dtype, device=fs.device)
         F = fs
     else:
-        M, F = segment_maps(q, k, v, log_alpha, beta, C=C, fwd=fwd)
-    # rank 0's entry is (0, S_end of rank 0), so the chain below starts from its true end state
-    Ms = [torch.empty_like(M) for _ in range(world)]
-    Fs = [torch.empty_like(F) for _ in range(world)]
-    dist.all_gather(Ms, M.contiguous(), group=group)
-    dist.all_gather(Fs, F.contiguous(), group=group)
+        M, F = segment_maps(q, k, v, log_alpha, beta, C=C, maps=maps)
+    Ml = [torch.empty_like(M) for _ in range(world)]
+    Fl = [torch.empty_like(F) for _ in range(world)]
+    dist.all_gather(Ml, M.contiguous(), group=group)
+    dist.all_gather(Fl, F.contiguous(), group=group)
+    Ms, Fs = torch.stack(Ml), torch.stack(Fl)
     if rank == 0:
         return o, fs
-    S = Fs[0]
-    for r in range(1, rank):
-        S = torch.matmul(Ms[r], S) + Fs[r]
+    # segments 0 .. rank-1 from a zero state (segment 0's map is (0, its end state))
+    S = start_states(Ms[:rank], Fs[:rank], None, compose=compose)[rank]
     return fwd(q, k, v, log_alpha, beta, init_state=S.contiguous(), C=C)
