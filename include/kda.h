@@ -180,6 +180,24 @@ KDA_API kda_status kda_chunk_simt_offsets(int B, int T, int H, int dk, int dv, i
 KDA_API kda_status kda_set_timing_events(void* const* events, int n_events);
 
 /*
+ * Test hook for the failure path of the bounded device-side waits (no
+ * counterpart on the pages; it exists so that tests can make a wait expire
+ * without breaking anything on the GPU).  Arms, for the next tensor-core
+ * prefill (kda_chunk_fwd / _ex / _prep / _noalloc) called from this host
+ * thread, one extra wait in the first CTA of the chosen kernels on a barrier
+ * that nothing ever completes, bounded by limit_ns.  That wait expires: the
+ * kernel records KDA_ERR_TIMEOUT (read back with kda_chunk_fwd_device_status),
+ * waits for the copies and products it has already issued, frees its tensor
+ * memory and returns; the call's outputs are then undefined.  The next call is
+ * unaffected.
+ *   kernels  : bit 0 the chunk-local kernel (tc_intra), bit 1 the state carry
+ *              (tc_recur); 0 disarms
+ *   limit_ns : 1 .. 1e9 (ignored when kernels == 0)
+ * Errors: KDA_ERR_SHAPE for unknown bits or a limit out of range.
+ */
+KDA_API kda_status kda_set_test_wait_limit(unsigned int kernels, unsigned long long limit_ns);
+
+/*
  * Number of kernels kda_chunk_fwd_ex launches for this problem and algorithm
  * (after AUTO resolution), and their names through names[i] (static strings;
  * names may be NULL, at most max_names entries are written).  Returns the
@@ -202,14 +220,20 @@ KDA_API int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kd
  * device memory that the library itself declares.  Every device that loads the
  * library holds that array until the process exits.
  *
- *   - Problems whose kda_chunk_fwd_workspace_size() exceeds
- *     KDA_NOALLOC_SCRATCH_BYTES are rejected with KDA_ERR_SCRATCH before
- *     anything is launched (about 16 K token-heads at dk = dv = 128 on the
- *     CUDA-core path, e.g. B = 1, T = 1024, H = 16).
+ *   - A problem fits exactly when kda_chunk_fwd_workspace_size() <=
+ *     KDA_NOALLOC_SCRATCH_BYTES; larger ones are rejected with KDA_ERR_SCRATCH
+ *     before anything is launched.  From the scratch layouts: the tensor-core
+ *     path (bf16, dk = dv = 128) needs 147,968 bytes per (64-token chunk, head),
+ *     about 450 chunk-heads (e.g. B = 1, T = 1792, H = 16); the CUDA-core path
+ *     needs 4 (3 dk + 2 dv) bytes per token-head plus 4 dk dv bytes per
+ *     (chunk, head), about 18.7 K token-heads at dk = dv = 128, C = 64 and about
+ *     43 K at dk = dv = 64, C = 64; packed batches add 32 bytes per sequence.
  *   - The call never calls cudaMalloc, cudaFree or any allocating routine.
  *   - The first call on a device looks up the array's device address with that
- *     device current (cudaGetSymbolAddress) and caches it; make that first call
- *     before any stream capture on the device.
+ *     device current (cudaGetSymbolAddress) and caches it for the process; make
+ *     that first call before any stream capture on the device.  Destroying the
+ *     device's primary context between calls (cudaDeviceReset) is not
+ *     supported: the cached address would no longer be valid.
  *   - All calls share the one array, and it keeps the last call's contents
  *     (the prefill writes every scratch byte before reading it, so nothing needs
  *     clearing).  Calls whose execution overlaps on the GPU -- on different

@@ -94,6 +94,8 @@ def _declare(lib):
     lib.kda_chunk_segment_map.restype = c_int
     lib.kda_compose_states.argtypes = [vp, vp, vp] + [c_int] * 5 + [vp, vp]
     lib.kda_compose_states.restype = c_int
+    lib.kda_set_test_wait_limit.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+    lib.kda_set_test_wait_limit.restype = c_int
     return lib
 
 
@@ -127,7 +129,8 @@ def exported_symbols():
             "kda_chunk_simt_offsets", "kda_decode_step", "kda_set_timing_events", "kda_chunk_fwd_kernels",
             "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep", "kda_chunk_bwd_workspace_size",
             "kda_chunk_bwd", "kda_chunk_fwd_device_status", "kda_chunk_bwd_device_status",
-            "kda_chunk_fwd_noalloc_device_status", "kda_chunk_segment_map", "kda_compose_states"]
+            "kda_chunk_fwd_noalloc_device_status", "kda_chunk_segment_map", "kda_compose_states",
+            "kda_set_test_wait_limit"]
 
 
 def _ptr(t):
@@ -207,6 +210,16 @@ def chunk_kernels(B, T, H, dk, dv, C, dtype, cu_seqlens=None, algo="auto"):
     if cnt < 0:
         raise KdaError(cnt, "kda_chunk_fwd_kernels")
     return [names[i].decode() for i in range(cnt)]
+
+
+def set_test_wait_limit(kernels: int, limit_ns: int):
+    """Failure-path test hook (``kda_set_test_wait_limit``): the next
+    tensor-core prefill from this thread makes a bounded wait expire in the
+    first CTA of the chosen kernels (bit 0 tc_intra, bit 1 tc_recur) and records
+    KDA_ERR_TIMEOUT; 0 disarms."""
+    st = lib().kda_set_test_wait_limit(int(kernels), int(limit_ns))
+    if st != 0:
+        raise KdaError(st, "kda_set_test_wait_limit")
 
 
 def set_timing_events(events):

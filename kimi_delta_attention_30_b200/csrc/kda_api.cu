@@ -13,7 +13,8 @@ namespace kda {
 cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                               const float* init_state, void* o, float* final_state, const ChunkMap& cmap,
                               const SeqMap& smap, int n_chunks, int n_seqs, int H, int C, void* tc_ws,
-                              unsigned prep, cudaStream_t stream);
+                              unsigned prep, cudaStream_t stream, unsigned long long stall_intra_ns,
+                              unsigned long long stall_recur_ns);
 size_t tc_workspace_bytes(int n_chunks, int H, int C);
 bool tc_available();
 bool tc_supports(int C);
@@ -22,6 +23,17 @@ int tc_chunk();
 TimingHook& timing_hook() {
     static thread_local TimingHook hook{{nullptr}, 0, 0};
     return hook;
+}
+
+// kda_set_test_wait_limit: armed per host thread, consumed by the next
+// tensor-core prefill from that thread.
+struct TestWait {
+    unsigned kernels;
+    unsigned long long ns;
+};
+TestWait& test_wait() {
+    static thread_local TestWait w{0u, 0ull};
+    return w;
 }
 
 extern const char* const kTcKernelNames[];
@@ -327,8 +339,11 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
         err = launch_simt_prefill(dtype, q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap,
                                   p.n_chunks, p.n_seqs, H, dk, dv, C, w, s);
     } else {
+        const TestWait tw = test_wait();
+        test_wait() = TestWait{0u, 0ull};
         err = launch_tc_prefill(q, k, v, log_alpha, beta, init_state, o, final_state, cmap, smap, p.n_chunks,
-                                p.n_seqs, H, C, ws + table_bytes(p), prep, s);
+                                p.n_seqs, H, C, ws + table_bytes(p), prep, s, (tw.kernels & 1u) ? tw.ns : 0ull,
+                                (tw.kernels & 2u) ? tw.ns : 0ull);
     }
     timing_hook().n = 0;
     timing_hook().base = 0;
@@ -436,6 +451,13 @@ kda_status kda_chunk_fwd(const void* q, const void* k, const void* v, const void
                          size_t workspace_bytes, void* stream) {
     return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, dtype, init_state, cu_seqlens_host, n_seqs, B, T, H, dk, dv,
                             C, o, final_state, workspace, workspace_bytes, stream, KDA_ALGO_AUTO);
+}
+
+kda_status kda_set_test_wait_limit(unsigned int kernels, unsigned long long limit_ns) {
+    if (kernels & ~3u) return KDA_ERR_SHAPE;
+    if (kernels != 0u && (limit_ns == 0ull || limit_ns > 1000000000ull)) return KDA_ERR_SHAPE;
+    test_wait() = TestWait{kernels, kernels ? limit_ns : 0ull};
+    return KDA_OK;
 }
 
 kda_status kda_set_timing_events(void* const* events, int n_events) {

@@ -300,25 +300,35 @@ __global__ void __launch_bounds__(kTW, 2) kb_chain(const float* __restrict__ Qg,
         }
         __syncthreads();
         // dW = P^T dO + Kd dS' (P is zero above its diagonal): thread t forms column
-        // t % 32 of rows t / 32 + 16 m
+        // t % 32 of rows 4 (t / 32) .. 4 (t / 32) + 3, so the rows of P and Kd it reads
+        // are one float4 (the same for the whole warp) per column or channel group
         {
-            const int j = tid & 31, i0 = tid >> 5;
-            float acc[kBwdC / 16];
-#pragma unroll
-            for (int m = 0; m < kBwdC / 16; ++m) acc[m] = 0.f;
+            const int j = tid & 31, i0 = 4 * (tid >> 5);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
             for (int r = 0; r < L; ++r) {
                 const float o = dOs[r * kBV + j];
-#pragma unroll
-                for (int m = 0; m < kBwdC / 16; ++m) acc[m] = fmaf(Ps[r * C + i0 + 16 * m], o, acc[m]);
+                const float4 p = *reinterpret_cast<const float4*>(Ps + r * C + i0);
+                acc[0] = fmaf(p.x, o, acc[0]);
+                acc[1] = fmaf(p.y, o, acc[1]);
+                acc[2] = fmaf(p.z, o, acc[2]);
+                acc[3] = fmaf(p.w, o, acc[3]);
             }
-            for (int c = 0; c < dk; ++c) {
-                const float ds = dS[c * kBV + j];
+            for (int c = 0; c < dk; c += 4) {
+                float ds[4];
 #pragma unroll
-                for (int m = 0; m < kBwdC / 16; ++m) acc[m] = fmaf(M1[(i0 + 16 * m) * dk + c], ds, acc[m]);
+                for (int u = 0; u < 4; ++u) ds[u] = dS[(c + u) * kBV + j];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float4 kd = *reinterpret_cast<const float4*>(M1 + (i0 + m) * dk + c);
+                    acc[m] = fmaf(kd.x, ds[0], acc[m]);
+                    acc[m] = fmaf(kd.y, ds[1], acc[m]);
+                    acc[m] = fmaf(kd.z, ds[2], acc[m]);
+                    acc[m] = fmaf(kd.w, ds[3], acc[m]);
+                }
             }
 #pragma unroll
-            for (int m = 0; m < kBwdC / 16; ++m) {
-                const int i = i0 + 16 * m;
+            for (int m = 0; m < 4; ++m) {
+                const int i = i0 + m;
                 if (i < L) {
                     dWs[i * kBV + j] = acc[m];
                     dW[tok_off(t0 + i, H, h, dv) + j0 + j] = acc[m];
@@ -333,27 +343,27 @@ __global__ void __launch_bounds__(kTW, 2) kb_chain(const float* __restrict__ Qg,
         }
         __syncthreads();
         // dS = Diag(Gam) dS' + Qg^T dO - Wk^T dW: thread t forms column t % 32 of
-        // rows t / 32 + 16 m (each element is read and written by its own thread)
+        // channels 8 (t / 32) .. 8 (t / 32) + 7, read as two float4 of each of Qg and
+        // Wk per row (each element is read and written by its own thread)
         {
-            const int j = tid & 31, c0 = tid >> 5;
-            float acc[kMaxDK / 16];
+            const int j = tid & 31, c0 = 8 * (tid >> 5);
+            if (c0 < dk) {
+                float acc[8];
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 16; ++m) {
-                const int c = c0 + 16 * m;
-                acc[m] = c < dk ? exp_g(gC[c], gCl[c]) * dS[c * kBV + j] : 0.f;
-            }
-            for (int r = 0; r < L; ++r) {
-                const float o = dOs[r * kBV + j], w = dWs[r * kBV + j];
+                for (int m = 0; m < 8; ++m) acc[m] = exp_g(gC[c0 + m], gCl[c0 + m]) * dS[(c0 + m) * kBV + j];
+                for (int r = 0; r < L; ++r) {
+                    const float o = dOs[r * kBV + j], w = dWs[r * kBV + j];
+                    const float4 qa = *reinterpret_cast<const float4*>(M1 + r * dk + c0);
+                    const float4 qb = *reinterpret_cast<const float4*>(M1 + r * dk + c0 + 4);
+                    const float4 wa = *reinterpret_cast<const float4*>(M2 + r * dk + c0);
+                    const float4 wb = *reinterpret_cast<const float4*>(M2 + r * dk + c0 + 4);
+                    const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                    const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                for (int m = 0; m < kMaxDK / 16; ++m) {
-                    const int c = c0 + 16 * m;
-                    if (c < dk) acc[m] += M1[r * dk + c] * o - M2[r * dk + c] * w;
+                    for (int m = 0; m < 8; ++m) acc[m] += qv[m] * o - wv[m] * w;
                 }
-            }
 #pragma unroll
-            for (int m = 0; m < kMaxDK / 16; ++m) {
-                const int c = c0 + 16 * m;
-                if (c < dk) dS[c * kBV + j] = acc[m];
+                for (int m = 0; m < 8; ++m) dS[(c0 + m) * kBV + j] = acc[m];
             }
         }
         __syncthreads();
@@ -492,7 +502,7 @@ __global__ void __launch_bounds__(kT) kb_a(const Tin* __restrict__ d_o, const fl
 // by one float against bank conflicts); U and Wk are read through L1 (98 KB of
 // shared memory at d = 128, so two blocks share an SM).
 template <typename Tin>
-__global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin* __restrict__ v,
+__global__ void __launch_bounds__(kT, 2) kb_b(const Tin* __restrict__ k, const Tin* __restrict__ v,
                                            const Tin* __restrict__ beta, const float* __restrict__ g,
                                            const float* __restrict__ gl, const float* __restrict__ Atg,
                                            const float* __restrict__ U, const float* __restrict__ Wk,
@@ -554,27 +564,32 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
         if (lane == 0) db[r] = s;
     }
     __syncthreads();   // the rows of X are read by other threads below (and dA is overwritten)
-    // dA = -(Y U^T + Z Wk^T), i < r: thread t forms rows t / 16 + 16 m, columns t % 16 + 16 n
-    {
-        const int rb = tid >> 4, ib = tid & 15;
+    // dA = -(Y U^T + Z Wk^T), i < r: one warp per 4 x 4 tile of the lower triangle
+    // (rows 4a..4a+3, columns 4b..4b+3, b <= a), its lanes splitting the columns of
+    // [Y | Z] and [U | Wk], so each load of a U or Wk row is one coalesced line;
+    // five shuffle rounds add the lanes' partial sums.  Rows i >= len of U and Wk
+    // are read as zero; the tiles above the diagonal are set to zero.
+    for (int t = warp; t < 136; t += kT / 32) {
+        int a = 0;
+        while ((a + 1) * (a + 2) / 2 <= t) ++a;
+        const int b = t - a * (a + 1) / 2;
+        const float* urow[4];
+        const float* wrow[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            const int i = 4 * b + n;
+            urow[n] = i < len ? U + tok_off(tok0 + i, H, h, dv) : nullptr;
+            wrow[n] = i < len ? Wk + tok_off(tok0 + i, H, h, dk) : nullptr;
+        }
         float acc[4][4];
 #pragma unroll
         for (int m = 0; m < 4; ++m)
 #pragma unroll
             for (int n = 0; n < 4; ++n) acc[m][n] = 0.f;
-        // rows i >= len of U, Wk are read as zero
-        const float* urow[4];
-        const float* wrow[4];
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            const int i = ib + 16 * n;
-            urow[n] = i < len ? U + tok_off(tok0 + i, H, h, dv) : nullptr;
-            wrow[n] = i < len ? Wk + tok_off(tok0 + i, H, h, dk) : nullptr;
-        }
-        for (int j = 0; j < ncol; ++j) {
+        for (int j = lane; j < ncol; j += 32) {
             float xr[4], ui[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) xr[m] = X[(rb + 16 * m) * xs + j];
+            for (int m = 0; m < 4; ++m) xr[m] = X[(4 * a + m) * xs + j];
 #pragma unroll
             for (int n = 0; n < 4; ++n)
                 ui[n] = urow[n] ? (j < dv ? __ldg(urow[n] + j) : __ldg(wrow[n] + j - dv)) : 0.f;
@@ -586,10 +601,23 @@ __global__ void __launch_bounds__(kT) kb_b(const Tin* __restrict__ k, const Tin*
 #pragma unroll
         for (int m = 0; m < 4; ++m)
 #pragma unroll
-            for (int n = 0; n < 4; ++n) {
-                const int r = rb + 16 * m, i = ib + 16 * n;
-                dA[r * C + i] = (r < len && i < r) ? -acc[m][n] : 0.f;
+            for (int n = 0; n < 4; ++n) acc[m][n] = wsum(acc[m][n]);
+        if (lane == 0) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int r = 4 * a + m, i0 = 4 * b;
+                float4 o;
+                o.x = (r < len && i0 < r) ? -acc[m][0] : 0.f;
+                o.y = (r < len && i0 + 1 < r) ? -acc[m][1] : 0.f;
+                o.z = (r < len && i0 + 2 < r) ? -acc[m][2] : 0.f;
+                o.w = (r < len && i0 + 3 < r) ? -acc[m][3] : 0.f;
+                *reinterpret_cast<float4*>(dA + r * C + i0) = o;
             }
+        }
+    }
+    for (int e4 = tid; e4 < C * C / 4; e4 += kT) {
+        const int r = e4 >> 4, bb = e4 & 15;
+        if (bb > (r >> 2)) *reinterpret_cast<float4*>(dA + r * C + 4 * bb) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
     float* dAc = dAt + ((size_t)blockIdx.x * H + h) * C * C;
@@ -626,7 +654,8 @@ constexpr int kCH = 64;          // kb_c: channels per pass
 // channel-major ([c][r], row stride kPS), padded rows as in kb_p.  The dAt and
 // dP tiles are staged with their masks applied (zero for i >= r, resp. i > r, and
 // for rows past the end of the chunk).
-// Shared: Qt, Kt, Gt, GLt [kCH][kPS], dAs, dPs [C][C], Fs, Ys, Xs [C][kCH].
+// Shared: Qt, Kt, Gt, GLt [kCH][kPS], dAs, dPs [C][C], Fs, Ys, Xs, dQs, dKgs, dKds
+// [C][kCH], PX, PY [8][kCH] (the dlog alpha scan's segment sums).
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, const Tin* __restrict__ k,
                                                      const Tin* __restrict__ la, const float* __restrict__ g,
@@ -648,6 +677,11 @@ __global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, 
     float* Fs = dPs + C * C;
     float* Ys = Fs + C * kCH;
     float* Xs = Ys + C * kCH;
+    float* dQs = Xs + C * kCH;       // this pass's dQg, dKg, dKd [C][kCH]
+    float* dKgs = dQs + C * kCH;
+    float* dKds = dKgs + C * kCH;
+    float* PX = dKds + C * kCH;      // per-segment sums of the dlog alpha scan [8][kCH]
+    float* PY = PX + 8 * kCH;
     int seq, tok0, len, idx;
     cmap.locate(blockIdx.x, seq, tok0, len, idx);
     const int h = blockIdx.y, tid = threadIdx.x;
@@ -700,6 +734,13 @@ __global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, 
             }
         }
         for (int e = tid; e < 2 * C * kCH; e += kCThreads) Fs[e] = 0.f;   // Fs and Ys
+        for (int e4 = tid; e4 < len * kCH / 4; e4 += kCThreads) {
+            const int r = e4 / (kCH / 4), cq = 4 * (e4 - r * (kCH / 4));
+            const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + cq;
+            *reinterpret_cast<float4*>(dQs + r * kCH + cq) = *reinterpret_cast<const float4*>(dQg + off);
+            *reinterpret_cast<float4*>(dKgs + r * kCH + cq) = *reinterpret_cast<const float4*>(dKg + off);
+            *reinterpret_cast<float4*>(dKds + r * kCH + cq) = *reinterpret_cast<const float4*>(dKd + off);
+        }
         __syncthreads();
 
         const float* qc = Qt + c * kPS;
@@ -734,19 +775,21 @@ __global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, 
                     const float4 a4 = *reinterpret_cast<const float4*>(dAs + (4 * a + x) * C + 4 * b);
                     const float4 p4 = *reinterpret_cast<const float4*>(dPs + (4 * a + x) * C + 4 * b);
                     const float da[4] = {a4.x, a4.y, a4.z, a4.w}, dp[4] = {p4.x, p4.y, p4.z, p4.w};
-                    float rowT = 0.f;
+                    float tx[4];
 #pragma unroll
                     for (int y = 0; y < 4; ++y) {
+                        // with w = dAt k_r + dP q_r: T_ri = w k_i E and the column term is w E
                         const float e = exp_gdiff(gr[x], lr[x], gi[y], li[y]);
                         const float ke = ki[y] * e;
-                        const float av = da[y] * ke, bv = dp[y] * ke;
-                        x1[x] += av;
-                        x2[x] += bv;
-                        const float t = fmaf(kr[x], av, qr[x] * bv);
-                        rowT += t;
-                        colT[y] += t;
-                        yc[y] = fmaf(fmaf(da[y], kr[x], dp[y] * qr[x]), e, yc[y]);
+                        x1[x] = fmaf(da[y], ke, x1[x]);
+                        x2[x] = fmaf(dp[y], ke, x2[x]);
+                        const float w = fmaf(da[y], kr[x], dp[y] * qr[x]);
+                        yc[y] = fmaf(w, e, yc[y]);
+                        tx[y] = w * ke;
                     }
+                    const float rowT = (tx[0] + tx[1]) + (tx[2] + tx[3]);
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) colT[y] += tx[y];
                     // rows x >= u of this tile count for F(4a + u)
 #pragma unroll
                     for (int u = 0; u <= x; ++u) rs[u] += rowT;
@@ -793,39 +836,62 @@ __global__ void __launch_bounds__(kCThreads, 1) kb_c(const Tin* __restrict__ q, 
                 Xs[r * kCH + c] = x1[x];
                 if (r < len) {
                     const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + c;
-                    dq_out[off] = from_f32<Tin>(x2[x] + dQg[off] * exp_g(gr[x], lr[x]));
+                    dq_out[off] = from_f32<Tin>(x2[x] + dQs[r * kCH + c] * exp_g(gr[x], lr[x]));
                 }
             }
         }
         __syncthreads();
         // dk, and the per-(row, channel) terms of dlog alpha (into Xs and Ys, which
         // each element's thread has just read)
-        const float gC = Gt[c * kPS + len - 1], gCl = GLt[c * kPS + len - 1];   // used by ap == 0 below
         for (int e = tid; e < len * kCH; e += kCThreads) {
             const int r = e / kCH, cc = e - r * kCH;
             const size_t off = tok_off(tok0 + r, H, h, DK) + c0 + cc;
             const float gv = Gt[cc * kPS + r], lv = GLt[cc * kPS + r];
             const float eg = exp_g(gv, lv);
             const float ed = exp_gdiff(Gt[cc * kPS + len - 1], GLt[cc * kPS + len - 1], gv, lv);
-            const float dkg = dKg[off], dkd = dKd[off];
+            const float dkg = dKgs[e], dkd = dKds[e];
             dk_out[off] = from_f32<Tin>(Xs[e] + Ys[e] + dkg * eg + dkd * ed);
-            Xs[e] = dkd * Kt[cc * kPS + r] * ed;                               // dKd Kd
-            Ys[e] = (dQg[off] * Qt[cc * kPS + r] + dkg * Kt[cc * kPS + r]) * eg;   // dQg Qg + dKg Kg
+            Xs[e] = dkd * Kt[cc * kPS + r] * ed;                              // dKd Kd
+            Ys[e] = (dQs[e] * Qt[cc * kPS + r] + dkg * Kt[cc * kPS + r]) * eg;   // dQg Qg + dKg Kg
         }
         __syncthreads();
-        // dlog alpha, one thread per channel (zero where the forward's floor on log alpha was active)
-        if (ap == 0) {
-            float pre = 0.f;   // sum_{r<j} dKd Kd
-            for (int j = 0; j < len; ++j) {
-                Fs[j * kCH + c] += pre;
-                pre += Xs[j * kCH + c];
+        // dlog alpha (zero where the forward's floor on log alpha was active):
+        //   F(j) + sum_{r<j} dKd Kd + sum_{r>=j} (dQg Qg + dKg Kg) + dGam Gam,
+        // the two sums as scans over 8 segments of 8 rows per channel
+        const int seg = ap, j0 = 8 * seg;
+        {
+            float sx = 0.f, sy = 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (j0 + u < len) {
+                    sx += Xs[(j0 + u) * kCH + c];
+                    sy += Ys[(j0 + u) * kCH + c];
+                }
+            PX[seg * kCH + c] = sx;
+            PY[seg * kCH + c] = sy;
+        }
+        __syncthreads();
+        if (j0 < len) {
+            float pre = 0.f, suf = 0.f;   // sum of the segments before / after this one
+            for (int s2 = 0; s2 < seg; ++s2) pre += PX[s2 * kCH + c];
+            for (int s2 = seg + 1; s2 < 8; ++s2) suf += PY[s2 * kCH + c];
+            const float gam = dGam[(chunk * H + h) * DK + c0 + c] *
+                              exp_g(Gt[c * kPS + len - 1], GLt[c * kPS + len - 1]);
+            float prej[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                prej[u] = pre;
+                if (j0 + u < len) pre += Xs[(j0 + u) * kCH + c];
             }
-            const float gam = dGam[(chunk * H + h) * DK + c0 + c] * exp_g(gC, gCl);
-            float suf = 0.f;   // sum_{r>=j} (dQg Qg + dKg Kg)
-            for (int j = len - 1; j >= 0; --j) {
-                const size_t off = tok_off(tok0 + j, H, h, DK) + c0 + c;
-                suf += Ys[j * kCH + c];
-                dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor ? Fs[j * kCH + c] + suf + gam : 0.f);
+#pragma unroll
+            for (int u = 7; u >= 0; --u) {
+                const int j = j0 + u;
+                if (j < len) {
+                    suf += Ys[j * kCH + c];
+                    const size_t off = tok_off(tok0 + j, H, h, DK) + c0 + c;
+                    dla_out[off] = from_f32<Tin>(to_f32(la[off]) >= kLogAlphaFloor
+                                                     ? Fs[j * kCH + c] + prej[u] + suf + gam : 0.f);
+                }
             }
         }
     }
@@ -838,7 +904,8 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     constexpr int C = 64;
     const size_t smem_a = sizeof(float) * (2 * (size_t)kBV * (DK + 1) + 3 * (size_t)C * kBP);
     const size_t smem_b = sizeof(float) * (2 * (size_t)C * C + 2 * C + (size_t)C * (dv + DK + 1));
-    const size_t smem_c = sizeof(float) * (4 * (size_t)kCH * kPS + 2 * (size_t)C * C + 3 * (size_t)C * kCH);
+    const size_t smem_c = sizeof(float) * (4 * (size_t)kCH * kPS + 2 * (size_t)C * C + 6 * (size_t)C * kCH +
+                                           2 * 8 * (size_t)kCH);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kb_a<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a))) return e;
     if ((e = cudaFuncSetAttribute(kb_b<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
-         int H, unsigned prep_flags) {
+         int H, unsigned prep_flags, unsigned long long stall_ns) {
     // PREP = false is the plain operator: no preprocessing code is compiled in
     const unsigned prep = PREP ? prep_flags : 0u;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -229,6 +229,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     uint64_t& mbar = reinterpret_cast<uint64_t*>(sm + kIntraBars)[0];      // tensor-core products, in issue order
     uint64_t& mbar_k = reinterpret_cast<uint64_t*>(sm + kIntraBars)[1];    // the second half of the last product
     uint64_t& mbar_la = reinterpret_cast<uint64_t*>(sm + kIntraBars)[2];   // log alpha rows landed
+    uint64_t& mbar_never = reinterpret_cast<uint64_t*>(sm + kIntraBars)[3];  // completed by nothing (failure test)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // this thread: rows [8 w, 8 w + 8) of 16-row block I = w / 2, and channels
@@ -250,6 +251,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         mbar_init(&mbar, 1);
         mbar_init(&mbar_k, 1);
         mbar_init(&mbar_la, 64);
+        mbar_init(&mbar_never, 1);
         mbar_init_fence();
     }
     if (warp == 0) {
@@ -338,6 +340,13 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         inv_nk[tid] = 1.f;   // inv_nk [0, 64) and inv_nq [64, 128) are adjacent
     }
     if (!mbar_wait(&mbar_la, 0)) {
+        record_error(err, KDA_ERR_TIMEOUT);
+        atomicExch(&sflags[1], 1u);
+    }
+    // test of the failure path (stall_ns != 0, set through kda_set_test_wait_limit):
+    // the first CTA waits, bounded by stall_ns, on a barrier that nothing completes,
+    // then records the timeout and takes the abort path like any expired wait
+    if (stall_ns != 0ull && blockIdx.x == 0 && tid == 0 && !mbar_wait(&mbar_never, 0, stall_ns)) {
         record_error(err, KDA_ERR_TIMEOUT);
         atomicExch(&sflags[1], 1u);
     }
@@ -925,7 +934,7 @@ template <int BV, int MODE>
 __global__ void __launch_bounds__(kRecurThreads, 1)
 tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, float* __restrict__ final_state,
          __nv_bfloat16* __restrict__ o, int* __restrict__ err, SeqMap smap, int H, float* __restrict__ s_store,
-         float* __restrict__ w_store) {
+         float* __restrict__ w_store, unsigned long long stall_ns) {
     constexpr bool STORE = MODE == 1, MAP = MODE == 2;
     using Lay = RecurLayout<BV>;
     constexpr int HB = BV / 2;          // state columns per thread
@@ -944,6 +953,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     uint64_t* p_full = bars + 7;      // P landed
     uint64_t* d_issued = bars + 8;    // the chunk's first product has been issued
     uint32_t* sflags = reinterpret_cast<uint32_t*>(bars + 9);        // [0] tmem base, [1] abort
+    uint64_t* never = bars + 10;      // completed by nothing (failure test)
     uint8_t* s_h = sm + Lay::kS;
     uint8_t* s_l = s_h + 16384;
     auto w_hi = [&](int n) { return sm + Lay::kW + (n & 1) * 16384; };   // lo parts 8 KB further
@@ -965,6 +975,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
 
     if (tid == 0) {
         for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
+        mbar_init(never, 1);
         sflags[1] = 0;
         mbar_init_fence();
     }
@@ -1102,6 +1113,9 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
             tmem_st16(tmem_addr(t_s, 32 * sp, cq + 16 * g), t);
         }
         tmem_st_wait();
+        // test of the failure path (stall_ns != 0): the first CTA waits, bounded, on a
+        // barrier that nothing completes before its first product, then aborts
+        if (stall_ns != 0ull && n == 0 && blockIdx.x == 0 && tid == 0 && !mbar_wait(never, 0, stall_ns)) fail();
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -1228,14 +1242,14 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
 template <int BV, int MODE = 0>
 cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* final_state, __nv_bfloat16* o, int* err,
                          const SeqMap& smap, int n_seqs, int H, cudaStream_t stream, float* s_store = nullptr,
-                         float* w_store = nullptr) {
+                         float* w_store = nullptr, unsigned long long stall_ns = 0ull) {
     using Lay = RecurLayout<BV>;
     cudaError_t e =
         cudaFuncSetAttribute(tc_recur<BV, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Lay::kAlloc);
     if (e != cudaSuccess) return e;
     const unsigned tiles = (MODE == 2 ? 2u : 1u) * (unsigned)(kD / BV);
     tc_recur<BV, MODE><<<dim3((unsigned)(n_seqs * H) * tiles), kRecurThreads, Lay::kAlloc, stream>>>(
-        ws, init_state, final_state, o, err, smap, H, s_store, w_store);
+        ws, init_state, final_state, o, err, smap, H, s_store, w_store, stall_ns);
     return cudaGetLastError();
 }
 
@@ -1287,7 +1301,8 @@ size_t tc_workspace_bytes(int n_chunks, int H, int C) {
 cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                               const float* init_state, void* o, float* final_state, const ChunkMap& cmap,
                               const SeqMap& smap, int n_chunks, int n_seqs, int H, int C, void* tc_ws,
-                              unsigned prep, cudaStream_t stream) {
+                              unsigned prep, cudaStream_t stream, unsigned long long stall_intra_ns,
+                              unsigned long long stall_recur_ns) {
     if (C != kC) return cudaErrorNotSupported;
     int* err = reinterpret_cast<int*>(tc_ws);
     uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
@@ -1299,7 +1314,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         kern<<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, prep);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, prep, stall_intra_ns);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1307,9 +1322,11 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
     if (n_seqs > 0) {
         const long units = (long)n_seqs * H;
         if (units * 4 <= sm_count())
-            e = launch_recur<32>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream);
+            e = launch_recur<32>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream,
+                                 nullptr, nullptr, stall_recur_ns);
         else
-            e = launch_recur<64>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream);
+            e = launch_recur<64>(ws, init_state, final_state, (__nv_bfloat16*)o, err, smap, n_seqs, H, stream,
+                                 nullptr, nullptr, stall_recur_ns);
         if (e != cudaSuccess) return e;
     }
     timing_mark(stream, 2);
@@ -1332,7 +1349,7 @@ cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const 
         if (e != cudaSuccess) return e;
         tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         tc_unpack_u_wk<<<dim3(n_chunks, H), 256, 0, stream>>>(ws, U, Wk, cmap, H);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1363,7 +1380,7 @@ cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, c
         if (e != cudaSuccess) return e;
         tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     timing_mark(stream, 1);

@@ -251,3 +251,13 @@ def test_device_status_validates_on_the_host():
     # zero sequences launch nothing, on either path
     assert _status_bwd(dtype=0, dk=128, dv=128, B=0) == OK
     assert _status_fwd(dtype=0, dk=128, dv=128, B=0) == OK
+
+
+def test_test_wait_limit_arguments():
+    """kda_set_test_wait_limit checks its arguments on the host and disarms with 0."""
+    lib = kda.lib()
+    assert lib.kda_set_test_wait_limit(4, 1000) == E_SHAPE          # unknown kernel bit
+    assert lib.kda_set_test_wait_limit(1, 0) == E_SHAPE             # zero limit
+    assert lib.kda_set_test_wait_limit(2, 2_000_000_000) == E_SHAPE  # above one second
+    assert lib.kda_set_test_wait_limit(3, 1000) == OK
+    assert lib.kda_set_test_wait_limit(0, 0) == OK                  # disarm

@@ -353,3 +353,23 @@ def test_varlen_call_returns_before_earlier_work_finishes(cuda_ok, call):
     assert pending, "the call waited for earlier work on its stream"
     if call == "fwd":
         _check_all(inp, out[0], out[1], TOL["bf16"], label="varlen async call")
+
+
+@pytest.mark.parametrize("kernels", [1, 2, 3])
+def test_device_wait_timeout_is_reported_and_recoverable(cuda_ok, kernels):
+    """The failure path of the bounded device-side waits, without breaking the
+    GPU: kda_set_test_wait_limit makes one wait in the first CTA of tc_intra
+    (1), tc_recur (2) or both (3) wait 1 ms on a barrier that nothing completes.
+    The call then reports KDA_ERR_TIMEOUT through the device status, and the
+    next call on the same stream and workspace is normal and matches the
+    oracle."""
+    inp = _to(make_prefill("prefill", B=2, T=300, H=4, seed=61), DEV)
+    B, T, H, dk = inp.q.shape
+    ws = torch.empty(kda.workspace_size(B, T, H, dk, dk, 64, torch.bfloat16), dtype=torch.uint8, device=DEV)
+    args = (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta)
+    kda.set_test_wait_limit(kernels, 1_000_000)
+    kda.chunk_fwd(*args, init_state=inp.init_state, C=64, workspace=ws)
+    assert kda.device_status("fwd", ws, torch.bfloat16, B, T, H, dk, dk, 64) == kda.KDA_ERR_TIMEOUT
+    o, fs = kda.chunk_fwd(*args, init_state=inp.init_state, C=64, workspace=ws)
+    assert kda.device_status("fwd", ws, torch.bfloat16, B, T, H, dk, dk, 64) == 0
+    _check_all(inp, o, fs, TOL["bf16"], label=f"after a timeout in kernels {kernels}")

@@ -32,6 +32,19 @@ def test_noalloc_rejects_oversized_problem_before_launch():
     assert "SCRATCH" in lib.kda_status_string(E_SCRATCH).decode()
 
 
+def test_noalloc_limits_stated_in_the_header():
+    """The per-path bounds the header states follow from the workspace sizes:
+    450 tensor-core chunk-heads fit, the CUDA-core path holds about 18.7 K
+    token-heads at d = 128 and 43 K at d = 64 (host computation only)."""
+    lim = kda.NOALLOC_SCRATCH_BYTES
+    assert kda.workspace_size(1, 1792, 16, 128, 128, 64, torch.bfloat16) <= lim < \
+        kda.workspace_size(1, 1792 + 64, 16, 128, 128, 64, torch.bfloat16)
+    assert kda.workspace_size(1, 18 * 1024, 1, 128, 128, 64, torch.float32) <= lim < \
+        kda.workspace_size(1, 19 * 1024, 1, 128, 128, 64, torch.float32)
+    assert kda.workspace_size(1, 42 * 1024, 1, 64, 64, 64, torch.float32) <= lim < \
+        kda.workspace_size(1, 44 * 1024, 1, 64, 64, 64, torch.float32)
+
+
 def _args(inp):
     return (inp.q, inp.k, inp.v, inp.log_alpha, inp.beta)
 
