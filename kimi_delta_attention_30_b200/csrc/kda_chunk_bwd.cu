@@ -31,6 +31,7 @@
 // the tensor-core forward (bf16, d = 128; g by the CUDA-core K1) or by the
 // CUDA-core forward kernels.
 #include <algorithm>
+#include <type_traits>
 
 #include "kda_internal.cuh"
 
@@ -41,7 +42,7 @@ constexpr int kT = 256;
 constexpr int kTW = 512;      // kb_chain: more warps to hide latency
 constexpr int kBV = 32;       // d_v columns per chain block / per tile
 constexpr int kBP = kBV + 1;  // padded row stride of the d_v tiles
-constexpr int kMaxDK = 128;
+
 constexpr int kBwdC = 64;     // the backward kernels tile by 64 tokens
 
 __device__ __forceinline__ float wsum(float x) {
@@ -911,8 +912,15 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     if ((e = cudaFuncSetAttribute(kb_b<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_b))) return e;
     if ((e = cudaFuncSetAttribute(kb_c<Tin, DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c))) return e;
     const dim3 grid(n_chunks, H);
-    kb_a<Tin, DK><<<grid, kT, smem_a, stream>>>(d_o, ws.fwd.W, ws.dW, ws.fwd.S_chunk, ws.dS_chunk, ws.dQg, ws.dKd,
-                                               ws.dWk, ws.dGam, ws.P, cmap, H, dv);
+    if (std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && dv == 128 && ws.tc_ws) {
+        // bf16, d = 128: the four chunk-local products on the tensor cores
+        e = launch_kb_a_tc(d_o, ws.fwd.W, ws.dW, ws.fwd.S_chunk, ws.dS_chunk, ws.dQg, ws.dKd, ws.dWk, ws.dGam, ws.P,
+                           reinterpret_cast<int*>(ws.tc_ws), cmap, n_chunks, H, stream);
+        if (e != cudaSuccess) return e;
+    } else {
+        kb_a<Tin, DK><<<grid, kT, smem_a, stream>>>(d_o, ws.fwd.W, ws.dW, ws.fwd.S_chunk, ws.dS_chunk, ws.dQg,
+                                                   ws.dKd, ws.dWk, ws.dGam, ws.P, cmap, H, dv);
+    }
     timing_mark(stream, 4);
     kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
                                             ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);

@@ -219,6 +219,12 @@ cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, 
                                  const SeqMap& smap, int n_chunks, int n_seqs, int H, int dkk, int dvv, int C,
                                  const BwdWorkspace& ws, cudaStream_t stream);
 
+// Tensor-core chunk-local products of the backward pass (bf16, d = 128):
+// dQg = dO S^T, dWk = -dW S^T, dKd = W dS'^T, dP = dO W^T, dGam = rowsum(dS' . S).
+cudaError_t launch_kb_a_tc(const void* d_o, const float* W, const float* dW, const float* S_chunk,
+                           const float* dS_chunk, float* dQg, float* dKd, float* dWk, float* dGam, float* dP, int* err,
+                           const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream);
+
 // A segment's affine map S_end = M S_start + F (M [N, H, dk, dk], F [N, H, dk, dv]).
 cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
                                   const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,
