@@ -236,7 +236,7 @@ def design_bytes(kernel: str, g: Geometry, in_bytes=2):
 def _tc_digest():
     csrc = os.path.join(ROOT, "kimi_delta_attention_30_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("kda_chunk_tc.cu", "kda_tc.cuh"):
+    for f in ("kda_chunk_tc.cu", "kda_tc.cuh", "kda_tc_image.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -155,7 +155,7 @@ SimtLayout simt_layout(const Plan& p, int H, int dk, int dv) {
 struct BwdLayout {
     SimtLayout fwd;
     size_t off[12];
-    size_t tc = 0, o_scratch = 0;   // tensor-core recompute (0: not used)
+    size_t tc = 0, o_scratch = 0, T = 0;   // tensor-core recompute (0: not used)
     size_t total;
 };
 
@@ -179,6 +179,8 @@ BwdLayout bwd_layout(const Plan& p, int H, int dk, int dv, int C, bool tc = fals
         o = align_up(o + tc_workspace_bytes(p.n_chunks, H, C));
         L.o_scratch = o;
         o = align_up(o + tok * dv * sizeof(uint16_t));
+        L.T = o;                                   // (I + A)^-1 per (chunk, head), fp32
+        o = align_up(o + ch * C * C * sizeof(float));
     }
     L.total = o;
     return L;
@@ -550,6 +552,7 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     w.Kd = f(L.off[11]);
     w.tc_ws = use_tc ? (void*)(ws + L.tc) : nullptr;
     w.o_scratch = use_tc ? (void*)(ws + L.o_scratch) : nullptr;
+    w.T = use_tc ? (float*)(ws + L.T) : nullptr;
     timing_mark(s, 0);
     cudaError_t err = launch_simt_backward(dtype, q, k, v, log_alpha, beta, init_state, d_o, d_final_state, dq,
                                            dk_out, dv_out, dlog_alpha, dbeta, d_init_state, cmap, smap, p.n_chunks,

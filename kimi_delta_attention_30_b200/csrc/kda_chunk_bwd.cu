@@ -922,8 +922,15 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
                                                    ws.dKd, ws.dWk, ws.dGam, ws.P, cmap, H, dv);
     }
     timing_mark(stream, 4);
-    kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
-                                            ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
+    if (std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && dv == 128 && ws.tc_ws && ws.T) {
+        // bf16, d = 128: the back substitution as two tensor-core products with T
+        e = launch_kb_b_tc(ws.T, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW, ws.dWk, k, v, beta, ws.fwd.g, ws.fwd.gl, dv_,
+                           dbeta, ws.dKg, ws.dAt, reinterpret_cast<int*>(ws.tc_ws), cmap, n_chunks, H, stream);
+        if (e != cudaSuccess) return e;
+    } else {
+        kb_b<Tin><<<grid, kT, smem_b, stream>>>(k, v, beta, ws.fwd.g, ws.fwd.gl, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW,
+                                                ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
+    }
     timing_mark(stream, 5);
     kb_c<Tin, DK><<<grid, kCThreads, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd,
                                                      ws.dKg, ws.dGam, dq, dk_, dla, cmap, H);
@@ -942,7 +949,7 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
         // bf16, d = 128: the tensor-core forward recomputes U, Wk, W and the chunk start states
         if ((e = launch_simt_g(dtype, la, cmap, n_chunks, H, dk, ws.fwd, stream)) != cudaSuccess) return e;
         e = launch_tc_states(q, k, v, la, beta, init_state, ws.o_scratch, cmap, smap, n_chunks, n_seqs, H, ws.tc_ws,
-                             ws.fwd.S_chunk, ws.fwd.W, ws.fwd.U, ws.fwd.Wk, stream);
+                             ws.fwd.S_chunk, ws.fwd.W, ws.fwd.U, ws.fwd.Wk, ws.T, ws.At, stream);
     } else {
         e = launch_simt_states(dtype, k, v, la, beta, init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws.fwd,
                                stream);
@@ -958,14 +965,25 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
         return e;
     // two chain blocks per SM (115,712 bytes each at d = 128) need the whole shared-memory carveout
     if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100))) return e;
-    if (n_chunks > 0)
+    // (the tensor-core path takes At from the recompute and P from its images, and
+    // kb_a_tc writes the whole dP buffer: no pairwise pass is needed here)
+    const bool tc_chain = std::is_same<Tin, __nv_bfloat16>::value && dk == 128 && dv == 128 && ws.tc_ws;
+    if (n_chunks > 0 && !tc_chain)
         kern_p<<<dim3(n_chunks, H), kPThreads, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg,
                                                                  ws.Kd, cmap, H);
     timing_mark(stream, 2);
-    if (n_seqs > 0)
-        kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kTW, smem_chain, stream>>>(
-            ws.Qg, ws.Kd, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, H, dk,
-            dv, C);
+    if (n_seqs > 0) {
+        if (std::is_same<Tin, __nv_bfloat16>::value && dk == 128 && dv == 128 && ws.tc_ws) {
+            // bf16, d = 128: the reverse chain on the tensor cores, from the recompute's images
+            if ((e = launch_tc_chain(ws.tc_ws, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, n_seqs, H, stream)) !=
+                cudaSuccess)
+                return e;
+        } else {
+            kb_chain<Tin><<<dim3(n_seqs, H, dv / kBV), kTW, smem_chain, stream>>>(
+                ws.Qg, ws.Kd, ws.fwd.g, ws.fwd.gl, ws.fwd.Wk, ws.P, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap,
+                H, dk, dv, C);
+        }
+    }
     timing_mark(stream, 3);
     if ((e = cudaGetLastError()) != cudaSuccess || n_chunks == 0) return e;
     if (dk == 128) return run_bwd_dk<Tin, 128>(q, k, v, la, beta, d_o, dq, dk_, dv_, dla, dbeta, cmap, n_chunks, H, dv,

@@ -44,6 +44,7 @@
 // nats has its diagonal A / P entries recomputed pairwise on CUDA cores.
 #include "kda_internal.cuh"
 #include "kda_tc.cuh"
+#include "kda_tc_image.cuh"
 
 namespace kda {
 
@@ -53,28 +54,11 @@ extern const int kTcKernelCount = 2;
 namespace {
 
 using namespace tc;
+using namespace tcimg;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr float kDiagRange = 80.0f;
-
-// ---- workspace image of one (chunk, head) --------------------------------------
-constexpr uint32_t kOffWkQh = 0;         // [128 rows][128 k] bf16 SW128 K-major: rows 0-63 Wk, 64-127 Q exp(g) (hi)
-constexpr uint32_t kOffWkQl = 32768;     // lo parts
-constexpr uint32_t kOffKdTh = 65536;     // [128 rows (channel)][64 k (token)] bf16 SW128 K-major (hi)
-constexpr uint32_t kOffKdTl = 81920;     // lo parts
-constexpr uint32_t kOffU = 98304;        // U : fp32, see u_index()
-constexpr uint32_t kOffPh = 131072;      // P [64 rows][64 k] bf16 SW128 K-major (hi)
-constexpr uint32_t kOffPl = 139264;      // lo parts
-constexpr uint32_t kOffGam = 147456;     // Gamma_C fp32 [128]
-constexpr uint32_t kChunkBytes = 147968;
-constexpr uint32_t kErrHeader = 256;     // first bytes of the TC scratch: error word
-
-// U tiles: [4 column blocks of 32][64 rows][8 chunks of 4 floats], chunk
-// permuted by row % 8 so that row-per-thread float4 reads hit distinct banks.
-__host__ __device__ __forceinline__ int u_index(int r, int j) {   // j % 4 == 0
-    return (j >> 5) * 2048 + r * 32 + (((((j & 31) >> 2)) ^ (r & 7)) << 2);
-}
 
 // ---- tc_intra shared memory (byte offsets from a 1024-aligned base) -----------
 constexpr int kIntraThreads = 256;
@@ -208,7 +192,8 @@ __global__ void __launch_bounds__(kIntraThreads, 2)
 tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
          const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ la,
          const __nv_bfloat16* __restrict__ beta, uint8_t* __restrict__ ws, int* __restrict__ err, ChunkMap cmap,
-         int H, unsigned prep_flags, unsigned long long stall_ns) {
+         int H, unsigned prep_flags, unsigned long long stall_ns, float* __restrict__ t_store,
+         float* __restrict__ at_store) {
     // PREP = false is the plain operator: no preprocessing code is compiled in
     const unsigned prep = PREP ? prep_flags : 0u;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -550,6 +535,14 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             if (!is_p) {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) As[r * kAS + i0 + e] = (i0 + e < r) ? br * vals[e] : 0.f;
+                if (at_store) {   // the backward pass: the key products before the beta scaling
+                    float* dst = at_store + ((size_t)chunk * H + h) * (kC * kC) + r * kC + i0;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) =
+                            make_float4((i0 + e < r) ? vals[e] : 0.f, (i0 + e + 1 < r) ? vals[e + 1] : 0.f,
+                                        (i0 + e + 2 < r) ? vals[e + 2] : 0.f, (i0 + e + 3 < r) ? vals[e + 3] : 0.f);
+                }
             } else {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) vals[e] = (i0 + e <= r) ? vals[e] : 0.f;
@@ -563,6 +556,11 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 if (!is_p) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) As[r * kAS + i + e] = 0.f;
+                    if (at_store) {
+                        float* dst = at_store + ((size_t)chunk * H + h) * (kC * kC) + r * kC + i;
+                        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4*>(dst + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
                 } else {
                     store8_split(sm + kPh, sm + kPl, sw128_chunk(r, i, 64), zero);
                 }
@@ -666,6 +664,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                     const int row = 16 * R + r, col = 16 * R + i;
                     if (!is_p) {
                         As[row * kAS + col] = (i < r && row < len) ? sbeta[row] * val : 0.f;
+                        if (at_store)
+                            at_store[((size_t)chunk * H + h) * (kC * kC) + row * kC + col] =
+                                (i < r && row < len) ? val : 0.f;
                     } else {
                         __nv_bfloat16 ph, pl;
                         split1(row < len ? val : 0.f, ph, pl);
@@ -745,6 +746,16 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         else
             tsolve_cols<4>(As, Ts, Yw, 2, 32 + 8 * (warp - 6), lane);
         __syncthreads();
+        // for the backward pass: T itself, fp32 [64][64] per (chunk, head)
+        if (t_store) {
+            float* dst = t_store + ((size_t)chunk * H + h) * (kC * kC);
+            for (int e = tid; e < kC * kC / 4; e += kIntraThreads) {
+                const int rr = e >> 4, c4 = (e & 15) * 4;
+                const float4 x = ((c4 >> 4) <= (rr >> 4)) ? *reinterpret_cast<const float4*>(Ts + rr * kTS + c4)
+                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(dst + rr * kC + c4) = x;
+            }
+        }
         // T (hi/lo) as a K-major tile; blocks above the diagonal are zero
         for (int e = tid; e < 64 * 8; e += kIntraThreads) {
             const int rr = e >> 3, k8 = (e & 7) * 8;
@@ -1314,7 +1325,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         kern<<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, prep, stall_intra_ns);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, prep, stall_intra_ns, nullptr, nullptr);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1339,7 +1350,7 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
 cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
                              int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
-                             float* Wk, cudaStream_t stream) {
+                             float* Wk, float* T_store, float* At_store, cudaStream_t stream) {
     int* err = reinterpret_cast<int*>(tc_ws);
     uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
@@ -1349,7 +1360,7 @@ cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const 
         if (e != cudaSuccess) return e;
         tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull, T_store, At_store);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         tc_unpack_u_wk<<<dim3(n_chunks, H), 256, 0, stream>>>(ws, U, Wk, cmap, H);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1380,7 +1391,7 @@ cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, c
         if (e != cudaSuccess) return e;
         tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull);
+            (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull, nullptr, nullptr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     timing_mark(stream, 1);

@@ -198,6 +198,7 @@ struct BwdWorkspace {
     float* Qg;          // [tokens, H, dk] q . exp(g)
     float* Kd;          // [tokens, H, dk] k . exp(g_C - g)
     void* tc_ws;        // tensor-core workspace for the recompute (bf16, d = 128), or null
+    float* T;           // [chunks, H, C, C] (I + A)^-1 from that recompute (tensor-core path only)
     void* o_scratch;    // outputs of that recompute [tokens, H, dv] bf16 (unused)
 };
 
@@ -210,7 +211,7 @@ cudaError_t launch_simt_g(kda_dtype dtype, const void* log_alpha, const ChunkMap
 cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
                              int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
-                             float* Wk, cudaStream_t stream);
+                             float* Wk, float* T_store, float* At_store, cudaStream_t stream);
 
 cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
                                  const void* log_alpha, const void* beta, const float* init_state,
@@ -221,6 +222,20 @@ cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, 
 
 // Tensor-core chunk-local products of the backward pass (bf16, d = 128):
 // dQg = dO S^T, dWk = -dW S^T, dKd = W dS'^T, dP = dO W^T, dGam = rowsum(dS' . S).
+// Tensor-core reverse chain of the backward pass (bf16, d = 128): from the
+// per-chunk images of the recompute, dW = Kd dS' + P^T dO and dS = Gamma dS' +
+// Qg^T dO - Wk^T dW per chunk, storing dS_chunk, dW and the initial-state gradient.
+cudaError_t launch_tc_chain(void* tc_ws, const void* d_o, const float* d_final, float* dS_chunk, float* dW,
+                            float* d_init, const SeqMap& smap, int n_seqs, int H, cudaStream_t stream);
+
+// Tensor-core back substitution of the backward pass (bf16, d = 128):
+// [Y | Z] = T^T [dW | dWk], dA = -(Y U^T + Z Wk^T) (i < r), dv = beta Y, dKg = beta Z,
+// dbeta_r = v_r.Y_r + Kg_r.Z_r + sum_i dA_ri At_ri, dAt = Diag(beta) dA.
+cudaError_t launch_kb_b_tc(const float* T, const float* At, const float* U, const float* Wk, const float* dW,
+                           const float* dWk, const void* k, const void* v, const void* beta, const float* g,
+                           const float* gl, void* dv_out, void* dbeta_out, float* dKg, float* dAt, int* err,
+                           const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream);
+
 cudaError_t launch_kb_a_tc(const void* d_o, const float* W, const float* dW, const float* S_chunk,
                            const float* dS_chunk, float* dQg, float* dKd, float* dWk, float* dGam, float* dP, int* err,
                            const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream);
