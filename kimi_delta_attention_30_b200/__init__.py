@@ -300,11 +300,24 @@ BWD_KERNELS_TC = ["k1_cumsum", "tc_intra", "tc_unpack_u_wk", "tc_recur", "kb_cha
 BWD_KERNELS = ["k1_cumsum", "k2_wy", "k3_state", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
 # the timing hook's marks of kda_chunk_bwd: start, recompute, kb_p, kb_chain, kb_a, kb_b, kb_c
 BWD_TIMED = ["recompute", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
+# the same marks on the tensor-core path, where nothing runs between the second and third
+# (None): the recompute already stored the key products and the chain reads P from its images
+BWD_TIMED_TC = ["recompute", None, "kb_chain_tc", "kb_a_tc", "kb_b_tc", "kb_c"]
+
+
+def _bwd_tc(dtype, dk, dv) -> bool:
+    return dtype == torch.bfloat16 and dk == 128 and dv == 128
 
 
 def bwd_kernels(dtype, dk, dv):
     """The kernels one kda_chunk_bwd call launches for this problem."""
-    return BWD_KERNELS_TC if (dtype == torch.bfloat16 and dk == 128 and dv == 128) else BWD_KERNELS
+    return BWD_KERNELS_TC if _bwd_tc(dtype, dk, dv) else BWD_KERNELS
+
+
+def bwd_timed(dtype, dk, dv):
+    """Labels of the intervals between kda_chunk_bwd's timing marks for this problem
+    (None where no kernel runs in the interval)."""
+    return BWD_TIMED_TC if _bwd_tc(dtype, dk, dv) else BWD_TIMED
 
 
 def bwd_workspace_size(B, T, H, dk, dv, C=64, cu_seqlens=None) -> int:

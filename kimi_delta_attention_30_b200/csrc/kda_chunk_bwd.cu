@@ -959,21 +959,23 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
     const size_t smem_p = sizeof(float) * 4 * (size_t)kPS * dk;
     const size_t smem_chain = sizeof(float) * ((size_t)dk * kBV + 2 * (size_t)C * dk + 2 * (size_t)C * kBV +
                                                (size_t)C * C + 2 * dk);
-    auto kern_p = dk == 128 ? kb_p<Tin, 128> : kb_p<Tin, 64>;
-    if ((e = cudaFuncSetAttribute(kern_p, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
-    if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
-        return e;
-    // two chain blocks per SM (115,712 bytes each at d = 128) need the whole shared-memory carveout
-    if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100))) return e;
-    // (the tensor-core path takes At from the recompute and P from its images, and
-    // kb_a_tc writes the whole dP buffer: no pairwise pass is needed here)
+    // the tensor-core path takes At from the recompute and P from its images, and kb_a_tc
+    // writes the whole dP buffer: no pairwise pass runs there
     const bool tc_chain = std::is_same<Tin, __nv_bfloat16>::value && dk == 128 && dv == 128 && ws.tc_ws;
-    if (n_chunks > 0 && !tc_chain)
-        kern_p<<<dim3(n_chunks, H), kPThreads, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg,
-                                                                 ws.Kd, cmap, H);
+    if (!tc_chain) {
+        auto kern_p = dk == 128 ? kb_p<Tin, 128> : kb_p<Tin, 64>;
+        if ((e = cudaFuncSetAttribute(kern_p, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_p))) return e;
+        if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_chain)))
+            return e;
+        // two chain blocks per SM (115,712 bytes each at d = 128) need the whole shared-memory carveout
+        if ((e = cudaFuncSetAttribute(kb_chain<Tin>, cudaFuncAttributePreferredSharedMemoryCarveout, 100))) return e;
+        if (n_chunks > 0)
+            kern_p<<<dim3(n_chunks, H), kPThreads, smem_p, stream>>>(q, k, ws.fwd.g, ws.fwd.gl, ws.P, ws.At, ws.Qg,
+                                                                     ws.Kd, cmap, H);
+    }
     timing_mark(stream, 2);
     if (n_seqs > 0) {
-        if (std::is_same<Tin, __nv_bfloat16>::value && dk == 128 && dv == 128 && ws.tc_ws) {
+        if (tc_chain) {
             // bf16, d = 128: the reverse chain on the tensor cores, from the recompute's images
             if ((e = launch_tc_chain(ws.tc_ws, d_o, d_final, ws.dS_chunk, ws.dW, d_init, smap, n_seqs, H, stream)) !=
                 cudaSuccess)
