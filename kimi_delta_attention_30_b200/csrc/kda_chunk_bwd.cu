@@ -932,8 +932,15 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
                                                 ws.dWk, dv_, dbeta, ws.dKg, ws.dAt, cmap, H, DK, dv, C);
     }
     timing_mark(stream, 5);
-    kb_c<Tin, DK><<<grid, kCThreads, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd,
-                                                     ws.dKg, ws.dGam, dq, dk_, dla, cmap, H);
+    if (std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && dv == 128 && ws.tc_ws) {
+        // bf16, d = 128: the pairwise terms as block-referenced tensor-core products
+        e = launch_kb_c_tc(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg, ws.dKd, ws.dKg, ws.dGam, dq, dk_, dla,
+                           reinterpret_cast<int*>(ws.tc_ws), cmap, n_chunks, H, stream);
+        if (e != cudaSuccess) return e;
+    } else {
+        kb_c<Tin, DK><<<grid, kCThreads, smem_c, stream>>>(q, k, la, ws.fwd.g, ws.fwd.gl, ws.dAt, ws.P, ws.dQg,
+                                                         ws.dKd, ws.dKg, ws.dGam, dq, dk_, dla, cmap, H);
+    }
     timing_mark(stream, 6);
     return cudaGetLastError();
 }

@@ -240,6 +240,14 @@ cudaError_t launch_kb_a_tc(const void* d_o, const float* W, const float* dW, con
                            const float* dS_chunk, float* dQg, float* dKd, float* dWk, float* dGam, float* dP, int* err,
                            const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream);
 
+// Tensor-core pairwise gradient terms of the backward pass (bf16, d = 128): from dAt,
+// dP (strictly lower parts in the products, dP's diagonal elementwise) and the
+// gradients of the elementwise factors, dq, dk and dlog alpha.
+cudaError_t launch_kb_c_tc(const void* q, const void* k, const void* la, const float* g, const float* gl,
+                           const float* dAt, const float* dP, const float* dQg, const float* dKd, const float* dKg,
+                           const float* dGam, void* dq, void* dk, void* dla, int* err, const ChunkMap& cmap,
+                           int n_chunks, int H, cudaStream_t stream);
+
 // A segment's affine map S_end = M S_start + F (M [N, H, dk, dk], F [N, H, dk, dv]).
 cudaError_t launch_tc_segment_map(const void* q, const void* k, const void* v, const void* log_alpha,
                                   const void* beta, const ChunkMap& cmap, const SeqMap& smap, int n_chunks,

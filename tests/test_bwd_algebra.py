@@ -148,3 +148,89 @@ def test_dlog_alpha_prefix_assembled_from_tiles():
             E[r, i] = 1.0
             want = ((i < j) & (j <= r)).astype(float)
             np.testing.assert_array_equal(tile_assembled_F(E), want, err_msg=f"pair ({r}, {i})")
+
+
+def tc_pairwise_terms(kk, qq, g, dAt, dP, L, range_max=80.0):
+    """The pairwise gradient stage as the tensor-core kernel forms it, in fp64, for
+    one 64-row chunk whose first L rows exist: X1, X2 (row sums) and Y (column sums)
+    of the strictly lower dAt and dP as block-referenced products (row block I's
+    keys scaled by e^{gb_I - g_i}, gb_I = g at row 16 I - 1 or 0; key block J's rows
+    scaled by e^{g_r - ge_J}, ge_J = g at row 16 J + 15; references clamped to the
+    last row), blocks spanning more than `range_max` nats summed pairwise, dP's
+    diagonal added elementwise, and F(j) = sum_{r >= j} D_r with
+    D_r = k_r X1_r + q_r X2_r - k_r Y_r (X2, Y without the diagonal)."""
+    C, dk = 64, kk.shape[1]
+    kp = np.zeros((C, dk)); kp[:L] = kk[:L]
+    qp = np.zeros((C, dk)); qp[:L] = qq[:L]
+    gp = np.vstack([g[:L], np.repeat(g[L - 1:L], C - L, axis=0)])
+    low = np.tril(np.ones((C, C)), -1)
+    A = np.zeros((C, C)); A[:L, :L] = dAt[:L, :L]; A *= low
+    Pm = np.zeros((C, C)); Pm[:L, :L] = dP[:L, :L]; Pm *= low
+    dPd = np.zeros(C); dPd[:L] = np.diag(dP)[:L]
+    ref = [gp[min(16 * j + 15, L - 1)] for j in range(4)]
+    gb = [np.zeros(dk)] + ref[:3]
+    flag = [np.max(gb[I] - ref[I]) > range_max for I in range(4)]
+    X1, X2, Y = np.zeros((C, dk)), np.zeros((C, dk)), np.zeros((C, dk))
+    for I in range(4):
+        rows, nk = slice(16 * I, 16 * I + 16), 16 * (I + 1)
+        KV = kp[:nk] * np.exp(gb[I][None, :] - gp[:nk])
+        if flag[I]:
+            KV[16 * I:] = 0.0
+        sc = np.exp(gp[rows] - gb[I][None, :])
+        X1[rows] = (A[rows, :nk] @ KV) * sc
+        X2[rows] = (Pm[rows, :nk] @ KV) * sc
+    for J in range(4):
+        keys, r0 = slice(16 * J, 16 * J + 16), 16 * J
+        f = np.exp(gp[r0:] - ref[J][None, :])
+        RK, RQ = kp[r0:] * f, qp[r0:] * f
+        if flag[J]:
+            RK[:16] = 0.0
+            RQ[:16] = 0.0
+        Y[keys] = (A[r0:, keys].T @ RK + Pm[r0:, keys].T @ RQ) * np.exp(ref[J][None, :] - gp[keys])
+    for I in range(4):
+        if not flag[I]:
+            continue
+        for x in range(16 * I + 1, 16 * I + 16):
+            for y in range(16 * I, x):
+                e = np.exp(gp[x] - gp[y])
+                X1[x] += A[x, y] * kp[y] * e
+                X2[x] += Pm[x, y] * kp[y] * e
+                Y[y] += (A[x, y] * kp[x] + Pm[x, y] * qp[x]) * e
+    D = kp * X1 + qp * X2 - kp * Y
+    F = np.cumsum(D[::-1], axis=0)[::-1]
+    return X1[:L], X2[:L] + dPd[:L, None] * kp[:L], Y[:L] + dPd[:L, None] * qp[:L], F[:L], flag
+
+
+@pytest.mark.parametrize("L,regime", [(64, "moderate"), (64, "near0"), (50, "mixed")])
+def test_tensor_core_pairwise_form_matches_the_pairs(L, regime):
+    """The block-referenced form of the pairwise gradient terms (versions and their
+    references, the diagonal of dP outside the products, the pairwise path of
+    large-range blocks, dlog alpha's pairwise share as a suffix sum of row sums
+    minus column sums) equals the direct pairwise sums in fp64.  The near-0 case
+    sends every diagonal block down the pairwise path; the mixed case one of them."""
+    rng = np.random.default_rng(L + len(regime))
+    dk = 8
+    kk = rng.standard_normal((L, dk))
+    qq = rng.standard_normal((L, dk))
+    if regime == "moderate":
+        la = -np.logaddexp(0.0, rng.standard_normal((L, dk)) + 2.0)
+    elif regime == "near0":
+        la = -8.0 - 8.0 * rng.random((L, dk))
+    else:
+        la = -np.logaddexp(0.0, rng.standard_normal((L, dk)) + 2.0)
+        la[16:32] = -8.0 - 8.0 * rng.random((16, dk))
+    g = np.cumsum(la, axis=0)
+    dAt = rng.standard_normal((L, L))
+    dP = rng.standard_normal((L, L))
+    X1, X2, Y, F, flag = tc_pairwise_terms(kk, qq, g, dAt, dP, L)
+    assert any(flag) == (regime != "moderate")
+    E = np.exp(np.minimum(g[:, None, :] - g[None, :, :], 0.0))
+    low, inc = np.tril(np.ones((L, L)), -1), np.tril(np.ones((L, L)))
+    A, P = dAt * low, dP * inc
+    np.testing.assert_allclose(X1, np.einsum('ri,ic,ric->rc', A, kk, E), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(X2, np.einsum('ri,ic,ric->rc', P, kk, E), rtol=1e-9, atol=1e-12)
+    Yd = np.einsum('ri,rc,ric->ic', A, kk, E) + np.einsum('ri,rc,ric->ic', P, qq, E)
+    np.testing.assert_allclose(Y, Yd, rtol=1e-9, atol=1e-12)
+    Tp = (A[:, :, None] * kk[:, None, :] + P[:, :, None] * qq[:, None, :]) * kk[None, :, :] * E
+    Fd = np.array([Tp[j:, :j].sum(axis=(0, 1)) for j in range(L)])
+    np.testing.assert_allclose(F, Fd, rtol=1e-8, atol=1e-10)
