@@ -575,30 +575,40 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     // factor is 2^(a - b) of two sums over at most 16 tokens).  Warp w forms the
     // 17 pairs (r, i <= r) of rows w and 15 - w, each lane over 4 channels; the 34
     // per-lane sums (A and P of each pair) are reduced across the warp by halving
-    // exchanges, after which lane l holds sum number l.
+    // exchanges, after which lane l holds sum number l.  (Splitting each pair's
+    // factor at a 4-row sub-block boundary, so that the exponentials are formed per
+    // row instead of per pair, measured slower: each key version serves about three
+    // pairs, so building the versions costs what the pairs save.)
     if (!abort && fbmask) {
         float* fk = reinterpret_cast<float*>(sm + kFbStage);   // [16][128] k
         float* fq = fk + 16 * 128;                              // [16][128] q
         float* fg = fq + 16 * 128;                              // [16][128] block-local g * log2 e
-        for (int R = 0; R < 4; ++R) {
-            if (!(fbmask & (1u << R))) continue;
+        // thread: one row, 8 consecutive channels of k, q and log alpha; the next
+        // flagged block's are loaded while the current one's pairs are formed
+        const int frow = tid >> 4, fc8 = (tid & 15) * 8;
+        uint4 nk8, nq8, nl8;
+        auto fetch = [&](int Rf) {
+            const int rr = 16 * Rf + frow;
+            nk8 = nq8 = nl8 = make_uint4(0u, 0u, 0u, 0u);
+            if (rr < len) {
+                const size_t off = ((size_t)(tok0 + rr) * H + h) * kD + fc8;
+                nk8 = *reinterpret_cast<const uint4*>(k + off);
+                nq8 = *reinterpret_cast<const uint4*>(q + off);
+                nl8 = *reinterpret_cast<const uint4*>(la + off);
+            }
+        };
+        int R = __ffs(fbmask) - 1;
+        fetch(R);
+        while (R < 4) {
             {
-                // thread: one row, 8 consecutive channels of k, q and log alpha
-                const int row = tid >> 4, c8 = (tid & 15) * 8, rr = 16 * R + row;
-                uint4 k8 = make_uint4(0u, 0u, 0u, 0u), q8 = k8, l8 = k8;
-                if (rr < len) {
-                    const size_t off = ((size_t)(tok0 + rr) * H + h) * kD + c8;
-                    k8 = *reinterpret_cast<const uint4*>(k + off);
-                    q8 = *reinterpret_cast<const uint4*>(q + off);
-                    l8 = *reinterpret_cast<const uint4*>(la + off);
-                }
+                const int rr = 16 * R + frow;
                 const float2 sk = PREP ? make_float2(inv_nk[rr], inv_nk[rr]) : make_float2(1.f, 1.f);
                 const float2 sq = PREP ? make_float2(inv_nq[rr], inv_nq[rr]) : make_float2(1.f, 1.f);
-                const uint32_t kw[4] = {k8.x, k8.y, k8.z, k8.w}, qw[4] = {q8.x, q8.y, q8.z, q8.w};
-                const uint32_t lw[4] = {l8.x, l8.y, l8.z, l8.w};
-                float* dk_ = fk + row * 128 + c8;
-                float* dq_ = fq + row * 128 + c8;
-                float* dg_ = fg + row * 128 + c8;
+                const uint32_t kw[4] = {nk8.x, nk8.y, nk8.z, nk8.w}, qw[4] = {nq8.x, nq8.y, nq8.z, nq8.w};
+                const uint32_t lw[4] = {nl8.x, nl8.y, nl8.z, nl8.w};
+                float* dk_ = fk + frow * 128 + fc8;
+                float* dq_ = fq + frow * 128 + fc8;
+                float* dg_ = fg + frow * 128 + fc8;
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     *reinterpret_cast<float2*>(dk_ + 2 * m) = mul2(unpack_bf16x2(kw[m]), sk);
@@ -607,6 +617,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                     *reinterpret_cast<float2*>(dg_ + 2 * m) = (rr < len) ? l2 : make_float2(0.f, 0.f);
                 }
             }
+            const unsigned rest = fbmask & ~((2u << R) - 1u);
+            const int Rn = rest ? __ffs(rest) - 1 : 4;
+            if (Rn < 4) fetch(Rn);
             __syncthreads();
             if (tid < 128) {
                 float acc = 0.f;
@@ -619,15 +632,22 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
             __syncthreads();
             {
                 const int ra = warp, rb = 15 - warp;
+                // the two rows' values, read once; the pairs select between them
+                const float4 gra = *reinterpret_cast<const float4*>(fg + ra * 128 + 4 * lane);
+                const float4 kra = *reinterpret_cast<const float4*>(fk + ra * 128 + 4 * lane);
+                const float4 qra = *reinterpret_cast<const float4*>(fq + ra * 128 + 4 * lane);
+                const float4 grb = *reinterpret_cast<const float4*>(fg + rb * 128 + 4 * lane);
+                const float4 krb = *reinterpret_cast<const float4*>(fk + rb * 128 + 4 * lane);
+                const float4 qrb = *reinterpret_cast<const float4*>(fq + rb * 128 + 4 * lane);
                 float v[34];
 #pragma unroll
                 for (int jj = 0; jj < 17; ++jj) {
                     const bool first = jj <= ra;
-                    const int r = first ? ra : rb, i = first ? jj : jj - ra - 1;
-                    const float4 gr = *reinterpret_cast<const float4*>(fg + r * 128 + 4 * lane);
+                    const int i = first ? jj : jj - ra - 1;
+                    const float4 gr = first ? gra : grb;
+                    const float4 kr = first ? kra : krb;
+                    const float4 qr = first ? qra : qrb;
                     const float4 gi = *reinterpret_cast<const float4*>(fg + i * 128 + 4 * lane);
-                    const float4 kr = *reinterpret_cast<const float4*>(fk + r * 128 + 4 * lane);
-                    const float4 qr = *reinterpret_cast<const float4*>(fq + r * 128 + 4 * lane);
                     const float4 ki = *reinterpret_cast<const float4*>(fk + i * 128 + 4 * lane);
                     // 2^(g_r - g_i) <= 1 (i <= r)
                     const float2 d0 = fma2(make_float2(gi.x, gi.y), make_float2(-1.f, -1.f), make_float2(gr.x, gr.y));
@@ -681,6 +701,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 }
             }
             __syncthreads();
+            R = Rn;
         }
     }
 
