@@ -566,26 +566,24 @@ def main():
             host = {n: getattr(hl_inp, n).to("cpu").pin_memory() for n in names}
             host["init_state"] = hl_inp.init_state.to("cpu").pin_memory()
             B, T, H, dk = hl_inp.q.shape
-            o = torch.empty(hl_inp.v.shape, dtype=hl_inp.v.dtype, device=dev)
-            fs = torch.empty(hl_inp.init_state.shape, dtype=torch.float32, device=dev)
-            o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-            fs_h = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-            ws = torch.empty(kda.workspace_size(B, T, H, dk, dk, 64, torch.bfloat16, cu_seqlens=hl_inp.cu_seqlens),
-                             dtype=torch.uint8, device=dev)
+            o_h = torch.empty(hl_inp.v.shape, dtype=hl_inp.v.dtype).pin_memory()
+            fs_h = torch.empty(hl_inp.init_state.shape, dtype=torch.float32).pin_memory()
+            # the device copies of the inputs are not needed for this part
+            for n in names:
+                setattr(hl_inp, n, None)
+            hl_inp.init_state = None
+            torch.cuda.empty_cache()
+            e2e_groups = 8
+            buf = torch.empty(kda.host_buffer_size(hl_inp.cu_seqlens, H, dk, dk, 64, torch.bfloat16, e2e_groups),
+                              dtype=torch.uint8, device=dev)
             h2d = sum(t.numel() * t.element_size() for t in host.values())
             d2h = o_h.numel() * o_h.element_size() + fs_h.numel() * fs_h.element_size()
             e2e_steps = max(3, min(a.steps, 10))
 
             def e2e_step():
-                # the device buffers of the inputs are overwritten with the same values
-                for n in names:
-                    getattr(hl_inp, n).copy_(host[n], non_blocking=True)
-                hl_inp.init_state.copy_(host["init_state"], non_blocking=True)
-                kda.chunk_fwd(hl_inp.q, hl_inp.k, hl_inp.v, hl_inp.log_alpha, hl_inp.beta,
-                              init_state=hl_inp.init_state, cu_seqlens=hl_inp.cu_seqlens, C=64, o=o,
-                              final_state=fs, workspace=ws)
-                o_h.copy_(o, non_blocking=True)
-                fs_h.copy_(fs, non_blocking=True)
+                kda.chunk_fwd_host(host["q"], host["k"], host["v"], host["log_alpha"], host["beta"],
+                                   hl_inp.cu_seqlens, init_state=host["init_state"], C=64, o=o_h, final_state=fs_h,
+                                   n_groups=e2e_groups, device_buffer=buf, stream=stream, synchronize=False)
 
             for _ in range(a.warmup):
                 e2e_step()
@@ -601,8 +599,11 @@ def main():
             et = max_over_ranks(e0.elapsed_time(e1))
             e2e = {"value": job_throughput(world, sum(lengths), e2e_steps, et), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": et / e2e_steps,
-                   "steps": e2e_steps, "path": "kda_chunk_fwd (public API) with pinned host buffers"}
-            del host, o_h, fs_h, ws, o, fs
+                   "steps": e2e_steps, "n_groups": e2e_groups,
+                   "path": "kda_chunk_fwd_host (public API): pinned host buffers in, the packed batch in "
+                           f"{e2e_groups} groups of sequences whose copies both ways overlap the kernels, "
+                           "pinned host buffers out"}
+            del host, o_h, fs_h, buf
     if hl_inp is not None:
         del hl_inp
     torch.cuda.empty_cache()

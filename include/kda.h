@@ -152,6 +152,51 @@ KDA_API kda_status kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                             size_t workspace_bytes, void* stream, kda_algo algo);
 
 /*
+ * Prefill of a packed batch held in HOST memory, with the transfers overlapped
+ * with the computation.  The sequences are taken in `n_groups` groups of
+ * consecutive sequences with about equal token counts; while group g is
+ * computed (on `stream`), group g + 1's inputs are copied to the device and
+ * group g - 1's outputs back to the host, on two streams of the library's own,
+ * so that both copy directions and the kernels run at once.  Each group is one
+ * kda_chunk_fwd call on device staging inside `device_buffer`, so every output
+ * equals, bit for bit, the device call's on the whole batch (a sequence's
+ * result does not depend on the other sequences).  This is the library's
+ * transfer pipeline around the operation, not part of the pages' method.
+ *
+ *   q, k, v, log_alpha, beta : HOST inputs, layouts as kda_chunk_fwd with B = 1;
+ *                     page-locked memory (cudaHostAlloc / cudaHostRegister) lets
+ *                     the copies overlap; pageable memory works, serialised
+ *   init_state      : HOST [N, H, dk, dv] fp32, or NULL for zero states
+ *   cu_seqlens_host : HOST n_seqs + 1 int32 offsets (as kda_chunk_fwd; required)
+ *   o               : HOST output [1, T, H, dv], dtype `dtype`
+ *   final_state     : HOST [N, H, dk, dv] fp32, or NULL
+ *   n_groups        : >= 1; more groups overlap more but each call costs a
+ *                     launch sequence (8 suits batches of ~10^6 tokens); values
+ *                     above n_seqs act as n_seqs
+ *   device_buffer   : device scratch of kda_chunk_fwd_host_buffer_size() bytes
+ *                     (same sizes and n_groups), 256-byte aligned; ownership
+ *                     stays with the caller, contents on entry are ignored
+ *   stream          : cudaStream_t (as void*): the call's work starts after the
+ *                     work already on `stream`, and `stream` waits for all of it
+ *                     (copies back included); the call returns without waiting,
+ *                     so the host buffers must stay valid until `stream` is done
+ * Errors: as kda_chunk_fwd (KDA_ERR_SEQLENS for a NULL cu_seqlens_host,
+ * KDA_ERR_WORKSPACE for a short device_buffer), KDA_ERR_CUDA if a stream, event
+ * or copy cannot be made.  A bounded device wait that expired in any group is
+ * reported by kda_chunk_fwd_host_device_status.
+ */
+KDA_API size_t kda_chunk_fwd_host_buffer_size(kda_dtype dtype, const int32_t* cu_seqlens_host, int n_seqs,
+                                              int H, int dk, int dv, int C, int n_groups);
+KDA_API kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const void* log_alpha,
+                                      const void* beta, kda_dtype dtype, const float* init_state,
+                                      const int32_t* cu_seqlens_host, int n_seqs, int H, int dk, int dv,
+                                      int C, void* o, float* final_state, int n_groups, void* device_buffer,
+                                      size_t device_buffer_bytes, void* stream);
+/* Synchronises `stream`; KDA_OK, or the first error a group's kernels recorded
+ * (KDA_ERR_TIMEOUT) in the last kda_chunk_fwd_host call that used device_buffer. */
+KDA_API kda_status kda_chunk_fwd_host_device_status(const void* device_buffer, void* stream);
+
+/*
  * Byte offsets, inside the workspace of the SIMT algorithm, of the
  * intermediates that its four kernels exchange (for inspection by tests):
  *   offsets[0] g       fp32 [T_total, H, dk]  chunk-local inclusive cumulative log decay

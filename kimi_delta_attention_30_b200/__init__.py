@@ -96,6 +96,13 @@ def _declare(lib):
     lib.kda_compose_states.restype = c_int
     lib.kda_set_test_wait_limit.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
     lib.kda_set_test_wait_limit.restype = c_int
+    lib.kda_chunk_fwd_host_buffer_size.argtypes = [c_int, i32p, c_int] + [c_int] * 5
+    lib.kda_chunk_fwd_host_buffer_size.restype = c_size
+    lib.kda_chunk_fwd_host.argtypes = [vp] * 5 + [c_int, vp, i32p, c_int] + [c_int] * 4 + [vp, vp, c_int, vp,
+                                                                                          c_size, vp]
+    lib.kda_chunk_fwd_host.restype = c_int
+    lib.kda_chunk_fwd_host_device_status.argtypes = [vp, vp]
+    lib.kda_chunk_fwd_host_device_status.restype = c_int
     return lib
 
 
@@ -130,7 +137,8 @@ def exported_symbols():
             "kda_chunk_fwd_noalloc", "kda_chunk_fwd_prep", "kda_decode_step_prep", "kda_chunk_bwd_workspace_size",
             "kda_chunk_bwd", "kda_chunk_fwd_device_status", "kda_chunk_bwd_device_status",
             "kda_chunk_fwd_noalloc_device_status", "kda_chunk_segment_map", "kda_compose_states",
-            "kda_set_test_wait_limit"]
+            "kda_set_test_wait_limit", "kda_chunk_fwd_host_buffer_size", "kda_chunk_fwd_host",
+            "kda_chunk_fwd_host_device_status"]
 
 
 def _ptr(t):
@@ -291,6 +299,82 @@ def chunk_fwd(q, k, v, log_alpha, beta, init_state=None, cu_seqlens=None, C: int
     if st != 0:
         raise KdaError(st, what)
     return o, final_state
+
+
+def host_buffer_size(cu_seqlens, H, dk, dv, C: int = 64, dtype=torch.bfloat16, n_groups: int = 8) -> int:
+    """Device bytes chunk_fwd_host needs for this batch (kda_chunk_fwd_host_buffer_size)."""
+    cu, n, _keep = _cu_arg(cu_seqlens)
+    return int(lib().kda_chunk_fwd_host_buffer_size(_DTYPES[dtype], cu, n, H, dk, dv, C, n_groups))
+
+
+def _check_host(name, t, dtype=None):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def chunk_fwd_host(q, k, v, log_alpha, beta, cu_seqlens, init_state=None, C: int = 64, o=None,
+                   final_state=None, output_final_state: bool = True, n_groups: int = 8, device_buffer=None,
+                   device=None, stream=None, synchronize: bool = True):
+    """Prefill of a packed batch held in host memory (``kda_chunk_fwd_host``):
+    the library copies group after group of sequences to the device, computes
+    them and copies the results back, with the copies of neighbouring groups
+    overlapping the computation.
+
+    q, k, log_alpha ``[1, T, H, dk]``, v ``[1, T, H, dv]``, beta ``[1, T, H]``:
+    CPU tensors of one dtype (page-locked for the copies to overlap);
+    ``cu_seqlens`` host offsets (N + 1); ``init_state`` CPU ``[N, H, dk, dv]``
+    fp32 or None.  Returns CPU ``(o, final_state)``.  With ``synchronize`` the
+    call waits for the stream, so the results are ready; without it the caller
+    must keep every tensor alive and wait for ``stream`` before reading them.
+    """
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("log_alpha", log_alpha), ("beta", beta)):
+        _check_host(name, t, dt)
+    if cu_seqlens is None:
+        raise ValueError("chunk_fwd_host takes a packed batch: cu_seqlens is required")
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu, n_seqs, _keep = _cu_arg(cu_seqlens)
+    _check_host("init_state", init_state, torch.float32)
+    if o is None:
+        o = torch.empty((1, T, H, dv), dtype=dt).pin_memory()
+    if final_state is None and output_final_state:
+        final_state = torch.empty((n_seqs, H, dk, dv), dtype=torch.float32).pin_memory()
+    _check_host("o", o, dt)
+    _check_host("final_state", final_state, torch.float32)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with _launch_on(dev, stream, (("device_buffer", device_buffer),)) as (s, allocated):
+        need = lib().kda_chunk_fwd_host_buffer_size(_DTYPES[dt], cu, n_seqs, H, dk, dv, C, n_groups)
+        if device_buffer is None:
+            device_buffer = torch.empty(max(int(need), 256), dtype=torch.uint8, device=dev)
+            allocated.append(device_buffer)
+        _check_cuda("device_buffer", device_buffer)
+        st = lib().kda_chunk_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), log_alpha.data_ptr(),
+                                      beta.data_ptr(), _DTYPES[dt],
+                                      init_state.data_ptr() if init_state is not None else None, cu, n_seqs, H,
+                                      dk, dv, C, o.data_ptr(), final_state.data_ptr() if final_state is not None
+                                      else None, int(n_groups), _ptr(device_buffer),
+                                      device_buffer.numel() * device_buffer.element_size(), _stream_handle(s))
+        if st == 0 and synchronize:
+            s.synchronize()
+    if st != 0:
+        raise KdaError(st, "kda_chunk_fwd_host")
+    return o, final_state
+
+
+def host_device_status(device_buffer, stream=None) -> int:
+    """kda_chunk_fwd_host_device_status: 0, or the error a bounded device wait
+    recorded during the last chunk_fwd_host call that used ``device_buffer``."""
+    with _launch_on(device_buffer.device, stream, ()) as (s, _allocated):
+        return int(lib().kda_chunk_fwd_host_device_status(_ptr(device_buffer), _stream_handle(s)))
 
 
 # kernels of one kda_chunk_bwd call: the recompute (bf16 with d = 128: k1 and the tensor-core

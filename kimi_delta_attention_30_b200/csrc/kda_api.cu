@@ -641,3 +641,222 @@ kda_status kda_decode_step_prep(const void* q, const void* k, const void* v, con
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// kda_chunk_fwd_host: the prefill of a host-resident packed batch, in groups of
+// sequences whose copies overlap the computation of their neighbours.
+// ---------------------------------------------------------------------------
+namespace kda {
+// The first error a group's kernels recorded, kept in the host buffer's status word.
+__global__ void accumulate_status(const int* __restrict__ word, int* __restrict__ acc) {
+    const int w = *word;
+    if (w != 0) atomicCAS(acc, 0, w);
+}
+}  // namespace kda
+
+namespace {
+
+struct HostGroup {
+    int s0, s1;   // sequences [s0, s1)
+};
+
+// Consecutive sequences in groups of about equal token counts (at most n_groups,
+// none empty of sequences).
+std::vector<HostGroup> host_groups(const int32_t* cu, int n_seqs, int n_groups) {
+    std::vector<HostGroup> g;
+    const int G = std::max(1, std::min(n_groups, n_seqs));
+    const long long T = cu[n_seqs];
+    int s0 = 0;
+    for (int i = 0; i < G && s0 < n_seqs; ++i) {
+        int s1;
+        if (i == G - 1) {
+            s1 = n_seqs;
+        } else {
+            const long long target = T * (i + 1) / G;
+            s1 = s0 + 1;
+            while (s1 < n_seqs - (G - 1 - i) && cu[s1] < target) ++s1;
+        }
+        g.push_back(HostGroup{s0, s1});
+        s0 = s1;
+    }
+    return g;
+}
+
+// Device buffer: [status word][workspace][slot 0][slot 1]; a slot holds one group's
+// q, k, log alpha, v, beta, initial states, o and final states.
+struct HostLayout {
+    size_t ws_off = 0, ws_bytes = 0, slot_off[2] = {0, 0}, total = 0;
+    size_t q = 0, k = 0, la = 0, v = 0, beta = 0, init = 0, o = 0, fin = 0;   // offsets inside a slot
+};
+
+kda_status host_layout(kda_dtype dtype, const int32_t* cu, int n_seqs, int H, int dk, int dv, int C,
+                       const std::vector<HostGroup>& groups, HostLayout& L) {
+    const size_t es = dtype == KDA_BF16 ? 2 : 4;
+    long long max_tok = 0, max_seq = 0;
+    size_t ws = 0;
+    for (const HostGroup& g : groups) {
+        const int ns = g.s1 - g.s0;
+        std::vector<int32_t> cg(ns + 1);
+        for (int i = 0; i <= ns; ++i) cg[i] = cu[g.s0 + i] - cu[g.s0];
+        const size_t w = kda_chunk_fwd_workspace_size(1, cg[ns], H, dk, dv, C, dtype, cg.data(), ns);
+        if (w == 0) return KDA_ERR_SHAPE;
+        ws = std::max(ws, w);
+        max_tok = std::max<long long>(max_tok, cg[ns]);
+        max_seq = std::max<long long>(max_seq, ns);
+    }
+    const size_t tok = (size_t)max_tok * H, st = (size_t)max_seq * H * dk * dv * sizeof(float);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes);
+        return at;
+    };
+    L.q = take(tok * dk * es);
+    L.k = take(tok * dk * es);
+    L.la = take(tok * dk * es);
+    L.v = take(tok * dv * es);
+    L.beta = take(tok * es);
+    L.init = take(st);
+    L.o = take(tok * dv * es);
+    L.fin = take(st);
+    L.ws_off = kAlign;
+    L.ws_bytes = ws;
+    L.slot_off[0] = align_up(L.ws_off + ws);
+    L.slot_off[1] = L.slot_off[0] + o;
+    L.total = L.slot_off[1] + o;
+    return KDA_OK;
+}
+
+// Streams and events of one call; destroyed when the call returns (the runtime
+// releases them once the work queued on them has finished).
+struct HostStreams {
+    cudaStream_t in = nullptr, out = nullptr;
+    std::vector<cudaEvent_t> ev;
+    ~HostStreams() {
+        for (cudaEvent_t e : ev) cudaEventDestroy(e);
+        if (in) cudaStreamDestroy(in);
+        if (out) cudaStreamDestroy(out);
+    }
+    cudaError_t make(int n_events) {
+        cudaError_t e;
+        if ((e = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        ev.assign(n_events, nullptr);
+        for (cudaEvent_t& x : ev)
+            if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) return e;
+        return cudaSuccess;
+    }
+};
+
+cudaError_t copy_async(void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, cudaStream_t s) {
+    return bytes ? cudaMemcpyAsync(dst, src, bytes, kind, s) : cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_chunk_fwd_host_buffer_size(kda_dtype dtype, const int32_t* cu_seqlens_host, int n_seqs, int H, int dk,
+                                      int dv, int C, int n_groups) {
+    if ((dtype != KDA_BF16 && dtype != KDA_F32) || !cu_seqlens_host || n_groups < 1) return 0;
+    Plan p;
+    if (make_plan(1, cu_seqlens_host[n_seqs >= 1 ? n_seqs : 0], H, dk, dv, C, cu_seqlens_host, n_seqs, p) != KDA_OK)
+        return 0;
+    HostLayout L;
+    if (host_layout(dtype, cu_seqlens_host, n_seqs, H, dk, dv, C, host_groups(cu_seqlens_host, n_seqs, n_groups), L) !=
+        KDA_OK)
+        return 0;
+    return L.total;
+}
+
+kda_status kda_chunk_fwd_host(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
+                              kda_dtype dtype, const float* init_state, const int32_t* cu_seqlens_host, int n_seqs,
+                              int H, int dk, int dv, int C, void* o, float* final_state, int n_groups,
+                              void* device_buffer, size_t device_buffer_bytes, void* stream) {
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_DTYPE;
+    if (!cu_seqlens_host || n_seqs < 1) return KDA_ERR_SEQLENS;
+    if (n_groups < 1) return KDA_ERR_SHAPE;
+    const int T = cu_seqlens_host[n_seqs];
+    Plan p;
+    kda_status st = make_plan(1, T, H, dk, dv, C, cu_seqlens_host, n_seqs, p);
+    if (st != KDA_OK) return st;
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
+    if (!device_buffer) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(device_buffer) & (kAlign - 1)) != 0) return KDA_ERR_ALIGN;
+    const std::vector<HostGroup> groups = host_groups(cu_seqlens_host, n_seqs, n_groups);
+    HostLayout L;
+    if ((st = host_layout(dtype, cu_seqlens_host, n_seqs, H, dk, dv, C, groups, L)) != KDA_OK) return st;
+    if (device_buffer_bytes < L.total) return KDA_ERR_WORKSPACE;
+    if ((st = check_device()) != KDA_OK) return st;
+
+    const size_t es = dtype == KDA_BF16 ? 2 : 4;
+    const size_t sb = (size_t)H * dk * dv * sizeof(float);
+    const int G = (int)groups.size();
+    cudaStream_t s = (cudaStream_t)stream;
+    char* buf = (char*)device_buffer;
+    HostStreams hs;
+    // events: start, then per group: inputs in, computed, outputs out
+    if (hs.make(1 + 3 * G) != cudaSuccess) return KDA_ERR_CUDA;
+    cudaEvent_t ev0 = hs.ev[0];
+    auto ev_in = [&](int g) { return hs.ev[1 + 3 * g]; };
+    auto ev_comp = [&](int g) { return hs.ev[2 + 3 * g]; };
+    auto ev_out = [&](int g) { return hs.ev[3 + 3 * g]; };
+    const bool tc = resolve(KDA_ALGO_AUTO, dtype, dk, dv, C) == KDA_ALGO_TC;
+
+    cudaError_t e = cudaMemsetAsync(buf, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaEventRecord(ev0, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.in, ev0, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.out, ev0, 0);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    for (int g = 0; g < G; ++g) {
+        const int s0 = groups[g].s0, ns = groups[g].s1 - s0;
+        const long long t0 = cu_seqlens_host[s0], nt = cu_seqlens_host[s0 + ns] - t0;
+        char* sl = buf + L.slot_off[g & 1];
+        const size_t tk = (size_t)nt * H, ok = (size_t)t0 * H;
+        // inputs, once the computation that last read this slot is done
+        if (g >= 2) e = cudaStreamWaitEvent(hs.in, ev_comp(g - 2), 0);
+        if (e == cudaSuccess) e = copy_async(sl + L.q, (const char*)q + ok * dk * es, tk * dk * es, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess) e = copy_async(sl + L.k, (const char*)k + ok * dk * es, tk * dk * es, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess)
+            e = copy_async(sl + L.la, (const char*)log_alpha + ok * dk * es, tk * dk * es, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess) e = copy_async(sl + L.v, (const char*)v + ok * dv * es, tk * dv * es, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess) e = copy_async(sl + L.beta, (const char*)beta + ok * es, tk * es, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess && init_state)
+            e = copy_async(sl + L.init, init_state + (size_t)s0 * H * dk * dv, (size_t)ns * sb, cudaMemcpyHostToDevice, hs.in);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in(g), hs.in);
+        // the computation, once the inputs are in and this slot's previous outputs are out
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in(g), 0);
+        if (e == cudaSuccess && g >= 2) e = cudaStreamWaitEvent(s, ev_out(g - 2), 0);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+        std::vector<int32_t> cg(ns + 1);
+        for (int i = 0; i <= ns; ++i) cg[i] = cu_seqlens_host[s0 + i] - (int32_t)t0;
+        st = chunk_fwd_impl(sl + L.q, sl + L.k, sl + L.v, sl + L.la, sl + L.beta, dtype, 0u,
+                            init_state ? (const float*)(sl + L.init) : nullptr, cg.data(), ns, 1, (int)nt, H, dk, dv,
+                            C, sl + L.o, final_state ? (float*)(sl + L.fin) : nullptr, buf + L.ws_off, L.ws_bytes,
+                            stream, KDA_ALGO_AUTO);
+        if (st != KDA_OK) return st;
+        if (tc && ns > 0) {
+            Plan pg;
+            if ((st = make_plan(1, (int)nt, H, dk, dv, tc_chunk(), cg.data(), ns, pg)) != KDA_OK) return st;
+            accumulate_status<<<1, 1, 0, s>>>((const int*)(buf + L.ws_off + table_bytes(pg)), (int*)buf);
+            if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+        }
+        if ((e = cudaEventRecord(ev_comp(g), s)) != cudaSuccess) return KDA_ERR_CUDA;
+        // the outputs, once computed
+        e = cudaStreamWaitEvent(hs.out, ev_comp(g), 0);
+        if (e == cudaSuccess) e = copy_async((char*)o + ok * dv * es, sl + L.o, tk * dv * es, cudaMemcpyDeviceToHost, hs.out);
+        if (e == cudaSuccess && final_state)
+            e = copy_async(final_state + (size_t)s0 * H * dk * dv, sl + L.fin, (size_t)ns * sb, cudaMemcpyDeviceToHost, hs.out);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out(g), hs.out);
+        if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    // the caller's stream ends after the last copy back (the output stream runs in order)
+    return cudaStreamWaitEvent(s, ev_out(G - 1), 0) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_chunk_fwd_host_device_status(const void* device_buffer, void* stream) {
+    if (!device_buffer) return KDA_ERR_NULL;
+    return read_error_word(device_buffer, 0, stream);
+}
+
+}  // extern "C"

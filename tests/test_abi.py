@@ -261,3 +261,42 @@ def test_test_wait_limit_arguments():
     assert lib.kda_set_test_wait_limit(2, 2_000_000_000) == E_SHAPE  # above one second
     assert lib.kda_set_test_wait_limit(3, 1000) == OK
     assert lib.kda_set_test_wait_limit(0, 0) == OK                  # disarm
+
+
+def _host_call(cu=(0, 100, 300, 700), n_groups=3, buf=0x100000, bufb=1 << 40, dtype=0, H=2, dk=128, dv=128):
+    lib = kda.lib()
+    vp = ctypes.c_void_p
+    cua = None if cu is None else (ctypes.c_int32 * len(cu))(*cu)
+    n = 0 if cu is None else len(cu) - 1
+    args = [vp(0x10000)] * 5
+    return lib.kda_chunk_fwd_host(*args, dtype, None, cua, n, H, dk, dv, 64, vp(0x20000), None, n_groups,
+                                  None if buf is None else vp(buf), bufb, None)
+
+
+def test_host_pipeline_buffer_size_and_rejections():
+    """kda_chunk_fwd_host_buffer_size / kda_chunk_fwd_host check their arguments on
+    the host: the buffer holds at least one workspace for the largest group and two
+    staging slots, and shrinks as the batch is cut into more groups."""
+    lib = kda.lib()
+    cu = [0, 1000, 2000, 3000, 4000, 5000, 6000, 7000, 8000]
+    cua = (ctypes.c_int32 * len(cu))(*cu)
+    H, d = 4, 128
+    one = lib.kda_chunk_fwd_host_buffer_size(0, cua, 8, H, d, d, 64, 1)
+    four = lib.kda_chunk_fwd_host_buffer_size(0, cua, 8, H, d, d, 64, 4)
+    eight = lib.kda_chunk_fwd_host_buffer_size(0, cua, 8, H, d, d, 64, 8)
+    whole = lib.kda_chunk_fwd_workspace_size(1, 8000, H, d, d, 64, 0, cua, 8)
+    io = 8000 * H * d * 2 * 5 + 8000 * H * 2 + 2 * 8 * H * d * d * 4   # q k log_alpha v o, beta, states
+    assert one >= whole + 2 * io
+    assert one > four > eight > 0
+    assert lib.kda_chunk_fwd_host_buffer_size(0, None, 8, H, d, d, 64, 4) == 0
+    assert lib.kda_chunk_fwd_host_buffer_size(0, cua, 8, H, d, d, 64, 0) == 0
+    assert lib.kda_chunk_fwd_host_buffer_size(5, cua, 8, H, d, d, 64, 4) == 0
+    # rejections before anything touches a device
+    assert _host_call(cu=None) == E_SEQ
+    assert _host_call(cu=(0, 100, 50)) == E_SEQ
+    assert _host_call(n_groups=0) == E_SHAPE
+    assert _host_call(dtype=5) == E_DTYPE
+    assert _host_call(buf=None) == E_WS
+    assert _host_call(bufb=1024) == E_WS
+    assert _host_call(buf=0x100010) == E_ALIGN
+    assert lib.kda_chunk_fwd_host_device_status(None, None) == E_NULL
