@@ -213,7 +213,6 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     uint32_t* sflags = reinterpret_cast<uint32_t*>(inv_nq + 64);      // [0] fallback mask, [1] abort, [2] tmem base
     uint64_t& mbar = reinterpret_cast<uint64_t*>(sm + kIntraBars)[0];      // tensor-core products, in issue order
     uint64_t& mbar_k = reinterpret_cast<uint64_t*>(sm + kIntraBars)[1];    // the second half of the last product
-    uint64_t& mbar_la = reinterpret_cast<uint64_t*>(sm + kIntraBars)[2];   // log alpha rows landed
     uint64_t& mbar_never = reinterpret_cast<uint64_t*>(sm + kIntraBars)[3];  // completed by nothing (failure test)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -235,7 +234,6 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         sflags[1] = 0;
         mbar_init(&mbar, 1);
         mbar_init(&mbar_k, 1);
-        mbar_init(&mbar_la, 64);
         mbar_init(&mbar_never, 1);
         mbar_init_fence();
     }
@@ -244,14 +242,14 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         tmem_relinquish();
     }
     __syncthreads();   // barriers initialised
-    // log alpha rows by the bulk-copy engine (one 256-byte row per thread of the first two warps)
-    if (tid < 64) {
-        if (tid < len) {
-            mbar_arrive_expect_tx(&mbar_la, 256);
-            bulk_g2s(sm + kLaStage + tid * 256, la + ((size_t)(tok0 + tid) * H + h) * kD, 256, &mbar_la);
-        } else {
-            mbar_arrive(&mbar_la);
-        }
+    // log alpha rows by plain 16-byte loads (thread: 4 pieces of 8 channels), staged below;
+    // the SM's bulk-copy engine is busy with the other CTA's workspace stores
+    uint4 la_pc[4];
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int e = tid + 256 * it, r = e >> 4, c8 = (e & 15) * 8;
+        la_pc[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (r < len) la_pc[it] = *reinterpret_cast<const uint4*>(la + ((size_t)(tok0 + r) * H + h) * kD + c8);
     }
     // key / query rows for the normalisation, read row-wise (coalesced) before anything
     // waits: warp w takes rows 16 (w % 4) .. + 15 of k (w < 4) or q (w >= 4), lane l
@@ -324,10 +322,12 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     } else if (PREP && tid < 128) {
         inv_nk[tid] = 1.f;   // inv_nk [0, 64) and inv_nq [64, 128) are adjacent
     }
-    if (!mbar_wait(&mbar_la, 0)) {
-        record_error(err, KDA_ERR_TIMEOUT);
-        atomicExch(&sflags[1], 1u);
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int e = tid + 256 * it, r = e >> 4, c8 = (e & 15) * 8;
+        *reinterpret_cast<uint4*>(sm + kLaStage + r * 256 + c8 * 2) = la_pc[it];
     }
+    __syncthreads();
     // test of the failure path (stall_ns != 0, set through kda_set_test_wait_limit):
     // the first CTA waits, bounded by stall_ns, on a barrier that nothing completes,
     // then records the timeout and takes the abort path like any expired wait
