@@ -573,7 +573,7 @@ def main():
                 setattr(hl_inp, n, None)
             hl_inp.init_state = None
             torch.cuda.empty_cache()
-            e2e_groups = 8
+            e2e_groups = 16
             buf = torch.empty(kda.host_buffer_size(hl_inp.cu_seqlens, H, dk, dk, 64, torch.bfloat16, e2e_groups),
                               dtype=torch.uint8, device=dev)
             h2d = sum(t.numel() * t.element_size() for t in host.values())
