@@ -68,3 +68,17 @@ def test_host_pipeline_without_initial_or_final_state():
     o_ref, _ = kda.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], init_state=None,
                              cu_seqlens=inp.cu_seqlens, C=64)
     assert torch.equal(o, o_ref.cpu())
+
+
+def test_host_pipeline_from_pageable_memory():
+    """Pageable (not page-locked) host tensors work too: the copies then do not
+    overlap, the results are the same."""
+    inp = make_prefill(replace(WORKLOADS["varlen"], H=2), seed=11, lengths=[130, 64, 1, 500])
+    q, k, v, la, b = (getattr(inp, n).contiguous() for n in ("q", "k", "v", "log_alpha", "beta"))
+    assert not q.is_pinned()
+    o, fs = kda.chunk_fwd_host(q, k, v, la, b, inp.cu_seqlens, init_state=inp.init_state.contiguous(), C=64,
+                               n_groups=3, o=torch.empty(v.shape, dtype=v.dtype),
+                               final_state=torch.empty(inp.init_state.shape, dtype=torch.float32))
+    o_ref, fs_ref = _device_call(inp)
+    assert torch.equal(o, o_ref)
+    assert torch.equal(fs, fs_ref)
