@@ -1226,10 +1226,15 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         }
         if (!mbar_wait(bar_s, par)) fail();
         tc_fence_after();
-        __syncthreads();   // every thread is past its reads of this chunk's U stage
-        if (tid == 0) {
-            if (n + 1 < nch) load_kdt(n + 1);          // the S update is done with Kd^T
-            if (n + 2 < nch) load_uu(n + 2, stage);
+        if (sp < 2) {
+            // the W warps are past their reads of this chunk's U stage (the other warps
+            // read only its Gamma, before the barrier ahead of this chunk's first
+            // product), so the output warps do not hold the chain up here
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (tid == 0) {
+                if (n + 1 < nch) load_kdt(n + 1);          // the S update is done with Kd^T
+                if (n + 2 < nch) load_uu(n + 2, stage);
+            }
         }
         {
             float t[NG][16];
