@@ -380,8 +380,7 @@ def host_device_status(device_buffer, stream=None) -> int:
 # kernels of one kda_chunk_bwd call: the recompute (bf16 with d = 128: k1 and the tensor-core
 # forward with its states, T and the key products stored; otherwise the CUDA-core k1-k3),
 # then the gradient kernels (bf16 with d = 128: all four on the tensor cores)
-BWD_KERNELS_TC = ["k1_cumsum", "tc_intra", "tc_unpack_u_wk", "tc_recur", "kb_chain_tc", "kb_a_tc", "kb_b_tc",
-                  "kb_c_tc"]
+BWD_KERNELS_TC = ["k1_cumsum", "tc_intra", "tc_recur", "kb_chain_tc", "kb_a_tc", "kb_b_tc", "kb_c_tc"]
 BWD_KERNELS = ["k1_cumsum", "k2_wy", "k3_state", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]
 # the timing hook's marks of kda_chunk_bwd: start, recompute, kb_p, kb_chain, kb_a, kb_b, kb_c
 BWD_TIMED = ["recompute", "kb_p", "kb_chain", "kb_a", "kb_b", "kb_c"]

@@ -924,7 +924,7 @@ cudaError_t run_bwd_dk(const Tin* q, const Tin* k, const Tin* v, const Tin* la, 
     timing_mark(stream, 4);
     if (std::is_same<Tin, __nv_bfloat16>::value && DK == 128 && dv == 128 && ws.tc_ws && ws.T) {
         // bf16, d = 128: the back substitution as two tensor-core products with T
-        e = launch_kb_b_tc(ws.T, ws.At, ws.fwd.U, ws.fwd.Wk, ws.dW, ws.dWk, k, v, beta, ws.fwd.g, ws.fwd.gl, dv_,
+        e = launch_kb_b_tc(ws.T, ws.At, ws.tc_ws, ws.dW, ws.dWk, k, v, beta, ws.fwd.g, ws.fwd.gl, dv_,
                            dbeta, ws.dKg, ws.dAt, reinterpret_cast<int*>(ws.tc_ws), cmap, n_chunks, H, stream);
         if (e != cudaSuccess) return e;
     } else {
@@ -956,7 +956,7 @@ cudaError_t run_bwd(const Tin* q, const Tin* k, const Tin* v, const Tin* la, con
         // bf16, d = 128: the tensor-core forward recomputes U, Wk, W and the chunk start states
         if ((e = launch_simt_g(dtype, la, cmap, n_chunks, H, dk, ws.fwd, stream)) != cudaSuccess) return e;
         e = launch_tc_states(q, k, v, la, beta, init_state, ws.o_scratch, cmap, smap, n_chunks, n_seqs, H, ws.tc_ws,
-                             ws.fwd.S_chunk, ws.fwd.W, ws.fwd.U, ws.fwd.Wk, ws.T, ws.At, stream);
+                             ws.fwd.S_chunk, ws.fwd.W, ws.T, ws.At, stream);
     } else {
         e = launch_simt_states(dtype, k, v, la, beta, init_state, cmap, smap, n_chunks, n_seqs, H, dk, dv, C, ws.fwd,
                                stream);

@@ -27,7 +27,8 @@
 //     [Y | Z] = T^T [dW | dWk]          (M =  64, N = 256, K =  64)
 //     dA = -[Y | Z] [U | Wk]^T, i < r   (M =  64, N =  64, K = 256)
 // then dv = beta Y, dKg = beta Z, dbeta_r = v_r.Y_r + Kg_r.Z_r + sum_i dA_ri At_ri
-// and dAt = Diag(beta) dA on CUDA cores.  T's row-major image is the MN-major A
+// and dAt = Diag(beta) dA on CUDA cores.  U and Wk come straight from the
+// recompute's per-chunk image (U fp32, Wk as its hi/lo bf16 rows).  T's row-major image is the MN-major A
 // operand of the first product, [dW | dWk] its MN-major B operand; the second
 // reads [Y | Z] (from tensor memory, split into bf16 hi/lo) as its K-major A
 // operand and [U | Wk] as its K-major B operand.
@@ -298,9 +299,35 @@ __device__ __forceinline__ void stage_pair(uint8_t* hi, uint8_t* lo, const float
     }
 }
 
+// [U | Wk] (64 token rows x 256, K-major) straight from the recompute's image of
+// this (chunk, head): U from its fp32 tile, split as above; Wk's hi and lo bf16
+// chunks copied as they are (rows 0-63 of the [Wk ; Q exp(g)] image); rows past
+// the chunk's end zero.
+__device__ __forceinline__ void stage_u_wk_image(uint8_t* hi, uint8_t* lo, const uint8_t* img, int len, int tid) {
+    const float* u = reinterpret_cast<const float*>(img + kOffU);
+#pragma unroll 4
+    for (int it = 0; it < 8; ++it) {
+        const int e = tid + kAThreads * it, i = e >> 5, j4 = (e & 31) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < len) x = *reinterpret_cast<const float4*>(u + u_index(i, j4));
+        store4_split(hi, lo, sw128_offset(i, j4, 64), x);
+    }
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+        const int e = tid + kAThreads * it, i = e >> 4, j8 = (e & 15) * 8;
+        uint4 xh = make_uint4(0u, 0u, 0u, 0u), xl = xh;
+        if (i < len) {
+            xh = *reinterpret_cast<const uint4*>(img + kOffWkQh + sw128_chunk(i, j8, 128));
+            xl = *reinterpret_cast<const uint4*>(img + kOffWkQl + sw128_chunk(i, j8, 128));
+        }
+        *reinterpret_cast<uint4*>(hi + sw128_chunk(i, kD + j8, 64)) = xh;
+        *reinterpret_cast<uint4*>(lo + sw128_chunk(i, kD + j8, 64)) = xl;
+    }
+}
+
 __global__ void __launch_bounds__(kAThreads, 1)
-kb_b_tc(const float* __restrict__ T, const float* __restrict__ At, const float* __restrict__ U,
-        const float* __restrict__ Wk, const float* __restrict__ dW, const float* __restrict__ dWk,
+kb_b_tc(const float* __restrict__ T, const float* __restrict__ At, const uint8_t* __restrict__ images,
+        const float* __restrict__ dW, const float* __restrict__ dWk,
         const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
         const __nv_bfloat16* __restrict__ beta, const float* __restrict__ g, const float* __restrict__ gl,
         __nv_bfloat16* __restrict__ dv_out, __nv_bfloat16* __restrict__ dbeta_out, float* __restrict__ dKg,
@@ -338,7 +365,7 @@ kb_b_tc(const float* __restrict__ T, const float* __restrict__ At, const float* 
         store4_split(sm + kBTh, sm + kBTl, sw128_offset(i, c4, 64), x);
     }
     stage_pair(sm + kBXh, sm + kBXl, dW, dWk, tok0, len, H, h, tid);
-    stage_pair(sm + kBUh, sm + kBUl, U, Wk, tok0, len, H, h, tid);
+    stage_u_wk_image(sm + kBUh, sm + kBUl, images + (chunk * H + h) * (size_t)kChunkBytes, len, tid);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -772,15 +799,16 @@ cudaError_t launch_chain(const uint8_t* ws, const void* d_o, const float* d_fina
 
 }  // namespace
 
-cudaError_t launch_kb_b_tc(const float* T, const float* At, const float* U, const float* Wk, const float* dW,
+cudaError_t launch_kb_b_tc(const float* T, const float* At, const void* tc_ws, const float* dW,
                            const float* dWk, const void* k, const void* v, const void* beta, const float* g,
                            const float* gl, void* dv_out, void* dbeta_out, float* dKg, float* dAt, int* err,
                            const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream) {
     if (n_chunks == 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kb_b_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBSmem);
     if (e != cudaSuccess) return e;
+    const uint8_t* images = reinterpret_cast<const uint8_t*>(tc_ws) + kErrHeader;
     kb_b_tc<<<dim3(n_chunks, H), kAThreads, kBSmem, stream>>>(
-        T, At, U, Wk, dW, dWk, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)beta, g, gl,
+        T, At, images, dW, dWk, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, (const __nv_bfloat16*)beta, g, gl,
         (__nv_bfloat16*)dv_out, (__nv_bfloat16*)dbeta_out, dKg, dAt, err, cmap, H);
     return cudaGetLastError();
 }

@@ -1290,24 +1290,6 @@ cudaError_t launch_recur(const uint8_t* ws, const float* init_state, float* fina
     return cudaGetLastError();
 }
 
-// U (fp32, row-swizzled) and Wk (rows 0-63 of the [Wk ; Q exp(g)] hi/lo images) of
-// every chunk-head as plain token-major fp32 arrays [tokens, H, 128].
-__global__ void __launch_bounds__(256) tc_unpack_u_wk(const uint8_t* __restrict__ ws, float* __restrict__ U,
-                                                      float* __restrict__ Wk, ChunkMap cmap, int H) {
-    int seq, tok0, len, idx;
-    cmap.locate(blockIdx.x, seq, tok0, len, idx);
-    const int h = blockIdx.y;
-    const uint8_t* src = ws + ((size_t)blockIdx.x * H + h) * kChunkBytes;
-    const float* uo = reinterpret_cast<const float*>(src + kOffU);
-    for (int e = threadIdx.x; e < len * kD; e += 256) {
-        const int r = e >> 7, j = e & 127;
-        const size_t off = ((size_t)(tok0 + r) * H + h) * kD + j;
-        U[off] = uo[u_index(r, j & ~3) + (j & 3)];
-        const uint32_t b = sw128_offset(r, j, 128);
-        Wk[off] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(src + kOffWkQh + b)) +
-                  __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(src + kOffWkQl + b));
-    }
-}
 
 // multiprocessors of the current device, looked up once per device
 int sm_count() {
@@ -1371,12 +1353,13 @@ cudaError_t launch_tc_prefill(const void* q, const void* k, const void* v, const
 }
 
 // The forward intermediates the backward pass needs, from the tensor-core path:
-// every chunk's start state and W (fp32, from the state carry) and U, Wk (fp32,
-// unpacked from the per-chunk workspace).  o_scratch receives the outputs.
+// the per-chunk images (read again by the gradient kernels), T and the key
+// products, and every chunk's start state and W (fp32, from the state carry).
+// o_scratch receives the outputs.
 cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
-                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
-                             float* Wk, float* T_store, float* At_store, cudaStream_t stream) {
+                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W,
+                             float* T_store, float* At_store, cudaStream_t stream) {
     int* err = reinterpret_cast<int*>(tc_ws);
     uint8_t* ws = reinterpret_cast<uint8_t*>(tc_ws) + kErrHeader;
     cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
@@ -1387,8 +1370,6 @@ cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const 
         tc_intra<false><<<(unsigned)((long)n_chunks * H), kIntraThreads, kIntraAlloc, stream>>>(
             (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
             (const __nv_bfloat16*)log_alpha, (const __nv_bfloat16*)beta, ws, err, cmap, H, 0u, 0ull, T_store, At_store);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        tc_unpack_u_wk<<<dim3(n_chunks, H), 256, 0, stream>>>(ws, U, Wk, cmap, H);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (n_seqs > 0) {

@@ -206,12 +206,13 @@ struct BwdWorkspace {
 cudaError_t launch_simt_g(kda_dtype dtype, const void* log_alpha, const ChunkMap& cmap, int n_chunks, int H, int dk,
                           const SimtWorkspace& ws, cudaStream_t stream);
 
-// Tensor-core recompute for the backward pass (bf16, d = 128): chunk start
-// states and W from the state carry, U and Wk unpacked from the workspace.
+// Tensor-core recompute for the backward pass (bf16, d = 128): the per-chunk
+// images in tc_ws, T and the key products, and the chunk start states and W
+// from the state carry.
 cudaError_t launch_tc_states(const void* q, const void* k, const void* v, const void* log_alpha, const void* beta,
                              const float* init_state, void* o_scratch, const ChunkMap& cmap, const SeqMap& smap,
-                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W, float* U,
-                             float* Wk, float* T_store, float* At_store, cudaStream_t stream);
+                             int n_chunks, int n_seqs, int H, void* tc_ws, float* S_chunk, float* W,
+                             float* T_store, float* At_store, cudaStream_t stream);
 
 cudaError_t launch_simt_backward(kda_dtype dtype, const void* q, const void* k, const void* v,
                                  const void* log_alpha, const void* beta, const float* init_state,
@@ -231,7 +232,7 @@ cudaError_t launch_tc_chain(void* tc_ws, const void* d_o, const float* d_final, 
 // Tensor-core back substitution of the backward pass (bf16, d = 128):
 // [Y | Z] = T^T [dW | dWk], dA = -(Y U^T + Z Wk^T) (i < r), dv = beta Y, dKg = beta Z,
 // dbeta_r = v_r.Y_r + Kg_r.Z_r + sum_i dA_ri At_ri, dAt = Diag(beta) dA.
-cudaError_t launch_kb_b_tc(const float* T, const float* At, const float* U, const float* Wk, const float* dW,
+cudaError_t launch_kb_b_tc(const float* T, const float* At, const void* tc_ws, const float* dW,
                            const float* dWk, const void* k, const void* v, const void* beta, const float* g,
                            const float* gl, void* dv_out, void* dbeta_out, float* dKg, float* dAt, int* err,
                            const ChunkMap& cmap, int n_chunks, int H, cudaStream_t stream);
