@@ -120,6 +120,17 @@ __device__ __forceinline__ void store8_split(uint8_t* hi_tile, uint8_t* lo_tile,
     *reinterpret_cast<uint4*>(lo_tile + off) = lv;
 }
 
+// The same with the hi and lo values at different offsets of their tiles.
+__device__ __forceinline__ void store8_split2(uint8_t* hi, uint32_t ohi, uint8_t* lo, uint32_t olo, const float* x) {
+    uint4 hv, lv;
+    split2(x[0], x[1], hv.x, lv.x);
+    split2(x[2], x[3], hv.y, lv.y);
+    split2(x[4], x[5], hv.z, lv.z);
+    split2(x[6], x[7], hv.w, lv.w);
+    *reinterpret_cast<uint4*>(hi + ohi) = hv;
+    *reinterpret_cast<uint4*>(lo + olo) = lv;
+}
+
 __device__ __forceinline__ void record_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
@@ -136,6 +147,22 @@ __device__ __forceinline__ void mma3(uint32_t d, uint32_t ah, uint32_t al, int a
         mma_bf16(d, dah, dbh, idesc, acc0);
         mma_bf16(d, dah, dbl, idesc, 1u);
         mma_bf16(d, dal, dbh, idesc, 1u);
+    }
+}
+
+// The same three terms with B MN-major and its hi and lo tiles side by side as one
+// operand [B_hi | B_lo] of width 2N (the lo tile one 64-wide block after the hi
+// tile): D[0, N) (+)= A_hi B_hi + A_lo B_hi and D[N, 2N) (+)= A_hi B_lo, two MMAs
+// per K-slice instead of three (each A tile read once); the caller adds the two
+// halves of D.
+__device__ __forceinline__ void mma2w(uint32_t d, uint32_t ah, uint32_t al, int arows, uint32_t bh, int brows,
+                                      int ksteps, uint32_t idesc_wide, uint32_t idesc_narrow, bool accumulate) {
+    for (int s = 0; s < ksteps; ++s) {
+        const uint32_t acc0 = (accumulate || s > 0) ? 1u : 0u;
+        const uint64_t dah = sw128_desc_k(ah, arows, s), dal = sw128_desc_k(al, arows, s);
+        const uint64_t db = mn_desc_k(bh, brows, s);
+        mma_bf16(d, dah, db, idesc_wide, acc0);
+        mma_bf16(d, dal, db, idesc_narrow, 1u);
     }
 }
 
@@ -952,7 +979,13 @@ struct RecurLayout {
     static constexpr uint32_t kBars = kW + 2 * 2 * 8192;
     static constexpr uint32_t kSmem = kBars + 128;
     static constexpr uint32_t kAlloc = kSmem + 1024;
-    static constexpr uint32_t kTmemCols = (3 * BV <= 32) ? 32 : (3 * BV <= 64) ? 64 : (3 * BV <= 128) ? 128 : 256;
+    // The products take [hi | lo] B operands (mma2w): D and S in two column ranges each
+    // (D buffers 2 x 2 BV, S 2 BV).  At 64 columns the lo tiles of S and W are the
+    // 64-wide blocks after the hi tiles; at 32 the second halves of the same rows.
+    static_assert(BV == 32 || BV == 64, "state column tiles of 32 or 64");
+    static constexpr uint32_t kCols = 6 * BV;
+    static constexpr uint32_t kTmemCols = (kCols <= 32) ? 32 : (kCols <= 64) ? 64 : (kCols <= 128) ? 128
+                                                       : (kCols <= 256) ? 256 : 512;
 };
 
 // MODE 0: the prefill.  MODE 1 (for the backward pass): also every chunk's start
@@ -1025,7 +1058,20 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sflags[0];
-    const uint32_t t_s = tbase + 2 * BV;     // S (columns [2 BV, 3 BV)); D of chunk n: columns [BV (n % 2), + BV)
+    // D of chunk n: columns [DW (n % 2), + DW); S: from 2 DW.  D and S are each the sum
+    // of two BV-column ranges (the A_hi B_lo term of the products in the second).
+    constexpr uint32_t DW = 2 * BV;
+    const uint32_t t_s = tbase + 2 * DW;
+    auto t_dbuf = [&](int m) { return tbase + (uint32_t)(DW * (m & 1)); };
+    // 16 columns of D or S at column offset col: the sum of the two ranges
+    auto ld_sum16 = [&](uint32_t t, int col, float (&v)[16]) {
+        float w[16];
+        tmem_ld16(tmem_addr(t, 32 * sp, col), v);
+        tmem_ld16(tmem_addr(t, 32 * sp, BV + col), w);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] += w[e];
+    };
 
     auto chunk_src = [&](int n) {
         return ws + (size_t)((size_t)(sq.chunk0 + n) * H + h) * kChunkBytes;
@@ -1091,17 +1137,17 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         } else {
             const uint32_t a = smem_u32(sm + Lay::kP);
             const uint32_t wh = smem_u32(w_hi(m));
-            mma3(tbase + (uint32_t)(BV * (m & 1)), a, a + 16384, 128, wh, wh + 8192, 64, true, kC / 16,
-                 idesc_bf16_f32_bmn(128, BV), true);
+            mma2w(t_dbuf(m), a, a + 16384, 128, wh, 64, kC / 16, idesc_bf16_f32_bmn(128, 2 * BV),
+                  idesc_bf16_f32_bmn(128, BV), true);
         }
         mma_commit(bar_o);
     };
     // O rows of chunk m out of D (warps with sp >= 2: rows 64-127 = token rows 0-63)
     auto emit_o = [&](int m) {
-        const uint32_t t_d = tbase + (uint32_t)(BV * (m & 1));
+        const uint32_t t_d = t_dbuf(m);
         float d[NG][16];
 #pragma unroll
-        for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
+        for (int g = 0; g < NG; ++g) ld_sum16(t_d, cq + 16 * g, d[g]);
         tmem_ld_wait();
         const int r = c - 64;
         if (r < min(kC, sq.len - m * kC)) {
@@ -1124,16 +1170,18 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         const int stage = n & 1;
         const uint8_t* uu = sm + Lay::kUU + stage * Lay::kUStage;
         const uint32_t par = (uint32_t)n & 1u;
-        const uint32_t t_d = tbase + (uint32_t)(BV * (n & 1));
+        const uint32_t t_d = t_dbuf(n);
         if (STORE) {
             float* dst = s_store + ((((size_t)sq.chunk0 + n) * H + h) * kD + c) * kD + j0 + cq;
 #pragma unroll
             for (int j = 0; j < HB; j += 4)
                 *reinterpret_cast<float4*>(dst + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
         }
-        // S_n as the MN-major B operand (K = channel row c, N = columns)
+        // S_n as the MN-major B operand (K = channel row c, N = columns), hi and lo tiles
 #pragma unroll
-        for (int j = 0; j < HB; j += 8) store8_split(s_h, s_l, mn_chunk(c, cq + j, 128), s + j);
+        for (int j = 0; j < HB; j += 8)
+            store8_split2(s_h, mn_chunk(c, cq + j, 128), BV == 32 ? s_h : s_l,
+                          mn_chunk(c, (BV == 32 ? 32 : 0) + cq + j, 128), s + j);
         if (!mbar_wait(&uu_full[stage], (uint32_t)(n >> 1) & 1u)) fail();
         // Diag(Gamma_C) S_n into TMEM; the S update accumulates on top of it
         const float gam = reinterpret_cast<const float*>(uu + Lay::kUtile)[c];
@@ -1143,6 +1191,10 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
 #pragma unroll
             for (int e = 0; e < 16; ++e) t[e] = gam * s[16 * g + e];
             tmem_st16(tmem_addr(t_s, 32 * sp, cq + 16 * g), t);
+            // the second range starts from zero (one accumulate flag covers both)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) t[e] = 0.f;
+            tmem_st16(tmem_addr(t_s, 32 * sp, BV + cq + 16 * g), t);
         }
         tmem_st_wait();
         // test of the failure path (stall_ns != 0): the first CTA waits, bounded, on a
@@ -1158,8 +1210,8 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                 fail();
             } else {
                 const uint32_t a = smem_u32(sm + Lay::kWkQ);
-                mma3(t_d, a, a + 32768, 128, smem_u32(s_h), smem_u32(s_l), 128, true, kD / 16,
-                     idesc_bf16_f32_bmn(128, BV), false);
+                mma2w(t_d, a, a + 32768, 128, smem_u32(s_h), 128, kD / 16, idesc_bf16_f32_bmn(128, 2 * BV),
+                      idesc_bf16_f32_bmn(128, BV), false);
             }
             mma_commit(bar_d);
             mbar_arrive(d_issued);   // the previous chunk's output product may follow it
@@ -1174,7 +1226,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
             uint8_t* w_h = w_hi(n);
             float d[NG][16];
 #pragma unroll
-            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_d, 32 * sp, cq + 16 * g), d[g]);
+            for (int g = 0; g < NG; ++g) ld_sum16(t_d, cq + 16 * g, d[g]);
             tmem_ld_wait();
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
@@ -1186,8 +1238,10 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                     d[g][e] = u.x - d[g][e]; d[g][e + 1] = u.y - d[g][e + 1];
                     d[g][e + 2] = u.z - d[g][e + 2]; d[g][e + 3] = u.w - d[g][e + 3];
                 }
-                store8_split(w_h, w_h + 8192, mn_chunk(r, jb, 64), d[g]);
-                store8_split(w_h, w_h + 8192, mn_chunk(r, jb + 8, 64), d[g] + 8);
+                uint8_t* w_l = BV == 32 ? w_h : w_h + 8192;
+                const int lc = BV == 32 ? 32 : 0;
+                store8_split2(w_h, mn_chunk(r, jb, 64), w_l, mn_chunk(r, lc + jb, 64), d[g]);
+                store8_split2(w_h, mn_chunk(r, jb + 8, 64), w_l, mn_chunk(r, lc + jb + 8, 64), d[g] + 8);
                 if (STORE && r < min(kC, sq.len - n * kC)) {
                     float* dst = w_store + ((size_t)(sq.tok0 + n * kC + r) * H + h) * kD + j0 + jb;
 #pragma unroll
@@ -1204,8 +1258,8 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
                     fail();
                 } else {
                     const uint32_t a = smem_u32(sm + Lay::kKdT);
-                    mma3(t_s, a, a + 16384, 128, smem_u32(w_h), smem_u32(w_h) + 8192, 64, true, kC / 16,
-                         idesc_bf16_f32_bmn(128, BV), true);
+                    mma2w(t_s, a, a + 16384, 128, smem_u32(w_h), 64, kC / 16, idesc_bf16_f32_bmn(128, 2 * BV),
+                          idesc_bf16_f32_bmn(128, BV), true);
                 }
                 mma_commit(bar_s);
             }
@@ -1239,7 +1293,7 @@ tc_recur(const uint8_t* __restrict__ ws, const float* __restrict__ init_state, f
         {
             float t[NG][16];
 #pragma unroll
-            for (int g = 0; g < NG; ++g) tmem_ld16(tmem_addr(t_s, 32 * sp, cq + 16 * g), t[g]);
+            for (int g = 0; g < NG; ++g) ld_sum16(t_s, cq + 16 * g, t[g]);
             tmem_ld_wait();
 #pragma unroll
             for (int g = 0; g < NG; ++g)
