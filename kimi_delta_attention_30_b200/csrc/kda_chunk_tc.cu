@@ -598,18 +598,19 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 
     // ---- diagonal blocks with a large decay range: pairwise on CUDA cores ----------
     // Block R's 16 rows are staged in shared memory (k and q in fp32, normalised
-    // when asked, and the block-local cumulative log decay times log2 e, so every
-    // factor is 2^(a - b) of two sums over at most 16 tokens).  Warp w forms the
-    // 17 pairs (r, i <= r) of rows w and 15 - w, each lane over 4 channels; the 34
-    // per-lane sums (A and P of each pair) are reduced across the warp by halving
-    // exchanges, after which lane l holds sum number l.  (Splitting each pair's
-    // factor at a 4-row sub-block boundary, so that the exponentials are formed per
-    // row instead of per pair, measured slower: each key version serves about three
-    // pairs, so building the versions costs what the pairs save.)
+    // when asked, and each token's decay alpha = exp(log alpha) per channel).  Warp w
+    // forms the 17 pairs (r, i <= r) of rows w and 15 - w, each lane over 4 channels,
+    // walking i down from r: the factor prod_{i < j <= r} alpha_j starts at 1 on the
+    // diagonal and takes one more alpha per step, so a block costs one exponential
+    // per (row, channel) instead of one per (pair, channel), and each factor carries
+    // at most 15 roundings (the difference of two cumulative sums carries their
+    // absolute error, up to 16 |log alpha| ulps, into the exponent).  The 34 per-lane
+    // sums (A and P of each pair) are reduced across the warp by halving exchanges,
+    // after which lane l holds sum number l.
     if (!abort && fbmask) {
         float* fk = reinterpret_cast<float*>(sm + kFbStage);   // [16][128] k
         float* fq = fk + 16 * 128;                              // [16][128] q
-        float* fg = fq + 16 * 128;                              // [16][128] block-local g * log2 e
+        float* fa = fq + 16 * 128;                              // [16][128] alpha
         // thread: one row, 8 consecutive channels of k, q and log alpha; the next
         // flagged block's are loaded while the current one's pairs are formed
         const int frow = tid >> 4, fc8 = (tid & 15) * 8;
@@ -635,52 +636,45 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 const uint32_t lw[4] = {nl8.x, nl8.y, nl8.z, nl8.w};
                 float* dk_ = fk + frow * 128 + fc8;
                 float* dq_ = fq + frow * 128 + fc8;
-                float* dg_ = fg + frow * 128 + fc8;
+                float* da_ = fa + frow * 128 + fc8;
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     *reinterpret_cast<float2*>(dk_ + 2 * m) = mul2(unpack_bf16x2(kw[m]), sk);
                     *reinterpret_cast<float2*>(dq_ + 2 * m) = mul2(unpack_bf16x2(qw[m]), sq);
+                    // rows past the end are never a factor of a kept pair
                     const float2 l2 = prep_log_alpha2(unpack_bf16x2(lw[m]), prep);
-                    *reinterpret_cast<float2*>(dg_ + 2 * m) = (rr < len) ? l2 : make_float2(0.f, 0.f);
+                    *reinterpret_cast<float2*>(da_ + 2 * m) =
+                        make_float2(ex2_approx(l2.x * kLog2e), ex2_approx(l2.y * kLog2e));
                 }
             }
             const unsigned rest = fbmask & ~((2u << R) - 1u);
             const int Rn = rest ? __ffs(rest) - 1 : 4;
             if (Rn < 4) fetch(Rn);
             __syncthreads();
-            if (tid < 128) {
-                float acc = 0.f;
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    acc += fg[rr * 128 + tid];
-                    fg[rr * 128 + tid] = acc * kLog2e;
-                }
-            }
-            __syncthreads();
             {
                 const int ra = warp, rb = 15 - warp;
                 // the two rows' values, read once; the pairs select between them
-                const float4 gra = *reinterpret_cast<const float4*>(fg + ra * 128 + 4 * lane);
                 const float4 kra = *reinterpret_cast<const float4*>(fk + ra * 128 + 4 * lane);
                 const float4 qra = *reinterpret_cast<const float4*>(fq + ra * 128 + 4 * lane);
-                const float4 grb = *reinterpret_cast<const float4*>(fg + rb * 128 + 4 * lane);
                 const float4 krb = *reinterpret_cast<const float4*>(fk + rb * 128 + 4 * lane);
                 const float4 qrb = *reinterpret_cast<const float4*>(fq + rb * 128 + 4 * lane);
                 float v[34];
+                float2 e0 = make_float2(1.f, 1.f), e1 = e0;
 #pragma unroll
                 for (int jj = 0; jj < 17; ++jj) {
+                    // pair jj: row ra with i = ra - jj, then row rb with i = 16 - jj
                     const bool first = jj <= ra;
-                    const int i = first ? jj : jj - ra - 1;
-                    const float4 gr = first ? gra : grb;
+                    const int i = first ? ra - jj : 16 - jj;
                     const float4 kr = first ? kra : krb;
                     const float4 qr = first ? qra : qrb;
-                    const float4 gi = *reinterpret_cast<const float4*>(fg + i * 128 + 4 * lane);
                     const float4 ki = *reinterpret_cast<const float4*>(fk + i * 128 + 4 * lane);
-                    // 2^(g_r - g_i) <= 1 (i <= r)
-                    const float2 d0 = fma2(make_float2(gi.x, gi.y), make_float2(-1.f, -1.f), make_float2(gr.x, gr.y));
-                    const float2 d1 = fma2(make_float2(gi.z, gi.w), make_float2(-1.f, -1.f), make_float2(gr.z, gr.w));
-                    const float2 e0 = make_float2(ex2_approx(d0.x), ex2_approx(d0.y));
-                    const float2 e1 = make_float2(ex2_approx(d1.x), ex2_approx(d1.y));
+                    if (jj == 0 || jj == ra + 1) {   // the diagonal pair of a row
+                        e0 = e1 = make_float2(1.f, 1.f);
+                    } else {                          // one more token's decay
+                        const float4 ai = *reinterpret_cast<const float4*>(fa + (i + 1) * 128 + 4 * lane);
+                        e0 = mul2(e0, make_float2(ai.x, ai.y));
+                        e1 = mul2(e1, make_float2(ai.z, ai.w));
+                    }
                     const float2 ke0 = mul2(make_float2(ki.x, ki.y), e0), ke1 = mul2(make_float2(ki.z, ki.w), e1);
                     float2 a2 = mul2(make_float2(kr.x, kr.y), ke0), p2 = mul2(make_float2(qr.x, qr.y), ke0);
                     a2 = fma2(make_float2(kr.z, kr.w), ke1, a2);
@@ -707,7 +701,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 }
                 auto put = [&](int jj, bool is_p, float val) {
                     const bool first = jj <= ra;
-                    const int r = first ? ra : rb, i = first ? jj : jj - ra - 1;
+                    const int r = first ? ra : rb, i = first ? ra - jj : 16 - jj;
                     const int row = 16 * R + r, col = 16 * R + i;
                     if (!is_p) {
                         As[row * kAS + col] = (i < r && row < len) ? sbeta[row] * val : 0.f;
