@@ -229,6 +229,7 @@ def design_bytes(kernel: str, g: Geometry, in_bytes=2):
         + 2 * g.state_bytes,
         "k4_output": th * (2 * g.dk * in_bytes + 8 * g.dk + 4 * g.dv + g.dv * in_bytes) + schunk,
         "seq_table_write": 0,
+        "chunk_table_fill": 0,
     }
     return table.get(kernel, None) if kernel != "simt" else simt_ws
 
@@ -293,7 +294,7 @@ def prefill_report(g: Geometry, C_req: int, C_run: int, kernels, k_avg_ms, ms_pe
     t = ms_per_step / 1e3
     algo_b = minimal_bytes(g)
     flops = algorithmic_flops(g, C_run)
-    timed = [j for j, n in enumerate(kernels) if n != "seq_table_write"]
+    timed = [j for j, n in enumerate(kernels) if n not in ("seq_table_write", "chunk_table_fill")]
     dom = max(timed, key=lambda j: k_avg_ms[j])
     dom_s = k_avg_ms[dom] / 1e3
     ach = algo_b / dom_s / 1e9

@@ -62,10 +62,30 @@ __global__ void __launch_bounds__(256) seq_table_write(SeqInfo* __restrict__ dst
     for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = b.e[i];
 }
 
-// natural order then longest first, 2 n_seqs entries at `dst`; returns the number of
-// launches (with `mark`, timing-hook event i follows the i-th of them)
+// The per-chunk table (first token, length, sequence, index in the sequence), one
+// thread per chunk, from the natural-order sequence table written just before.
+__global__ void __launch_bounds__(256) chunk_table_fill(const SeqInfo* __restrict__ seqs, int n_seqs, int n_chunks,
+                                                        int C, int4* __restrict__ dst) {
+    const int c = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+    if (c >= n_chunks) return;
+    int lo = 0, hi = n_seqs - 1;
+    while (lo < hi) {   // last sequence whose first chunk is <= c
+        const int mid = (lo + hi + 1) >> 1;
+        if (seqs[mid].chunk0 <= c) lo = mid; else hi = mid - 1;
+    }
+    const SeqInfo sq = seqs[lo];
+    const int idx = c - sq.chunk0;
+    dst[c] = make_int4(sq.tok0 + idx * C, min(C, sq.len - idx * C), sq.seq, idx);
+}
+
+// the per-chunk table follows the two sequence tables
+int4* chunk_table(SeqInfo* tables, size_t n_seqs) { return reinterpret_cast<int4*>(tables + 2 * n_seqs); }
+
+// natural order then longest first, 2 n_seqs entries at `dst`, then the per-chunk
+// table of n_chunks entries of C tokens; returns the number of launches (with `mark`,
+// timing-hook event i follows the i-th of them)
 int upload_tables(SeqInfo* dst, const std::vector<SeqInfo>& natural, const std::vector<SeqInfo>& by_len,
-                  cudaStream_t s, cudaError_t* err, bool mark = false) {
+                  int n_chunks, int C, cudaStream_t s, cudaError_t* err, bool mark = false) {
     const size_t n = natural.size();
     int launches = 0;
     TableBatch b;
@@ -80,11 +100,20 @@ int upload_tables(SeqInfo* dst, const std::vector<SeqInfo>& natural, const std::
         if ((*err = cudaGetLastError()) != cudaSuccess) return launches;
         if (mark) timing_mark_abs(s, launches);
     }
+    if (n_chunks > 0) {
+        chunk_table_fill<<<(n_chunks + 255) / 256, 256, 0, s>>>(dst, (int)n, n_chunks, C, chunk_table(dst, n));
+        ++launches;
+        if ((*err = cudaGetLastError()) != cudaSuccess) return launches;
+        if (mark) timing_mark_abs(s, launches);
+    }
     *err = cudaSuccess;
     return launches;
 }
 
-int table_launches(size_t n_seqs) { return (int)((2 * n_seqs + kTableBatch - 1) / kTableBatch); }
+// launches of upload_tables: the sequence-table batches, then the chunk table
+int table_launches(size_t n_seqs, int n_chunks) {
+    return (int)((2 * n_seqs + kTableBatch - 1) / kTableBatch) + (n_chunks > 0 ? 1 : 0);
+}
 
 // Problem geometry shared by the workspace query and the launch.
 struct Plan {
@@ -129,8 +158,10 @@ kda_status make_plan(int B, int T, int H, int dk, int dv, int C, const int32_t* 
     return KDA_OK;
 }
 
-// Workspace layout: [sequence tables][algorithm scratch]
-size_t table_bytes(const Plan& p) { return p.varlen ? align_up(2 * sizeof(SeqInfo) * (size_t)p.n_seqs) : 0; }
+// Workspace layout: [sequence tables, chunk table][algorithm scratch]
+size_t table_bytes(const Plan& p) {
+    return p.varlen ? align_up(2 * sizeof(SeqInfo) * (size_t)p.n_seqs + sizeof(int4) * (size_t)p.n_chunks) : 0;
+}
 
 struct SimtLayout {
     size_t off[6];
@@ -324,13 +355,14 @@ kda_status chunk_fwd_impl(const void* q, const void* k, const void* v, const voi
     timing_mark(s, 0);
     if (p.varlen) {
         cudaError_t terr;
-        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr, true);
+        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, p.n_chunks, C, s, &terr, true);
         if (terr != cudaSuccess) {
             timing_hook().n = 0;
             timing_hook().base = 0;
             return KDA_ERR_CUDA;
         }
         cmap.seqs = (const SeqInfo*)ws;
+        cmap.chunks = chunk_table((SeqInfo*)ws, p.n_seqs);
         smap.order = (const SeqInfo*)ws + p.n_seqs;
     }
     cudaError_t err;
@@ -383,13 +415,14 @@ kda_status segment_map_impl(const void* q, const void* k, const void* v, const v
     timing_mark(s, 0);
     if (p.varlen) {
         cudaError_t terr;
-        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr, true);
+        timing_hook().base = upload_tables((SeqInfo*)ws, p.natural, p.by_len, p.n_chunks, C, s, &terr, true);
         if (terr != cudaSuccess) {
             timing_hook().n = 0;
             timing_hook().base = 0;
             return KDA_ERR_CUDA;
         }
         cmap.seqs = (const SeqInfo*)ws;
+        cmap.chunks = chunk_table((SeqInfo*)ws, p.n_seqs);
         smap.order = (const SeqInfo*)ws + p.n_seqs;
     }
     cudaError_t err;
@@ -480,9 +513,11 @@ int kda_chunk_fwd_kernels(int B, int T, int H, int dk, int dv, int C, kda_dtype 
     if (st != KDA_OK) return st;
     algo = resolve(algo, dtype, dk, dv, C);
     const char* const* list = (algo == KDA_ALGO_TC) ? kTcKernelNames : kSimtKernelNames;
-    const int nt = p.varlen ? table_launches(p.natural.size()) : 0;   // sequence-table writes come first
+    // the table writes come first: sequence-table batches, then the chunk table
+    const int nt = p.varlen ? table_launches(p.natural.size(), p.n_chunks) : 0;
     const int n = (algo == KDA_ALGO_TC) ? kTcKernelCount : 4;
-    for (int i = 0; names && i < nt + n && i < max_names; ++i) names[i] = i < nt ? "seq_table_write" : list[i - nt];
+    for (int i = 0; names && i < nt + n && i < max_names; ++i)
+        names[i] = i < nt ? (p.n_chunks > 0 && i == nt - 1 ? "chunk_table_fill" : "seq_table_write") : list[i - nt];
     return nt + n;
 }
 
@@ -529,9 +564,10 @@ kda_status kda_chunk_bwd(const void* q, const void* k, const void* v, const void
     SeqMap smap{nullptr, T, Cb, ncps};
     if (p.varlen) {
         cudaError_t terr;
-        upload_tables((SeqInfo*)ws, p.natural, p.by_len, s, &terr);
+        upload_tables((SeqInfo*)ws, p.natural, p.by_len, p.n_chunks, Cb, s, &terr);
         if (terr != cudaSuccess) return KDA_ERR_CUDA;
         cmap.seqs = (const SeqInfo*)ws;
+        cmap.chunks = chunk_table((SeqInfo*)ws, p.n_seqs);
         smap.order = (const SeqInfo*)ws + p.n_seqs;
     }
     auto f = [&](size_t off) { return (float*)(ws + off); };

@@ -600,13 +600,14 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     // Block R's 16 rows are staged in shared memory (k and q in fp32, normalised
     // when asked, and each token's decay alpha = exp(log alpha) per channel).  Warp w
     // forms the 17 pairs (r, i <= r) of rows w and 15 - w, each lane over 4 channels,
-    // walking i down from r: the factor prod_{i < j <= r} alpha_j starts at 1 on the
-    // diagonal and takes one more alpha per step, so a block costs one exponential
-    // per (row, channel) instead of one per (pair, channel), and each factor carries
-    // at most 15 roundings (the difference of two cumulative sums carries their
-    // absolute error, up to 16 |log alpha| ulps, into the exponent).  The 34 per-lane
-    // sums (A and P of each pair) are reduced across the warp by halving exchanges,
-    // after which lane l holds sum number l.
+    // walking i down from r: the factor prod_{i < j <= r} alpha_j, carried already
+    // multiplied into k_r and q_r, starts at 1 on the diagonal and takes one more
+    // alpha per step.  A block so costs one exponential per (row, channel) instead of
+    // one per (pair, channel), and each factor carries at most 15 roundings (the
+    // difference of two cumulative sums would carry their absolute error, up to
+    // 16 |log alpha| ulps, into the exponent).  The 34 per-lane sums (A and P of each
+    // pair) are reduced across the warp by halving exchanges, after which lane l
+    // holds sum number l.
     if (!abort && fbmask) {
         float* fk = reinterpret_cast<float*>(sm + kFbStage);   // [16][128] k
         float* fq = fk + 16 * 128;                              // [16][128] q
@@ -659,26 +660,31 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
                 const float4 krb = *reinterpret_cast<const float4*>(fk + rb * 128 + 4 * lane);
                 const float4 qrb = *reinterpret_cast<const float4*>(fq + rb * 128 + 4 * lane);
                 float v[34];
-                float2 e0 = make_float2(1.f, 1.f), e1 = e0;
+                // k_r and q_r times the decay from row r down to token i: the diagonal
+                // pair starts them at k_r, q_r and every later pair of the row multiplies
+                // in one more alpha (warp w's rows switch after pair w, a uniform branch)
+                float4 fA = kra, fP = qra;
 #pragma unroll
                 for (int jj = 0; jj < 17; ++jj) {
                     // pair jj: row ra with i = ra - jj, then row rb with i = 16 - jj
-                    const bool first = jj <= ra;
+                    const bool first = jj < 8 && jj <= ra;
                     const int i = first ? ra - jj : 16 - jj;
-                    const float4 kr = first ? kra : krb;
-                    const float4 qr = first ? qra : qrb;
-                    const float4 ki = *reinterpret_cast<const float4*>(fk + i * 128 + 4 * lane);
-                    if (jj == 0 || jj == ra + 1) {   // the diagonal pair of a row
-                        e0 = e1 = make_float2(1.f, 1.f);
-                    } else {                          // one more token's decay
-                        const float4 ai = *reinterpret_cast<const float4*>(fa + (i + 1) * 128 + 4 * lane);
-                        e0 = mul2(e0, make_float2(ai.x, ai.y));
-                        e1 = mul2(e1, make_float2(ai.z, ai.w));
+                    if (jj > 0) {
+                        // the row switch is a select (8 per pair of the first 8): a branch here
+                        // keeps the compiler from overlapping consecutive pairs
+                        const bool sw = jj <= 8 && jj == ra + 1;
+                        const float4 ai = *reinterpret_cast<const float4*>(fa + min(i + 1, 15) * 128 + 4 * lane);
+                        const float2 a01 = make_float2(ai.x, ai.y), a23 = make_float2(ai.z, ai.w);
+                        const float2 A01 = mul2(make_float2(fA.x, fA.y), a01), A23 = mul2(make_float2(fA.z, fA.w), a23);
+                        const float2 P01 = mul2(make_float2(fP.x, fP.y), a01), P23 = mul2(make_float2(fP.z, fP.w), a23);
+                        fA = sw ? krb : make_float4(A01.x, A01.y, A23.x, A23.y);
+                        fP = sw ? qrb : make_float4(P01.x, P01.y, P23.x, P23.y);
                     }
-                    const float2 ke0 = mul2(make_float2(ki.x, ki.y), e0), ke1 = mul2(make_float2(ki.z, ki.w), e1);
-                    float2 a2 = mul2(make_float2(kr.x, kr.y), ke0), p2 = mul2(make_float2(qr.x, qr.y), ke0);
-                    a2 = fma2(make_float2(kr.z, kr.w), ke1, a2);
-                    p2 = fma2(make_float2(qr.z, qr.w), ke1, p2);
+                    const float4 ki = *reinterpret_cast<const float4*>(fk + i * 128 + 4 * lane);
+                    float2 a2 = mul2(make_float2(ki.x, ki.y), make_float2(fA.x, fA.y));
+                    float2 p2 = mul2(make_float2(ki.x, ki.y), make_float2(fP.x, fP.y));
+                    a2 = fma2(make_float2(ki.z, ki.w), make_float2(fA.z, fA.w), a2);
+                    p2 = fma2(make_float2(ki.z, ki.w), make_float2(fP.z, fP.w), p2);
                     v[2 * jj] = a2.x + a2.y;
                     v[2 * jj + 1] = p2.x + p2.y;
                 }

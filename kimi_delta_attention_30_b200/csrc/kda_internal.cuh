@@ -27,6 +27,10 @@ struct ChunkMap {
     int T;          // tokens per sequence (equal-length case)
     int C;
     int ncps;       // chunks per sequence (equal-length case)
+    // packed batches: per chunk (first token, length, sequence, index in the sequence),
+    // filled once per call so that a kernel's first loads wait on one lookup instead of
+    // a search's chain of dependent loads; nullptr falls back to the search
+    const int4* chunks = nullptr;
 
     __device__ __forceinline__ void locate(int chunk, int& seq, int& tok0, int& len, int& idx) const {
         if (seqs == nullptr) {
@@ -34,6 +38,12 @@ struct ChunkMap {
             idx = chunk - seq * ncps;
             tok0 = seq * T + idx * C;
             len = min(C, T - idx * C);
+        } else if (chunks != nullptr) {
+            const int4 e = __ldg(chunks + chunk);
+            tok0 = e.x;
+            len = e.y;
+            seq = e.z;
+            idx = e.w;
         } else {
             int lo = 0, hi = n_seqs - 1;
             while (lo < hi) {            // last s with chunk0 <= chunk
