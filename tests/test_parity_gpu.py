@@ -227,7 +227,8 @@ def test_prefill_resume_and_handoff(cuda_ok):
     o2, s2 = kda.chunk_fwd(sl(inp.q, t1, 260), sl(inp.k, t1, 260), sl(inp.v, t1, 260),
                            sl(inp.log_alpha, t1, 260), sl(inp.beta, t1, 260), init_state=s1)
     torch.cuda.synchronize()
-    assert rel_err(to_f64(torch.cat([o1, o2], 1)), to_f64(o_all), stored_as="bf16") <= 2e-2
+    # two stored bf16 outputs: the storage half-ulp of each side is allowed
+    assert rel_err(to_f64(torch.cat([o1, o2], 1)), to_f64(o_all), stored_as="bf16", both_stored=True) <= 2e-2
     assert rel_err(to_f64(s2), to_f64(fs_all)) <= 2e-2
     # prefill 250 tokens, then 10 decode steps
     o_p, st = kda.chunk_fwd(sl(inp.q, 0, 250), sl(inp.k, 0, 250), sl(inp.v, 0, 250), sl(inp.log_alpha, 0, 250),
@@ -237,7 +238,7 @@ def test_prefill_resume_and_handoff(cuda_ok):
         outs.append(kda.decode_step(inp.q[:, t].contiguous(), inp.k[:, t].contiguous(), inp.v[:, t].contiguous(),
                                     inp.log_alpha[:, t].contiguous(), inp.beta[:, t].contiguous(), st))
     torch.cuda.synchronize()
-    assert rel_err(to_f64(torch.stack(outs, 1)), to_f64(o_all[:, 250:]), stored_as="bf16") <= 2e-2
+    assert rel_err(to_f64(torch.stack(outs, 1)), to_f64(o_all[:, 250:]), stored_as="bf16", both_stored=True) <= 2e-2
     assert rel_err(to_f64(st), to_f64(fs_all)) <= 2e-2
 
 
