@@ -449,8 +449,9 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
     // ---- first MMA in two channel halves --------------------------------------------
     // Round hr: every thread reads k and q of its 8 rows for its two channels in
     // half hr, builds that half's MMA operands and writes its Q exp(g) and Kd
-    // values to the workspace.
-#pragma unroll
+    // values to the workspace.  (The two rounds share one copy of the code: the
+    // kernel's largest stall is instruction fetch.)
+#pragma unroll 1
     for (int hr = 0; hr < 2; ++hr) {
         const int ch = 64 * hr + kc;
         // e = exp(g - gb[I]), f = exp(gb[I+1] - g)
@@ -471,7 +472,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int r = r0 + j;
-            const float2 gj = make_float2(g[j][2 * hr], g[j][2 * hr + 1]);
+            const float2 gj = hr ? make_float2(g[j][2], g[j][3]) : make_float2(g[j][0], g[j][1]);
             const float2 e = exp_diff2(gj, gref), f = exp_diff2(glast, gj);
             float2 k2 = unpack_bf16x2(kv[j]), q2 = unpack_bf16x2(qv[j]);
             if (PREP) {
