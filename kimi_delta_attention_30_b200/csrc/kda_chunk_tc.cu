@@ -790,10 +790,8 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         float* Yw = scr + warp * 128;   // [16][8] per warp
         if (warp < 4)
             tsolve_cols<2>(As, Ts, Yw, 0, 4 * warp, lane);
-        else if (warp < 6)
-            tsolve_cols<4>(As, Ts, Yw, 1, 16 + 8 * (warp - 4), lane);
-        else
-            tsolve_cols<4>(As, Ts, Yw, 2, 32 + 8 * (warp - 6), lane);
+        else   // one inlined copy for both block columns
+            tsolve_cols<4>(As, Ts, Yw, warp < 6 ? 1 : 2, warp < 6 ? 16 + 8 * (warp - 4) : 32 + 8 * (warp - 6), lane);
         __syncthreads();
         // for the backward pass: T itself, fp32 [64][64] per (chunk, head)
         if (t_store) {
@@ -907,7 +905,7 @@ tc_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ 
         const bool row_lane = lane < 16;
         const int cg = (warp >> 2) * 64;
         float* uo = reinterpret_cast<float*>(st_u);
-#pragma unroll
+#pragma unroll 1
         for (int bt = 0; bt < 2; ++bt) {
             const int j0 = cg + 32 * bt;
             float vals[2][16];
