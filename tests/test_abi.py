@@ -74,6 +74,27 @@ def test_tensor_core_path_serves_both_chunk_sizes_with_64_token_chunks():
         _ws(B=2, T=300, H=3, dk=128, dv=128, C=128, dtype=0, algo="simt")
 
 
+def test_packed_batches_launch_the_table_writes_first():
+    """A packed batch starts with the sequence-table write and the per-chunk table
+    (one 16-byte entry per chunk in the workspace); an equal-length batch has
+    neither."""
+    import torch
+    H, d = 3, 128
+    cu = [0, 100, 300, 301, 301, 365]          # an empty sequence included
+    for algo, first in (("tc", "tc_intra"), ("simt", "k1_cumsum")):
+        names = kda.chunk_kernels(1, 365, H, d, d, 64, torch.bfloat16, cu_seqlens=cu, algo=algo)
+        assert names[:3] == ["seq_table_write", "chunk_table_fill", first], names
+        names = kda.chunk_kernels(2, 365, H, d, d, 64, torch.bfloat16, algo=algo)
+        assert names[0] == first and "chunk_table_fill" not in names, names
+    # the two sequence tables (16 bytes per sequence each) and the chunk table sit
+    # ahead of the scratch: one more 64-token chunk adds its 16-byte entry besides
+    # the scratch it needs
+    w = _ws(B=1, T=365, H=H, dk=d, dv=d, C=64, dtype=0, cu=cu, algo="tc")
+    w_more = _ws(B=1, T=429, H=H, dk=d, dv=d, C=64, dtype=0, cu=cu[:-1] + [365, 429], algo="tc")
+    w_eq = _ws(B=1, T=365, H=H, dk=d, dv=d, C=64, dtype=0, algo="tc")
+    assert w > w_eq and w_more > w
+
+
 def test_simt_offsets_are_disjoint_and_ordered():
     off = kda.simt_offsets(2, 200, 3, 64, 64, 64)
     assert off == sorted(off) and len(set(off)) == 5
